@@ -1,0 +1,363 @@
+"""Pins for the fp64 oracle: facts fixed by the pages and by the mathematics.
+
+None of these tests re-types the oracle's formulas. Each one checks a closed
+form, a conservation law, a special case, an invariance or finite differences,
+chosen so that a dropped term, a wrong sign or index, a transposed operand or
+the wrong softmax axis fails at least one of them.
+
+Source: SequenceO1 (arXiv 2609.08443) §3.1 Eq. (7)-(9) (SA), §2.3 (STCA),
+§5.1 Table 1 (token-wise "vanilla" normalisation as the comparator).
+"""
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.sa import NORM_PROTO, NORM_TOKEN
+
+RNG = np.random.default_rng(1234)
+
+
+def _rand_problem(lengths, H=2, d=8, kp=5, per_user_q=False, seed=0, sigma_q=0.7):
+    rng = np.random.default_rng(seed)
+    T = int(sum(lengths))
+    B = len(lengths)
+    q = rng.standard_normal((B, H, kp, d) if per_user_q else (H, kp, d)) * sigma_q
+    k = rng.standard_normal((T, H, d))
+    v = rng.standard_normal((T, H, d))
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    return q, k, v, cu
+
+
+# ---------------------------------------------------------------- hand example
+# d = 2. Keys are one-hot so that S_{j,i} = q_j[c(i)]: k_0 = e_0, k_1 = e_1,
+# k_2 = e_0. Prototypes q_0 = (0, ln 2), q_1 = (ln 3, 0). Scores (rows j, cols i):
+#   S = [[0, ln2, 0], [ln3, 0, ln3]]
+# PROTO (down each column): exp -> [[1,2,1],[3,1,3]] -> A = [[1/4,2/3,1/4],[3/4,1/3,3/4]]
+# TOKEN (along each row):   A = [[1/4,1/2,1/4],[3/7,1/7,3/7]]
+# Values v_0 = (4,0), v_1 = (0,3), v_2 = (8,4).
+HAND_Q = np.array([[[0.0, math.log(2.0)], [math.log(3.0), 0.0]]])      # [H=1,k=2,d=2]
+HAND_K = np.array([[[1.0, 0.0]], [[0.0, 1.0]], [[1.0, 0.0]]])           # [T=3,H=1,d=2]
+HAND_V = np.array([[[4.0, 0.0]], [[0.0, 3.0]], [[8.0, 4.0]]])
+HAND_CU = np.array([0, 3])
+
+
+def _frac(a):
+    return np.array([[float(Fraction(x)) for x in row] for row in a])
+
+
+def test_hand_example_proto():
+    sk, lse, mass = oracle.sa_forward_proto(HAND_Q, HAND_K, HAND_V, HAND_CU)
+    # sketch_0 = 1/4 v0 + 2/3 v1 + 1/4 v2 = (3, 3); sketch_1 = 3/4 v0 + 1/3 v1 + 3/4 v2 = (9, 4)
+    np.testing.assert_allclose(sk[0, 0], [[3.0, 3.0], [9.0, 4.0]], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(mass[0, 0], [7 / 6, 11 / 6], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[:, 0], [math.log(4), math.log(3), math.log(4)], atol=1e-12)
+
+
+def test_hand_example_token():
+    sk, lse, mass = oracle.sa_forward_token(HAND_Q, HAND_K, HAND_V, HAND_CU)
+    # sketch_0 = (1/4)(4,0) + (1/2)(0,3) + (1/4)(8,4) = (3, 5/2)
+    # sketch_1 = (3/7)(4,0) + (1/7)(0,3) + (3/7)(8,4) = (36/7, 15/7)
+    np.testing.assert_allclose(sk[0, 0], _frac([["3", "5/2"], ["36/7", "15/7"]]), atol=1e-12)
+    np.testing.assert_allclose(mass[0, 0], [1.0, 1.0], atol=1e-12)
+    np.testing.assert_allclose(lse[0, 0], [math.log(4), math.log(7)], atol=1e-12)
+
+
+def test_hand_example_backward_proto_value():
+    # With dO = e_{j=0, c=0} the loss is sketch[0,0] = sum_i A_{0,i} v_i[0]; its
+    # gradient w.r.t. v_i[0] is A_{0,i} = (1/4, 2/3, 1/4) and 0 for v_i[1].
+    dO = np.zeros((1, 1, 2, 2))
+    dO[0, 0, 0, 0] = 1.0
+    _, _, dv = oracle.sa_backward_proto(HAND_Q, HAND_K, HAND_V, HAND_CU, None, dO)
+    np.testing.assert_allclose(dv[:, 0, 0], [0.25, 2 / 3, 0.25], atol=1e-12)
+    np.testing.assert_allclose(dv[:, 0, 1], 0.0, atol=1e-12)
+
+
+# ---------------------------------------------------------- conservation laws
+@pytest.mark.parametrize("scale", [1.0, 0.35])
+def test_proto_conservation_identity_values(scale):
+    """Eq. (8): with V = I the sketch is A itself, so each token's column sums to 1."""
+    n, d, kp = 6, 8, 5
+    q, k, _, cu = _rand_problem([n], H=1, d=d, kp=kp, seed=3)
+    v = np.zeros((n, 1, d))
+    for i in range(n):
+        v[i, 0, i] = 1.0
+    sk, _, _ = oracle.sa_forward_proto(q, k, v, cu, scale=scale)
+    A = sk[0, 0, :, :n]
+    np.testing.assert_allclose(A.sum(axis=0), 1.0, atol=1e-13)
+    assert (A > 0).all()
+
+
+def test_token_conservation_identity_values():
+    """Token-wise comparator: with V = I each prototype's row of A sums to 1."""
+    n, d, kp = 6, 8, 5
+    q, k, _, cu = _rand_problem([n], H=1, d=d, kp=kp, seed=4)
+    v = np.zeros((n, 1, d))
+    for i in range(n):
+        v[i, 0, i] = 1.0
+    sk, _, mass = oracle.sa_forward_token(q, k, v, cu)
+    np.testing.assert_allclose(sk[0, 0, :, :n].sum(axis=1), 1.0, atol=1e-13)
+    np.testing.assert_allclose(mass, 1.0, atol=1e-13)
+
+
+def test_proto_sum_over_prototypes_is_value_sum():
+    """Summing Eq. (9) over j and using Eq. (8): sum_j X~_j = sum_i x_i (valid i only)."""
+    lengths = [7, 1, 12]
+    used = [5, 1, 12]
+    q, k, v, cu = _rand_problem(lengths, H=3, d=8, kp=6, seed=5)
+    sk, _, mass = oracle.sa_forward_proto(q, k, v, cu, used)
+    for b in range(3):
+        lo = cu[b]
+        np.testing.assert_allclose(sk[b].sum(axis=1), v[lo:lo + used[b]].sum(axis=0), atol=1e-12)
+        np.testing.assert_allclose(mass[b].sum(axis=1), used[b], atol=1e-12)
+
+
+def test_token_ones_column():
+    """TOKEN: a value column of all ones gives a sketch column of ones."""
+    q, k, v, cu = _rand_problem([9, 4], H=2, d=8, kp=3, seed=6)
+    v[:, :, 2] = 1.0
+    sk, _, _ = oracle.sa_forward_token(q, k, v, cu)
+    np.testing.assert_allclose(sk[:, :, :, 2], 1.0, atol=1e-13)
+
+
+# ------------------------------------------------------------- special cases
+def test_proto_single_prototype_is_sum_pooling():
+    """k = 1: each token gives all its mass to the one prototype; X~ = sum_i x_i."""
+    q, k, v, cu = _rand_problem([10, 3], H=2, d=8, kp=1, seed=7)
+    sk, lse, _ = oracle.sa_forward_proto(q, k, v, cu, scale=0.5)
+    for b in range(2):
+        np.testing.assert_allclose(sk[b, :, 0], v[cu[b]:cu[b + 1]].sum(axis=0), atol=1e-12)
+    # lse_i = the single score 0.5 <q, k_i>
+    np.testing.assert_allclose(lse[:, 0], 0.5 * (k[:, 0] * q[0, 0][None, :]).sum(axis=1), atol=1e-12)
+
+
+def test_proto_zero_queries_split_evenly():
+    q, k, v, cu = _rand_problem([10], H=1, d=8, kp=4, seed=8)
+    q[:] = 0.0
+    sk, lse, mass = oracle.sa_forward_proto(q, k, v, cu)
+    np.testing.assert_allclose(sk[0, 0], np.tile(v[:, 0].sum(axis=0) / 4, (4, 1)), atol=1e-12)
+    np.testing.assert_allclose(lse[:, 0], math.log(4), atol=1e-13)
+    np.testing.assert_allclose(mass, 10 / 4, atol=1e-12)
+
+
+def test_token_zero_queries_mean_pooling():
+    q, k, v, cu = _rand_problem([10], H=1, d=8, kp=4, seed=9)
+    q[:] = 0.0
+    sk, lse, _ = oracle.sa_forward_token(q, k, v, cu)
+    np.testing.assert_allclose(sk[0, 0], np.tile(v[:, 0].mean(axis=0), (4, 1)), atol=1e-12)
+    np.testing.assert_allclose(lse[0, 0], math.log(10), atol=1e-13)
+
+
+def test_token_single_token():
+    q, k, v, cu = _rand_problem([1], H=2, d=8, kp=4, seed=10)
+    sk, lse, _ = oracle.sa_forward_token(q, k, v, cu, scale=0.3)
+    for h in range(2):
+        np.testing.assert_allclose(sk[0, h], np.tile(v[0, h], (4, 1)), atol=1e-13)
+        np.testing.assert_allclose(lse[0, h], 0.3 * q[h] @ k[0, h], atol=1e-13)
+
+
+def test_proto_hard_assignment_limit():
+    """Large scale: Eq. (8) tends to a one-hot assignment of each token to its best prototype."""
+    q, k, v, cu = _rand_problem([40], H=1, d=8, kp=5, seed=11)
+    scale = 1.0e5
+    sk, _, mass = oracle.sa_forward_proto(q, k, v, cu, scale=scale)
+    s = k[:, 0] @ q[0].T           # [n, k], an independent recomputation of the ordering only
+    best = s.argmax(axis=1)
+    gap = np.sort(s, axis=1)[:, -1] - np.sort(s, axis=1)[:, -2]
+    assert gap.min() * scale > 60   # every token's runner-up weight is < e^-60
+    want = np.zeros((5, 8))
+    for i, j in enumerate(best):
+        want[j] += v[i, 0]
+    np.testing.assert_allclose(sk[0, 0], want, atol=1e-10)
+    np.testing.assert_allclose(mass[0, 0], np.bincount(best, minlength=5), atol=1e-10)
+
+
+def test_token_hard_assignment_limit():
+    """Large scale: each prototype copies the value of its best-scoring token."""
+    q, k, v, cu = _rand_problem([40], H=1, d=8, kp=5, seed=12)
+    scale = 1.0e5
+    sk, _, _ = oracle.sa_forward_token(q, k, v, cu, scale=scale)
+    s = q[0] @ k[:, 0].T           # [k, n]
+    best = s.argmax(axis=1)
+    srt = np.sort(s, axis=1)
+    assert ((srt[:, -1] - srt[:, -2]) * scale).min() > 60
+    np.testing.assert_allclose(sk[0, 0], v[best, 0], atol=1e-10)
+
+
+def test_empty_user():
+    q, k, v, cu = _rand_problem([5, 0, 3], H=2, d=8, kp=3, seed=13)
+    sk, lse, mass = oracle.sa_forward_proto(q, k, v, cu)
+    assert (sk[1] == 0).all() and (mass[1] == 0).all()
+    skt, lset, masst = oracle.sa_forward_token(q, k, v, cu)
+    assert (skt[1] == 0).all() and np.isneginf(lset[1]).all()
+
+
+# ------------------------------------------------------------ invariances
+@pytest.mark.parametrize("norm", [NORM_PROTO, NORM_TOKEN])
+def test_permutation_invariance(norm):
+    """Eq. (7)-(9) have no positional term: permuting a user's tokens keeps the sketch."""
+    q, k, v, cu = _rand_problem([11, 6], H=2, d=8, kp=4, seed=14)
+    perm = np.concatenate([RNG.permutation(11), 11 + RNG.permutation(6)])
+    a = oracle.sa_forward(q, k, v, cu, None, 0.9, norm)
+    b = oracle.sa_forward(q, k[perm], v[perm], cu, None, 0.9, norm)
+    np.testing.assert_allclose(a[0], b[0], atol=1e-12)
+    if norm == NORM_PROTO:
+        np.testing.assert_allclose(a[1][perm], b[1], atol=1e-12)
+
+
+@pytest.mark.parametrize("norm", [NORM_PROTO, NORM_TOKEN])
+def test_padding_has_no_effect(norm):
+    q, k, v, cu = _rand_problem([9, 7], H=2, d=8, kp=4, seed=15)
+    used = [6, 7]
+    a = oracle.sa_forward(q, k, v, cu, used, 1.0, norm)
+    k2, v2 = k.copy(), v.copy()
+    k2[6:9] = 1e3
+    v2[6:9] = -7e2
+    b = oracle.sa_forward(q, k2, v2, cu, used, 1.0, norm)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+    # and equals the problem with the padding cut away
+    c = oracle.sa_forward(q, np.concatenate([k[:6], k[9:]]), np.concatenate([v[:6], v[9:]]),
+                          [0, 6, 13], None, 1.0, norm)
+    np.testing.assert_allclose(a[0], c[0], atol=1e-13)
+    if norm == NORM_PROTO:
+        assert np.isneginf(a[1][6:9]).all()
+
+
+def test_users_are_independent():
+    q, k, v, cu = _rand_problem([8, 5, 6], H=2, d=8, kp=3, seed=16)
+    a = oracle.sa_forward_proto(q, k, v, cu)
+    k2 = k.copy()
+    k2[8:13] += 1.0
+    b = oracle.sa_forward_proto(q, k2, v, cu)
+    np.testing.assert_array_equal(a[0][[0, 2]], b[0][[0, 2]])
+    assert not np.allclose(a[0][1], b[0][1])
+
+
+def test_heads_are_independent_problems():
+    q, k, v, cu = _rand_problem([8], H=3, d=8, kp=3, seed=17)
+    full = oracle.sa_forward_proto(q, k, v, cu)
+    one = oracle.sa_forward_proto(q[1:2], k[:, 1:2], v[:, 1:2], cu)
+    np.testing.assert_allclose(full[0][:, 1:2], one[0], atol=1e-14)
+
+
+def test_scale_folds_into_queries():
+    q, k, v, cu = _rand_problem([8, 3], H=2, d=8, kp=3, seed=18)
+    a = oracle.sa_forward_token(q, k, v, cu, scale=0.125)
+    b = oracle.sa_forward_token(q * 0.125, k, v, cu, scale=1.0)
+    np.testing.assert_allclose(a[0], b[0], atol=1e-13)
+
+
+def test_per_user_queries_match_shared_when_equal():
+    q, k, v, cu = _rand_problem([8, 3], H=2, d=8, kp=3, seed=19)
+    qb = np.stack([q, q])
+    np.testing.assert_allclose(oracle.sa_forward_proto(q, k, v, cu)[0],
+                               oracle.sa_forward_proto(qb, k, v, cu)[0], atol=0)
+
+
+# --------------------------------------------------------- finite differences
+def _fd_check(norm, per_user_q):
+    lengths, used = [5, 4], [4, 4]
+    q, k, v, cu = _rand_problem(lengths, H=2, d=4, kp=3, per_user_q=per_user_q, seed=20)
+    rng = np.random.default_rng(21)
+    dO = rng.standard_normal((2, 2, 3, 4))
+    scale = 0.8
+    dq, dk, dv = oracle.sa_backward(q, k, v, cu, used, dO, scale, norm)
+
+    def loss(q_, k_, v_):
+        return float((oracle.sa_forward(q_, k_, v_, cu, used, scale, norm)[0] * dO).sum())
+
+    eps = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = x.copy(); xp[idx] += eps
+            xm = x.copy(); xm[idx] -= eps
+            args = {"q": (q, k, v), "k": (q, k, v), "v": (q, k, v)}[name]
+            ap = list(args); am = list(args)
+            pos = "qkv".index(name)
+            ap[pos] = xp; am[pos] = xm
+            num[idx] = (loss(*ap) - loss(*am)) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8, err_msg=name)
+    # padding rows get zero gradient
+    assert (dk[4] == 0).all() and (dv[4] == 0).all()
+
+
+@pytest.mark.parametrize("norm", [NORM_PROTO, NORM_TOKEN])
+def test_backward_finite_differences_shared_q(norm):
+    _fd_check(norm, per_user_q=False)
+
+
+@pytest.mark.parametrize("norm", [NORM_PROTO, NORM_TOKEN])
+def test_backward_finite_differences_per_user_q(norm):
+    _fd_check(norm, per_user_q=True)
+
+
+# ---------------------------------------------------------------------- STCA
+def _stca_problem(targets, hist, ks, H=2, d=8, seed=30):
+    rng = np.random.default_rng(seed)
+    B = len(targets)
+    q = rng.standard_normal((sum(targets), H, d))
+    kh = rng.standard_normal((sum(hist), H, d))
+    vh = rng.standard_normal((sum(hist), H, d))
+    ksk = rng.standard_normal((B, H, ks, d))
+    vsk = rng.standard_normal((B, H, ks, d))
+    cut = np.concatenate([[0], np.cumsum(targets)])
+    cuh = np.concatenate([[0], np.cumsum(hist)])
+    return q, cut, kh, vh, cuh, ksk, vsk
+
+
+def test_stca_single_key_returns_its_value():
+    q, cut, kh, vh, cuh, ksk, vsk = _stca_problem([3], [1], 0)
+    out, lse = oracle.stca_forward(q, cut, kh, vh, cuh, ksk, vsk, 0.5)
+    np.testing.assert_allclose(out, np.broadcast_to(vh[0], out.shape), atol=1e-14)
+    np.testing.assert_allclose(lse, 0.5 * (q * kh[0][None]).sum(axis=2), atol=1e-13)
+
+
+def test_stca_zero_query_is_mean_of_all_keys():
+    q, cut, kh, vh, cuh, ksk, vsk = _stca_problem([2, 3], [5, 4], 3)
+    q[:] = 0
+    out, lse = oracle.stca_forward(q, cut, kh, vh, cuh, ksk, vsk, 1.0)
+    for b, (t0, t1, h0, h1) in enumerate([(0, 2, 0, 5), (2, 5, 5, 9)]):
+        allv = np.concatenate([vh[h0:h1], vsk[b].transpose(1, 0, 2)], axis=0)
+        np.testing.assert_allclose(out[t0:t1], np.broadcast_to(allv.mean(axis=0), out[t0:t1].shape), atol=1e-13)
+        np.testing.assert_allclose(lse[t0:t1], math.log(allv.shape[0]), atol=1e-13)
+
+
+def test_stca_segment_merge_law():
+    """Softmax over [suffix; sketch] = lse-weighted merge of the two one-segment results."""
+    q, cut, kh, vh, cuh, ksk, vsk = _stca_problem([4, 2], [6, 3], 5)
+    out, lse = oracle.stca_forward(q, cut, kh, vh, cuh, ksk, vsk, 0.7)
+    o1, l1 = oracle.stca_forward(q, cut, kh, vh, cuh, ksk[:, :, :0], vsk[:, :, :0], 0.7)
+    o2, l2 = oracle.stca_forward(q, cut, kh[:0], vh[:0], np.zeros_like(cuh), ksk, vsk, 0.7)
+    lm = np.logaddexp(l1, l2)
+    np.testing.assert_allclose(lse, lm, atol=1e-12)
+    merged = np.exp(l1 - lm)[..., None] * o1 + np.exp(l2 - lm)[..., None] * o2
+    np.testing.assert_allclose(out, merged, atol=1e-12)
+
+
+def test_stca_equals_token_sa_with_one_prototype():
+    """One target over one user's suffix is token-wise SA with that target as the only prototype."""
+    q, cut, kh, vh, cuh, ksk, vsk = _stca_problem([1], [7], 0, H=2)
+    out, lse = oracle.stca_forward(q, cut, kh, vh, cuh, ksk, vsk, 0.6)
+    sk, lse_t, _ = oracle.sa_forward_token(q[0][:, None, :], kh, vh, cuh, None, 0.6)
+    np.testing.assert_allclose(out[0], sk[0, :, 0], atol=1e-13)
+    np.testing.assert_allclose(lse[0], lse_t[0, :, 0], atol=1e-13)
+
+
+def test_stca_kv_len_is_truncation():
+    q, cut, kh, vh, cuh, ksk, vsk = _stca_problem([1, 1], [6, 5], 2)
+    out, lse = oracle.stca_forward(q, cut, kh, vh, cuh, ksk, vsk, 1.0, target_kv_len=[3, 5])
+    o2, l2 = oracle.stca_forward(q, cut, np.concatenate([kh[:3], kh[6:]]),
+                                 np.concatenate([vh[:3], vh[6:]]), [0, 3, 8], ksk, vsk, 1.0)
+    np.testing.assert_allclose(out, o2, atol=1e-14)
+
+
+def test_stca_no_keys():
+    q, cut, kh, vh, cuh, ksk, vsk = _stca_problem([2], [0], 0)
+    out, lse = oracle.stca_forward(q, cut, kh, vh, cuh, ksk, vsk, 1.0)
+    assert (out == 0).all() and np.isneginf(lse).all()
