@@ -1,0 +1,183 @@
+/*
+ * sketch_attn.h — C ABI of libska.so: Sketch Attention (SA) and STCA on NVIDIA B200 (sm_100a).
+ *
+ * The operations are those of "SequenceO1: End-to-End Ultra-Long (100K) Sequence Modeling in
+ * Recommendation with Low-Rank Caching" (arXiv 2609.08443):
+ *
+ *   SA (§3.1, Eq. (7)-(9)): for a user with history keys K = X W_K (n x d) and values V (the
+ *   history X itself in the paper) and prototypes Q = P W_Q (k x d),
+ *       S = scale * Q K^T                         (k x n; the paper's scale is 1/sqrt(d))
+ *       A = softmax_proto(S), sum_j A[j,i] = 1    (prototype-wise: over j for every token i)
+ *       sketch = A V                              (k x d; fixed size, target-agnostic)
+ *   FlashSA (§4.4) computes this in one streaming pass: block-wise affinities, softmax
+ *   statistics (max and log-sum-exp) and aggregation, without storing the k x n scores.
+ *
+ *   SKA_NORM_TOKEN selects the token-wise ("vanilla attention") normalisation that §5.1 / Table 1
+ *   compares against: A = softmax over the valid tokens i for every prototype j.
+ *
+ *   STCA (§2.3; used on the recent suffix and on the sketch in §3.4, batched per user by MRLB in
+ *   §4.2): out_t = softmax(scale * q_t K^T) V over the keys [suffix rows of the target's user ;
+ *   that user's sketch rows], one softmax per (target, head).
+ *
+ * Heads: H heads are H independent problems on d-wide slices (the paper's SA is single-head).
+ *
+ * Conventions shared by every entry point
+ *   Memory     All tensor arguments are DEVICE pointers owned by the caller, row-major and
+ *              contiguous, 16-byte aligned. Integer index arrays are int32 on the device. The
+ *              library never reads device memory from the host; sizes (total_*, max_*) come in
+ *              the descriptor. The library allocates nothing: scratch memory is the caller's
+ *              workspace `ws` of at least *_workspace_size() bytes (256-byte aligned).
+ *   Execution  Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *              stream) and returns before the work finishes. Calls are reentrant; two calls must
+ *              not share a workspace while both are in flight.
+ *   Errors     Invalid arguments are reported before anything is launched (SKA_ERR_INVALID_VALUE,
+ *              SKA_ERR_UNSUPPORTED, SKA_ERR_WORKSPACE_TOO_SMALL); a failed launch returns
+ *              SKA_ERR_CUDA. A kernel that waits longer than its time budget on a pipeline
+ *              barrier stops, records SKA_ERR_DEVICE_TIMEOUT in the workspace status word and
+ *              exits; ska_read_device_status() reports it.
+ *   Outputs    Outputs are fully overwritten (zeros for empty users). No output may alias an
+ *              input. k and v may alias each other (the paper's V = X).
+ *   Padding    Tokens of user b at positions >= seqused[b] take no part in the result, but their
+ *              rows must hold finite numbers (a zero weight times a non-finite value is NaN).
+ *   Determinism  Results are bitwise reproducible run to run (fixed-order reductions).
+ */
+#ifndef SKETCH_ATTN_H_
+#define SKETCH_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SKA_OK = 0,
+  SKA_ERR_INVALID_VALUE = 1,       /* bad pointer, size, stride or alignment */
+  SKA_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. head_dim not 64/128) */
+  SKA_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < *_workspace_size(desc) */
+  SKA_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+  SKA_ERR_DEVICE_TIMEOUT = 5       /* a kernel gave up waiting on a pipeline barrier */
+} ska_status;
+
+typedef enum { SKA_BF16 = 0, SKA_F32 = 1 } ska_dtype;
+
+typedef enum {
+  SKA_NORM_PROTO = 0, /* the paper's Eq. (8): softmax over prototypes for every token */
+  SKA_NORM_TOKEN = 1  /* §5.1 comparator: softmax over tokens for every prototype */
+} ska_norm;
+
+/* One batched SA problem: num_users ragged users, each with its own history.
+ *   num_heads    H >= 1
+ *   head_dim     d, 64 or 128
+ *   num_protos   k: a multiple of 16 in [16, 256], or 512, 1024, 2048 (k/ceil(k/256) a
+ *                multiple of 16)
+ *   total_tokens rows of k and v (= cu_seqlens[num_users]); < 2^31
+ *   max_seqlen   an upper bound on any user's length (informational; may be 0)
+ *   scale        multiplies Q K^T; must be > 0 and finite (1/sqrt(d) in Eq. (7))
+ *   norm         ska_norm
+ *   in_dtype     ska_dtype of q, k, v (SKA_F32 inputs are rounded to bf16 in the workspace)
+ *   q_per_user   0: q is [H, k, d], the prototypes shared by every user (layer 0, Eq. (6));
+ *                1: q is [B, H, k, d], per-user queries (a refinement layer, §3.3)          */
+typedef struct {
+  int32_t num_users;
+  int32_t num_heads;
+  int32_t head_dim;
+  int32_t num_protos;
+  int64_t total_tokens;
+  int32_t max_seqlen;
+  float scale;
+  int32_t norm;
+  int32_t in_dtype;
+  int32_t q_per_user;
+  int32_t reserved;
+} ska_sa_desc;
+
+/* Bytes of workspace sa_forward needs for this descriptor (0 if the descriptor is invalid). */
+size_t sa_forward_workspace_size(const ska_sa_desc* desc);
+
+/* SA forward (FlashSA), §3.1 Eq. (7)-(9) and §4.4.
+ *   q           [H,k,d] or [B,H,k,d] (q_per_user), in_dtype
+ *   k, v        [total_tokens, H, d], in_dtype; user b owns rows [cu_seqlens[b], cu_seqlens[b+1])
+ *   cu_seqlens  int32 [B+1], non-decreasing, cu_seqlens[0] = 0
+ *   seqused     int32 [B] or NULL: only the first min(seqused[b], len_b) rows of user b count
+ *   sketch      out, fp32 [B, H, k, d]
+ *   lse         out, fp32, may be NULL. PROTO: [total_tokens, H], the per-token log-sum-exp over
+ *               the k prototypes (-inf on padding rows). TOKEN: [B, H, k], the per-prototype
+ *               log-sum-exp over the valid tokens (-inf for an empty user). The backward pass
+ *               needs it.
+ *   mass        out, fp32 [B, H, k] or NULL: sum_i A[j,i], the mass each prototype received.  */
+ska_status sa_forward(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
+                      const int32_t* cu_seqlens, const int32_t* seqused, float* sketch, float* lse,
+                      float* mass, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace sa_backward needs (0 if the descriptor is invalid). */
+size_t sa_backward_workspace_size(const ska_sa_desc* desc);
+
+/* SA backward: gradients of <dsketch, sketch> through Eq. (7)-(9) (SA is trained end to end,
+ * App. A.4). Inputs as in sa_forward plus the forward's lse; bf16 inputs only.
+ *   dsketch  bf16 [B, H, k, d]
+ *   dq       out, fp32, q's shape: [H,k,d] summed over all users when the prototypes are shared,
+ *            else [B,H,k,d]
+ *   dk, dv   out, fp32 [total_tokens, H, d]; zero rows on padding tokens                      */
+ska_status sa_backward(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
+                       const int32_t* cu_seqlens, const int32_t* seqused, const float* lse,
+                       const void* dsketch, float* dq, float* dk, float* dv, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* One batched STCA problem (§2.3, §3.4, MRLB §4.2): num_users users, each with a block of
+ * target queries that share the user's keys.
+ *   head_dim 64 or 128; num_sketch = k_s sketch rows per user (0 allowed, a multiple of 8 else);
+ *   total_targets = cu_targets[B]; total_hist = cu_hist[B]; scale > 0 (1/sqrt(d_h) in §2.3). */
+typedef struct {
+  int32_t num_users;
+  int32_t num_heads;
+  int32_t head_dim;
+  int32_t num_sketch;
+  int64_t total_targets;
+  int64_t total_hist;
+  int32_t max_targets;
+  int32_t max_hist;
+  float scale;
+  int32_t reserved;
+} ska_stca_desc;
+
+size_t stca_forward_workspace_size(const ska_stca_desc* desc);
+
+/* STCA forward. All bf16 except the fp32 outputs.
+ *   q              [total_targets, H, d]; targets of user b are rows [cu_targets[b], cu_targets[b+1])
+ *   k_hist, v_hist [total_hist, H, d]; the recent suffix of user b is rows [cu_hist[b], cu_hist[b+1])
+ *   target_kv_len  int32 [total_targets] or NULL: target t sees only the first target_kv_len[t]
+ *                  suffix rows of its user (request-aware masking, §4.2)
+ *   k_sk, v_sk     [B, H, num_sketch, d] (NULL when num_sketch == 0)
+ *   out            fp32 [total_targets, H, d];  lse  fp32 [total_targets, H] or NULL          */
+ska_status stca_forward(const ska_stca_desc* desc, const void* q, const int32_t* cu_targets,
+                        const void* k_hist, const void* v_hist, const int32_t* cu_hist,
+                        const int32_t* target_kv_len, const void* k_sk, const void* v_sk, float* out,
+                        float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* ska_status_string(ska_status status);
+
+/* Reads the device status word of a workspace after synchronising `stream`; returns SKA_OK or
+ * the first device-side error a kernel recorded there (e.g. SKA_ERR_DEVICE_TIMEOUT), and
+ * clears it. Test and debug helper: it blocks the host. */
+ska_status ska_read_device_status(void* ws, void* stream);
+
+/* Test hook (process-wide, not synchronised with concurrent calls): the time budget in ns of
+ * every barrier wait in later launches (0 restores the default of 4 s), and debug flags
+ * (1 = the load producer of later SA forward launches withholds its first arrival, so that
+ * the consumers' bounded waits must run out and report SKA_ERR_DEVICE_TIMEOUT). */
+void ska_set_debug(uint64_t wait_budget_ns, uint32_t flags);
+
+/* Bench hook (process-wide): while both handles are non-NULL, every later call records
+ * `start_event` on its stream immediately before its fused main kernel and `stop_event`
+ * immediately after it (cudaEvent_t handles created by the caller), so that the main kernel
+ * can be timed on its own stream with CUDA events. Pass NULL, NULL to stop recording. */
+void ska_set_timing_events(void* start_event, void* stop_event);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SKETCH_ATTN_H_ */

@@ -1,0 +1,112 @@
+"""Torch-facing binding of the C ABI: takes device tensors, passes their pointers and the
+current CUDA stream to libska.so, and returns the outputs. No computation happens here."""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import SaDesc, SkaError, StcaDesc
+
+_NORMS = {"proto": _lib.SKA_NORM_PROTO, "token": _lib.SKA_NORM_TOKEN,
+          _lib.SKA_NORM_PROTO: _lib.SKA_NORM_PROTO, _lib.SKA_NORM_TOKEN: _lib.SKA_NORM_TOKEN}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev_tensor(name, t, dtypes):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+
+
+def _check(rc: int, what: str):
+    if rc != _lib.SKA_OK:
+        raise SkaError(rc, what)
+
+
+def sa_desc(q, k, cu_seqlens, *, scale, norm, max_seqlen=0) -> SaDesc:
+    per_user = q.dim() == 4
+    d = SaDesc()
+    d.num_users = cu_seqlens.numel() - 1
+    d.num_heads = k.shape[1]
+    d.head_dim = k.shape[2]
+    d.num_protos = q.shape[-2]
+    d.total_tokens = k.shape[0]
+    d.max_seqlen = int(max_seqlen)
+    d.scale = float(scale)
+    d.norm = _NORMS[norm]
+    d.in_dtype = _lib.SKA_F32 if q.dtype == torch.float32 else _lib.SKA_BF16
+    d.q_per_user = 1 if per_user else 0
+    d.reserved = 0
+    return d
+
+
+def sa_forward_workspace_size(desc: SaDesc) -> int:
+    return int(_lib.lib().sa_forward_workspace_size(ctypes.byref(desc)))
+
+
+def sa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+               seqused: Optional[torch.Tensor] = None, *, scale: float = 1.0, norm="proto",
+               want_lse: bool = True, want_mass: bool = False, workspace: Optional[torch.Tensor] = None,
+               out: Optional[torch.Tensor] = None, lse_out: Optional[torch.Tensor] = None, stream=None):
+    """Sketch Attention forward (SequenceO1 §3.1 Eq. (7)-(9), FlashSA §4.4).
+
+    q [H,k,d] or [B,H,k,d]; k, v [T,H,d] (bf16, or fp32 rounded to bf16 on the device);
+    cu_seqlens int32 [B+1]; seqused int32 [B] or None. Returns (sketch fp32 [B,H,k,d],
+    lse or None, mass or None).
+    """
+    dts = (torch.bfloat16, torch.float32)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _dev_tensor(name, t, dts)
+    _dev_tensor("cu_seqlens", cu_seqlens, (torch.int32,))
+    _dev_tensor("seqused", seqused, (torch.int32,))
+    desc = sa_desc(q, k, cu_seqlens, scale=scale, norm=norm)
+    B, H, D, kp, T = desc.num_users, desc.num_heads, desc.head_dim, desc.num_protos, desc.total_tokens
+    dev = k.device
+    need = sa_forward_workspace_size(desc)
+    if need == 0 and B > 0:
+        raise SkaError(_lib.SKA_ERR_UNSUPPORTED, "sa_forward_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    sketch = out if out is not None else torch.empty((B, H, kp, D), dtype=torch.float32, device=dev)
+    lse = None
+    if want_lse:
+        shape = (T, H) if desc.norm == _lib.SKA_NORM_PROTO else (B, H, kp)
+        lse = lse_out if lse_out is not None else torch.empty(shape, dtype=torch.float32, device=dev)
+    mass = torch.empty((B, H, kp), dtype=torch.float32, device=dev) if want_mass else None
+    rc = _lib.lib().sa_forward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                               _ptr(seqused), _ptr(sketch), _ptr(lse), _ptr(mass), _ptr(workspace),
+                               ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check(rc, "sa_forward")
+    return sketch, lse, mass
+
+
+def read_device_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(_lib.lib().ska_read_device_status(_ptr(workspace), _stream(stream)))
+
+
+def set_debug(wait_budget_ns: int = 0, flags: int = 0) -> None:
+    _lib.lib().ska_set_debug(ctypes.c_uint64(wait_budget_ns), ctypes.c_uint32(flags))
+
+
+def set_timing_events(start=None, stop=None) -> None:
+    """Bench hook: record these torch.cuda.Events around the fused main kernel of later calls."""
+    a = ctypes.c_void_p(start.cuda_event) if start is not None else ctypes.c_void_p(0)
+    b = ctypes.c_void_p(stop.cuda_event) if stop is not None else ctypes.c_void_p(0)
+    _lib.lib().ska_set_timing_events(a, b)

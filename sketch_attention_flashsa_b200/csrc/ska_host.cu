@@ -1,0 +1,321 @@
+// C-ABI host layer of libska.so: argument validation, workspace carving, TMA descriptor
+// encoding and kernel launches. Everything here runs on the host and only enqueues work on
+// the caller's stream; no device memory is read or allocated.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "ska_internal.h"
+
+using namespace ska;
+
+namespace {
+
+std::atomic<uint64_t> g_budget_ns{0};
+std::atomic<uint32_t> g_debug_flags{0};
+std::atomic<void*> g_ev_start{nullptr};
+std::atomic<void*> g_ev_stop{nullptr};
+
+struct TimedRegion {
+  cudaStream_t s;
+  cudaEvent_t stop;
+  explicit TimedRegion(cudaStream_t st) : s(st), stop(nullptr) {
+    cudaEvent_t a = static_cast<cudaEvent_t>(g_ev_start.load(std::memory_order_relaxed));
+    cudaEvent_t b = static_cast<cudaEvent_t>(g_ev_stop.load(std::memory_order_relaxed));
+    if (a && b) {
+      cudaEventRecord(a, s);
+      stop = b;
+    }
+  }
+  ~TimedRegion() {
+    if (stop) cudaEventRecord(stop, s);
+  }
+};
+
+uint64_t wait_budget() {
+  const uint64_t b = g_budget_ns.load(std::memory_order_relaxed);
+  return b ? b : kDefaultBudgetNs;
+}
+
+int device_sm_count() {
+  static int cache[64];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [rows, inner] tensor with 128-byte swizzle.
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_elems,
+               uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_elems * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Validation shared by forward and backward descriptors.
+ska_status check_sa_desc(const ska_sa_desc* d) {
+  if (!d) return SKA_ERR_INVALID_VALUE;
+  if (d->num_users < 0 || d->num_heads < 1 || d->total_tokens < 0 || d->total_tokens >= (int64_t(1) << 31))
+    return SKA_ERR_INVALID_VALUE;
+  if (!(d->scale > 0.f) || !std::isfinite(d->scale)) return SKA_ERR_INVALID_VALUE;
+  if (d->norm != SKA_NORM_PROTO && d->norm != SKA_NORM_TOKEN) return SKA_ERR_INVALID_VALUE;
+  if (d->in_dtype != SKA_BF16 && d->in_dtype != SKA_F32) return SKA_ERR_INVALID_VALUE;
+  if (d->q_per_user != 0 && d->q_per_user != 1) return SKA_ERR_INVALID_VALUE;
+  if (d->num_protos < 1) return SKA_ERR_INVALID_VALUE;
+  if (d->head_dim != 64 && d->head_dim != 128) return SKA_ERR_UNSUPPORTED;
+  if (int64_t(d->num_users) * d->num_heads >= (int64_t(1) << 30)) return SKA_ERR_INVALID_VALUE;
+  return SKA_OK;
+}
+
+struct FwdWs {
+  size_t hdr, prefix, partial, mass_partial, qb, kb, vb, total;
+};
+
+bool fwd_ws_layout(const ska_sa_desc* d, const ProtoFwdLaunch& L, FwdWs* w) {
+  const size_t B = d->num_users, H = d->num_heads, D = d->head_dim, k = d->num_protos;
+  const size_t T = d->total_tokens;
+  const size_t slots = B * H + L.num_clusters;
+  size_t off = 0;
+  w->hdr = off;
+  off += sizeof(WsHeader);
+  w->prefix = off;
+  off = align256(off + (B + 1) * 4);
+  w->partial = off;
+  off = align256(off + slots * k * D * 4);
+  w->mass_partial = off;
+  off = align256(off + slots * k * 4);
+  w->qb = w->kb = w->vb = 0;
+  if (d->in_dtype == SKA_F32) {
+    const size_t qn = (d->q_per_user ? B : 1) * H * k * D;
+    w->qb = off;
+    off = align256(off + qn * 2);
+    w->kb = off;
+    off = align256(off + T * H * D * 2);
+    w->vb = off;
+    off = align256(off + T * H * D * 2);
+  }
+  w->total = off;
+  return true;
+}
+
+bool plan_forward(const ska_sa_desc* d, ProtoFwdLaunch* L, int* nk, int* nv) {
+  const int sms = device_sm_count();
+  if (sms <= 0) return false;
+  return proto_fwd_plan(d->head_dim, d->num_protos, sms, L, nk, nv);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ska_status_string(ska_status s) {
+  switch (s) {
+    case SKA_OK: return "SKA_OK";
+    case SKA_ERR_INVALID_VALUE: return "SKA_ERR_INVALID_VALUE";
+    case SKA_ERR_UNSUPPORTED: return "SKA_ERR_UNSUPPORTED";
+    case SKA_ERR_WORKSPACE_TOO_SMALL: return "SKA_ERR_WORKSPACE_TOO_SMALL";
+    case SKA_ERR_CUDA: return "SKA_ERR_CUDA";
+    case SKA_ERR_DEVICE_TIMEOUT: return "SKA_ERR_DEVICE_TIMEOUT";
+  }
+  return "SKA_ERR_UNKNOWN";
+}
+
+void ska_set_timing_events(void* start_event, void* stop_event) {
+  g_ev_start.store(start_event, std::memory_order_relaxed);
+  g_ev_stop.store(stop_event, std::memory_order_relaxed);
+}
+
+void ska_set_debug(uint64_t wait_budget_ns, uint32_t flags) {
+  g_budget_ns.store(wait_budget_ns, std::memory_order_relaxed);
+  g_debug_flags.store(flags, std::memory_order_relaxed);
+}
+
+ska_status ska_read_device_status(void* ws, void* stream) {
+  if (!ws) return SKA_ERR_INVALID_VALUE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SKA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SKA_ERR_CUDA;
+  if (v != 0) {
+    const int32_t zero = 0;
+    if (cudaMemcpyAsync(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice, st) != cudaSuccess) return SKA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SKA_ERR_CUDA;
+  }
+  return static_cast<ska_status>(v);
+}
+
+size_t sa_forward_workspace_size(const ska_sa_desc* d) {
+  if (check_sa_desc(d) != SKA_OK) return 0;
+  if (d->norm != SKA_NORM_PROTO) return 0;
+  ProtoFwdLaunch L;
+  int nk, nv;
+  if (!plan_forward(d, &L, &nk, &nv)) return 0;
+  FwdWs w;
+  fwd_ws_layout(d, L, &w);
+  return w.total;
+}
+
+ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                      const int32_t* seqused, float* sketch, float* lse, float* mass, void* ws, size_t ws_bytes,
+                      void* stream) {
+  ska_status st = check_sa_desc(d);
+  if (st != SKA_OK) return st;
+  if (d->norm != SKA_NORM_PROTO) return SKA_ERR_UNSUPPORTED;
+  if (mass) return SKA_ERR_UNSUPPORTED;
+  const int B = d->num_users, H = d->num_heads, D = d->head_dim, kp = d->num_protos;
+  const int64_t T = d->total_tokens;
+  if (B == 0) return SKA_OK;
+  ProtoFwdLaunch L;
+  int nk = 0, nv = 0;
+  if (!plan_forward(d, &L, &nk, &nv)) return SKA_ERR_UNSUPPORTED;
+  // pointers and alignment
+  if (!q || !cu_seqlens || !sketch || !ws) return SKA_ERR_INVALID_VALUE;
+  if (T > 0 && (!k || !v)) return SKA_ERR_INVALID_VALUE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(sketch) || !aligned16(lse) ||
+      !aligned16(mass) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seqused) & 3u))
+    return SKA_ERR_INVALID_VALUE;
+  FwdWs w;
+  fwd_ws_layout(d, L, &w);
+  if (ws_bytes < w.total) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  const size_t esz = d->in_dtype == SKA_F32 ? 4 : 2;
+  const size_t qn = size_t(d->q_per_user ? B : 1) * H * kp * D;
+  const size_t kvn = size_t(T) * H * D;
+  const size_t sk_bytes = size_t(B) * H * kp * D * 4;
+  const size_t lse_bytes = size_t(T) * H * 4;
+  if (overlaps(sketch, sk_bytes, q, qn * esz) || overlaps(sketch, sk_bytes, k, kvn * esz) ||
+      overlaps(sketch, sk_bytes, v, kvn * esz) || overlaps(lse, lse_bytes, q, qn * esz) ||
+      overlaps(lse, lse_bytes, k, kvn * esz) || overlaps(lse, lse_bytes, v, kvn * esz) ||
+      overlaps(lse, lse_bytes, sketch, sk_bytes) || overlaps(ws, w.total, sketch, sk_bytes) ||
+      overlaps(ws, w.total, lse, lse_bytes) || overlaps(ws, w.total, q, qn * esz) ||
+      overlaps(ws, w.total, k, kvn * esz) || overlaps(ws, w.total, v, kvn * esz))
+    return SKA_ERR_INVALID_VALUE;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb + w.hdr);
+  int32_t* prefix = reinterpret_cast<int32_t*>(wsb + w.prefix);
+  float* partial = reinterpret_cast<float*>(wsb + w.partial);
+  float* mass_partial = reinterpret_cast<float*>(wsb + w.mass_partial);
+
+  const void* qb = q;
+  const void* kb = k;
+  const void* vb = v;
+  if (d->in_dtype == SKA_F32) {
+    if (launch_cast_f32_bf16(static_cast<const float*>(q), wsb + w.qb, int64_t(qn), s) != cudaSuccess)
+      return SKA_ERR_CUDA;
+    if (launch_cast_f32_bf16(static_cast<const float*>(k), wsb + w.kb, int64_t(kvn), s) != cudaSuccess)
+      return SKA_ERR_CUDA;
+    if (launch_cast_f32_bf16(static_cast<const float*>(v), wsb + w.vb, int64_t(kvn), s) != cudaSuccess)
+      return SKA_ERR_CUDA;
+    qb = wsb + w.qb;
+    kb = wsb + w.kb;
+    vb = wsb + w.vb;
+  }
+
+  if (launch_schedule(cu_seqlens, seqused, B, H, L.num_clusters, prefix, hdr, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (T > 0) {
+    CUtensorMap mQ, mK, mV;
+    const uint64_t qrows = uint64_t(d->q_per_user ? B : 1) * H * kp;
+    if (!encode_2d(&mQ, qb, D, qrows, D, 64, L.kc)) return SKA_ERR_CUDA;
+    if (!encode_2d(&mK, kb, uint64_t(H) * D, T, uint64_t(H) * D, 64, kTileTokens)) return SKA_ERR_CUDA;
+    if (!encode_2d(&mV, vb, uint64_t(H) * D, T, uint64_t(H) * D, 64, kTileTokens)) return SKA_ERR_CUDA;
+    ProtoFwdParams p{};
+    p.cu_seqlens = cu_seqlens;
+    p.seqused = seqused;
+    p.tile_prefix = prefix;
+    p.hdr = hdr;
+    p.partial = partial;
+    p.lse = lse;
+    p.mass_partial = nullptr;
+    p.B = B;
+    p.H = H;
+    p.k = kp;
+    p.total_tokens = static_cast<int>(T);
+    p.q_per_user = d->q_per_user;
+    p.nk_slots = nk;
+    p.nv_entries = nv;
+    p.scale_log2 = d->scale * 1.4426950408889634f;
+    p.budget_ns = wait_budget();
+    p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
+    cudaError_t e;
+    {
+      TimedRegion tr(s);
+      e = launch_proto_fwd(D, L, mQ, mK, mV, p, s);
+    }
+    if (e != cudaSuccess) return SKA_ERR_CUDA;
+  }
+  if (launch_proto_combine(prefix, hdr, partial, nullptr, B, H, kp, D, sketch, nullptr, s) != cudaSuccess)
+    return SKA_ERR_CUDA;
+  if (lse && T > 0) {
+    if (launch_fill_padding_lse(cu_seqlens, seqused, B, H, T, lse, s) != cudaSuccess) return SKA_ERR_CUDA;
+  }
+  return SKA_OK;
+}
+
+size_t sa_backward_workspace_size(const ska_sa_desc* d) {
+  (void)d;
+  return 0;
+}
+
+ska_status sa_backward(const ska_sa_desc* d, const void*, const void*, const void*, const int32_t*, const int32_t*,
+                       const float*, const void*, float*, float*, float*, void*, size_t, void*) {
+  ska_status st = check_sa_desc(d);
+  if (st != SKA_OK) return st;
+  return SKA_ERR_UNSUPPORTED;
+}
+
+size_t stca_forward_workspace_size(const ska_stca_desc* d) {
+  (void)d;
+  return 0;
+}
+
+ska_status stca_forward(const ska_stca_desc* d, const void*, const int32_t*, const void*, const void*,
+                        const int32_t*, const int32_t*, const void*, const void*, float*, float*, void*, size_t,
+                        void*) {
+  if (!d) return SKA_ERR_INVALID_VALUE;
+  return SKA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

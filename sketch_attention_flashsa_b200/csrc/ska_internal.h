@@ -1,0 +1,68 @@
+// Internal interfaces between the C-ABI host layer and the kernels of libska.so.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/sketch_attn.h"
+
+namespace ska {
+
+constexpr int kTileTokens = 128;       // history tokens per pipeline tile
+constexpr int kMaxProtosPerCta = 256;  // prototypes one CTA holds in TMEM
+constexpr uint64_t kDefaultBudgetNs = 4000000000ull;
+
+// Workspace header (first 256 bytes of every workspace).
+struct WsHeader {
+  int32_t status;      // first device-side error (ska_status), 0 if none
+  int32_t total_tiles; // written by the scheduling kernel
+  int32_t tiles_per_cluster;
+  int32_t pad[61];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+// Parameters of the prototype-wise (paper Eq. (8)) fused forward kernel.
+struct ProtoFwdParams {
+  const int32_t* cu_seqlens;   // [B+1]
+  const int32_t* seqused;      // [B] or null
+  const int32_t* tile_prefix;  // [B+1] exclusive prefix of per-user tile counts
+  WsHeader* hdr;               // status + schedule
+  float* partial;              // [(num_segments + num_clusters) * k * D] fp32
+  float* lse;                  // [T, H] or null
+  float* mass_partial;         // [(num_segments + num_clusters) * k] or null
+  int B, H, k;
+  int total_tokens;
+  int q_per_user;
+  int nk_slots;                // K ring: 16 KB slots
+  int nv_entries;              // V ring: entries of D/64 x 16 KB
+  float scale_log2;            // scale * log2(e)
+  uint64_t budget_ns;
+  uint32_t debug_flags;
+};
+
+struct ProtoFwdLaunch {
+  int cluster;          // CTAs per cluster (prototype groups)
+  int kc;               // prototypes per CTA
+  int num_clusters;     // persistent clusters
+  size_t smem_bytes;
+};
+
+// Host-side planning (no device access).
+bool proto_fwd_plan(int head_dim, int num_protos, int num_sms, ProtoFwdLaunch* out, int* nk_slots,
+                    int* nv_entries);
+
+cudaError_t launch_proto_fwd(int head_dim, const ProtoFwdLaunch& L, const CUtensorMap& mapQ,
+                             const CUtensorMap& mapK, const CUtensorMap& mapV, const ProtoFwdParams& p,
+                             cudaStream_t stream);
+
+// Small kernels (ska_small.cu).
+cudaError_t launch_schedule(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,
+                            int num_clusters, int32_t* tile_prefix, WsHeader* hdr, cudaStream_t stream);
+cudaError_t launch_proto_combine(const int32_t* tile_prefix, const WsHeader* hdr, const float* partial,
+                                 const float* mass_partial, int B, int H, int k, int D, float* sketch,
+                                 float* mass, cudaStream_t stream);
+cudaError_t launch_fill_padding_lse(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,
+                                    int64_t T, float* lse, cudaStream_t stream);
+cudaError_t launch_cast_f32_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream);
+
+}  // namespace ska

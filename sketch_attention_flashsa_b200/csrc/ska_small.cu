@@ -1,0 +1,142 @@
+// Small SIMT kernels around the fused SA kernels: tile scheduling from cu_seqlens, the
+// fixed-order combine of per-cluster partial sketches, -inf padding of the per-token lse,
+// and the fp32 -> bf16 input conversion.
+#include <algorithm>
+
+#include <cuda_bf16.h>
+
+#include "ska_internal.h"
+
+namespace ska {
+
+namespace {
+
+__device__ __forceinline__ int used_len(const int32_t* cu, const int32_t* seqused, int b) {
+  int len = cu[b + 1] - cu[b];
+  if (seqused) len = min(len, seqused[b]);
+  return max(len, 0);
+}
+
+// One block. tile_prefix[b] = sum_{b' < b} ceil(used_b' / 128); header gets the stream size and
+// the number of tiles each persistent cluster takes. Also clears the device status word.
+__global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restrict__ cu,
+                                                        const int32_t* __restrict__ seqused, int B, int H,
+                                                        int num_clusters, int32_t* __restrict__ prefix,
+                                                        WsHeader* hdr) {
+  __shared__ int part[1024];
+  const int t = threadIdx.x;
+  const int per = (B + 1023) / 1024;
+  const int lo = min(B, t * per), hi = min(B, lo + per);
+  int s = 0;
+  for (int b = lo; b < hi; ++b) s += (used_len(cu, seqused, b) + kTileTokens - 1) / kTileTokens;
+  part[t] = s;
+  __syncthreads();
+  // inclusive scan of the 1024 partial sums (Hillis-Steele)
+  for (int off = 1; off < 1024; off <<= 1) {
+    int v = (t >= off) ? part[t - off] : 0;
+    __syncthreads();
+    part[t] += v;
+    __syncthreads();
+  }
+  int run = (t == 0) ? 0 : part[t - 1];
+  for (int b = lo; b < hi; ++b) {
+    prefix[b] = run;
+    run += (used_len(cu, seqused, b) + kTileTokens - 1) / kTileTokens;
+  }
+  if (t == 1023) {
+    prefix[B] = part[1023];
+    const int total = H * part[1023];
+    hdr->total_tiles = total;
+    hdr->tiles_per_cluster = (total + num_clusters - 1) / num_clusters;
+    hdr->status = 0;
+  }
+}
+
+// sketch[s, :, :] = sum over the clusters p that touched segment s of partial[s + p, :, :],
+// in increasing p. Segment s = b*H + h covers global tiles [H*prefix[b] + h*n_b, ... + n_b).
+__global__ void proto_combine_kernel(const int32_t* __restrict__ prefix, const WsHeader* __restrict__ hdr,
+                                     const float* __restrict__ partial, const float* __restrict__ mass_partial,
+                                     int B, int H, int k, int D, float* __restrict__ sketch,
+                                     float* __restrict__ mass) {
+  const int s = blockIdx.x;
+  const int b = s / H, h = s - b * H;
+  const int nb = prefix[b + 1] - prefix[b];
+  const int W = hdr->tiles_per_cluster;
+  const int64_t per = static_cast<int64_t>(k) * D;
+  int p0 = 0, p1 = -1;
+  if (nb > 0 && W > 0) {
+    const int t0 = H * prefix[b] + h * nb;
+    p0 = t0 / W;
+    p1 = (t0 + nb - 1) / W;
+  }
+  for (int64_t e = (static_cast<int64_t>(blockIdx.y) * blockDim.x + threadIdx.x) * 4; e < per;
+       e += static_cast<int64_t>(gridDim.y) * blockDim.x * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int pc = p0; pc <= p1; ++pc) {
+      const float4 v = *reinterpret_cast<const float4*>(partial + (static_cast<int64_t>(s + pc) * per + e));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    *reinterpret_cast<float4*>(sketch + static_cast<int64_t>(s) * per + e) = acc;
+  }
+  if (mass && blockIdx.y == 0) {
+    for (int j = threadIdx.x; j < k; j += blockDim.x) {
+      float acc = 0.f;
+      for (int pc = p0; pc <= p1; ++pc) acc += mass_partial[static_cast<int64_t>(s + pc) * k + j];
+      mass[static_cast<int64_t>(s) * k + j] = acc;
+    }
+  }
+}
+
+// lse rows of padding tokens (positions >= seqused[b] inside user b) are -inf.
+__global__ void fill_padding_lse_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ seqused,
+                                        int B, int H, int64_t T, float* __restrict__ lse) {
+  const int b = blockIdx.x;
+  if (b >= B) return;
+  const int64_t lo = cu[b] + used_len(cu, seqused, b);
+  const int64_t hi = (static_cast<int64_t>(cu[b + 1]) < T) ? static_cast<int64_t>(cu[b + 1]) : T;
+  if (hi <= lo) return;
+  const int64_t n = static_cast<int64_t>(hi - lo) * H;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) lse[lo * H + i] = -INFINITY;
+}
+
+__global__ void cast_f32_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+}  // namespace
+
+cudaError_t launch_schedule(const int32_t* cu, const int32_t* seqused, int B, int H, int num_clusters,
+                            int32_t* prefix, WsHeader* hdr, cudaStream_t stream) {
+  schedule_kernel<<<1, 1024, 0, stream>>>(cu, seqused, B, H, num_clusters, prefix, hdr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_proto_combine(const int32_t* prefix, const WsHeader* hdr, const float* partial,
+                                 const float* mass_partial, int B, int H, int k, int D, float* sketch,
+                                 float* mass, cudaStream_t stream) {
+  const int per4 = (k * D) / 4;
+  const int threads = 256;
+  const int bx = std::min(32, (per4 + threads - 1) / threads);
+  dim3 grid(B * H, bx, 1);
+  proto_combine_kernel<<<grid, threads, 0, stream>>>(prefix, hdr, partial, mass_partial, B, H, k, D, sketch, mass);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_padding_lse(const int32_t* cu, const int32_t* seqused, int B, int H, int64_t T,
+                                    float* lse, cudaStream_t stream) {
+  fill_padding_lse_kernel<<<B, 256, 0, stream>>>(cu, seqused, B, H, T, lse);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cast_f32_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 148 * 16);
+  cast_f32_bf16_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+      src, static_cast<__nv_bfloat16*>(dst), n);
+  return cudaGetLastError();
+}
+
+}  // namespace ska
