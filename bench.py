@@ -38,6 +38,8 @@ WORKLOADS = {
     "sa_fwd_b8_l100k_h8_d128_k512_masked": ([100_000] * 8, 8, 128, 512, [70_000] + [100_000] * 7),
     "sa_fwd_b64_ragged_h4_d64_k256": ("ragged64", 4, 64, 256, None),
     "sa_fwd_paper_h1_d128_k1024": ("paper", 1, 128, 1024, None),
+    # profiling size: same per-tile work as the headline, 205 MB of K+V (> L2), ~0.25 ms
+    "sa_fwd_b2_l100k_h2_d128_k512": ([100_000] * 2, 2, 128, 512, None),
 }
 DEFAULT_WORKLOAD = "sa_fwd_b8_l100k_h8_d128_k512"
 

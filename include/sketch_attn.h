@@ -39,6 +39,10 @@
  *              input. k and v may alias each other (the paper's V = X).
  *   Padding    Tokens of user b at positions >= seqused[b] take no part in the result, but their
  *              rows must hold finite numbers (a zero weight times a non-finite value is NaN).
+ *   Precision  Scores S = scale Q K^T are exact products of the bf16 inputs summed in fp32; the
+ *              softmax runs in fp32; the aggregation A V multiplies fp16-rounded weights A with
+ *              the values converted to fp16 (exact for |v| in [2^-14, 65504]; larger magnitudes
+ *              saturate to 65504) and accumulates in fp32.
  *   Determinism  Results are bitwise reproducible run to run (fixed-order reductions).
  */
 #ifndef SKETCH_ATTN_H_

@@ -11,13 +11,17 @@
 //         exchange of (max, sum) with the other CTAs of the cluster through distributed
 //         shared memory, then P[tok, j] = exp(S - lse_tok) in bf16 to shared memory.
 //   MMA2  O^T[dd, j]  += V_tile[tok, dd]^T . P[tok, j]    M=D, N=KC, K=128 tokens   (TMEM)
+//         in fp16: P is rounded to fp16 (11 significant bits, eight times finer than bf16) and
+//         the bf16 V tile is rewritten in place as fp16 (exact inside the fp16 range) by two
+//         converter warps, so that the aggregation keeps ~5e-4 relative precision per weight.
 // Tiles of all (user, head) segments are concatenated and split evenly over the persistent
 // clusters; a cluster writes one fp32 partial sketch per segment it touches, and a second
 // kernel sums the partials of each segment in a fixed order (a plain sum: each token's
 // normalisation is complete inside the tile that holds it).
 //
 // Warp roles (384 threads): warp 0 = TMA producer, warp 1 = TMEM owner + MMA issuer,
-// warps 2-3 idle, warps 4-11 = two softmax warpgroups (each owns half of the KC columns).
+// warps 2-3 = V converters, warps 4-11 = two softmax warpgroups (each owns half of the KC
+// columns).
 #include <cstdio>
 
 #include "ska_internal.h"
@@ -29,6 +33,8 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kSoftmaxThreads = 256;
+constexpr int kConvThreads = 64;
+constexpr int kPrefetchTiles = 3;  // L2 prefetch distance of the producer, in tiles
 constexpr int kSlotBytes = 16384;  // one [128 rows x 64 bf16] swizzled block
 constexpr int kMaxRing = 8;
 
@@ -56,7 +62,7 @@ __host__ __device__ inline SmemLayout smem_layout(int D, int KC, int CS, int nk,
 
 struct Bars {
   uint64_t kfull[kMaxRing], kempty[kMaxRing];
-  uint64_t vfull[kMaxRing], vempty[kMaxRing];
+  uint64_t vfull[kMaxRing], vempty[kMaxRing], vconv[kMaxRing];
   uint64_t qfull, qfree, sfull, sfree, pfull, pfree, ofull, ofree, drain;
   uint64_t xbar[2];
   uint32_t tmem_base;
@@ -159,7 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.nk_slots; ++i) { mbar_init(&bars.kfull[i], 1); mbar_init(&bars.kempty[i], 1); }
-    for (int i = 0; i < p.nv_entries; ++i) { mbar_init(&bars.vfull[i], 1); mbar_init(&bars.vempty[i], 1); }
+    for (int i = 0; i < p.nv_entries; ++i) {
+      mbar_init(&bars.vfull[i], 1);
+      mbar_init(&bars.vempty[i], 1);
+      mbar_init(&bars.vconv[i], kConvThreads);
+    }
     mbar_init(&bars.qfull, 1);
     mbar_init(&bars.qfree, 1);
     mbar_init(&bars.sfull, 1);
@@ -200,15 +210,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&mapQ);
       tma_prefetch_desc(&mapK);
       tma_prefetch_desc(&mapV);
-      TilePos tk, tv;
+      TilePos tk, tv, tp;
       tile_seek(p, g0, tk);
       tv = tk;
+      tp = tk;
+      int ip = 0;  // next tile to prefetch into L2 (rank 0 of the cluster only)
+      auto prefetch_to = [&](int upto) {
+        while (ip < ntiles && ip < upto) {
+          const int tok0 = p.cu_seqlens[tp.b] + tp.j * kTileTokens;
+          for (int kb = 0; kb < KB; ++kb) {
+            tma_prefetch_l2_2d(&mapK, tp.h * D + kb * 64, tok0);
+            tma_prefetch_l2_2d(&mapV, tp.h * D + kb * 64, tok0);
+          }
+          ++ip;
+          tile_next(p, tp);
+        }
+      };
       int kslot = 0, kuse = 0;  // K ring position, number of slot fills issued
       int vent = 0, vuse = 0;
       int nseg = 0;
       bool skip_first = (p.debug_flags & 1u) != 0;
       bool ok = true;
       for (int i = 0; i <= ntiles && ok; ++i) {
+        if (rank == 0) prefetch_to(i + kPrefetchTiles);
         if (i < ntiles) {
           const bool first = (tk.j == 0) || (i == 0);
           if (first) {
@@ -265,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && ntiles > 0) {
       constexpr uint32_t idesc1 = idesc_bf16_f32(128, KC, false, false);
-      constexpr uint32_t idesc2 = idesc_bf16_f32(D, KC, true, true);
+      constexpr uint32_t idesc2 = idesc_bf16_f32(D, KC, true, true, /*f16_inputs=*/true);
       TilePos t1, t2;
       tile_seek(p, g0, t1);
       t2 = t1;
@@ -312,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool last = (t2.j == t2.nb - 1) || (i == ntiles);
           ok = wait(&bars.pfull, (i - 1) & 1);
           if (!ok) break;
-          ok = wait(&bars.vfull[vent], (vuse / p.nv_entries) & 1);
+          ok = wait(&bars.vconv[vent], (vuse / p.nv_entries) & 1);
           if (!ok) break;
           if (first && nseg2 > 0) {
             ok = wait(&bars.ofree, (nseg2 - 1) & 1);
@@ -341,6 +365,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Drain every MMA this thread issued before TMEM is released.
       umma_commit(&bars.drain);
       wait(&bars.drain, 0, false, true);
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ V converters: bf16 -> fp16
+    const int ct = threadIdx.x - 64;
+    int vent = 0, vuse = 0;
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      ok = __all_sync(0xffffffffu, wait(&bars.vfull[vent], (vuse / p.nv_entries) & 1));
+      if (!ok) break;
+      uint4* base = reinterpret_cast<uint4*>(sV + vent * KB * kSlotBytes);
+      constexpr int kChunks = KB * kSlotBytes / 16;
+#pragma unroll 4
+      for (int c = ct; c < kChunks; c += kConvThreads) {
+        uint4 w = base[c];
+        w.x = bf16x2_to_f16x2(w.x);
+        w.y = bf16x2_to_f16x2(w.y);
+        w.z = bf16x2_to_f16x2(w.z);
+        w.w = bf16x2_to_f16x2(w.w);
+        base[c] = w;
+      }
+      fence_async_shared();
+      mbar_arrive(&bars.vconv[vent]);
+      vent = (vent + 1 == p.nv_entries) ? 0 : vent + 1;
+      ++vuse;
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax warpgroups
@@ -409,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float f = valid ? ex2_approx(m2 - M) / Lsum : 0.f;
 
-      // P[tok, j] = A_{j,tok} as bf16 into the swizzled MN-major operand of MMA2.
+      // P[tok, j] = A_{j,tok} as fp16 into the swizzled MN-major operand of MMA2.
       if (i > 0) {
         ok = __all_sync(0xffffffffu, wait(&bars.pfree, (i - 1) & 1));
         if (!ok) break;
@@ -418,10 +466,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < NCOL; c += 8) {
         const int jj = col0 + c;
         uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(sv[c + 0]) * f, __uint_as_float(sv[c + 1]) * f);
-        w.y = pack_bf16x2(__uint_as_float(sv[c + 2]) * f, __uint_as_float(sv[c + 3]) * f);
-        w.z = pack_bf16x2(__uint_as_float(sv[c + 4]) * f, __uint_as_float(sv[c + 5]) * f);
-        w.w = pack_bf16x2(__uint_as_float(sv[c + 6]) * f, __uint_as_float(sv[c + 7]) * f);
+        w.x = pack_f16x2(__uint_as_float(sv[c + 0]) * f, __uint_as_float(sv[c + 1]) * f);
+        w.y = pack_f16x2(__uint_as_float(sv[c + 2]) * f, __uint_as_float(sv[c + 3]) * f);
+        w.z = pack_f16x2(__uint_as_float(sv[c + 4]) * f, __uint_as_float(sv[c + 5]) * f);
+        w.w = pack_f16x2(__uint_as_float(sv[c + 6]) * f, __uint_as_float(sv[c + 7]) * f);
         if (!valid) w = make_uint4(0, 0, 0, 0);
         uint8_t* dst = sP + (jj >> 6) * kSlotBytes + sw128_offset(r, (jj & 63) * 2);
         *reinterpret_cast<uint4*>(dst) = w;

@@ -53,6 +53,7 @@ def assert_close(got, want, what):
     mx = float(err.max())
     denom = float(np.linalg.norm(want[fin]))
     rel = float(np.linalg.norm(got[fin] - want[fin]) / denom) if denom > 0 else float(np.linalg.norm(got[fin]))
+    print(f"[parity] {what}: max abs {mx:.3e}, rel L2 {rel:.3e}, max |want| {np.abs(want[fin]).max():.3e}")
     assert mx <= MAX_ABS and rel <= REL_L2, f"{what}: max abs {mx:.3e}, rel L2 {rel:.3e}"
     return mx, rel
 
