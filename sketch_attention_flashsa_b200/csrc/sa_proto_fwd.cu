@@ -33,6 +33,7 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kSoftmaxThreads = 256;
+constexpr int kSoftmaxWarps = 8;
 constexpr int kConvThreads = 64;
 constexpr int kPrefetchTiles = 3;  // L2 prefetch distance of the producer, in tiles
 constexpr int kSlotBytes = 16384;  // one [128 rows x 64 bf16] swizzled block
@@ -173,14 +174,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars.qfull, 1);
     mbar_init(&bars.qfree, 1);
     mbar_init(&bars.sfull, 1);
-    mbar_init(&bars.sfree, kSoftmaxThreads);
-    mbar_init(&bars.pfull, kSoftmaxThreads);
+    mbar_init(&bars.sfree, kSoftmaxWarps);
+    mbar_init(&bars.pfull, kSoftmaxWarps);
     mbar_init(&bars.pfree, 1);
     mbar_init(&bars.ofull, 1);
-    mbar_init(&bars.ofree, kSoftmaxThreads);
+    mbar_init(&bars.ofree, kSoftmaxWarps);
     mbar_init(&bars.drain, 1);
-    mbar_init(&bars.xbar[0], CS * kSoftmaxThreads);
-    mbar_init(&bars.xbar[1], CS * kSoftmaxThreads);
+    mbar_init(&bars.xbar[0], 1);  // one arming arrival + CS * 256 * 8 transaction bytes
+    mbar_init(&bars.xbar[1], 1);
     bars.abort_flag = 0;
     fence_mbar_init();
   }
@@ -398,18 +399,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int col0 = g * NCOL;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const float c2 = p.scale_log2;
+    const uint64_t c2x2 = f2_pack(c2, c2);
     TilePos t;
     if (ntiles > 0) tile_seek(p, g0, t);
     int nseg = 0;
     bool ok = true;
     const uint32_t xbase = smem_u32(sX);
     const uint32_t xbar_local[2] = {smem_u32(&bars.xbar[0]), smem_u32(&bars.xbar[1])};
+    const bool x_owner = (threadIdx.x == 128);  // arms the exchange barrier's byte count
+    constexpr uint32_t kXBytesPerCta = kSoftmaxThreads * 8;
+    int cur_b = -1, used = 0, tok_base = 0;
     for (int i = 0; i < ntiles && ok; ++i) {
-      const int used = user_used(p, t.b);
+      if (t.b != cur_b) {
+        cur_b = t.b;
+        used = user_used(p, t.b);
+        tok_base = p.cu_seqlens[t.b];
+      }
       const int nvalid = min(kTileTokens, used - t.j * kTileTokens);
       const bool valid = r < nvalid;
-      const int tok = p.cu_seqlens[t.b] + t.j * kTileTokens + r;
+      const int tok = tok_base + t.j * kTileTokens + r;
       const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
+      const int par = i & 1;
+      if (x_owner) mbar_expect_tx(&bars.xbar[par], kXBytesPerCta * CS);
 
       ok = __all_sync(0xffffffffu, wait(&bars.sfull, i & 1));
       if (!ok) break;
@@ -423,29 +434,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (NCOL > R16) tmem_ld8(tS + lane_off + col0 + R16, sv + R16);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&bars.sfree);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.sfree);
 
       // Local statistics in the log2 domain: m2 = max_j s_j * c2, l = sum_j 2^(s_j c2 - m2).
+      // Four independent max chains and two packed-pair sum chains keep latency off the path.
       float m2 = -INFINITY, lsum = 0.f;
       if (valid) {
-        float mx = __uint_as_float(sv[0]);
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int c = 1; c < NCOL; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
-        m2 = mx * c2;
-#pragma unroll
-        for (int c = 0; c < NCOL; ++c) {
-          const float e = ex2_approx(fmaf(__uint_as_float(sv[c]), c2, -m2));
-          sv[c] = __float_as_uint(e);
-          lsum += e;
+        for (int c = 0; c < NCOL; c += 8) {
+          mx0 = max3f(mx0, __uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
+          mx1 = max3f(mx1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
+          mx2 = max3f(mx2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
+          mx3 = max3f(mx3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
         }
+        m2 = fmaxf(max3f(mx0, mx1, mx2), mx3) * c2;
+        const uint64_t negm = f2_pack(-m2, -m2);
+        uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+        for (int c = 0; c < NCOL; c += 4) {
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), c2x2, negm), x0, x1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), c2x2, negm), x2, x3);
+          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1), e2 = ex2_approx(x2), e3 = ex2_approx(x3);
+          sv[c] = __float_as_uint(e0);
+          sv[c + 1] = __float_as_uint(e1);
+          sv[c + 2] = __float_as_uint(e2);
+          sv[c + 3] = __float_as_uint(e3);
+          acc0 = f2_add(acc0, f2_pack(e0, e1));
+          acc1 = f2_add(acc1, f2_pack(e2, e3));
+        }
+        float a0, a1, b0, b1;
+        f2_unpack(acc0, a0, a1);
+        f2_unpack(acc1, b0, b1);
+        lsum = (a0 + a1) + (b0 + b1);
       }
-      // Exchange (m2, l) with every warpgroup of every CTA of the cluster.
-      const int par = i & 1;
+      // Exchange (m2, l) with every warpgroup of every CTA of the cluster: asynchronous
+      // stores that count as transaction bytes on the destination CTA's exchange barrier.
       const uint32_t xoff = static_cast<uint32_t>((((par * CS + rank) * 2 + g) * 128 + r) * 8);
-      for (int c = 0; c < CS; ++c) {
-        st_cluster_f32x2(mapa_shared(xbase + xoff, c), m2, lsum);
-        mbar_arrive_remote(mapa_shared(xbar_local[par], c));
-      }
+      for (int c = 0; c < CS; ++c)
+        st_async_f32x2(mapa_shared(xbase + xoff, c), m2, lsum, mapa_shared(xbar_local[par], c));
       ok = __all_sync(0xffffffffu, wait(&bars.xbar[par], (i >> 1) & 1, true));
       if (!ok) break;
       float M = -INFINITY;
@@ -456,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         Lsum += e.y * ex2_approx(e.x - M);
       }
       const float f = valid ? ex2_approx(m2 - M) / Lsum : 0.f;
+      const uint64_t f2 = f2_pack(f, f);
 
       // P[tok, j] = A_{j,tok} as fp16 into the swizzled MN-major operand of MMA2.
       if (i > 0) {
@@ -466,16 +496,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < NCOL; c += 8) {
         const int jj = col0 + c;
         uint4 w;
-        w.x = pack_f16x2(__uint_as_float(sv[c + 0]) * f, __uint_as_float(sv[c + 1]) * f);
-        w.y = pack_f16x2(__uint_as_float(sv[c + 2]) * f, __uint_as_float(sv[c + 3]) * f);
-        w.z = pack_f16x2(__uint_as_float(sv[c + 4]) * f, __uint_as_float(sv[c + 5]) * f);
-        w.w = pack_f16x2(__uint_as_float(sv[c + 6]) * f, __uint_as_float(sv[c + 7]) * f);
+        float a0, a1;
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1])), f2), a0, a1);
+        w.x = pack_f16x2(a0, a1);
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), f2), a0, a1);
+        w.y = pack_f16x2(a0, a1);
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5])), f2), a0, a1);
+        w.z = pack_f16x2(a0, a1);
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7])), f2), a0, a1);
+        w.w = pack_f16x2(a0, a1);
         if (!valid) w = make_uint4(0, 0, 0, 0);
         uint8_t* dst = sP + (jj >> 6) * kSlotBytes + sw128_offset(r, (jj & 63) * 2);
         *reinterpret_cast<uint4*>(dst) = w;
       }
       fence_async_shared();
-      mbar_arrive(&bars.pfull);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.pfull);
 
       if (p.lse && valid && g == 0 && rank == 0 && tok < p.total_tokens)
         p.lse[static_cast<int64_t>(tok) * p.H + t.h] = (M + log2f(Lsum)) * 0.69314718055994531f;
@@ -499,7 +535,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(&bars.ofree);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.ofree);
         ++nseg;
       }
       tile_next(p, t);
