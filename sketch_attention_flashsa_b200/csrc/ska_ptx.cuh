@@ -353,6 +353,19 @@ __device__ __forceinline__ void st_async_f32x2(uint32_t dst_cluster_addr, float 
                : "memory");
 }
 
+// Two bf16 in one word, each multiplied by a fp32 pair `f2` (both halves equal), rounded once to
+// two fp16 (saturating at +-65504).
+__device__ __forceinline__ uint32_t scale_bf16x2_to_f16x2(uint32_t w, uint64_t f2) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(v) : "l"(v), "l"(f2));
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  uint32_t d;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
