@@ -174,6 +174,25 @@ ska_status ska_read_device_status(void* ws, void* stream);
  * the consumers' bounded waits must run out and report SKA_ERR_DEVICE_TIMEOUT). */
 void ska_set_debug(uint64_t wait_budget_ns, uint32_t flags);
 
+/* SA forward for callers that cannot allocate device memory (code running inside a memory
+ * pool it does not own, plugins that only receive input and output pointers, service paths
+ * that must not allocate after start-up). The paper has no counterpart: this is a deployment
+ * variant of sa_forward. It runs the same kernels with its scratch memory in a file-scope
+ * device array of sa_forward_noalloc_scratch_bytes() bytes (40 MiB) that every GPU loading this
+ * library holds until the process exits; it calls no allocator.
+ *   Arguments and outputs are those of sa_forward, without the workspace.
+ *   Returns SKA_ERR_WORKSPACE_TOO_SMALL, before any launch, when the problem needs more scratch
+ *   than the array holds (sa_forward_workspace_size(desc) > sa_forward_noalloc_scratch_bytes()).
+ *   The first call on a device looks up the array's address (cudaGetSymbolAddress); make it
+ *   before any stream capture. All calls on a device share the array: calls that overlap on
+ *   the GPU (other streams, other host threads) race and must be serialised by the caller.   */
+ska_status sa_forward_noalloc(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
+                              const int32_t* cu_seqlens, const int32_t* seqused, float* sketch,
+                              float* lse, float* mass, void* stream);
+
+/* Size in bytes of the device array that sa_forward_noalloc uses as scratch. */
+size_t sa_forward_noalloc_scratch_bytes(void);
+
 /* Bench hook (process-wide): while both handles are non-NULL, every later call records
  * `start_event` on its stream immediately before its fused main kernel and `stop_event`
  * immediately after it (cudaEvent_t handles created by the caller), so that the main kernel

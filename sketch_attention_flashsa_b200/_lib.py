@@ -21,7 +21,8 @@ SKA_NORM_TOKEN = 1
 
 EXPORTED = ("sa_forward_workspace_size", "sa_forward", "sa_backward_workspace_size", "sa_backward",
             "stca_forward_workspace_size", "stca_forward", "ska_status_string",
-            "ska_read_device_status", "ska_set_debug", "ska_set_timing_events")
+            "ska_read_device_status", "ska_set_debug", "ska_set_timing_events",
+            "sa_forward_noalloc", "sa_forward_noalloc_scratch_bytes")
 
 
 class SaDesc(ctypes.Structure):
@@ -77,6 +78,10 @@ def lib() -> ctypes.CDLL:
     L.ska_read_device_status.restype = ctypes.c_int
     L.ska_set_debug.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
     L.ska_set_debug.restype = None
+    L.sa_forward_noalloc.argtypes = [ctypes.POINTER(SaDesc), vp, vp, vp, i32p, i32p, vp, vp, vp, vp]
+    L.sa_forward_noalloc.restype = ctypes.c_int
+    L.sa_forward_noalloc_scratch_bytes.argtypes = []
+    L.sa_forward_noalloc_scratch_bytes.restype = sz
     L.ska_set_timing_events.argtypes = [vp, vp]
     L.ska_set_timing_events.restype = None
     _lib = L
