@@ -42,6 +42,12 @@ constexpr int kPrefetchTiles = 3;  // L2 prefetch distance of the producer, in t
 constexpr int kSlotBytes = 16384;  // one [128 rows x 64 bf16] swizzled block
 constexpr int kMaxRing = 8;
 
+// Three of every eight groups of four exponentials go to the FMA pipe (exp2_fma_pair), the rest
+// to MUFU: at d = 128 the MUFU time of a tile equals its MMA time, so the split leaves headroom.
+__host__ __device__ constexpr bool exp_on_fma(int group4) {
+  return (group4 & 7) == 2 || (group4 & 7) == 5 || (group4 & 7) == 7;
+}
+
 struct SmemLayout {
   uint32_t q_off, p_off, k_off, v_off, x_off, m_off, l_off, f_off, total;
 };
@@ -384,11 +390,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------ exchange + V converters (rows of this warp)
-    const int cw = warp - 2;                 // rows [64 cw, 64 cw + 64)
+    // Lane l owns token rows r0 = 64 cw + l and r1 = r0 + 32 of every tile: it converts their
+    // V rows to fp16 in registers as soon as the tile lands, forms their factors f once the
+    // cluster exchange completes, and writes f * v back in place.
+    const int cw = warp - 2;
+    const int rows[2] = {cw * 64 + lane, cw * 64 + 32 + lane};
     const float c2 = p.scale_log2;
     const uint32_t xbase = smem_u32(sX);
     const uint32_t xbar_local[2] = {smem_u32(&bars.xbar[0]), smem_u32(&bars.xbar[1])};
     constexpr uint32_t kXBytesPerCta = 128 * 8;
+    constexpr int kWords = KB * 2 * 8 * 4;  // 32-bit words of V this lane converts per tile
     TilePos t;
     if (ntiles > 0) tile_seek(p, g0, t);
     int vent = 0, vuse = 0;
@@ -403,13 +414,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nvalid = min(kTileTokens, used - t.j * kTileTokens);
       const int par = i & 1;
       if (CS > 1 && cw == 0 && lane == 0) mbar_expect_tx(&bars.xbar[par], kXBytesPerCta * CS);
+
+      // 1. this lane's V rows -> fp16 words in registers (unscaled)
+      ok = __all_sync(0xffffffffu, wait(&bars.vfull[vent], (vuse / p.nv_entries) & 1));
+      if (!ok) break;
+      uint8_t* vb = sV + vent * KB * kSlotBytes;
+      uint32_t vw[kWords];
+#pragma unroll
+      for (int b = 0; b < KB; ++b)
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int st = 0; st < 8; ++st) {
+            // chunk (st + lane) & 7 of the row: 8 neighbouring lanes touch 8 different banks
+            const uint4 w = *reinterpret_cast<const uint4*>(vb + b * kSlotBytes + rows[u] * 128 +
+                                                            (((st + lane) & 7) << 4));
+            const int o = ((b * 2 + u) * 8 + st) * 4;
+            vw[o + 0] = bf16x2_as_f16x2(w.x);
+            vw[o + 1] = bf16x2_as_f16x2(w.y);
+            vw[o + 2] = bf16x2_as_f16x2(w.z);
+            vw[o + 3] = bf16x2_as_f16x2(w.w);
+          }
+
+      // 2. row statistics of this CTA and the cluster exchange
       ok = __all_sync(0xffffffffu, wait(&bars.statsready[par], (i >> 1) & 1));
       if (!ok) break;
-      // this CTA's row statistics (log2 domain), two rows per lane
       float m2[2], l[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int r = cw * 64 + u * 32 + lane;
+        const int r = rows[u];
         m2[u] = fmaxf(sM[(par * 2 + 0) * 128 + r], sM[(par * 2 + 1) * 128 + r]) * c2;
         l[u] = sL[(par * 2 + 0) * 128 + r] + sL[(par * 2 + 1) * 128 + r];
       }
@@ -417,8 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (CS > 1) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const int r = cw * 64 + u * 32 + lane;
-          const uint32_t xoff = static_cast<uint32_t>(((par * CS + rank) * 128 + r) * 8);
+          const uint32_t xoff = static_cast<uint32_t>(((par * CS + rank) * 128 + rows[u]) * 8);
           for (int c = 0; c < CS; ++c)
             st_async_f32x2(mapa_shared(xbase + xoff, c), m2[u], l[u], mapa_shared(xbar_local[par], c));
         }
@@ -426,46 +458,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const int r = cw * 64 + u * 32 + lane;
           float M = -INFINITY;
-          for (int c = 0; c < CS; ++c) M = fmaxf(M, sX[(par * CS + c) * 128 + r].x);
+          for (int c = 0; c < CS; ++c) M = fmaxf(M, sX[(par * CS + c) * 128 + rows[u]].x);
           float Ls = 0.f;
           for (int c = 0; c < CS; ++c) {
-            const float2 e = sX[(par * CS + c) * 128 + r];
+            const float2 e = sX[(par * CS + c) * 128 + rows[u]];
             Ls += e.y * ex2_approx(e.x - M);
           }
           Mx[u] = M;
           Lx[u] = Ls;
         }
       }
+      uint32_t fh[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int r = cw * 64 + u * 32 + lane;
-        const bool valid = r < nvalid;
-        sF[r] = valid ? ex2_approx(m2[u] - Mx[u]) / Lx[u] : 0.f;
-        const int tok = tok_base + t.j * kTileTokens + r;
+        const bool valid = rows[u] < nvalid;
+        const float f = valid ? ex2_approx(m2[u] - Mx[u]) / Lx[u] : 0.f;
+        fh[u] = pack_f16x2(f, f);
+        const int tok = tok_base + t.j * kTileTokens + rows[u];
         if (p.lse && valid && rank == 0 && tok < p.total_tokens)
           p.lse[static_cast<int64_t>(tok) * p.H + t.h] = (Mx[u] + log2f(Lx[u])) * 0.69314718055994531f;
       }
-      __syncwarp();
-      // V rows of this warp -> fp16 rows f * v, in place
-      ok = __all_sync(0xffffffffu, wait(&bars.vfull[vent], (vuse / p.nv_entries) & 1));
-      if (!ok) break;
-      uint8_t* vb = sV + vent * KB * kSlotBytes;
-#pragma unroll 4
-      for (int q = lane; q < KB * 512; q += 32) {
-        const int blk = q >> 9;
-        const int rr = cw * 64 + ((q & 511) >> 3);
-        uint4* ptr = reinterpret_cast<uint4*>(vb + blk * kSlotBytes + rr * 128 + (q & 7) * 16);
-        const float f = sF[rr];
-        const uint64_t ff = f2_pack(f, f);
-        uint4 w = *ptr;
-        w.x = scale_bf16x2_to_f16x2(w.x, ff);
-        w.y = scale_bf16x2_to_f16x2(w.y, ff);
-        w.z = scale_bf16x2_to_f16x2(w.z, ff);
-        w.w = scale_bf16x2_to_f16x2(w.w, ff);
-        *ptr = w;
-      }
+
+      // 3. f * v back into the tile (fp16), then hand it to MMA2
+#pragma unroll
+      for (int b = 0; b < KB; ++b)
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int st = 0; st < 8; ++st) {
+            const int o = ((b * 2 + u) * 8 + st) * 4;
+            uint4 w;
+            w.x = hmul2(vw[o + 0], fh[u]);
+            w.y = hmul2(vw[o + 1], fh[u]);
+            w.z = hmul2(vw[o + 2], fh[u]);
+            w.w = hmul2(vw[o + 3], fh[u]);
+            *reinterpret_cast<uint4*>(vb + b * kSlotBytes + rows[u] * 128 + (((st + lane) & 7) << 4)) = w;
+          }
       fence_async_shared();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.vconv[vent]);
@@ -543,7 +572,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           float x0, x1, x2, x3;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), c2x2, negm), x0, x1);
           f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), c2x2, negm), x2, x3);
-          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1), e2 = ex2_approx(x2), e3 = ex2_approx(x3);
+          float e0, e1, e2, e3;
+          if (exp_on_fma(c / 4)) {
+            exp2_fma_pair(x0, x1, e0, e1);
+            exp2_fma_pair(x2, x3, e2, e3);
+          } else {
+            e0 = ex2_approx(x0);
+            e1 = ex2_approx(x1);
+            e2 = ex2_approx(x2);
+            e3 = ex2_approx(x3);
+          }
           sv[c] = __float_as_uint(e0);
           sv[c + 1] = __float_as_uint(e1);
           sv[c + 2] = __float_as_uint(e2);
