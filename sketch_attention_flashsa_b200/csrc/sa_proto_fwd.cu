@@ -7,24 +7,21 @@
 // Layout of the computation (one cluster of CS CTAs works on one stream of 128-token tiles;
 // CTA c of the cluster owns prototypes [c*KC, (c+1)*KC)):
 //   MMA1  S^T[tok, j]  = K_tile[tok, :] . Q_c[j, :]^T     M=128 tokens, N=KC, K=D   (TMEM)
-//   softmax threads own one token row each: the row max m over this CTA's KC prototypes
-//         (both warpgroups agree on it through shared memory), E[tok, j] = exp(S - m) written
-//         as fp16 to shared memory, and the row sum l of E.
-//   V     converter warps exchange (m, l) of every row with the other CTAs of the cluster
-//         through distributed shared memory (asynchronous stores counted on an mbarrier), form
-//         the per-token factor f = exp(m - M) / L with the row's global max M and total L, and
-//         rewrite the bf16 V tile in place as fp16 rows f * v. E[tok, j] * f[tok] is the
-//         paper's A[j, tok], so the normalisation over prototypes never waits on the cluster.
-//   MMA2  O^T[dd, j]  += V'[tok, dd]^T . E[tok, j]        M=D, N=KC, K=128 tokens   (TMEM)
-//         in fp16 (11 significant bits, eight times finer than bf16) with fp32 accumulation.
+//   softmax threads own one token row each: max and sum over this CTA's KC prototypes, an
+//         exchange of (max, sum) with the other CTAs of the cluster through distributed
+//         shared memory, then P[tok, j] = exp(S - lse_tok) in bf16 to shared memory.
+//   MMA2  O^T[dd, j]  += V_tile[tok, dd]^T . P[tok, j]    M=D, N=KC, K=128 tokens   (TMEM)
+//         in fp16: P is rounded to fp16 (11 significant bits, eight times finer than bf16) and
+//         the bf16 V tile is rewritten in place as fp16 (exact inside the fp16 range) by two
+//         converter warps, so that the aggregation keeps ~5e-4 relative precision per weight.
 // Tiles of all (user, head) segments are concatenated and split evenly over the persistent
 // clusters; a cluster writes one fp32 partial sketch per segment it touches, and a second
 // kernel sums the partials of each segment in a fixed order (a plain sum: each token's
 // normalisation is complete inside the tile that holds it).
 //
 // Warp roles (384 threads): warp 0 = TMA producer, warp 1 = TMEM owner + MMA issuer,
-// warps 2-3 = exchange + V converters (each owns 64 token rows), warps 4-11 = two softmax
-// warpgroups (each owns half of the KC columns of every row).
+// warps 2-3 = V converters, warps 4-11 = two softmax warpgroups (each owns half of the KC
+// columns).
 #include <cstdio>
 
 #include "ska_internal.h"
@@ -37,19 +34,21 @@ namespace {
 constexpr int kThreads = 384;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kSoftmaxWarps = 8;
-constexpr int kConvWarps = 2;
+constexpr int kConvThreads = 64;
 constexpr int kPrefetchTiles = 3;  // L2 prefetch distance of the producer, in tiles
 constexpr int kSlotBytes = 16384;  // one [128 rows x 64 bf16] swizzled block
 constexpr int kMaxRing = 8;
 
-// Three of every eight groups of four exponentials go to the FMA pipe (exp2_fma_pair), the rest
-// to MUFU: at d = 128 the MUFU time of a tile equals its MMA time, so the split leaves headroom.
-__host__ __device__ constexpr bool exp_on_fma(int group4) {
-  return (group4 & 7) == 2 || (group4 & 7) == 5 || (group4 & 7) == 7;
-}
+// Groups of four exponentials (out of every eight) computed on the FMA pipe by exp2_fma_pair
+// instead of MUFU. At d = 128 the MUFU time of a tile equals its MMA time, but in the present
+// pipeline the softmax is bound by its dependency chain, not by MUFU throughput: measured on
+// the 8 x 100K x 8-head workload, moving 3/8 of the exponentials to the FMA pipe made the
+// kernel slower (3.01 ms against 2.64 ms), so the split is off.
+constexpr int kExpFmaGroups = 0;
+__host__ __device__ constexpr bool exp_on_fma(int group4) { return (group4 & 7) < kExpFmaGroups; }
 
 struct SmemLayout {
-  uint32_t q_off, p_off, k_off, v_off, x_off, m_off, l_off, f_off, total;
+  uint32_t q_off, p_off, k_off, v_off, x_off, total;
 };
 
 __host__ __device__ inline SmemLayout smem_layout(int D, int KC, int CS, int nk, int nv) {
@@ -65,13 +64,7 @@ __host__ __device__ inline SmemLayout smem_layout(int D, int KC, int CS, int nk,
   L.v_off = off;
   off += nv * (D / 64) * kSlotBytes;
   L.x_off = off;
-  off += 2 * CS * 128 * 8;  // (max, sum) exchange: [parity][cta][row] float2
-  L.m_off = off;
-  off += 2 * 2 * 128 * 4;   // row max per warpgroup: [parity][wg][row]
-  L.l_off = off;
-  off += 2 * 2 * 128 * 4;   // row sum per warpgroup: [parity][wg][row]
-  L.f_off = off;
-  off += 128 * 4;           // per-token factor f
+  off += 2 * CS * 2 * 128 * 8;  // (max, sum) exchange: [parity][cta][wg][row]
   L.total = off;
   return L;
 }
@@ -80,7 +73,7 @@ struct Bars {
   uint64_t kfull[kMaxRing], kempty[kMaxRing];
   uint64_t vfull[kMaxRing], vempty[kMaxRing], vconv[kMaxRing];
   uint64_t qfull, qfree, sfull, sfree, pfull, pfree, ofull, ofree, drain;
-  uint64_t xbar[2], mready[2], statsready[2];
+  uint64_t xbar[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -175,9 +168,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = smem + L.k_off;
   uint8_t* sV = smem + L.v_off;
   float2* sX = reinterpret_cast<float2*>(smem + L.x_off);
-  float* sM = reinterpret_cast<float*>(smem + L.m_off);
-  float* sL = reinterpret_cast<float*>(smem + L.l_off);
-  float* sF = reinterpret_cast<float*>(smem + L.f_off);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -187,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < p.nv_entries; ++i) {
       mbar_init(&bars.vfull[i], 1);
       mbar_init(&bars.vempty[i], 1);
-      mbar_init(&bars.vconv[i], kConvWarps);
+      mbar_init(&bars.vconv[i], kConvThreads);
     }
     mbar_init(&bars.qfull, 1);
     mbar_init(&bars.qfree, 1);
@@ -198,11 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars.ofull, 1);
     mbar_init(&bars.ofree, kSoftmaxWarps);
     mbar_init(&bars.drain, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.xbar[i], 1);  // one arming arrival + CS * 128 * 8 transaction bytes
-      mbar_init(&bars.mready[i], kSoftmaxWarps);
-      mbar_init(&bars.statsready[i], kSoftmaxWarps);
-    }
+    mbar_init(&bars.xbar[0], 1);  // one arming arrival + CS * 256 * 8 transaction bytes
+    mbar_init(&bars.xbar[1], 1);
     bars.abort_flag = 0;
     fence_mbar_init();
   }
@@ -389,118 +376,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait(&bars.drain, 0, false, true);
     }
   } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------ exchange + V converters (rows of this warp)
-    // Lane l owns token rows r0 = 64 cw + l and r1 = r0 + 32 of every tile: it converts their
-    // V rows to fp16 in registers as soon as the tile lands, forms their factors f once the
-    // cluster exchange completes, and writes f * v back in place.
-    const int cw = warp - 2;
-    const int rows[2] = {cw * 64 + lane, cw * 64 + 32 + lane};
-    const float c2 = p.scale_log2;
-    const uint32_t xbase = smem_u32(sX);
-    const uint32_t xbar_local[2] = {smem_u32(&bars.xbar[0]), smem_u32(&bars.xbar[1])};
-    constexpr uint32_t kXBytesPerCta = 128 * 8;
-    constexpr int kWords = KB * 2 * 8 * 4;  // 32-bit words of V this lane converts per tile
-    TilePos t;
-    if (ntiles > 0) tile_seek(p, g0, t);
+    // ------------------------------------------------------------ V converters: bf16 -> fp16
+    const int ct = threadIdx.x - 64;
     int vent = 0, vuse = 0;
-    int cur_b = -1, used = 0, tok_base = 0;
     bool ok = true;
     for (int i = 0; i < ntiles && ok; ++i) {
-      if (t.b != cur_b) {
-        cur_b = t.b;
-        used = user_used(p, t.b);
-        tok_base = p.cu_seqlens[t.b];
-      }
-      const int nvalid = min(kTileTokens, used - t.j * kTileTokens);
-      const int par = i & 1;
-      if (CS > 1 && cw == 0 && lane == 0) mbar_expect_tx(&bars.xbar[par], kXBytesPerCta * CS);
-
-      // 1. this lane's V rows -> fp16 words in registers (unscaled)
       ok = __all_sync(0xffffffffu, wait(&bars.vfull[vent], (vuse / p.nv_entries) & 1));
       if (!ok) break;
-      uint8_t* vb = sV + vent * KB * kSlotBytes;
-      uint32_t vw[kWords];
-#pragma unroll
-      for (int b = 0; b < KB; ++b)
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-          for (int st = 0; st < 8; ++st) {
-            // chunk (st + lane) & 7 of the row: 8 neighbouring lanes touch 8 different banks
-            const uint4 w = *reinterpret_cast<const uint4*>(vb + b * kSlotBytes + rows[u] * 128 +
-                                                            (((st + lane) & 7) << 4));
-            const int o = ((b * 2 + u) * 8 + st) * 4;
-            vw[o + 0] = bf16x2_as_f16x2(w.x);
-            vw[o + 1] = bf16x2_as_f16x2(w.y);
-            vw[o + 2] = bf16x2_as_f16x2(w.z);
-            vw[o + 3] = bf16x2_as_f16x2(w.w);
-          }
-
-      // 2. row statistics of this CTA and the cluster exchange
-      ok = __all_sync(0xffffffffu, wait(&bars.statsready[par], (i >> 1) & 1));
-      if (!ok) break;
-      float m2[2], l[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int r = rows[u];
-        m2[u] = fmaxf(sM[(par * 2 + 0) * 128 + r], sM[(par * 2 + 1) * 128 + r]) * c2;
-        l[u] = sL[(par * 2 + 0) * 128 + r] + sL[(par * 2 + 1) * 128 + r];
+      uint4* base = reinterpret_cast<uint4*>(sV + vent * KB * kSlotBytes);
+      constexpr int kChunks = KB * kSlotBytes / 16;
+#pragma unroll 4
+      for (int c = ct; c < kChunks; c += kConvThreads) {
+        uint4 w = base[c];
+        w.x = bf16x2_to_f16x2(w.x);
+        w.y = bf16x2_to_f16x2(w.y);
+        w.z = bf16x2_to_f16x2(w.z);
+        w.w = bf16x2_to_f16x2(w.w);
+        base[c] = w;
       }
-      float Mx[2] = {m2[0], m2[1]}, Lx[2] = {l[0], l[1]};
-      if (CS > 1) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const uint32_t xoff = static_cast<uint32_t>(((par * CS + rank) * 128 + rows[u]) * 8);
-          for (int c = 0; c < CS; ++c)
-            st_async_f32x2(mapa_shared(xbase + xoff, c), m2[u], l[u], mapa_shared(xbar_local[par], c));
-        }
-        ok = __all_sync(0xffffffffu, wait(&bars.xbar[par], (i >> 1) & 1, true));
-        if (!ok) break;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          float M = -INFINITY;
-          for (int c = 0; c < CS; ++c) M = fmaxf(M, sX[(par * CS + c) * 128 + rows[u]].x);
-          float Ls = 0.f;
-          for (int c = 0; c < CS; ++c) {
-            const float2 e = sX[(par * CS + c) * 128 + rows[u]];
-            Ls += e.y * ex2_approx(e.x - M);
-          }
-          Mx[u] = M;
-          Lx[u] = Ls;
-        }
-      }
-      uint32_t fh[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const bool valid = rows[u] < nvalid;
-        const float f = valid ? ex2_approx(m2[u] - Mx[u]) / Lx[u] : 0.f;
-        fh[u] = pack_f16x2(f, f);
-        const int tok = tok_base + t.j * kTileTokens + rows[u];
-        if (p.lse && valid && rank == 0 && tok < p.total_tokens)
-          p.lse[static_cast<int64_t>(tok) * p.H + t.h] = (Mx[u] + log2f(Lx[u])) * 0.69314718055994531f;
-      }
-
-      // 3. f * v back into the tile (fp16), then hand it to MMA2
-#pragma unroll
-      for (int b = 0; b < KB; ++b)
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-          for (int st = 0; st < 8; ++st) {
-            const int o = ((b * 2 + u) * 8 + st) * 4;
-            uint4 w;
-            w.x = hmul2(vw[o + 0], fh[u]);
-            w.y = hmul2(vw[o + 1], fh[u]);
-            w.z = hmul2(vw[o + 2], fh[u]);
-            w.w = hmul2(vw[o + 3], fh[u]);
-            *reinterpret_cast<uint4*>(vb + b * kSlotBytes + rows[u] * 128 + (((st + lane) & 7) << 4)) = w;
-          }
       fence_async_shared();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.vconv[vent]);
+      mbar_arrive(&bars.vconv[vent]);
       vent = (vent + 1 == p.nv_entries) ? 0 : vent + 1;
       ++vuse;
-      tile_next(p, t);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax warpgroups
@@ -515,16 +412,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ntiles > 0) tile_seek(p, g0, t);
     int nseg = 0;
     bool ok = true;
-    int cur_b = -1, used = 0;
+    const uint32_t xbase = smem_u32(sX);
+    const uint32_t xbar_local[2] = {smem_u32(&bars.xbar[0]), smem_u32(&bars.xbar[1])};
+    const bool x_owner = (threadIdx.x == 128);  // arms the exchange barrier's byte count
+    constexpr uint32_t kXBytesPerCta = kSoftmaxThreads * 8;
+    int cur_b = -1, used = 0, tok_base = 0;
     for (int i = 0; i < ntiles && ok; ++i) {
       if (t.b != cur_b) {
         cur_b = t.b;
         used = user_used(p, t.b);
+        tok_base = p.cu_seqlens[t.b];
       }
       const int nvalid = min(kTileTokens, used - t.j * kTileTokens);
       const bool valid = r < nvalid;
+      const int tok = tok_base + t.j * kTileTokens + r;
       const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
       const int par = i & 1;
+      if (x_owner) mbar_expect_tx(&bars.xbar[par], kXBytesPerCta * CS);
 
       ok = __all_sync(0xffffffffu, wait(&bars.sfull, i & 1));
       if (!ok) break;
@@ -541,9 +445,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.sfree);
 
-      // Row max over this warpgroup's columns (four independent chains), shared with the other
-      // warpgroup so that both exponentiate against the CTA's row max.
-      float mloc = -INFINITY;
+      // Local statistics in the log2 domain: m2 = max_j s_j * c2, l = sum_j 2^(s_j c2 - m2).
+      // Four independent max chains and two packed-pair sum chains keep latency off the path.
+      float m2 = -INFINITY, lsum = 0.f;
       if (valid) {
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
@@ -553,18 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mx2 = max3f(mx2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
           mx3 = max3f(mx3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
         }
-        mloc = fmaxf(max3f(mx0, mx1, mx2), mx3);
-      }
-      sM[(par * 2 + g) * 128 + r] = mloc;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.mready[par]);
-      ok = __all_sync(0xffffffffu, wait(&bars.mready[par], (i >> 1) & 1));
-      if (!ok) break;
-      const float m2 = fmaxf(sM[(par * 2 + 0) * 128 + r], sM[(par * 2 + 1) * 128 + r]) * c2;
-
-      // E = 2^(s c2 - m2) and its row sum (two packed-pair chains).
-      float lsum = 0.f;
-      if (valid) {
+        m2 = fmaxf(max3f(mx0, mx1, mx2), mx3) * c2;
         const uint64_t negm = f2_pack(-m2, -m2);
         uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
@@ -594,11 +487,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         f2_unpack(acc1, b0, b1);
         lsum = (a0 + a1) + (b0 + b1);
       }
-      sL[(par * 2 + g) * 128 + r] = lsum;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.statsready[par]);
+      // Exchange (m2, l) with every warpgroup of every CTA of the cluster: asynchronous
+      // stores that count as transaction bytes on the destination CTA's exchange barrier.
+      const uint32_t xoff = static_cast<uint32_t>((((par * CS + rank) * 2 + g) * 128 + r) * 8);
+      for (int c = 0; c < CS; ++c)
+        st_async_f32x2(mapa_shared(xbase + xoff, c), m2, lsum, mapa_shared(xbar_local[par], c));
+      ok = __all_sync(0xffffffffu, wait(&bars.xbar[par], (i >> 1) & 1, true));
+      if (!ok) break;
+      float M = -INFINITY;
+      for (int c = 0; c < CS * 2; ++c) M = fmaxf(M, sX[(par * CS * 2 + c) * 128 + r].x);
+      float Lsum = 0.f;
+      for (int c = 0; c < CS * 2; ++c) {
+        const float2 e = sX[(par * CS * 2 + c) * 128 + r];
+        Lsum += e.y * ex2_approx(e.x - M);
+      }
+      const float f = valid ? ex2_approx(m2 - M) / Lsum : 0.f;
+      const uint64_t f2 = f2_pack(f, f);
 
-      // E[tok, j] as fp16 into the swizzled MN-major operand of MMA2.
+      // P[tok, j] = A_{j,tok} as fp16 into the swizzled MN-major operand of MMA2.
       if (i > 0) {
         ok = __all_sync(0xffffffffu, wait(&bars.pfree, (i - 1) & 1));
         if (!ok) break;
@@ -607,10 +513,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < NCOL; c += 8) {
         const int jj = col0 + c;
         uint4 w;
-        w.x = pack_f16x2(__uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
-        w.y = pack_f16x2(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
-        w.z = pack_f16x2(__uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
-        w.w = pack_f16x2(__uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
+        float a0, a1;
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1])), f2), a0, a1);
+        w.x = pack_f16x2(a0, a1);
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), f2), a0, a1);
+        w.y = pack_f16x2(a0, a1);
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5])), f2), a0, a1);
+        w.z = pack_f16x2(a0, a1);
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7])), f2), a0, a1);
+        w.w = pack_f16x2(a0, a1);
         if (!valid) w = make_uint4(0, 0, 0, 0);
         uint8_t* dst = sP + (jj >> 6) * kSlotBytes + sw128_offset(r, (jj & 63) * 2);
         *reinterpret_cast<uint4*>(dst) = w;
@@ -618,6 +529,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_shared();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.pfull);
+
+      if (p.lse && valid && g == 0 && rank == 0 && tok < p.total_tokens)
+        p.lse[static_cast<int64_t>(tok) * p.H + t.h] = (M + log2f(Lsum)) * 0.69314718055994531f;
 
       if (last) {
         // Segment epilogue: O^T (this CTA's KC prototypes) -> partial sketch slot.
