@@ -10,7 +10,8 @@ from ._lib import SkaError, LIB_PATH  # noqa: F401
 
 def __getattr__(name):
     if name in ("sa_forward", "sa_desc", "sa_forward_workspace_size", "read_device_status",
-                "set_debug", "sa_backward", "stca_forward"):
+                "set_debug", "sa_backward", "stca_forward", "stca_desc", "stca_forward_workspace_size",
+                "set_timing_events"):
         from . import api
         return getattr(api, name)
     raise AttributeError(name)

@@ -110,3 +110,52 @@ def set_timing_events(start=None, stop=None) -> None:
     a = ctypes.c_void_p(start.cuda_event) if start is not None else ctypes.c_void_p(0)
     b = ctypes.c_void_p(stop.cuda_event) if stop is not None else ctypes.c_void_p(0)
     _lib.lib().ska_set_timing_events(a, b)
+
+
+def stca_desc(q, k_hist, k_sk, cu_targets, cu_hist, *, scale) -> StcaDesc:
+    d = StcaDesc()
+    d.num_users = cu_targets.numel() - 1
+    d.num_heads = q.shape[1]
+    d.head_dim = q.shape[2]
+    d.num_sketch = k_sk.shape[2] if k_sk is not None else 0
+    d.total_targets = q.shape[0]
+    d.total_hist = k_hist.shape[0] if k_hist is not None else 0
+    d.max_targets = 0
+    d.max_hist = 0
+    d.scale = float(scale)
+    d.reserved = 0
+    return d
+
+
+def stca_forward_workspace_size(desc: StcaDesc) -> int:
+    return int(_lib.lib().stca_forward_workspace_size(ctypes.byref(desc)))
+
+
+def stca_forward(q: torch.Tensor, cu_targets: torch.Tensor, k_hist: torch.Tensor, v_hist: torch.Tensor,
+                 cu_hist: torch.Tensor, k_sk: Optional[torch.Tensor], v_sk: Optional[torch.Tensor], *,
+                 scale: float, target_kv_len: Optional[torch.Tensor] = None, want_lse: bool = True,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """STCA forward (SequenceO1 §2.3; the suffix and sketch branches of §3.4; MRLB §4.2).
+
+    q [Tq,H,d] bf16 with cu_targets int32 [B+1]; k_hist, v_hist [Th,H,d] bf16 with cu_hist;
+    k_sk, v_sk [B,H,ks,d] bf16 or None; target_kv_len int32 [Tq] or None.
+    Returns (out fp32 [Tq,H,d], lse fp32 [Tq,H] or None).
+    """
+    for name, t in (("q", q), ("k_hist", k_hist), ("v_hist", v_hist), ("k_sk", k_sk), ("v_sk", v_sk)):
+        _dev_tensor(name, t, (torch.bfloat16,))
+    for name, t in (("cu_targets", cu_targets), ("cu_hist", cu_hist), ("target_kv_len", target_kv_len)):
+        _dev_tensor(name, t, (torch.int32,))
+    desc = stca_desc(q, k_hist, k_sk, cu_targets, cu_hist, scale=scale)
+    dev = q.device
+    need = stca_forward_workspace_size(desc)
+    if need == 0 and desc.total_targets > 0:
+        raise SkaError(_lib.SKA_ERR_UNSUPPORTED, "stca_forward_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev) if want_lse else None
+    rc = _lib.lib().stca_forward(ctypes.byref(desc), _ptr(q), _ptr(cu_targets), _ptr(k_hist), _ptr(v_hist),
+                                 _ptr(cu_hist), _ptr(target_kv_len), _ptr(k_sk), _ptr(v_sk), _ptr(out),
+                                 _ptr(lse), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check(rc, "stca_forward")
+    return out, lse

@@ -1,0 +1,664 @@
+// Row-softmax forward on sm_100a, shared by two operations:
+//
+// * Token-wise SA: the "vanilla attention" normalisation that SequenceO1 §5.1 / Table 1
+//   compares with the paper's prototype-wise Eq. (8): every prototype j takes a softmax over
+//   the valid history tokens of its user, sketch_j = sum_i softmax_i(scale q_j . k_i) v_i.
+// * STCA (§2.3, applied in §3.4 to the recent suffix and to the sketch, many targets of one
+//   user batched by MRLB, §4.2): out_t = softmax(scale q_t K^T) V over the keys
+//   [suffix rows of the user (the first target_kv_len[t] of them) ; the user's sketch rows].
+//
+// A "stream" is one 128-row query tile of one (user, head): prototypes for SA, targets for
+// STCA. Streams are walked in 128-key tiles with an online (running max / running sum)
+// softmax; the key tiles of all streams are concatenated and split evenly across persistent
+// CTAs, each CTA writes an unnormalised partial (O, max, sum) per stream it touches, and a
+// combine kernel merges the partials of a stream by their log-sum-exp weights.
+//
+// Per key tile (one CTA, 256 threads):
+//   MMA1  S[q, key] = Q_tile . K_tile^T       M=128, N=128, K=d   -> TMEM (two buffers)
+//   softmax warpgroup (thread = query row): mask, running max (rescaling O in TMEM only when
+//         the max grows by more than 2^8), P = 2^(s c - m) as bf16 into shared memory
+//   MMA2  O[q, dd] += P . V_tile              M=128, N=d, K=128   -> TMEM
+// Warp 0: TMA producer; warp 1: TMEM owner + MMA issuer; warps 4-7: softmax.
+#include <algorithm>
+#include <cmath>
+
+#include "ska_internal.h"
+#include "ska_ptx.cuh"
+
+namespace ska {
+
+namespace {
+
+constexpr int kFaThreads = 256;
+constexpr int kFaSoftmaxWarps = 4;
+constexpr int kFaSlot = 16384;         // one [128 rows x 64 bf16] swizzled block
+constexpr int kFaMaxRing = 8;
+constexpr float kRescaleThreshold = 8.f;  // log2 units
+
+__host__ __device__ constexpr int fa_q_bytes(int D) { return 128 * D * 2; }
+
+struct FaLayout {
+  uint32_t q_off, p_off, k_off, v_off, total;
+};
+
+__host__ __device__ inline FaLayout fa_layout(int D, int nk, int nv) {
+  FaLayout L;
+  uint32_t off = 0;
+  L.q_off = off;
+  off += fa_q_bytes(D);
+  L.p_off = off;
+  off += 2 * kFaSlot;                 // P: 128 rows x 128 keys bf16, two 64-key blocks
+  L.k_off = off;
+  off += nk * (D / 64) * kFaSlot;     // K ring: tile entries
+  L.v_off = off;
+  off += nv * (D / 64) * kFaSlot;     // V ring: tile entries
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- per-user geometry
+__device__ __forceinline__ int fa_used(const FaFwdParams& p, int b) {
+  int len = p.cu_keys[b + 1] - p.cu_keys[b];
+  if (p.seqused) len = min(len, p.seqused[b]);
+  return max(len, 0);
+}
+
+// query tiles of user b
+__device__ __forceinline__ int fa_qtiles(const FaFwdParams& p, int b) {
+  if (p.mode == 0) return (p.k + 127) / 128;
+  return (max(p.cu_q[b + 1] - p.cu_q[b], 0) + 127) / 128;
+}
+
+// key tiles of user b: [history or suffix tiles ; sketch tiles (STCA)]
+__device__ __forceinline__ int fa_hist_tiles(const FaFwdParams& p, int b) { return (fa_used(p, b) + 127) / 128; }
+__device__ __forceinline__ int fa_ktiles(const FaFwdParams& p, int b) {
+  return fa_hist_tiles(p, b) + (p.mode == 1 ? (p.ks + 127) / 128 : 0);
+}
+
+struct FaPos {
+  int b, seg, j;     // user, stream index inside the user (h * QT + qt), key tile
+  int nb, nseg;      // key tiles per stream of user b, streams of user b
+  int qt_n;          // query tiles of user b
+};
+
+__device__ __forceinline__ void fa_seek(const FaFwdParams& p, int g, FaPos& t) {
+  int lo = 0, hi = p.B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.tile_prefix[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  t.b = lo;
+  t.qt_n = fa_qtiles(p, lo);
+  t.nb = fa_ktiles(p, lo);
+  t.nseg = p.H * t.qt_n;
+  const int off = g - p.tile_prefix[lo];
+  t.seg = off / t.nb;
+  t.j = off - t.seg * t.nb;
+}
+
+__device__ __forceinline__ void fa_next(const FaFwdParams& p, FaPos& t) {
+  if (++t.j < t.nb) return;
+  t.j = 0;
+  if (++t.seg < t.nseg) return;
+  t.seg = 0;
+  while (true) {
+    ++t.b;
+    if (t.b >= p.B) return;
+    t.qt_n = fa_qtiles(p, t.b);
+    t.nb = fa_ktiles(p, t.b);
+    t.nseg = p.H * t.qt_n;
+    if (t.nb > 0 && t.nseg > 0) return;
+  }
+}
+
+// ---------------------------------------------------------------- schedule
+// One block: per-user prefixes of key tiles and streams, totals, tiles per CTA; clears status.
+__global__ void __launch_bounds__(1024) fa_schedule_kernel(const FaFwdParams p, int num_ctas) {
+  __shared__ long long part_t[1024];
+  __shared__ int part_s[1024];
+  const int t = threadIdx.x;
+  const int per = (p.B + 1023) / 1024;
+  const int lo = min(p.B, t * per), hi = min(p.B, lo + per);
+  long long st = 0;
+  int ss = 0;
+  for (int b = lo; b < hi; ++b) {
+    const int ns = p.H * fa_qtiles(p, b);
+    st += static_cast<long long>(ns) * fa_ktiles(p, b);
+    ss += ns;
+  }
+  part_t[t] = st;
+  part_s[t] = ss;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const long long vt = (t >= off) ? part_t[t - off] : 0;
+    const int vs = (t >= off) ? part_s[t - off] : 0;
+    __syncthreads();
+    part_t[t] += vt;
+    part_s[t] += vs;
+    __syncthreads();
+  }
+  long long rt = (t == 0) ? 0 : part_t[t - 1];
+  int rs = (t == 0) ? 0 : part_s[t - 1];
+  for (int b = lo; b < hi; ++b) {
+    const_cast<int32_t*>(p.tile_prefix)[b] = static_cast<int32_t>(rt);
+    const_cast<int32_t*>(p.seg_prefix)[b] = rs;
+    const int ns = p.H * fa_qtiles(p, b);
+    rt += static_cast<long long>(ns) * fa_ktiles(p, b);
+    rs += ns;
+  }
+  if (t == 1023) {
+    const_cast<int32_t*>(p.tile_prefix)[p.B] = static_cast<int32_t>(part_t[1023]);
+    const_cast<int32_t*>(p.seg_prefix)[p.B] = part_s[1023];
+    const int total = static_cast<int>(part_t[1023]);
+    p.hdr->total_tiles = total;
+    p.hdr->tiles_per_cluster = (total + num_ctas - 1) / num_ctas;
+    p.hdr->status = 0;
+  }
+}
+
+// ---------------------------------------------------------------- combine
+// One block per stream (grid = an upper bound on the streams; extra blocks exit). Thread r of
+// 128 merges row r over the partial slots s + c of the CTAs c that walked part of stream s.
+__global__ void __launch_bounds__(128) fa_combine_kernel(const FaFwdParams p, int D, float* __restrict__ out,
+                                                         float* __restrict__ lse) {
+  const int s = blockIdx.x;
+  const int S = p.seg_prefix[p.B];
+  if (s >= S) return;
+  int lo = 0, hi = p.B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.seg_prefix[mid] <= s) lo = mid; else hi = mid - 1;
+  }
+  const int b = lo;
+  const int qt_n = fa_qtiles(p, b);
+  const int sin = s - p.seg_prefix[b];
+  const int h = sin / qt_n, qt = sin - h * qt_n;
+  const int nb = fa_ktiles(p, b);
+  const int W = p.hdr->tiles_per_cluster;
+  int c0 = 0, c1 = -1;
+  if (nb > 0 && W > 0) {
+    const int t0 = p.tile_prefix[b] + sin * nb;
+    c0 = t0 / W;
+    c1 = (t0 + nb - 1) / W;
+  }
+  const int r = threadIdx.x;
+  const int q = qt * 128 + r;
+  const int nq = (p.mode == 0) ? p.k : (p.cu_q[b + 1] - p.cu_q[b]);
+  if (q >= nq) return;
+  float M = -INFINITY;
+  for (int c = c0; c <= c1; ++c) M = fmaxf(M, p.part_ml[(static_cast<int64_t>(s + c) * 128 + r) * 2]);
+  float L = 0.f;
+  for (int c = c0; c <= c1; ++c) {
+    const float mc = p.part_ml[(static_cast<int64_t>(s + c) * 128 + r) * 2];
+    const float lc = p.part_ml[(static_cast<int64_t>(s + c) * 128 + r) * 2 + 1];
+    if (mc != -INFINITY) L += lc * exp2f(mc - M);
+  }
+  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  int64_t orow;
+  if (p.mode == 0) orow = (static_cast<int64_t>(b) * p.H + h) * p.k + q;
+  else orow = static_cast<int64_t>(p.cu_q[b] + q) * p.H + h;
+  float* dst = out + orow * D;
+  for (int dd = 0; dd < D; dd += 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = c0; c <= c1; ++c) {
+      const float mc = p.part_ml[(static_cast<int64_t>(s + c) * 128 + r) * 2];
+      if (mc == -INFINITY) continue;
+      const float wc = exp2f(mc - M);
+      const float4 v = *reinterpret_cast<const float4*>(p.part_o + (static_cast<int64_t>(s + c) * 128 + r) * D + dd);
+      acc.x += wc * v.x; acc.y += wc * v.y; acc.z += wc * v.z; acc.w += wc * v.w;
+    }
+    acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+    *reinterpret_cast<float4*>(dst + dd) = acc;
+  }
+  if (lse) lse[orow] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+
+struct FaBars {
+  uint64_t kfull[kFaMaxRing], kempty[kFaMaxRing], vfull[kFaMaxRing], vempty[kFaMaxRing];
+  uint64_t qfull, qfree, sfull[2], sfree[2], pfull, pfree, ofull, ofree, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct FaWaiter {
+  FaBars* bars;
+  int* status;
+  uint64_t budget;
+  __device__ __forceinline__ bool operator()(uint64_t* bar, uint32_t parity, bool drain = false) {
+    volatile int* ab = &bars->abort_flag;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (!drain && *ab) return false;
+      if (globaltimer_ns() - t0 > budget) {
+        atomicCAS(status, 0, (int)SKA_ERR_DEVICE_TIMEOUT);
+        *ab = 1;
+        return false;
+      }
+    }
+  }
+};
+
+// Q tile row (in the Q map) and column base for stream `seg` of user b.
+__device__ __forceinline__ void fa_q_coord(const FaFwdParams& p, const FaPos& t, int D, int& c0, int& row) {
+  const int h = t.seg / t.qt_n, qt = t.seg - h * t.qt_n;
+  if (p.mode == 0) {
+    c0 = 0;
+    row = (p.q_per_user ? t.b * p.H * p.k : 0) + h * p.k + qt * 128;
+  } else {
+    c0 = h * D;
+    row = p.cu_q[t.b] + qt * 128;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFaThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                  const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapKs,
+                  const __grid_constant__ CUtensorMap mapVs, const FaFwdParams p) {
+  constexpr int KB = D / 64;
+  constexpr int kTileBytes = KB * kFaSlot;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ FaBars bars;
+  const FaLayout L = fa_layout(D, p.nk_slots, p.nv_entries);
+  uint8_t* sQ = smem + L.q_off;
+  uint8_t* sP = smem + L.p_off;
+  uint8_t* sK = smem + L.k_off;
+  uint8_t* sV = smem + L.v_off;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.nk_slots; ++i) { mbar_init(&bars.kfull[i], 1); mbar_init(&bars.kempty[i], 1); }
+    for (int i = 0; i < p.nv_entries; ++i) { mbar_init(&bars.vfull[i], 1); mbar_init(&bars.vempty[i], 1); }
+    mbar_init(&bars.qfull, 1);
+    mbar_init(&bars.qfree, 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&bars.sfull[i], 1); mbar_init(&bars.sfree[i], kFaSoftmaxWarps); }
+    mbar_init(&bars.pfull, kFaSoftmaxWarps);
+    mbar_init(&bars.pfree, 1);
+    mbar_init(&bars.ofull, 1);
+    mbar_init(&bars.ofree, kFaSoftmaxWarps);
+    mbar_init(&bars.drain, 1);
+    bars.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = bars.tmem_base;
+  const uint32_t tO = tbase + 256;   // O: 128 lanes x D columns; S buffers at columns 0 and 128
+  FaWaiter wait{&bars, &p.hdr->status, p.budget_ns};
+  const int total = p.hdr->total_tiles;
+  const int W = p.hdr->tiles_per_cluster;
+  const int g0 = blockIdx.x * W;
+  const int ntiles = (W > 0 && g0 < total) ? (min(total, g0 + W) - g0) : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && ntiles > 0) {
+      FaPos tk, tv;
+      fa_seek(p, g0, tk);
+      tv = tk;
+      int kent = 0, kuse = 0, vent = 0, vuse = 0, nq = 0;
+      bool ok = true;
+      bool skip_first = (p.debug_flags & 1u) != 0;
+      auto kv_coord = [&](const FaPos& t, int& c0, int& row, const CUtensorMap*& mk, const CUtensorMap*& mv) {
+        const int h = t.seg / t.qt_n;
+        const int nh = fa_hist_tiles(p, t.b);
+        if (t.j < nh) {
+          c0 = h * D;
+          row = p.cu_keys[t.b] + t.j * 128;
+          mk = &mapK;
+          mv = &mapV;
+        } else {
+          c0 = 0;
+          row = (t.b * p.H + h) * p.ks + (t.j - nh) * 128;
+          mk = &mapKs;
+          mv = &mapVs;
+        }
+      };
+      for (int i = 0; i <= ntiles && ok; ++i) {
+        if (i < ntiles) {
+          if (tk.j == 0 || i == 0) {
+            if (nq > 0) ok = wait(&bars.qfree, (nq - 1) & 1);
+            if (!ok) break;
+            int qc0, qrow;
+            fa_q_coord(p, tk, D, qc0, qrow);
+            mbar_expect_tx(&bars.qfull, fa_q_bytes(D));
+            for (int kb = 0; kb < KB; ++kb) tma_load_2d(sQ + kb * kFaSlot, &mapQ, &bars.qfull, qc0 + kb * 64, qrow);
+            ++nq;
+          }
+          ok = wait(&bars.kempty[kent], ((kuse / p.nk_slots) & 1) ^ 1);
+          if (!ok) break;
+          int c0, row;
+          const CUtensorMap *mk, *mv;
+          kv_coord(tk, c0, row, mk, mv);
+          if (skip_first) {
+            skip_first = false;  // withhold this arrival: the MMA warp's wait must run out
+          } else {
+            mbar_expect_tx(&bars.kfull[kent], kTileBytes);
+            for (int kb = 0; kb < KB; ++kb)
+              tma_load_2d(sK + kent * kTileBytes + kb * kFaSlot, mk, &bars.kfull[kent], c0 + kb * 64, row);
+          }
+          kent = (kent + 1 == p.nk_slots) ? 0 : kent + 1;
+          ++kuse;
+          fa_next(p, tk);
+        }
+        if (i >= 1) {
+          ok = wait(&bars.vempty[vent], ((vuse / p.nv_entries) & 1) ^ 1);
+          if (!ok) break;
+          int c0, row;
+          const CUtensorMap *mk, *mv;
+          kv_coord(tv, c0, row, mk, mv);
+          mbar_expect_tx(&bars.vfull[vent], kTileBytes);
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_2d(sV + vent * kTileBytes + kb * kFaSlot, mv, &bars.vfull[vent], c0 + kb * 64, row);
+          vent = (vent + 1 == p.nv_entries) ? 0 : vent + 1;
+          ++vuse;
+          fa_next(p, tv);
+        }
+      }
+      for (int e = 0; e < p.nk_slots; ++e) {
+        const int fills = (kuse > e) ? (kuse - e - 1) / p.nk_slots + 1 : 0;
+        if (fills > 0) wait(&bars.kfull[e], (fills - 1) & 1, true);
+      }
+      for (int e = 0; e < p.nv_entries; ++e) {
+        const int fills = (vuse > e) ? (vuse - e - 1) / p.nv_entries + 1 : 0;
+        if (fills > 0) wait(&bars.vfull[e], (fills - 1) & 1, true);
+      }
+      if (nq > 0) wait(&bars.qfull, (nq - 1) & 1, true);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && ntiles > 0) {
+      constexpr uint32_t idesc1 = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
+      FaPos t1, t2;
+      fa_seek(p, g0, t1);
+      t2 = t1;
+      int kent = 0, kuse = 0, vent = 0, vuse = 0, nq = 0, nseg2 = 0;
+      bool ok = true;
+      for (int i = 0; i <= ntiles && ok; ++i) {
+        if (i < ntiles) {
+          const bool first = (t1.j == 0) || (i == 0);
+          const bool last = (t1.j == t1.nb - 1) || (i == ntiles - 1);
+          if (first) {
+            ok = wait(&bars.qfull, nq & 1);
+            if (!ok) break;
+            ++nq;
+          }
+          const int sb = i & 1;
+          if (i >= 2) {
+            ok = wait(&bars.sfree[sb], ((i >> 1) - 1) & 1);
+            if (!ok) break;
+          }
+          ok = wait(&bars.kfull[kent], (kuse / p.nk_slots) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t kbase = smem_u32(sK + kent * kTileBytes);
+#pragma unroll
+          for (int s = 0; s < D / 16; ++s) {
+            const uint64_t ad = sw128_desc(smem_u32(sQ) + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(kbase + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
+            umma_bf16(tbase + sb * 128, ad, bd, idesc1, s > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars.kempty[kent]);
+          umma_commit(&bars.sfull[sb]);
+          if (last) umma_commit(&bars.qfree);
+          kent = (kent + 1 == p.nk_slots) ? 0 : kent + 1;
+          ++kuse;
+          fa_next(p, t1);
+        }
+        if (i >= 1) {
+          const bool first = (t2.j == 0) || (i == 1);
+          const bool last = (t2.j == t2.nb - 1) || (i == ntiles);
+          ok = wait(&bars.pfull, (i - 1) & 1);
+          if (!ok) break;
+          ok = wait(&bars.vfull[vent], (vuse / p.nv_entries) & 1);
+          if (!ok) break;
+          if (first && nseg2 > 0) {
+            ok = wait(&bars.ofree, (nseg2 - 1) & 1);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          const uint32_t vbase = smem_u32(sV + vent * kTileBytes);
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint64_t ad = sw128_desc(smem_u32(sP) + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(vbase + s * 2048, kFaSlot, 1024);
+            umma_bf16(tO, ad, bd, idesc2, (first && s == 0) ? 0u : 1u);
+          }
+          umma_commit(&bars.vempty[vent]);
+          umma_commit(&bars.pfree);
+          if (last) {
+            umma_commit(&bars.ofull);
+            ++nseg2;
+          }
+          vent = (vent + 1 == p.nv_entries) ? 0 : vent + 1;
+          ++vuse;
+          fa_next(p, t2);
+        }
+      }
+      umma_commit(&bars.drain);
+      wait(&bars.drain, 0, true);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax warpgroup
+    // (continued below)
+    const int q4 = warp - 4;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    const float c2 = p.scale_log2;
+    const uint64_t c2x2 = f2_pack(c2, c2);
+    FaPos t;
+    if (ntiles > 0) fa_seek(p, g0, t);
+    float m = -INFINITY, l = 0.f;
+    int nseg = 0;
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const bool first = (t.j == 0) || (i == 0);
+      const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
+      if (first) {
+        m = -INFINITY;
+        l = 0.f;
+      }
+      // valid keys of this tile for this row
+      const int nh = fa_hist_tiles(p, t.b);
+      int kk0, vlen;
+      if (t.j < nh) {
+        kk0 = t.j * 128;
+        vlen = fa_used(p, t.b);
+        if (p.mode == 1 && p.kv_len) {
+          const int qt = t.seg % t.qt_n;
+          const int q = qt * 128 + r;
+          const int nq = p.cu_q[t.b + 1] - p.cu_q[t.b];
+          if (q < nq) vlen = min(vlen, max(p.kv_len[p.cu_q[t.b] + q], 0));
+        }
+      } else {
+        kk0 = (t.j - nh) * 128;
+        vlen = p.ks;
+      }
+      const int nvalid = vlen - kk0;  // keys [0, nvalid) of this tile count
+
+      const int sb = i & 1;
+      ok = __all_sync(0xffffffffu, wait(&bars.sfull[sb], (i >> 1) & 1));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[128];
+#pragma unroll
+      for (int c = 0; c < 128; c += 32) tmem_ld32(tbase + sb * 128 + lane_off + c, sv + c);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.sfree[sb]);
+
+      // mask and tile max
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        if (c >= nvalid) sv[c] = __float_as_uint(-INFINITY);
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+        mx0 = max3f(mx0, __uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
+        mx1 = max3f(mx1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
+        mx2 = max3f(mx2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
+        mx3 = max3f(mx3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
+      }
+      const float mt = fmaxf(max3f(mx0, mx1, mx2), mx3) * c2;
+      // lazy rescale: move the reference only when the max grows by more than 2^8
+      float factor = 1.f;
+      if (mt > m + kRescaleThreshold || (m == -INFINITY && mt > -INFINITY)) {
+        factor = (m == -INFINITY) ? 0.f : ex2_approx(m - mt);
+        m = mt;
+      }
+      const float mref = (m == -INFINITY) ? 0.f : m;
+      const uint64_t negm = f2_pack(-mref, -mref);
+      uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+      for (int c = 0; c < 128; c += 4) {
+        float x0, x1, x2, x3;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), c2x2, negm), x0, x1);
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), c2x2, negm), x2, x3);
+        const float e0 = ex2_approx(x0), e1 = ex2_approx(x1), e2 = ex2_approx(x2), e3 = ex2_approx(x3);
+        sv[c] = __float_as_uint(e0);
+        sv[c + 1] = __float_as_uint(e1);
+        sv[c + 2] = __float_as_uint(e2);
+        sv[c + 3] = __float_as_uint(e3);
+        acc0 = f2_add(acc0, f2_pack(e0, e1));
+        acc1 = f2_add(acc1, f2_pack(e2, e3));
+      }
+      float a0, a1, b0, b1;
+      f2_unpack(acc0, a0, a1);
+      f2_unpack(acc1, b0, b1);
+      l = l * factor + ((a0 + a1) + (b0 + b1));
+
+      if (i > 0) {
+        ok = __all_sync(0xffffffffu, wait(&bars.pfree, (i - 1) & 1));
+        if (!ok) break;
+      }
+      // O rows whose reference moved are rescaled in TMEM (MMA2 of the previous tile is done)
+      if (!first && __any_sync(0xffffffffu, factor != 1.f)) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + lane_off + c, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * factor);
+          tmem_st32(tO + lane_off + c, ov);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+      }
+      // P row as bf16 into the K-major A operand of MMA2
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
+        w.y = pack_bf16x2(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
+        w.z = pack_bf16x2(__uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
+        w.w = pack_bf16x2(__uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
+        *reinterpret_cast<uint4*>(sP + (c >> 6) * kFaSlot + sw128_offset(r, (c & 63) * 2)) = w;
+      }
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.pfull);
+
+      if (last) {
+        ok = __all_sync(0xffffffffu, wait(&bars.ofull, nseg & 1));
+        if (!ok) break;
+        tc_fence_after();
+        const int slot = p.seg_prefix[t.b] + t.seg + static_cast<int>(blockIdx.x);
+        float* dst = p.part_o + (static_cast<int64_t>(slot) * 128 + r) * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + lane_off + c, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; u += 4)
+            *reinterpret_cast<float4*>(dst + c + u) = make_float4(__uint_as_float(ov[u]), __uint_as_float(ov[u + 1]),
+                                                                  __uint_as_float(ov[u + 2]), __uint_as_float(ov[u + 3]));
+        }
+        p.part_ml[(static_cast<int64_t>(slot) * 128 + r) * 2] = m;
+        p.part_ml[(static_cast<int64_t>(slot) * 128 + r) * 2 + 1] = l;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.ofree);
+        ++nseg;
+      }
+      fa_next(p, t);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+template <int D>
+cudaError_t fa_launch_t(int num_ctas, size_t smem, const CUtensorMap& mQ, const CUtensorMap& mK,
+                        const CUtensorMap& mV, const CUtensorMap& mKs, const CUtensorMap& mVs,
+                        const FaFwdParams& p, cudaStream_t stream) {
+  auto kern = fa_fwd_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<num_ctas, kFaThreads, smem, stream>>>(mQ, mK, mV, mKs, mVs, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool fa_fwd_plan(int D, int num_sms, int* num_ctas, size_t* smem_bytes, int* nk, int* nv) {
+  if (D != 64 && D != 128) return false;
+  const size_t budget = 227 * 1024 - 1024 - 512;
+  int best_k = 0, best_v = 0;
+  for (int v = 1; v <= kFaMaxRing; ++v)
+    for (int k = 1; k <= kFaMaxRing; ++k) {
+      if (fa_layout(D, k, v).total > budget) continue;
+      const int score = std::min(k, v) * 100 + k + v;
+      if (best_k == 0 || score > std::min(best_k, best_v) * 100 + best_k + best_v) {
+        best_k = k;
+        best_v = v;
+      }
+    }
+  if (best_k == 0) return false;
+  *nk = best_k;
+  *nv = best_v;
+  *num_ctas = num_sms;
+  *smem_bytes = fa_layout(D, best_k, best_v).total + 1024;
+  return true;
+}
+
+cudaError_t launch_fa_fwd(int D, int num_ctas, size_t smem, const CUtensorMap& mQ, const CUtensorMap& mK,
+                          const CUtensorMap& mV, const CUtensorMap& mKs, const CUtensorMap& mVs,
+                          const FaFwdParams& p, cudaStream_t stream) {
+  if (D == 64) return fa_launch_t<64>(num_ctas, smem, mQ, mK, mV, mKs, mVs, p, stream);
+  if (D == 128) return fa_launch_t<128>(num_ctas, smem, mQ, mK, mV, mKs, mVs, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fa_schedule(const FaFwdParams& p, int num_ctas, cudaStream_t stream) {
+  fa_schedule_kernel<<<1, 1024, 0, stream>>>(p, num_ctas);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fa_combine(const FaFwdParams& p, int D, int max_streams, float* out, float* lse,
+                              cudaStream_t stream) {
+  if (max_streams <= 0) return cudaSuccess;
+  fa_combine_kernel<<<max_streams, 128, 0, stream>>>(p, D, out, lse);
+  return cudaGetLastError();
+}
+
+}  // namespace ska

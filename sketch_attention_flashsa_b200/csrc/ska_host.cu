@@ -1,6 +1,7 @@
 // C-ABI host layer of libska.so: argument validation, workspace carving, TMA descriptor
 // encoding and kernel launches. Everything here runs on the host and only enqueues work on
 // the caller's stream; no device memory is read or allocated.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -145,6 +146,137 @@ bool plan_forward(const ska_sa_desc* d, ProtoFwdLaunch* L, int* nk, int* nv) {
   return proto_fwd_plan(d->head_dim, d->num_protos, sms, L, nk, nv);
 }
 
+// ---------------------------------------------------------------- row-softmax engine (token SA, STCA)
+struct FaWs {
+  size_t hdr, tile_prefix, seg_prefix, part_o, part_ml, qb, kb, vb, total;
+};
+
+void fa_ws_layout(int B, int D, long long max_streams, int num_ctas, size_t cast_q, size_t cast_kv, FaWs* w) {
+  size_t off = 0;
+  w->hdr = off;
+  off += sizeof(WsHeader);
+  w->tile_prefix = off;
+  off = align256(off + size_t(B + 1) * 4);
+  w->seg_prefix = off;
+  off = align256(off + size_t(B + 1) * 4);
+  const size_t slots = size_t(max_streams) + size_t(num_ctas);
+  w->part_o = off;
+  off = align256(off + slots * 128 * D * 4);
+  w->part_ml = off;
+  off = align256(off + slots * 128 * 2 * 4);
+  w->qb = w->kb = w->vb = 0;
+  if (cast_q || cast_kv) {
+    w->qb = off;
+    off = align256(off + cast_q * 2);
+    w->kb = off;
+    off = align256(off + cast_kv * 2);
+    w->vb = off;
+    off = align256(off + cast_kv * 2);
+  }
+  w->total = off;
+}
+
+long long sa_token_streams(const ska_sa_desc* d) {
+  return (long long)d->num_users * d->num_heads * ((d->num_protos + 127) / 128);
+}
+
+size_t sa_token_ws_size(const ska_sa_desc* d, FaWs* w, int* ctas, size_t* smem, int* nk, int* nv) {
+  const int sms = device_sm_count();
+  if (sms <= 0 || !fa_fwd_plan(d->head_dim, sms, ctas, smem, nk, nv)) return 0;
+  const size_t qn = size_t(d->q_per_user ? d->num_users : 1) * d->num_heads * d->num_protos * d->head_dim;
+  const size_t kvn = size_t(d->total_tokens) * d->num_heads * d->head_dim;
+  fa_ws_layout(d->num_users, d->head_dim, sa_token_streams(d), *ctas, d->in_dtype == SKA_F32 ? qn : 0,
+               d->in_dtype == SKA_F32 ? kvn : 0, w);
+  return w->total;
+}
+
+ska_status sa_forward_token(const ska_sa_desc* d, const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens, const int32_t* seqused, float* sketch, float* lse,
+                            void* ws, size_t ws_bytes, cudaStream_t s) {
+  const int B = d->num_users, H = d->num_heads, D = d->head_dim, kp = d->num_protos;
+  const int64_t T = d->total_tokens;
+  FaWs w;
+  int ctas, nk, nv;
+  size_t smem;
+  if (sa_token_ws_size(d, &w, &ctas, &smem, &nk, &nv) == 0) return SKA_ERR_UNSUPPORTED;
+  if (ws_bytes < w.total) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const size_t qn = size_t(d->q_per_user ? B : 1) * H * kp * D;
+  const size_t kvn = size_t(T) * H * D;
+  const void* qb = q;
+  const void* kb = k;
+  const void* vb = v;
+  if (d->in_dtype == SKA_F32) {
+    if (launch_cast_f32_bf16(static_cast<const float*>(q), wsb + w.qb, int64_t(qn), s) != cudaSuccess ||
+        launch_cast_f32_bf16(static_cast<const float*>(k), wsb + w.kb, int64_t(kvn), s) != cudaSuccess ||
+        launch_cast_f32_bf16(static_cast<const float*>(v), wsb + w.vb, int64_t(kvn), s) != cudaSuccess)
+      return SKA_ERR_CUDA;
+    qb = wsb + w.qb;
+    kb = wsb + w.kb;
+    vb = wsb + w.vb;
+  }
+  FaFwdParams p{};
+  p.mode = 0;
+  p.cu_keys = cu_seqlens;
+  p.seqused = seqused;
+  p.cu_q = nullptr;
+  p.kv_len = nullptr;
+  p.tile_prefix = reinterpret_cast<int32_t*>(wsb + w.tile_prefix);
+  p.seg_prefix = reinterpret_cast<int32_t*>(wsb + w.seg_prefix);
+  p.hdr = reinterpret_cast<WsHeader*>(wsb + w.hdr);
+  p.part_o = reinterpret_cast<float*>(wsb + w.part_o);
+  p.part_ml = reinterpret_cast<float*>(wsb + w.part_ml);
+  p.B = B;
+  p.H = H;
+  p.k = kp;
+  p.ks = 0;
+  p.q_per_user = d->q_per_user;
+  p.nk_slots = nk;
+  p.nv_entries = nv;
+  p.scale_log2 = d->scale * 1.4426950408889634f;
+  p.budget_ns = wait_budget();
+  p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
+  if (launch_fa_schedule(p, ctas, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (T > 0) {
+    CUtensorMap mQ, mK, mV;
+    const uint64_t qrows = uint64_t(d->q_per_user ? B : 1) * H * kp;
+    if (!encode_2d(&mQ, qb, D, qrows, D, 64, 128)) return SKA_ERR_CUDA;
+    if (!encode_2d(&mK, kb, uint64_t(H) * D, T, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+    if (!encode_2d(&mV, vb, uint64_t(H) * D, T, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+    cudaError_t e;
+    {
+      TimedRegion tr(s);
+      e = launch_fa_fwd(D, ctas, smem, mQ, mK, mV, mK, mV, p, s);
+    }
+    if (e != cudaSuccess) return SKA_ERR_CUDA;
+  }
+  if (launch_fa_combine(p, D, int(sa_token_streams(d)), sketch, lse, s) != cudaSuccess) return SKA_ERR_CUDA;
+  return SKA_OK;
+}
+
+ska_status check_stca_desc(const ska_stca_desc* d) {
+  if (!d) return SKA_ERR_INVALID_VALUE;
+  if (d->num_users < 0 || d->num_heads < 1 || d->num_sketch < 0 || d->total_targets < 0 || d->total_hist < 0 ||
+      d->total_targets >= (int64_t(1) << 31) || d->total_hist >= (int64_t(1) << 31))
+    return SKA_ERR_INVALID_VALUE;
+  if (!(d->scale > 0.f) || !std::isfinite(d->scale)) return SKA_ERR_INVALID_VALUE;
+  if (d->head_dim != 64 && d->head_dim != 128) return SKA_ERR_UNSUPPORTED;
+  if (int64_t(d->num_users) * d->num_heads * std::max(d->num_sketch, 1) >= (int64_t(1) << 31))
+    return SKA_ERR_INVALID_VALUE;
+  return SKA_OK;
+}
+
+long long stca_max_streams(const ska_stca_desc* d) {
+  return (long long)d->num_heads * ((d->total_targets + 127) / 128 + d->num_users);
+}
+
+size_t stca_ws_size(const ska_stca_desc* d, FaWs* w, int* ctas, size_t* smem, int* nk, int* nv) {
+  const int sms = device_sm_count();
+  if (sms <= 0 || !fa_fwd_plan(d->head_dim, sms, ctas, smem, nk, nv)) return 0;
+  fa_ws_layout(d->num_users, d->head_dim, stca_max_streams(d), *ctas, 0, 0, w);
+  return w->total;
+}
+
 }  // namespace
 
 extern "C" {
@@ -187,7 +319,12 @@ ska_status ska_read_device_status(void* ws, void* stream) {
 
 size_t sa_forward_workspace_size(const ska_sa_desc* d) {
   if (check_sa_desc(d) != SKA_OK) return 0;
-  if (d->norm != SKA_NORM_PROTO) return 0;
+  if (d->norm == SKA_NORM_TOKEN) {
+    FaWs w;
+    int c, nk, nv;
+    size_t sm;
+    return sa_token_ws_size(d, &w, &c, &sm, &nk, &nv);
+  }
   ProtoFwdLaunch L;
   int nk, nv;
   if (!plan_forward(d, &L, &nk, &nv)) return 0;
@@ -201,14 +338,10 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
                       void* stream) {
   ska_status st = check_sa_desc(d);
   if (st != SKA_OK) return st;
-  if (d->norm != SKA_NORM_PROTO) return SKA_ERR_UNSUPPORTED;
   if (mass) return SKA_ERR_UNSUPPORTED;
   const int B = d->num_users, H = d->num_heads, D = d->head_dim, kp = d->num_protos;
   const int64_t T = d->total_tokens;
   if (B == 0) return SKA_OK;
-  ProtoFwdLaunch L;
-  int nk = 0, nv = 0;
-  if (!plan_forward(d, &L, &nk, &nv)) return SKA_ERR_UNSUPPORTED;
   // pointers and alignment
   if (!q || !cu_seqlens || !sketch || !ws) return SKA_ERR_INVALID_VALUE;
   if (T > 0 && (!k || !v)) return SKA_ERR_INVALID_VALUE;
@@ -216,23 +349,30 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
       !aligned16(mass) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
       (reinterpret_cast<uintptr_t>(seqused) & 3u))
     return SKA_ERR_INVALID_VALUE;
-  FwdWs w;
-  fwd_ws_layout(d, L, &w);
-  if (ws_bytes < w.total) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  const size_t ws_need = sa_forward_workspace_size(d);
+  if (ws_need == 0) return SKA_ERR_UNSUPPORTED;
+  if (ws_bytes < ws_need) return SKA_ERR_WORKSPACE_TOO_SMALL;
   const size_t esz = d->in_dtype == SKA_F32 ? 4 : 2;
   const size_t qn = size_t(d->q_per_user ? B : 1) * H * kp * D;
   const size_t kvn = size_t(T) * H * D;
   const size_t sk_bytes = size_t(B) * H * kp * D * 4;
-  const size_t lse_bytes = size_t(T) * H * 4;
+  const size_t lse_bytes = (d->norm == SKA_NORM_PROTO ? size_t(T) : size_t(B) * kp) * H * 4;
   if (overlaps(sketch, sk_bytes, q, qn * esz) || overlaps(sketch, sk_bytes, k, kvn * esz) ||
       overlaps(sketch, sk_bytes, v, kvn * esz) || overlaps(lse, lse_bytes, q, qn * esz) ||
       overlaps(lse, lse_bytes, k, kvn * esz) || overlaps(lse, lse_bytes, v, kvn * esz) ||
-      overlaps(lse, lse_bytes, sketch, sk_bytes) || overlaps(ws, w.total, sketch, sk_bytes) ||
-      overlaps(ws, w.total, lse, lse_bytes) || overlaps(ws, w.total, q, qn * esz) ||
-      overlaps(ws, w.total, k, kvn * esz) || overlaps(ws, w.total, v, kvn * esz))
+      overlaps(lse, lse_bytes, sketch, sk_bytes) || overlaps(ws, ws_need, sketch, sk_bytes) ||
+      overlaps(ws, ws_need, lse, lse_bytes) || overlaps(ws, ws_need, q, qn * esz) ||
+      overlaps(ws, ws_need, k, kvn * esz) || overlaps(ws, ws_need, v, kvn * esz))
     return SKA_ERR_INVALID_VALUE;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d->norm == SKA_NORM_TOKEN)
+    return sa_forward_token(d, q, k, v, cu_seqlens, seqused, sketch, lse, ws, ws_bytes, s);
+  ProtoFwdLaunch L;
+  int nk = 0, nv = 0;
+  if (!plan_forward(d, &L, &nk, &nv)) return SKA_ERR_UNSUPPORTED;
+  FwdWs w;
+  fwd_ws_layout(d, L, &w);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb + w.hdr);
   int32_t* prefix = reinterpret_cast<int32_t*>(wsb + w.prefix);
@@ -307,15 +447,96 @@ ska_status sa_backward(const ska_sa_desc* d, const void*, const void*, const voi
 }
 
 size_t stca_forward_workspace_size(const ska_stca_desc* d) {
-  (void)d;
-  return 0;
+  if (check_stca_desc(d) != SKA_OK) return 0;
+  FaWs w;
+  int c, nk, nv;
+  size_t sm;
+  return stca_ws_size(d, &w, &c, &sm, &nk, &nv);
 }
 
-ska_status stca_forward(const ska_stca_desc* d, const void*, const int32_t*, const void*, const void*,
-                        const int32_t*, const int32_t*, const void*, const void*, float*, float*, void*, size_t,
-                        void*) {
-  if (!d) return SKA_ERR_INVALID_VALUE;
-  return SKA_ERR_UNSUPPORTED;
+ska_status stca_forward(const ska_stca_desc* d, const void* q, const int32_t* cu_targets, const void* k_hist,
+                        const void* v_hist, const int32_t* cu_hist, const int32_t* target_kv_len, const void* k_sk,
+                        const void* v_sk, float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  ska_status st = check_stca_desc(d);
+  if (st != SKA_OK) return st;
+  const int B = d->num_users, H = d->num_heads, D = d->head_dim, ks = d->num_sketch;
+  const int64_t Tq = d->total_targets, Th = d->total_hist;
+  if (B == 0 || Tq == 0) return SKA_OK;
+  if (!q || !cu_targets || !cu_hist || !out || !ws) return SKA_ERR_INVALID_VALUE;
+  if (Th > 0 && (!k_hist || !v_hist)) return SKA_ERR_INVALID_VALUE;
+  if (ks > 0 && (!k_sk || !v_sk)) return SKA_ERR_INVALID_VALUE;
+  if (!aligned16(q) || !aligned16(k_hist) || !aligned16(v_hist) || !aligned16(k_sk) || !aligned16(v_sk) ||
+      !aligned16(out) || !aligned16(lse) || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
+      (reinterpret_cast<uintptr_t>(cu_targets) & 3u) || (reinterpret_cast<uintptr_t>(cu_hist) & 3u) ||
+      (reinterpret_cast<uintptr_t>(target_kv_len) & 3u))
+    return SKA_ERR_INVALID_VALUE;
+  FaWs w;
+  int ctas, nk, nv;
+  size_t smem;
+  if (stca_ws_size(d, &w, &ctas, &smem, &nk, &nv) == 0) return SKA_ERR_UNSUPPORTED;
+  if (ws_bytes < w.total) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  const size_t out_bytes = size_t(Tq) * H * D * 4, lse_bytes = size_t(Tq) * H * 4;
+  const size_t qb_ = size_t(Tq) * H * D * 2, hb = size_t(Th) * H * D * 2, sb = size_t(B) * H * ks * D * 2;
+  const void* ins[5] = {q, k_hist, v_hist, k_sk, v_sk};
+  const size_t insz[5] = {qb_, hb, hb, sb, sb};
+  for (int i = 0; i < 5; ++i)
+    if (overlaps(out, out_bytes, ins[i], insz[i]) || overlaps(lse, lse_bytes, ins[i], insz[i]) ||
+        overlaps(ws, w.total, ins[i], insz[i]))
+      return SKA_ERR_INVALID_VALUE;
+  if (overlaps(out, out_bytes, lse, lse_bytes) || overlaps(ws, w.total, out, out_bytes) ||
+      overlaps(ws, w.total, lse, lse_bytes))
+    return SKA_ERR_INVALID_VALUE;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  FaFwdParams p{};
+  p.mode = 1;
+  p.cu_keys = cu_hist;
+  p.seqused = nullptr;
+  p.cu_q = cu_targets;
+  p.kv_len = target_kv_len;
+  p.tile_prefix = reinterpret_cast<int32_t*>(wsb + w.tile_prefix);
+  p.seg_prefix = reinterpret_cast<int32_t*>(wsb + w.seg_prefix);
+  p.hdr = reinterpret_cast<WsHeader*>(wsb + w.hdr);
+  p.part_o = reinterpret_cast<float*>(wsb + w.part_o);
+  p.part_ml = reinterpret_cast<float*>(wsb + w.part_ml);
+  p.B = B;
+  p.H = H;
+  p.k = 0;
+  p.ks = ks;
+  p.q_per_user = 0;
+  p.nk_slots = nk;
+  p.nv_entries = nv;
+  p.scale_log2 = d->scale * 1.4426950408889634f;
+  p.budget_ns = wait_budget();
+  p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
+  if (launch_fa_schedule(p, ctas, s) != cudaSuccess) return SKA_ERR_CUDA;
+  CUtensorMap mQ, mK, mV, mKs, mVs;
+  if (!encode_2d(&mQ, q, uint64_t(H) * D, Tq, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+  // maps over absent segments point at q with one row; no tile of theirs is ever loaded
+  if (Th > 0) {
+    if (!encode_2d(&mK, k_hist, uint64_t(H) * D, Th, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+    if (!encode_2d(&mV, v_hist, uint64_t(H) * D, Th, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+  } else {
+    mK = mQ;
+    mV = mQ;
+  }
+  if (ks > 0) {
+    const uint64_t rows = uint64_t(B) * H * ks;
+    if (!encode_2d(&mKs, k_sk, D, rows, D, 64, 128)) return SKA_ERR_CUDA;
+    if (!encode_2d(&mVs, v_sk, D, rows, D, 64, 128)) return SKA_ERR_CUDA;
+  } else {
+    mKs = mQ;
+    mVs = mQ;
+  }
+  cudaError_t e;
+  {
+    TimedRegion tr(s);
+    e = launch_fa_fwd(D, ctas, smem, mQ, mK, mV, mKs, mVs, p, s);
+  }
+  if (e != cudaSuccess) return SKA_ERR_CUDA;
+  if (launch_fa_combine(p, D, int(stca_max_streams(d)), out, lse, s) != cudaSuccess) return SKA_ERR_CUDA;
+  return SKA_OK;
 }
 
 }  // extern "C"

@@ -55,6 +55,43 @@ cudaError_t launch_proto_fwd(int head_dim, const ProtoFwdLaunch& L, const CUtens
                              const CUtensorMap& mapK, const CUtensorMap& mapV, const ProtoFwdParams& p,
                              cudaStream_t stream);
 
+// Parameters of the row-softmax (FlashAttention-style) forward shared by token-wise SA and
+// STCA. A "stream" is one 128-row query tile of one (user, head): prototypes (SA) or targets
+// (STCA); its keys are the user's valid history (SA) or [suffix ; sketch] (STCA).
+struct FaFwdParams {
+  int mode;                    // 0 = SA token-wise, 1 = STCA
+  const int32_t* cu_keys;      // SA: cu_seqlens; STCA: cu_hist
+  const int32_t* seqused;      // SA only, nullable
+  const int32_t* cu_q;         // STCA: cu_targets; SA: null
+  const int32_t* kv_len;       // STCA: per-target suffix length, nullable
+  const int32_t* tile_prefix;  // [B+1] key tiles of all streams of users < b
+  const int32_t* seg_prefix;   // [B+1] streams of users < b
+  WsHeader* hdr;
+  float* part_o;               // [(max_streams + clusters) * 128 * D] unnormalised O
+  float* part_ml;              // [(max_streams + clusters) * 128 * 2] (max in log2 units, sum)
+  int B, H;
+  int k;                       // SA: prototypes
+  int ks;                      // STCA: sketch rows per (user, head)
+  int q_per_user;              // SA: q is [B,H,k,d]
+  int nk_slots, nv_entries;
+  float scale_log2;
+  uint64_t budget_ns;
+  uint32_t debug_flags;
+};
+
+bool fa_fwd_plan(int head_dim, int num_sms, int* num_ctas, size_t* smem_bytes, int* nk, int* nv);
+
+cudaError_t launch_fa_fwd(int head_dim, int num_ctas, size_t smem_bytes, const CUtensorMap& mapQ,
+                          const CUtensorMap& mapK, const CUtensorMap& mapV, const CUtensorMap& mapKs,
+                          const CUtensorMap& mapVs, const FaFwdParams& p, cudaStream_t stream);
+
+cudaError_t launch_fa_schedule(const FaFwdParams& p, int num_ctas, cudaStream_t stream);
+
+// LSE merge of the partials into the outputs. SA: out = sketch [B,H,k,D], lse [B,H,k].
+// STCA: out [total_targets, H, D], lse [total_targets, H].
+cudaError_t launch_fa_combine(const FaFwdParams& p, int head_dim, int max_streams, float* out, float* lse,
+                              cudaStream_t stream);
+
 // Small kernels (ska_small.cu).
 cudaError_t launch_schedule(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,
                             int num_clusters, int32_t* tile_prefix, WsHeader* hdr, cudaStream_t stream);
