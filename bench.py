@@ -292,6 +292,7 @@ def main():
     tflops = fl / (ms_per_step / 1e3) / 1e12
 
     peaks = load_peaks()
+    kname = "sa_proto_fwd_kernel" if args.norm == "proto" else "fa_fwd_kernel"
     t_tensor = fl / (peaks["bf16_tflops"] * 1e12)
     t_hbm = by / (peaks["hbm_gbs"] * 1e9)
     bound = "tensor" if t_tensor >= t_hbm else "hbm"
@@ -300,18 +301,22 @@ def main():
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": None,
                 "peak_source": f"{peaks['source']} bf16 dense (burst); sustained {peaks['bf16_tflops_sustained']}",
-                "kernel": "sa_proto_fwd_kernel", "kernel_ms": kern_mean}
+                "kernel": kname, "kernel_ms": kern_mean}
     else:
         achieved = by / (kern_mean / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
-                "kernel": "sa_proto_fwd_kernel", "kernel_ms": kern_mean}
+                "kernel": kname, "kernel_ms": kern_mean}
     traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(traffic_file):
+        import hashlib
         with open(traffic_file) as f:
             tr = json.load(f).get(args.workload, {}).get(args.norm)
         if tr:
-            roof["traffic"] = tr
+            with open(os.path.join(ROOT, tr["source"]), "rb") as f:
+                cur = hashlib.sha256(f.read()).hexdigest()[:16]
+            # counters are only valid for the kernel source they were taken on
+            roof["traffic"] = tr["bytes"] if cur == tr["source_sha256"] else None
 
     # End to end through the public API: pinned host inputs -> device, forward, sketch -> host.
     hq = inp["q"].cpu().pin_memory()
