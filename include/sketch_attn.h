@@ -131,8 +131,11 @@ ska_status sa_backward(const ska_sa_desc* desc, const void* q, const void* k, co
 
 /* One batched STCA problem (§2.3, §3.4, MRLB §4.2): num_users users, each with a block of
  * target queries that share the user's keys.
- *   head_dim 64 or 128; num_sketch = k_s sketch rows per user (0 allowed, a multiple of 8 else);
- *   total_targets = cu_targets[B]; total_hist = cu_hist[B]; scale > 0 (1/sqrt(d_h) in §2.3). */
+ *   head_dim 64 or 128; num_sketch = k_s sketch rows per user (0 allowed);
+ *   total_targets = cu_targets[B]; total_hist = cu_hist[B]; scale > 0 (1/sqrt(d_h) in §2.3);
+ *   max_targets: an upper bound on any user's target count (0: total_targets is used, which is
+ *   always a bound but leaves CTAs idle). A kernel that finds a user with more targets records
+ *   SKA_ERR_INVALID_VALUE in the device status word and computes nothing. max_hist: unused.  */
 typedef struct {
   int32_t num_users;
   int32_t num_heads;

@@ -112,7 +112,7 @@ def set_timing_events(start=None, stop=None) -> None:
     _lib.lib().ska_set_timing_events(a, b)
 
 
-def stca_desc(q, k_hist, k_sk, cu_targets, cu_hist, *, scale) -> StcaDesc:
+def stca_desc(q, k_hist, k_sk, cu_targets, cu_hist, *, scale, max_targets: int = 0) -> StcaDesc:
     d = StcaDesc()
     d.num_users = cu_targets.numel() - 1
     d.num_heads = q.shape[1]
@@ -120,7 +120,7 @@ def stca_desc(q, k_hist, k_sk, cu_targets, cu_hist, *, scale) -> StcaDesc:
     d.num_sketch = k_sk.shape[2] if k_sk is not None else 0
     d.total_targets = q.shape[0]
     d.total_hist = k_hist.shape[0] if k_hist is not None else 0
-    d.max_targets = 0
+    d.max_targets = int(max_targets)
     d.max_hist = 0
     d.scale = float(scale)
     d.reserved = 0
@@ -134,18 +134,21 @@ def stca_forward_workspace_size(desc: StcaDesc) -> int:
 def stca_forward(q: torch.Tensor, cu_targets: torch.Tensor, k_hist: torch.Tensor, v_hist: torch.Tensor,
                  cu_hist: torch.Tensor, k_sk: Optional[torch.Tensor], v_sk: Optional[torch.Tensor], *,
                  scale: float, target_kv_len: Optional[torch.Tensor] = None, want_lse: bool = True,
-                 workspace: Optional[torch.Tensor] = None, stream=None):
+                 max_targets: Optional[int] = None, workspace: Optional[torch.Tensor] = None, stream=None):
     """STCA forward (SequenceO1 §2.3; the suffix and sketch branches of §3.4; MRLB §4.2).
 
     q [Tq,H,d] bf16 with cu_targets int32 [B+1]; k_hist, v_hist [Th,H,d] bf16 with cu_hist;
-    k_sk, v_sk [B,H,ks,d] bf16 or None; target_kv_len int32 [Tq] or None.
+    k_sk, v_sk [B,H,ks,d] bf16 or None; target_kv_len int32 [Tq] or None; max_targets: an upper
+    bound on any user's target count (read from cu_targets when None).
     Returns (out fp32 [Tq,H,d], lse fp32 [Tq,H] or None).
     """
+    if max_targets is None:
+        max_targets = int((cu_targets[1:] - cu_targets[:-1]).max().item()) if cu_targets.numel() > 1 else 0
     for name, t in (("q", q), ("k_hist", k_hist), ("v_hist", v_hist), ("k_sk", k_sk), ("v_sk", v_sk)):
         _dev_tensor(name, t, (torch.bfloat16,))
     for name, t in (("cu_targets", cu_targets), ("cu_hist", cu_hist), ("target_kv_len", target_kv_len)):
         _dev_tensor(name, t, (torch.int32,))
-    desc = stca_desc(q, k_hist, k_sk, cu_targets, cu_hist, scale=scale)
+    desc = stca_desc(q, k_hist, k_sk, cu_targets, cu_hist, scale=scale, max_targets=max(max_targets, 1))
     dev = q.device
     need = stca_forward_workspace_size(desc)
     if need == 0 and desc.total_targets > 0:

@@ -75,123 +75,152 @@ __device__ __forceinline__ int fa_ktiles(const FaFwdParams& p, int b) {
   return fa_hist_tiles(p, b) + (p.mode == 1 ? (p.ks + 127) / 128 : 0);
 }
 
+// Work layout. Columns are the key tiles of every (user, head): user b contributes H * n_b
+// columns (n_b key tiles per head), in order (b, h, j). Persistent CTAs form groups of G (G =
+// the largest number of 128-row query tiles of any user); the CTAs of group g walk the same
+// contiguous column range together, CTA (g, qt) with query tile qt, so a K/V tile is read from
+// DRAM once and from L2 by the other G - 1 CTAs. Columns of users with fewer than qt + 1 query
+// tiles are skipped by that CTA.
 struct FaPos {
-  int b, seg, j;     // user, stream index inside the user (h * QT + qt), key tile
-  int nb, nseg;      // key tiles per stream of user b, streams of user b
-  int qt_n;          // query tiles of user b
+  int b, h, j;   // user, head, key tile
+  int nb, qtn;   // key tiles per head of user b, query tiles of user b
 };
 
-__device__ __forceinline__ void fa_seek(const FaFwdParams& p, int g, FaPos& t) {
+__device__ __forceinline__ void fa_user(const FaFwdParams& p, FaPos& t) {
+  t.nb = fa_ktiles(p, t.b);
+  t.qtn = fa_qtiles(p, t.b);
+}
+
+// First processable column at or after column g for query tile qt (t.b == B when none).
+__device__ __forceinline__ void fa_seek(const FaFwdParams& p, int g, int qt, FaPos& t) {
   int lo = 0, hi = p.B - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (p.tile_prefix[mid] <= g) lo = mid; else hi = mid - 1;
   }
   t.b = lo;
-  t.qt_n = fa_qtiles(p, lo);
-  t.nb = fa_ktiles(p, lo);
-  t.nseg = p.H * t.qt_n;
+  fa_user(p, t);
   const int off = g - p.tile_prefix[lo];
-  t.seg = off / t.nb;
-  t.j = off - t.seg * t.nb;
-}
-
-__device__ __forceinline__ void fa_next(const FaFwdParams& p, FaPos& t) {
-  if (++t.j < t.nb) return;
-  t.j = 0;
-  if (++t.seg < t.nseg) return;
-  t.seg = 0;
-  while (true) {
-    ++t.b;
-    if (t.b >= p.B) return;
-    t.qt_n = fa_qtiles(p, t.b);
-    t.nb = fa_ktiles(p, t.b);
-    t.nseg = p.H * t.qt_n;
-    if (t.nb > 0 && t.nseg > 0) return;
+  if (t.nb > 0 && off < p.H * t.nb) {
+    t.h = off / t.nb;
+    t.j = off - t.h * t.nb;
+  } else {
+    t.h = p.H;  // past this user
+    t.j = 0;
+  }
+  if (qt >= t.qtn || t.h >= p.H) {
+    t.h = 0;
+    t.j = 0;
+    do {
+      ++t.b;
+      if (t.b >= p.B) return;
+      fa_user(p, t);
+    } while (t.nb == 0 || qt >= t.qtn);
   }
 }
 
+__device__ __forceinline__ void fa_next(const FaFwdParams& p, int qt, FaPos& t) {
+  if (++t.j < t.nb) return;
+  t.j = 0;
+  if (++t.h < p.H) return;
+  t.h = 0;
+  do {
+    ++t.b;
+    if (t.b >= p.B) return;
+    fa_user(p, t);
+  } while (t.nb == 0 || qt >= t.qtn);
+}
+
+// Column index of a position.
+__device__ __forceinline__ int fa_col(const FaFwdParams& p, const FaPos& t) {
+  return p.tile_prefix[t.b] + t.h * t.nb + t.j;
+}
+
+// Number of columns in [c0, c1) that query tile qt processes.
+__device__ __forceinline__ int fa_count(const FaFwdParams& p, int qt, int c0, int c1) {
+  int n = 0;
+  int lo = 0, hi = p.B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.tile_prefix[mid] <= c0) lo = mid; else hi = mid - 1;
+  }
+  for (int b = lo; b < p.B; ++b) {
+    const int u0 = p.tile_prefix[b], u1 = p.tile_prefix[b + 1];
+    if (u0 >= c1) break;
+    if (qt < fa_qtiles(p, b)) n += max(0, min(u1, c1) - max(u0, c0));
+  }
+  return n;
+}
+
 // ---------------------------------------------------------------- schedule
-// One block: per-user prefixes of key tiles and streams, totals, tiles per CTA; clears status.
-__global__ void __launch_bounds__(1024) fa_schedule_kernel(const FaFwdParams p, int num_ctas) {
+// One block: tile_prefix[b] = sum_{b' < b} H * n_b'; columns per group; the largest number of
+// query tiles of any user (a device-side error when it exceeds the group size G); clears status.
+__global__ void __launch_bounds__(1024) fa_schedule_kernel(const FaFwdParams p, int num_groups, int G) {
   __shared__ long long part_t[1024];
-  __shared__ int part_s[1024];
+  __shared__ int part_q[1024];
   const int t = threadIdx.x;
   const int per = (p.B + 1023) / 1024;
   const int lo = min(p.B, t * per), hi = min(p.B, lo + per);
   long long st = 0;
-  int ss = 0;
+  int qmax = 0;
   for (int b = lo; b < hi; ++b) {
-    const int ns = p.H * fa_qtiles(p, b);
-    st += static_cast<long long>(ns) * fa_ktiles(p, b);
-    ss += ns;
+    st += static_cast<long long>(p.H) * fa_ktiles(p, b);
+    qmax = max(qmax, fa_qtiles(p, b));
   }
   part_t[t] = st;
-  part_s[t] = ss;
+  part_q[t] = qmax;
   __syncthreads();
   for (int off = 1; off < 1024; off <<= 1) {
     const long long vt = (t >= off) ? part_t[t - off] : 0;
-    const int vs = (t >= off) ? part_s[t - off] : 0;
+    const int vq = (t >= off) ? part_q[t - off] : 0;
     __syncthreads();
     part_t[t] += vt;
-    part_s[t] += vs;
+    part_q[t] = max(part_q[t], vq);
     __syncthreads();
   }
   long long rt = (t == 0) ? 0 : part_t[t - 1];
-  int rs = (t == 0) ? 0 : part_s[t - 1];
   for (int b = lo; b < hi; ++b) {
     const_cast<int32_t*>(p.tile_prefix)[b] = static_cast<int32_t>(rt);
-    const_cast<int32_t*>(p.seg_prefix)[b] = rs;
-    const int ns = p.H * fa_qtiles(p, b);
-    rt += static_cast<long long>(ns) * fa_ktiles(p, b);
-    rs += ns;
+    rt += static_cast<long long>(p.H) * fa_ktiles(p, b);
   }
   if (t == 1023) {
     const_cast<int32_t*>(p.tile_prefix)[p.B] = static_cast<int32_t>(part_t[1023]);
-    const_cast<int32_t*>(p.seg_prefix)[p.B] = part_s[1023];
     const int total = static_cast<int>(part_t[1023]);
     p.hdr->total_tiles = total;
-    p.hdr->tiles_per_cluster = (total + num_ctas - 1) / num_ctas;
-    p.hdr->status = 0;
+    p.hdr->tiles_per_cluster = (total + num_groups - 1) / num_groups;
+    p.hdr->status = (part_q[1023] > G) ? static_cast<int>(SKA_ERR_INVALID_VALUE) : 0;
   }
 }
 
 // ---------------------------------------------------------------- combine
-// One block per stream (grid = an upper bound on the streams; extra blocks exit). Thread r of
-// 128 merges row r over the partial slots s + c of the CTAs c that walked part of stream s.
-__global__ void __launch_bounds__(128) fa_combine_kernel(const FaFwdParams p, int D, float* __restrict__ out,
+// One block per (user, head, query tile) up to B * H * G; thread r merges row r of the stream
+// over the partial slots ((b H + h) + g) G + qt of the groups g that walked its columns.
+__global__ void __launch_bounds__(128) fa_combine_kernel(const FaFwdParams p, int D, int G, float* __restrict__ out,
                                                          float* __restrict__ lse) {
-  const int s = blockIdx.x;
-  const int S = p.seg_prefix[p.B];
-  if (s >= S) return;
-  int lo = 0, hi = p.B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.seg_prefix[mid] <= s) lo = mid; else hi = mid - 1;
-  }
-  const int b = lo;
-  const int qt_n = fa_qtiles(p, b);
-  const int sin = s - p.seg_prefix[b];
-  const int h = sin / qt_n, qt = sin - h * qt_n;
+  const int qt = blockIdx.x % G;
+  const int bh = blockIdx.x / G;
+  const int b = bh / p.H, h = bh - b * p.H;
+  if (b >= p.B) return;
+  if (qt >= fa_qtiles(p, b)) return;
   const int nb = fa_ktiles(p, b);
   const int W = p.hdr->tiles_per_cluster;
-  int c0 = 0, c1 = -1;
+  int g0 = 0, g1 = -1;
   if (nb > 0 && W > 0) {
-    const int t0 = p.tile_prefix[b] + sin * nb;
-    c0 = t0 / W;
-    c1 = (t0 + nb - 1) / W;
+    const int c0 = p.tile_prefix[b] + h * nb;
+    g0 = c0 / W;
+    g1 = (c0 + nb - 1) / W;
   }
   const int r = threadIdx.x;
   const int q = qt * 128 + r;
   const int nq = (p.mode == 0) ? p.k : (p.cu_q[b + 1] - p.cu_q[b]);
   if (q >= nq) return;
+  auto slot = [&](int g) { return (static_cast<int64_t>(bh + g) * G + qt) * 128 + r; };
   float M = -INFINITY;
-  for (int c = c0; c <= c1; ++c) M = fmaxf(M, p.part_ml[(static_cast<int64_t>(s + c) * 128 + r) * 2]);
+  for (int g = g0; g <= g1; ++g) M = fmaxf(M, p.part_ml[slot(g) * 2]);
   float L = 0.f;
-  for (int c = c0; c <= c1; ++c) {
-    const float mc = p.part_ml[(static_cast<int64_t>(s + c) * 128 + r) * 2];
-    const float lc = p.part_ml[(static_cast<int64_t>(s + c) * 128 + r) * 2 + 1];
-    if (mc != -INFINITY) L += lc * exp2f(mc - M);
+  for (int g = g0; g <= g1; ++g) {
+    const float mg = p.part_ml[slot(g) * 2];
+    if (mg != -INFINITY) L += p.part_ml[slot(g) * 2 + 1] * exp2f(mg - M);
   }
   const float inv = (L > 0.f) ? 1.f / L : 0.f;
   int64_t orow;
@@ -200,19 +229,18 @@ __global__ void __launch_bounds__(128) fa_combine_kernel(const FaFwdParams p, in
   float* dst = out + orow * D;
   for (int dd = 0; dd < D; dd += 4) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = c0; c <= c1; ++c) {
-      const float mc = p.part_ml[(static_cast<int64_t>(s + c) * 128 + r) * 2];
-      if (mc == -INFINITY) continue;
-      const float wc = exp2f(mc - M);
-      const float4 v = *reinterpret_cast<const float4*>(p.part_o + (static_cast<int64_t>(s + c) * 128 + r) * D + dd);
-      acc.x += wc * v.x; acc.y += wc * v.y; acc.z += wc * v.z; acc.w += wc * v.w;
+    for (int g = g0; g <= g1; ++g) {
+      const float mg = p.part_ml[slot(g) * 2];
+      if (mg == -INFINITY) continue;
+      const float wg = exp2f(mg - M);
+      const float4 v = *reinterpret_cast<const float4*>(p.part_o + slot(g) * D + dd);
+      acc.x += wg * v.x; acc.y += wg * v.y; acc.z += wg * v.z; acc.w += wg * v.w;
     }
     acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
     *reinterpret_cast<float4*>(dst + dd) = acc;
   }
   if (lse) lse[orow] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
-
 
 struct FaBars {
   uint64_t kfull[kFaMaxRing], kempty[kFaMaxRing], vfull[kFaMaxRing], vempty[kFaMaxRing];
@@ -242,8 +270,9 @@ struct FaWaiter {
 };
 
 // Q tile row (in the Q map) and column base for stream `seg` of user b.
-__device__ __forceinline__ void fa_q_coord(const FaFwdParams& p, const FaPos& t, int D, int& c0, int& row) {
-  const int h = t.seg / t.qt_n, qt = t.seg - h * t.qt_n;
+__device__ __forceinline__ void fa_q_coord(const FaFwdParams& p, const FaPos& t, int qt, int D, int& c0,
+                                           int& row) {
+  const int h = t.h;
   if (p.mode == 0) {
     c0 = 0;
     row = (p.q_per_user ? t.b * p.H * p.k : 0) + h * p.k + qt * 128;
@@ -295,22 +324,26 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   const uint32_t tbase = bars.tmem_base;
   const uint32_t tO = tbase + 256;   // O: 128 lanes x D columns; S buffers at columns 0 and 128
   FaWaiter wait{&bars, &p.hdr->status, p.budget_ns};
+  // group of G CTAs walking one column range; this CTA's query tile
+  const int G = p.group;
+  const int grp = blockIdx.x / G, qt = blockIdx.x % G;
+  const int ngroups = gridDim.x / G;
   const int total = p.hdr->total_tiles;
   const int W = p.hdr->tiles_per_cluster;
-  const int g0 = blockIdx.x * W;
-  const int ntiles = (W > 0 && g0 < total) ? (min(total, g0 + W) - g0) : 0;
+  const int c0 = grp * W, c1 = min(total, c0 + W);
+  const int ntiles = (grp < ngroups && W > 0 && c0 < total && p.hdr->status == 0) ? fa_count(p, qt, c0, c1) : 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && ntiles > 0) {
       FaPos tk, tv;
-      fa_seek(p, g0, tk);
+      fa_seek(p, c0, qt, tk);
       tv = tk;
       int kent = 0, kuse = 0, vent = 0, vuse = 0, nq = 0;
       bool ok = true;
       bool skip_first = (p.debug_flags & 1u) != 0;
       auto kv_coord = [&](const FaPos& t, int& c0, int& row, const CUtensorMap*& mk, const CUtensorMap*& mv) {
-        const int h = t.seg / t.qt_n;
+        const int h = t.h;
         const int nh = fa_hist_tiles(p, t.b);
         if (t.j < nh) {
           c0 = h * D;
@@ -330,7 +363,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
             if (nq > 0) ok = wait(&bars.qfree, (nq - 1) & 1);
             if (!ok) break;
             int qc0, qrow;
-            fa_q_coord(p, tk, D, qc0, qrow);
+            fa_q_coord(p, tk, qt, D, qc0, qrow);
             mbar_expect_tx(&bars.qfull, fa_q_bytes(D));
             for (int kb = 0; kb < KB; ++kb) tma_load_2d(sQ + kb * kFaSlot, &mapQ, &bars.qfull, qc0 + kb * 64, qrow);
             ++nq;
@@ -349,7 +382,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
           }
           kent = (kent + 1 == p.nk_slots) ? 0 : kent + 1;
           ++kuse;
-          fa_next(p, tk);
+          fa_next(p, qt, tk);
         }
         if (i >= 1) {
           ok = wait(&bars.vempty[vent], ((vuse / p.nv_entries) & 1) ^ 1);
@@ -362,7 +395,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
             tma_load_2d(sV + vent * kTileBytes + kb * kFaSlot, mv, &bars.vfull[vent], c0 + kb * 64, row);
           vent = (vent + 1 == p.nv_entries) ? 0 : vent + 1;
           ++vuse;
-          fa_next(p, tv);
+          fa_next(p, qt, tv);
         }
       }
       for (int e = 0; e < p.nk_slots; ++e) {
@@ -381,7 +414,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
       constexpr uint32_t idesc1 = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
       FaPos t1, t2;
-      fa_seek(p, g0, t1);
+      fa_seek(p, c0, qt, t1);
       t2 = t1;
       int kent = 0, kuse = 0, vent = 0, vuse = 0, nq = 0, nseg2 = 0;
       bool ok = true;
@@ -414,7 +447,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
           if (last) umma_commit(&bars.qfree);
           kent = (kent + 1 == p.nk_slots) ? 0 : kent + 1;
           ++kuse;
-          fa_next(p, t1);
+          fa_next(p, qt, t1);
         }
         if (i >= 1) {
           const bool first = (t2.j == 0) || (i == 1);
@@ -443,7 +476,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
           }
           vent = (vent + 1 == p.nv_entries) ? 0 : vent + 1;
           ++vuse;
-          fa_next(p, t2);
+          fa_next(p, qt, t2);
         }
       }
       umma_commit(&bars.drain);
@@ -458,7 +491,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
     const float c2 = p.scale_log2;
     const uint64_t c2x2 = f2_pack(c2, c2);
     FaPos t;
-    if (ntiles > 0) fa_seek(p, g0, t);
+    if (ntiles > 0) fa_seek(p, c0, qt, t);
     float m = -INFINITY, l = 0.f;
     int nseg = 0;
     bool ok = true;
@@ -476,7 +509,6 @@ __global__ void __launch_bounds__(kFaThreads, 1)
         kk0 = t.j * 128;
         vlen = fa_used(p, t.b);
         if (p.mode == 1 && p.kv_len) {
-          const int qt = t.seg % t.qt_n;
           const int q = qt * 128 + r;
           const int nq = p.cu_q[t.b + 1] - p.cu_q[t.b];
           if (q < nq) vlen = min(vlen, max(p.kv_len[p.cu_q[t.b] + q], 0));
@@ -576,7 +608,8 @@ __global__ void __launch_bounds__(kFaThreads, 1)
         ok = __all_sync(0xffffffffu, wait(&bars.ofull, nseg & 1));
         if (!ok) break;
         tc_fence_after();
-        const int slot = p.seg_prefix[t.b] + t.seg + static_cast<int>(blockIdx.x);
+        // slot of (column stream (b, h), group, query tile): unique along the column staircase
+        const int slot = ((t.b * p.H + t.h) + grp) * G + qt;
         float* dst = p.part_o + (static_cast<int64_t>(slot) * 128 + r) * D;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
@@ -595,7 +628,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
         if (lane == 0) mbar_arrive(&bars.ofree);
         ++nseg;
       }
-      fa_next(p, t);
+      fa_next(p, qt, t);
     }
   }
 
@@ -650,14 +683,14 @@ cudaError_t launch_fa_fwd(int D, int num_ctas, size_t smem, const CUtensorMap& m
 }
 
 cudaError_t launch_fa_schedule(const FaFwdParams& p, int num_ctas, cudaStream_t stream) {
-  fa_schedule_kernel<<<1, 1024, 0, stream>>>(p, num_ctas);
+  fa_schedule_kernel<<<1, 1024, 0, stream>>>(p, num_ctas / p.group, p.group);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fa_combine(const FaFwdParams& p, int D, int max_streams, float* out, float* lse,
                               cudaStream_t stream) {
   if (max_streams <= 0) return cudaSuccess;
-  fa_combine_kernel<<<max_streams, 128, 0, stream>>>(p, D, out, lse);
+  fa_combine_kernel<<<max_streams, 128, 0, stream>>>(p, D, p.group, out, lse);
   return cudaGetLastError();
 }
 

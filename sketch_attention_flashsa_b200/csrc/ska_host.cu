@@ -148,18 +148,17 @@ bool plan_forward(const ska_sa_desc* d, ProtoFwdLaunch* L, int* nk, int* nv) {
 
 // ---------------------------------------------------------------- row-softmax engine (token SA, STCA)
 struct FaWs {
-  size_t hdr, tile_prefix, seg_prefix, part_o, part_ml, qb, kb, vb, total;
+  size_t hdr, tile_prefix, part_o, part_ml, qb, kb, vb, total;
 };
 
-void fa_ws_layout(int B, int D, long long max_streams, int num_ctas, size_t cast_q, size_t cast_kv, FaWs* w) {
+// Slots: one per (column stream (b, h) + group, query tile) pair along the column staircase.
+void fa_ws_layout(int B, int H, int D, int G, int ngroups, size_t cast_q, size_t cast_kv, FaWs* w) {
   size_t off = 0;
   w->hdr = off;
   off += sizeof(WsHeader);
   w->tile_prefix = off;
   off = align256(off + size_t(B + 1) * 4);
-  w->seg_prefix = off;
-  off = align256(off + size_t(B + 1) * 4);
-  const size_t slots = size_t(max_streams) + size_t(num_ctas);
+  const size_t slots = (size_t(B) * H + size_t(ngroups)) * size_t(G);
   w->part_o = off;
   off = align256(off + slots * 128 * D * 4);
   w->part_ml = off;
@@ -176,16 +175,25 @@ void fa_ws_layout(int B, int D, long long max_streams, int num_ctas, size_t cast
   w->total = off;
 }
 
-long long sa_token_streams(const ska_sa_desc* d) {
-  return (long long)d->num_users * d->num_heads * ((d->num_protos + 127) / 128);
+// Group size (query tiles walked together) and CTA count of the row-softmax engine.
+bool fa_groups(int G, int sms, int* ctas, int* ngroups) {
+  if (G < 1 || G > sms) return false;
+  *ngroups = sms / G;
+  *ctas = *ngroups * G;
+  return true;
 }
+
+int sa_token_group(const ska_sa_desc* d) { return (d->num_protos + 127) / 128; }
 
 size_t sa_token_ws_size(const ska_sa_desc* d, FaWs* w, int* ctas, size_t* smem, int* nk, int* nv) {
   const int sms = device_sm_count();
-  if (sms <= 0 || !fa_fwd_plan(d->head_dim, sms, ctas, smem, nk, nv)) return 0;
+  int c0, ng;
+  if (sms <= 0 || !fa_fwd_plan(d->head_dim, sms, &c0, smem, nk, nv)) return 0;
+  const int G = sa_token_group(d);
+  if (!fa_groups(G, sms, ctas, &ng)) return 0;
   const size_t qn = size_t(d->q_per_user ? d->num_users : 1) * d->num_heads * d->num_protos * d->head_dim;
   const size_t kvn = size_t(d->total_tokens) * d->num_heads * d->head_dim;
-  fa_ws_layout(d->num_users, d->head_dim, sa_token_streams(d), *ctas, d->in_dtype == SKA_F32 ? qn : 0,
+  fa_ws_layout(d->num_users, d->num_heads, d->head_dim, G, ng, d->in_dtype == SKA_F32 ? qn : 0,
                d->in_dtype == SKA_F32 ? kvn : 0, w);
   return w->total;
 }
@@ -222,7 +230,7 @@ ska_status sa_forward_token(const ska_sa_desc* d, const void* q, const void* k, 
   p.cu_q = nullptr;
   p.kv_len = nullptr;
   p.tile_prefix = reinterpret_cast<int32_t*>(wsb + w.tile_prefix);
-  p.seg_prefix = reinterpret_cast<int32_t*>(wsb + w.seg_prefix);
+  p.group = sa_token_group(d);
   p.hdr = reinterpret_cast<WsHeader*>(wsb + w.hdr);
   p.part_o = reinterpret_cast<float*>(wsb + w.part_o);
   p.part_ml = reinterpret_cast<float*>(wsb + w.part_ml);
@@ -250,7 +258,7 @@ ska_status sa_forward_token(const ska_sa_desc* d, const void* q, const void* k, 
     }
     if (e != cudaSuccess) return SKA_ERR_CUDA;
   }
-  if (launch_fa_combine(p, D, int(sa_token_streams(d)), sketch, lse, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (launch_fa_combine(p, D, B * H * p.group, sketch, lse, s) != cudaSuccess) return SKA_ERR_CUDA;
   return SKA_OK;
 }
 
@@ -266,17 +274,21 @@ ska_status check_stca_desc(const ska_stca_desc* d) {
   return SKA_OK;
 }
 
-long long stca_max_streams(const ska_stca_desc* d) {
-  return (long long)d->num_heads * ((d->total_targets + 127) / 128 + d->num_users);
+// Query tiles walked together: from max_targets when given (an upper bound on any user's target
+// count), else from total_targets (always an upper bound, at the cost of idle CTAs).
+int stca_group(const ska_stca_desc* d) {
+  const int64_t mt = d->max_targets > 0 ? d->max_targets : d->total_targets;
+  return int((mt + 127) / 128);
 }
 
 size_t stca_ws_size(const ska_stca_desc* d, FaWs* w, int* ctas, size_t* smem, int* nk, int* nv) {
   const int sms = device_sm_count();
-  if (sms <= 0 || !fa_fwd_plan(d->head_dim, sms, ctas, smem, nk, nv)) return 0;
-  fa_ws_layout(d->num_users, d->head_dim, stca_max_streams(d), *ctas, 0, 0, w);
+  int c0, ng;
+  if (sms <= 0 || !fa_fwd_plan(d->head_dim, sms, &c0, smem, nk, nv)) return 0;
+  if (!fa_groups(stca_group(d), sms, ctas, &ng)) return 0;
+  fa_ws_layout(d->num_users, d->num_heads, d->head_dim, stca_group(d), ng, 0, 0, w);
   return w->total;
 }
-
 }  // namespace
 
 extern "C" {
@@ -496,7 +508,7 @@ ska_status stca_forward(const ska_stca_desc* d, const void* q, const int32_t* cu
   p.cu_q = cu_targets;
   p.kv_len = target_kv_len;
   p.tile_prefix = reinterpret_cast<int32_t*>(wsb + w.tile_prefix);
-  p.seg_prefix = reinterpret_cast<int32_t*>(wsb + w.seg_prefix);
+  p.group = stca_group(d);
   p.hdr = reinterpret_cast<WsHeader*>(wsb + w.hdr);
   p.part_o = reinterpret_cast<float*>(wsb + w.part_o);
   p.part_ml = reinterpret_cast<float*>(wsb + w.part_ml);
@@ -535,7 +547,7 @@ ska_status stca_forward(const ska_stca_desc* d, const void* q, const int32_t* cu
     e = launch_fa_fwd(D, ctas, smem, mQ, mK, mV, mKs, mVs, p, s);
   }
   if (e != cudaSuccess) return SKA_ERR_CUDA;
-  if (launch_fa_combine(p, D, int(stca_max_streams(d)), out, lse, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (launch_fa_combine(p, D, B * H * p.group, out, lse, s) != cudaSuccess) return SKA_ERR_CUDA;
   return SKA_OK;
 }
 

@@ -64,11 +64,11 @@ struct FaFwdParams {
   const int32_t* seqused;      // SA only, nullable
   const int32_t* cu_q;         // STCA: cu_targets; SA: null
   const int32_t* kv_len;       // STCA: per-target suffix length, nullable
-  const int32_t* tile_prefix;  // [B+1] key tiles of all streams of users < b
-  const int32_t* seg_prefix;   // [B+1] streams of users < b
+  const int32_t* tile_prefix;  // [B+1] key-tile columns (H per user) of users < b
+  int group;                   // CTAs per group = query tiles walked together
   WsHeader* hdr;
-  float* part_o;               // [(max_streams + clusters) * 128 * D] unnormalised O
-  float* part_ml;              // [(max_streams + clusters) * 128 * 2] (max in log2 units, sum)
+  float* part_o;               // [(B*H + groups) * group * 128 * D] unnormalised O
+  float* part_ml;              // [(B*H + groups) * group * 128 * 2] (max in log2 units, sum)
   int B, H;
   int k;                       // SA: prototypes
   int ks;                      // STCA: sketch rows per (user, head)
@@ -87,8 +87,8 @@ cudaError_t launch_fa_fwd(int head_dim, int num_ctas, size_t smem_bytes, const C
 
 cudaError_t launch_fa_schedule(const FaFwdParams& p, int num_ctas, cudaStream_t stream);
 
-// LSE merge of the partials into the outputs. SA: out = sketch [B,H,k,D], lse [B,H,k].
-// STCA: out [total_targets, H, D], lse [total_targets, H].
+// LSE merge of the partials into the outputs (max_streams = B * H * group blocks).
+// SA: out = sketch [B,H,k,D], lse [B,H,k]. STCA: out [total_targets, H, D], lse [total_targets, H].
 cudaError_t launch_fa_combine(const FaFwdParams& p, int head_dim, int max_streams, float* out, float* lse,
                               cudaStream_t stream);
 
