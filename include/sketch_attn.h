@@ -119,14 +119,20 @@ ska_status sa_forward(const ska_sa_desc* desc, const void* q, const void* k, con
 size_t sa_backward_workspace_size(const ska_sa_desc* desc);
 
 /* SA backward: gradients of <dsketch, sketch> through Eq. (7)-(9) (SA is trained end to end,
- * App. A.4). Inputs as in sa_forward plus the forward's lse; bf16 inputs only.
+ * App. A.4). Inputs as in sa_forward (bf16 only), plus:
+ *   sketch   fp32 [B, H, k, d], the forward output; read in TOKEN mode (D_j = dO_j . O_j), may
+ *            be NULL in PROTO mode
+ *   lse      fp32, the forward's lse (PROTO [total_tokens, H]; TOKEN [B, H, k])
  *   dsketch  bf16 [B, H, k, d]
  *   dq       out, fp32, q's shape: [H,k,d] summed over all users when the prototypes are shared,
  *            else [B,H,k,d]
- *   dk, dv   out, fp32 [total_tokens, H, d]; zero rows on padding tokens                      */
+ *   dk, dv   out, fp32 [total_tokens, H, d]; zero rows on padding tokens
+ * Supported: num_protos in {16, 32, 64, 128, 256} for head_dim 64, up to 128 for head_dim 128
+ * (SKA_ERR_UNSUPPORTED otherwise). dQ is formed from a two-term bf16 split of dS (16
+ * significant bits) and reduced over users in a fixed order.                                  */
 ska_status sa_backward(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
-                       const int32_t* cu_seqlens, const int32_t* seqused, const float* lse,
-                       const void* dsketch, float* dq, float* dk, float* dv, void* ws,
+                       const int32_t* cu_seqlens, const int32_t* seqused, const float* sketch,
+                       const float* lse, const void* dsketch, float* dq, float* dk, float* dv, void* ws,
                        size_t ws_bytes, void* stream);
 
 /* One batched STCA problem (§2.3, §3.4, MRLB §4.2): num_users users, each with a block of

@@ -66,7 +66,7 @@ def lib() -> ctypes.CDLL:
     L.sa_forward.restype = ctypes.c_int
     L.sa_backward_workspace_size.argtypes = [ctypes.POINTER(SaDesc)]
     L.sa_backward_workspace_size.restype = sz
-    L.sa_backward.argtypes = [ctypes.POINTER(SaDesc), vp, vp, vp, i32p, i32p, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.sa_backward.argtypes = [ctypes.POINTER(SaDesc), vp, vp, vp, i32p, i32p, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.sa_backward.restype = ctypes.c_int
     L.stca_forward_workspace_size.argtypes = [ctypes.POINTER(StcaDesc)]
     L.stca_forward_workspace_size.restype = sz

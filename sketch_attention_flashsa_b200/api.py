@@ -162,3 +162,35 @@ def stca_forward(q: torch.Tensor, cu_targets: torch.Tensor, k_hist: torch.Tensor
                                  _ptr(lse), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check(rc, "stca_forward")
     return out, lse
+
+
+def sa_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                seqused: Optional[torch.Tensor], lse: torch.Tensor, dsketch: torch.Tensor,
+                sketch: Optional[torch.Tensor] = None, *, scale: float = 1.0, norm="proto",
+                workspace: Optional[torch.Tensor] = None, stream=None):
+    """SA backward (gradients of <dsketch, sketch> through SequenceO1 §3.1 Eq. (7)-(9)).
+
+    bf16 q, k, v, dsketch; the forward's lse (and, for norm="token", its sketch).
+    Returns (dq fp32 shaped like q, dk fp32 [T,H,d], dv fp32 [T,H,d]).
+    """
+    for name, t in (("q", q), ("k", k), ("v", v), ("dsketch", dsketch)):
+        _dev_tensor(name, t, (torch.bfloat16,))
+    _dev_tensor("lse", lse, (torch.float32,))
+    _dev_tensor("sketch", sketch, (torch.float32,))
+    _dev_tensor("cu_seqlens", cu_seqlens, (torch.int32,))
+    _dev_tensor("seqused", seqused, (torch.int32,))
+    desc = sa_desc(q, k, cu_seqlens, scale=scale, norm=norm)
+    dev = k.device
+    need = int(_lib.lib().sa_backward_workspace_size(ctypes.byref(desc)))
+    if need == 0:
+        raise SkaError(_lib.SKA_ERR_UNSUPPORTED, "sa_backward_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    rc = _lib.lib().sa_backward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(seqused),
+                                _ptr(sketch), _ptr(lse), _ptr(dsketch), _ptr(dq), _ptr(dk), _ptr(dv),
+                                _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check(rc, "sa_backward")
+    return dq, dk, dv

@@ -1,0 +1,525 @@
+// SA backward on sm_100a: gradients of <dSketch, sketch> through SequenceO1 §3.1 Eq. (7)-(9)
+// (SA is trained end to end, App. A.4), for both normalisations.
+//
+// Per 128-token tile of one (user, head), one CTA holding all k <= 256 prototypes, tokens on
+// TMEM lanes (S^T orientation):
+//   MMA  S^T  = K . Q^T                        -> A = exp(scale s - lse) (PROTO: per-token lse;
+//                                                 TOKEN: per-prototype lse), A as bf16 to smem
+//   MMA  dV   = A^T . dO        (M=tok, N=d)   -> TMEM
+//   MMA  dA^T = V . dO^T        (M=tok, N=k)   -> TMEM (over S^T)
+//   softmax-gradient: PROTO dS = A (dA - delta_i) with delta_i = dV_i . v_i (equal to
+//        sum_j A_ji dA_ji, so no reduction over prototypes is needed); TOKEN dS = A (dA - D_j)
+//        with D_j = dO_j . O_j from the forward sketch. dS goes to smem as a bf16 pair
+//        hi + lo (hi = bf16(dS), lo = bf16(dS - hi)), 16 significant bits.
+//   MMA  dK   = dS^T . Q        (M=tok, N=d)   -> TMEM, scaled by `scale` on the way out
+//   MMA  dQ  += dS . K          (M=proto, N=d) -> TMEM, accumulated over the CTA's tiles of one
+//        segment with both halves of the pair; written to a partial slot at segment end.
+// Warps 0-7 (two warpgroups, each owning half of the prototype columns) do the elementwise
+// work; warp 8 issues TMA loads and MMAs. The phases of a tile run one after another.
+#include <algorithm>
+#include <cmath>
+
+#include "ska_internal.h"
+#include "ska_ptx.cuh"
+
+namespace ska {
+
+namespace {
+
+constexpr int kBwdWorkers = 256;
+constexpr int kBwdThreads = 288;
+constexpr int kBwdWarps = 8;
+constexpr int kBlk = 16384;  // [128 rows x 64 bf16] swizzled block
+
+struct BwdLayout {
+  uint32_t q_off, do_off, k_off, v_off, a_off, lo_off, lse_off, d_off, total;
+};
+
+// Q, dO: ceil(d/64) blocks of k rows x 128 B (k padded to a multiple of 8);
+// K, V: d/64 blocks of 128 rows; A / dS_hi and dS_lo: ceil(k/64) blocks of 128 rows.
+__host__ __device__ inline BwdLayout bwd_layout(int D, int k) {
+  BwdLayout L;
+  const uint32_t kb = D / 64, pb = (k + 63) / 64;
+  const uint32_t qbytes = kb * ((k * 128 + 1023) & ~1023u);
+  uint32_t off = 0;
+  L.q_off = off;
+  off += qbytes;
+  L.do_off = off;
+  off += qbytes;
+  L.k_off = off;
+  off += kb * kBlk;
+  L.v_off = off;
+  off += kb * kBlk;
+  L.a_off = off;
+  off += max(pb, 2u) * kBlk;  // MMA for dQ reads a full 128-prototype block
+  L.lo_off = off;
+  off += max(pb, 2u) * kBlk;
+  L.lse_off = off;
+  off += 256 * 4;
+  L.d_off = off;
+  off += 256 * 4;
+  L.total = off;
+  return L;
+}
+
+__host__ __device__ inline int bwd_tmem_cols(int D, int k) { return k + 2 * D + ((k + 127) / 128) * D; }
+
+struct BwdBars {
+  uint64_t ld, qd, m1, a, m2, ds, m3, out, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct BwdPos {
+  int b, h, j, nb;
+};
+
+__device__ __forceinline__ int bwd_used(const SaBwdParams& p, int b) {
+  int len = p.cu_seqlens[b + 1] - p.cu_seqlens[b];
+  if (p.seqused) len = min(len, p.seqused[b]);
+  return max(len, 0);
+}
+
+__device__ __forceinline__ void bwd_seek(const SaBwdParams& p, int g, BwdPos& t) {
+  int lo = 0, hi = p.B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.H * p.tile_prefix[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  t.b = lo;
+  t.nb = p.tile_prefix[lo + 1] - p.tile_prefix[lo];
+  const int off = g - p.H * p.tile_prefix[lo];
+  t.h = off / t.nb;
+  t.j = off - t.h * t.nb;
+}
+
+__device__ __forceinline__ void bwd_next(const SaBwdParams& p, BwdPos& t) {
+  if (++t.j < t.nb) return;
+  t.j = 0;
+  if (++t.h < p.H) return;
+  t.h = 0;
+  do {
+    ++t.b;
+    if (t.b >= p.B) return;
+    t.nb = p.tile_prefix[t.b + 1] - p.tile_prefix[t.b];
+  } while (t.nb == 0);
+}
+
+struct BwdWaiter {
+  BwdBars* bars;
+  int* status;
+  uint64_t budget;
+  __device__ __forceinline__ bool operator()(uint64_t* bar, uint32_t parity, bool drain = false) {
+    volatile int* ab = &bars->abort_flag;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (!drain && *ab) return false;
+      if (globaltimer_ns() - t0 > budget) {
+        atomicCAS(status, 0, (int)SKA_ERR_DEVICE_TIMEOUT);
+        *ab = 1;
+        return false;
+      }
+    }
+  }
+};
+
+
+template <int D, int KP>
+__global__ void __maxnreg__(224)
+    sa_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapDO,
+                  const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                  const SaBwdParams p) {
+  constexpr int KB = D / 64;
+  constexpr int PB = (KP + 63) / 64;
+  constexpr int NCOL = KP / 2;                  // prototype columns per worker thread
+  constexpr int QBLK = (KP * 128 + 1023) & ~1023;
+  constexpr int CV = (KP + 31) / 32 * 32;      // TMEM columns: S^T/dA^T at 0, dV, dK, dQ blocks
+  constexpr int CK = CV + D;
+  constexpr int CQ = CK + D;
+  constexpr int QBLOCKS = (KP + 127) / 128;
+  static_assert(CQ + QBLOCKS * D <= 512, "TMEM");
+  static_assert(NCOL % 8 == 0, "columns");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ BwdBars bars;
+  __shared__ uint64_t dready;
+  const BwdLayout L = bwd_layout(D, KP);
+  uint8_t* sQ = smem + L.q_off;
+  uint8_t* sDO = smem + L.do_off;
+  uint8_t* sK = smem + L.k_off;
+  uint8_t* sV = smem + L.v_off;
+  uint8_t* sA = smem + L.a_off;    // A, then dS hi
+  uint8_t* sLo = smem + L.lo_off;  // dS lo
+  float* sLse = reinterpret_cast<float*>(smem + L.lse_off);
+  float* sDj = reinterpret_cast<float*>(smem + L.d_off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.ld, 1);
+    mbar_init(&bars.qd, 1);
+    mbar_init(&bars.m1, 1);
+    mbar_init(&bars.m2, 1);
+    mbar_init(&bars.m3, 1);
+    mbar_init(&bars.a, kBwdWarps);
+    mbar_init(&bars.ds, kBwdWarps);
+    mbar_init(&bars.out, kBwdWarps);
+    mbar_init(&dready, kBwdWarps);
+    mbar_init(&bars.drain, 1);
+    bars.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(&bars.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = bars.tmem_base;
+  BwdWaiter wait{&bars, &p.hdr->status, p.budget_ns};
+  const int total = p.hdr->total_tiles;
+  const int W = p.hdr->tiles_per_cluster;
+  const int g0 = blockIdx.x * W;
+  const int ntiles = (W > 0 && g0 < total) ? (min(total, g0 + W) - g0) : 0;
+
+  if (warp == 8) {
+    // ---------------------------------------------------------------- control: TMA + MMA
+    if (lane == 0 && ntiles > 0) {
+      constexpr uint32_t i1 = idesc_bf16_f32(128, KP, false, false);
+      constexpr uint32_t iV = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t iQ = idesc_bf16_f32(128, D, true, true);
+      BwdPos t;
+      bwd_seek(p, g0, t);
+      int nseg = 0;
+      bool ok = true;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const bool first = (t.j == 0) || (i == 0);
+        if (first) {
+          const int qrow = (p.q_per_user ? t.b * p.H * p.k : 0) + t.h * p.k;
+          const int orow = (t.b * p.H + t.h) * p.k;
+          mbar_expect_tx(&bars.qd, 2 * KB * KP * 128);
+          for (int kb = 0; kb < KB; ++kb) {
+            tma_load_2d(sQ + kb * QBLK, &mapQ, &bars.qd, kb * 64, qrow);
+            tma_load_2d(sDO + kb * QBLK, &mapDO, &bars.qd, kb * 64, orow);
+          }
+        }
+        const int tok0 = p.cu_seqlens[t.b] + t.j * 128;
+        mbar_expect_tx(&bars.ld, 2 * KB * kBlk);
+        for (int kb = 0; kb < KB; ++kb) {
+          tma_load_2d(sK + kb * kBlk, &mapK, &bars.ld, t.h * D + kb * 64, tok0);
+          tma_load_2d(sV + kb * kBlk, &mapV, &bars.ld, t.h * D + kb * 64, tok0);
+        }
+        ok = wait(&bars.ld, i & 1);
+        if (ok && first) ok = wait(&bars.qd, nseg & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // S^T = K . Q^T
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s)
+          umma_bf16(tb, sw128_desc(smem_u32(sK) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                    sw128_desc(smem_u32(sQ) + (s / 4) * QBLK + (s % 4) * 32, 16, 1024), i1, s > 0);
+        umma_commit(&bars.m1);
+        ok = wait(&bars.a, i & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // dV = A^T . dO ; dA^T = V . dO^T (over S^T)
+#pragma unroll
+        for (int s = 0; s < KP / 16; ++s)
+          umma_bf16(tb + CV, sw128_desc(smem_u32(sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                    sw128_desc(smem_u32(sDO) + s * 2048, QBLK, 1024), iV, s > 0);
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s)
+          umma_bf16(tb, sw128_desc(smem_u32(sV) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                    sw128_desc(smem_u32(sDO) + (s / 4) * QBLK + (s % 4) * 32, 16, 1024), i1, s > 0);
+        umma_commit(&bars.m2);
+        ok = wait(&bars.ds, i & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // dK = dS^T . Q ; dQ += dS . K (hi and lo halves of dS)
+#pragma unroll
+        for (int s = 0; s < KP / 16; ++s)
+          umma_bf16(tb + CK, sw128_desc(smem_u32(sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                    sw128_desc(smem_u32(sQ) + s * 2048, QBLK, 1024), iV, s > 0);
+#pragma unroll
+        for (int g = 0; g < QBLOCKS; ++g)
+#pragma unroll
+          for (int half = 0; half < 2; ++half)
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+              const uint32_t abase = smem_u32(half == 0 ? sA : sLo) + 2 * g * kBlk;
+              umma_bf16(tb + CQ + g * D, sw128_desc(abase + s * 2048, kBlk, 1024),
+                        sw128_desc(smem_u32(sK) + s * 2048, kBlk, 1024), iQ,
+                        (first && half == 0 && s == 0) ? 0u : 1u);
+            }
+        umma_commit(&bars.m3);
+        ok = wait(&bars.out, i & 1);
+        if (!ok) break;
+        if (first) ++nseg;
+        bwd_next(p, t);
+      }
+      umma_commit(&bars.drain);  // completes when every MMA issued above has
+      wait(&bars.drain, 0, true);
+    }
+  } else {
+    // ---------------------------------------------------------------- workers
+    const int wg = warp >> 2, q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const int col0 = wg * NCOL;
+    const uint32_t loff = static_cast<uint32_t>(q4 * 32) << 16;
+    const float L2E = 1.4426950408889634f;
+    const float c2 = p.scale * L2E;
+    BwdPos t;
+    if (ntiles > 0) bwd_seek(p, g0, t);
+    int nseg = 0;
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const bool first = (t.j == 0) || (i == 0);
+      const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
+      const int used = bwd_used(p, t.b);
+      const int tok = p.cu_seqlens[t.b] + t.j * 128 + r;
+      const bool valid = (t.j * 128 + r) < used;
+      if (first && p.norm == SKA_NORM_TOKEN) {
+        // per-prototype lse (log2 units) and D_j = dO_j . O_j of this (user, head)
+        const int jj = threadIdx.x;
+        if (jj < p.k) {
+          const int64_t row = (static_cast<int64_t>(t.b) * p.H + t.h) * p.k + jj;
+          sLse[jj] = p.lse[row] * L2E;
+          float acc = 0.f;
+          for (int dd = 0; dd < D; ++dd)
+            acc += __bfloat162float(p.dsketch[row * D + dd]) * p.sketch[row * D + dd];
+          sDj[jj] = acc;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dready);
+        ok = __all_sync(0xffffffffu, wait(&dready, nseg & 1));
+        if (!ok) break;
+      }
+      ok = __all_sync(0xffffffffu, wait(&bars.m1, i & 1));
+      if (!ok) break;
+      tc_fence_after();
+      // A = exp(scale s - lse): PROTO per token row, TOKEN per prototype column
+      float a[NCOL];
+      {
+        uint32_t sv[NCOL];
+#pragma unroll
+        for (int c = 0; c < NCOL; c += 8) tmem_ld8(tb + loff + col0 + c, sv + c);
+        tmem_ld_wait();
+        const float lrow = (p.norm == SKA_NORM_PROTO && valid) ? p.lse[static_cast<int64_t>(tok) * p.H + t.h] * L2E : 0.f;
+#pragma unroll
+        for (int c = 0; c < NCOL; ++c) {
+          const float l2 = (p.norm == SKA_NORM_PROTO) ? lrow : sLse[col0 + c];
+          a[c] = valid ? ex2_approx(__uint_as_float(sv[c]) * c2 - l2) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < NCOL; c += 8) {
+        uint4 w;
+        w.x = pack_bf16x2(a[c + 0], a[c + 1]);
+        w.y = pack_bf16x2(a[c + 2], a[c + 3]);
+        w.z = pack_bf16x2(a[c + 4], a[c + 5]);
+        w.w = pack_bf16x2(a[c + 6], a[c + 7]);
+        const int jj = col0 + c;
+        *reinterpret_cast<uint4*>(sA + (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2)) = w;
+      }
+      fence_async_shared();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.a);
+      ok = __all_sync(0xffffffffu, wait(&bars.m2, i & 1));
+      if (!ok) break;
+      tc_fence_after();
+      // PROTO: delta_i = dV_i . v_i
+      float delta = 0.f;
+      if (p.norm == SKA_NORM_PROTO) {
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t dvr[32];
+          tmem_ld32(tb + loff + CV + c, dvr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; u += 8) {
+            const int dd = c + u;
+            const uint4 w = *reinterpret_cast<const uint4*>(sV + (dd >> 6) * kBlk + sw128_offset(r, (dd & 63) * 2));
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              delta = fmaf(__uint_as_float(dvr[u + 2 * e]), __uint_as_float(ww[e] << 16), delta);
+              delta = fmaf(__uint_as_float(dvr[u + 2 * e + 1]), __uint_as_float(ww[e] & 0xFFFF0000u), delta);
+            }
+          }
+        }
+      }
+      // dS = A (dA - delta) as a bf16 pair hi + lo
+#pragma unroll
+      for (int c = 0; c < NCOL; c += 8) {
+        uint32_t da[8];
+        tmem_ld8(tb + loff + col0 + c, da);
+        tmem_ld_wait();
+        float hi[8], lo[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float sub = (p.norm == SKA_NORM_PROTO) ? delta : sDj[col0 + c + u];
+          const float ds = a[c + u] * (__uint_as_float(da[u]) - sub);
+          hi[u] = __bfloat162float(__float2bfloat16_rn(ds));
+          lo[u] = ds - hi[u];
+        }
+        const int jj = col0 + c;
+        uint4 wh, wl;
+        wh.x = pack_bf16x2(hi[0], hi[1]); wh.y = pack_bf16x2(hi[2], hi[3]);
+        wh.z = pack_bf16x2(hi[4], hi[5]); wh.w = pack_bf16x2(hi[6], hi[7]);
+        wl.x = pack_bf16x2(lo[0], lo[1]); wl.y = pack_bf16x2(lo[2], lo[3]);
+        wl.z = pack_bf16x2(lo[4], lo[5]); wl.w = pack_bf16x2(lo[6], lo[7]);
+        const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
+        *reinterpret_cast<uint4*>(sA + off) = wh;
+        *reinterpret_cast<uint4*>(sLo + off) = wl;
+      }
+      fence_async_shared();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.ds);
+      ok = __all_sync(0xffffffffu, wait(&bars.m3, i & 1));
+      if (!ok) break;
+      tc_fence_after();
+      // dK (scaled) and dV rows: warpgroup wg writes channels [wg D/2, (wg+1) D/2)
+#pragma unroll
+      for (int c = 0; c < D / 2; c += 32) {
+        const int cc = wg * (D / 2) + c;
+        uint32_t kr[32], vr[32];
+        tmem_ld32(tb + loff + CK + cc, kr);
+        tmem_ld32(tb + loff + CV + cc, vr);
+        tmem_ld_wait();
+        if (tok < p.total_tokens && (t.j * 128 + r) < (p.cu_seqlens[t.b + 1] - p.cu_seqlens[t.b])) {
+          float* dk = p.dk + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
+          float* dv = p.dv + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) {
+            *reinterpret_cast<float4*>(dk + u) =
+                make_float4(p.scale * __uint_as_float(kr[u]), p.scale * __uint_as_float(kr[u + 1]),
+                            p.scale * __uint_as_float(kr[u + 2]), p.scale * __uint_as_float(kr[u + 3]));
+            *reinterpret_cast<float4*>(dv + u) = make_float4(__uint_as_float(vr[u]), __uint_as_float(vr[u + 1]),
+                                                             __uint_as_float(vr[u + 2]), __uint_as_float(vr[u + 3]));
+          }
+        }
+      }
+      if (last && wg < QBLOCKS) {
+        // dQ block wg (prototypes 128 wg + r) of this segment -> partial slot (scaled)
+        const int jrow = wg * 128 + r;
+        const int slot = (t.b * p.H + t.h) + static_cast<int>(blockIdx.x);
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t qr[32];
+          tmem_ld32(tb + loff + CQ + wg * D + c, qr);
+          tmem_ld_wait();
+          if (jrow < p.k) {
+            float* dst = p.dq_partial + (static_cast<int64_t>(slot) * p.k + jrow) * D + c;
+#pragma unroll
+            for (int u = 0; u < 32; u += 4)
+              *reinterpret_cast<float4*>(dst + u) =
+                  make_float4(p.scale * __uint_as_float(qr[u]), p.scale * __uint_as_float(qr[u + 1]),
+                              p.scale * __uint_as_float(qr[u + 2]), p.scale * __uint_as_float(qr[u + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.out);
+      if (first) ++nseg;
+      bwd_next(p, t);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tb, 512);
+  }
+}
+
+// dq[(b?) h] = sum over the segments it collects of their partial slots, fixed order.
+__global__ void sa_bwd_dq_reduce(const SaBwdParams p, int D, float* __restrict__ dq) {
+  const int64_t per = static_cast<int64_t>(p.k) * D;
+  const int qsets = p.q_per_user ? p.B * p.H : p.H;
+  const int64_t n = static_cast<int64_t>(qsets) * per;
+  const int W = p.hdr->tiles_per_cluster;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int qs = static_cast<int>(e / per);
+    const int64_t within = e - static_cast<int64_t>(qs) * per;
+    const int b0 = p.q_per_user ? qs / p.H : 0, b1 = p.q_per_user ? b0 + 1 : p.B;
+    const int h = p.q_per_user ? qs % p.H : qs;
+    float acc = 0.f;
+    for (int b = b0; b < b1; ++b) {
+      const int nb = p.tile_prefix[b + 1] - p.tile_prefix[b];
+      if (nb == 0 || W == 0) continue;
+      const int t0 = p.H * p.tile_prefix[b] + h * nb;
+      const int s = b * p.H + h;
+      for (int c = t0 / W; c <= (t0 + nb - 1) / W; ++c) acc += p.dq_partial[static_cast<int64_t>(s + c) * per + within];
+    }
+    dq[e] = acc;
+  }
+}
+
+// dK, dV rows of padding tokens (positions >= seqused inside a user) are zero.
+__global__ void sa_bwd_zero_padding(const SaBwdParams p, int D) {
+  const int b = blockIdx.x;
+  const int64_t lo = p.cu_seqlens[b] + bwd_used(p, b);
+  const int64_t hi = (static_cast<int64_t>(p.cu_seqlens[b + 1]) < p.total_tokens) ? p.cu_seqlens[b + 1] : p.total_tokens;
+  // rows inside the last partial tile are written by the main kernel; zero from the next tile on
+  const int64_t first_untouched = p.cu_seqlens[b] + ((bwd_used(p, b) + 127) / 128) * 128;
+  const int64_t z0 = (lo > first_untouched) ? lo : first_untouched;
+  for (int64_t i = z0 * p.H * D + threadIdx.x; i < hi * p.H * D; i += blockDim.x) {
+    p.dk[i] = 0.f;
+    p.dv[i] = 0.f;
+  }
+}
+
+template <int D, int KP>
+cudaError_t bwd_launch_t(int num_ctas, const CUtensorMap& mQ, const CUtensorMap& mDO, const CUtensorMap& mK,
+                         const CUtensorMap& mV, const SaBwdParams& p, cudaStream_t stream) {
+  auto kern = sa_bwd_kernel<D, KP>;
+  const size_t smem = bwd_layout(D, KP).total + 1024;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<num_ctas, kBwdThreads, smem, stream>>>(mQ, mDO, mK, mV, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool sa_bwd_supported(int D, int k) {
+  if (D != 64 && D != 128) return false;
+  if (!(k == 16 || k == 32 || k == 64 || k == 128 || k == 256)) return false;
+  if (bwd_tmem_cols(D, k) + ((k + 31) / 32 * 32 - k) > 512) return false;
+  return bwd_layout(D, k).total + 1024 <= 227 * 1024 - 512;
+}
+
+size_t sa_bwd_smem_bytes(int D, int k) { return bwd_layout(D, k).total + 1024; }
+
+cudaError_t launch_sa_bwd(int D, int num_ctas, const CUtensorMap& mQ, const CUtensorMap& mDO,
+                          const CUtensorMap& mK, const CUtensorMap& mV, const SaBwdParams& p,
+                          cudaStream_t stream) {
+#define SKA_BWD_CASE(DD, KK) \
+  if (D == DD && p.k == KK) return bwd_launch_t<DD, KK>(num_ctas, mQ, mDO, mK, mV, p, stream);
+  SKA_BWD_CASE(64, 16)
+  SKA_BWD_CASE(64, 32)
+  SKA_BWD_CASE(64, 64)
+  SKA_BWD_CASE(64, 128)
+  SKA_BWD_CASE(64, 256)
+  SKA_BWD_CASE(128, 16)
+  SKA_BWD_CASE(128, 32)
+  SKA_BWD_CASE(128, 64)
+  SKA_BWD_CASE(128, 128)
+#undef SKA_BWD_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_sa_bwd_finish(const SaBwdParams& p, int D, float* dq, cudaStream_t stream) {
+  sa_bwd_dq_reduce<<<592, 256, 0, stream>>>(p, D, dq);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (p.B > 0) sa_bwd_zero_padding<<<p.B, 256, 0, stream>>>(p, D);
+  return cudaGetLastError();
+}
+
+}  // namespace ska

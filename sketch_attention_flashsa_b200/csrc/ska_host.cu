@@ -447,15 +447,94 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
 }
 
 size_t sa_backward_workspace_size(const ska_sa_desc* d) {
-  (void)d;
-  return 0;
+  if (check_sa_desc(d) != SKA_OK) return 0;
+  if (d->in_dtype != SKA_BF16 || !sa_bwd_supported(d->head_dim, d->num_protos)) return 0;
+  const int sms = device_sm_count();
+  if (sms <= 0) return 0;
+  size_t off = sizeof(WsHeader);
+  off = align256(off + size_t(d->num_users + 1) * 4);
+  off = align256(off + (size_t(d->num_users) * d->num_heads + sms) * d->num_protos * d->head_dim * 4);
+  return off;
 }
 
-ska_status sa_backward(const ska_sa_desc* d, const void*, const void*, const void*, const int32_t*, const int32_t*,
-                       const float*, const void*, float*, float*, float*, void*, size_t, void*) {
+ska_status sa_backward(const ska_sa_desc* d, const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                       const int32_t* seqused, const float* sketch, const float* lse, const void* dsketch, float* dq,
+                       float* dk, float* dv, void* ws, size_t ws_bytes, void* stream) {
   ska_status st = check_sa_desc(d);
   if (st != SKA_OK) return st;
-  return SKA_ERR_UNSUPPORTED;
+  if (d->in_dtype != SKA_BF16 || !sa_bwd_supported(d->head_dim, d->num_protos)) return SKA_ERR_UNSUPPORTED;
+  const int B = d->num_users, H = d->num_heads, D = d->head_dim, kp = d->num_protos;
+  const int64_t T = d->total_tokens;
+  if (!q || !dq || !cu_seqlens || !ws || !lse) return SKA_ERR_INVALID_VALUE;
+  if (B > 0 && !dsketch) return SKA_ERR_INVALID_VALUE;
+  if (T > 0 && (!k || !v || !dk || !dv)) return SKA_ERR_INVALID_VALUE;
+  if (d->norm == SKA_NORM_TOKEN && B > 0 && !sketch) return SKA_ERR_INVALID_VALUE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(sketch) || !aligned16(lse) ||
+      !aligned16(dsketch) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seqused) & 3u))
+    return SKA_ERR_INVALID_VALUE;
+  const size_t need = sa_backward_workspace_size(d);
+  if (need == 0) return SKA_ERR_UNSUPPORTED;
+  if (ws_bytes < need) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  const size_t qn = size_t(d->q_per_user ? B : 1) * H * kp * D, kvn = size_t(T) * H * D;
+  const size_t outs[3][2] = {{reinterpret_cast<uintptr_t>(dq), qn * 4}, {reinterpret_cast<uintptr_t>(dk), kvn * 4},
+                             {reinterpret_cast<uintptr_t>(dv), kvn * 4}};
+  const void* ins[7] = {q, k, v, sketch, lse, dsketch, ws};
+  const size_t insz[7] = {qn * 2, kvn * 2, kvn * 2, size_t(B) * H * kp * D * 4,
+                          (d->norm == SKA_NORM_PROTO ? size_t(T) : size_t(B) * kp) * H * 4,
+                          size_t(B) * H * kp * D * 2, need};
+  for (int o = 0; o < 3; ++o) {
+    for (int i = 0; i < 7; ++i)
+      if (overlaps(reinterpret_cast<void*>(outs[o][0]), outs[o][1], ins[i], insz[i])) return SKA_ERR_INVALID_VALUE;
+    for (int o2 = o + 1; o2 < 3; ++o2)
+      if (overlaps(reinterpret_cast<void*>(outs[o][0]), outs[o][1], reinterpret_cast<void*>(outs[o2][0]),
+                   outs[o2][1]))
+        return SKA_ERR_INVALID_VALUE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (B == 0) return SKA_OK;
+  const int sms = device_sm_count();
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
+  int32_t* prefix = reinterpret_cast<int32_t*>(wsb + sizeof(WsHeader));
+  float* dqp = reinterpret_cast<float*>(wsb + align256(sizeof(WsHeader) + size_t(B + 1) * 4));
+  if (launch_schedule(cu_seqlens, seqused, B, H, sms, prefix, hdr, s) != cudaSuccess) return SKA_ERR_CUDA;
+  SaBwdParams p{};
+  p.norm = d->norm;
+  p.cu_seqlens = cu_seqlens;
+  p.seqused = seqused;
+  p.tile_prefix = prefix;
+  p.hdr = hdr;
+  p.lse = lse;
+  p.sketch = sketch;
+  p.dsketch = static_cast<const __nv_bfloat16*>(dsketch);
+  p.dk = dk;
+  p.dv = dv;
+  p.dq_partial = dqp;
+  p.B = B;
+  p.H = H;
+  p.k = kp;
+  p.total_tokens = static_cast<int>(T);
+  p.q_per_user = d->q_per_user;
+  p.scale = d->scale;
+  p.budget_ns = wait_budget();
+  if (T > 0) {
+    CUtensorMap mQ, mDO, mK, mV;
+    const uint64_t qrows = uint64_t(d->q_per_user ? B : 1) * H * kp;
+    if (!encode_2d(&mQ, q, D, qrows, D, 64, kp)) return SKA_ERR_CUDA;
+    if (!encode_2d(&mDO, dsketch, D, uint64_t(B) * H * kp, D, 64, kp)) return SKA_ERR_CUDA;
+    if (!encode_2d(&mK, k, uint64_t(H) * D, T, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+    if (!encode_2d(&mV, v, uint64_t(H) * D, T, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+    cudaError_t e;
+    {
+      TimedRegion tr(s);
+      e = launch_sa_bwd(D, sms, mQ, mDO, mK, mV, p, s);
+    }
+    if (e != cudaSuccess) return SKA_ERR_CUDA;
+  }
+  if (launch_sa_bwd_finish(p, D, dq, s) != cudaSuccess) return SKA_ERR_CUDA;
+  return SKA_OK;
 }
 
 size_t stca_forward_workspace_size(const ska_stca_desc* d) {

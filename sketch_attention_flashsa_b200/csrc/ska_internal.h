@@ -3,6 +3,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 
 #include "../../include/sketch_attn.h"
 
@@ -91,6 +92,33 @@ cudaError_t launch_fa_schedule(const FaFwdParams& p, int num_ctas, cudaStream_t 
 // SA: out = sketch [B,H,k,D], lse [B,H,k]. STCA: out [total_targets, H, D], lse [total_targets, H].
 cudaError_t launch_fa_combine(const FaFwdParams& p, int head_dim, int max_streams, float* out, float* lse,
                               cudaStream_t stream);
+
+// Parameters of the SA backward (both normalisations).
+struct SaBwdParams {
+  int norm;                    // SKA_NORM_PROTO or SKA_NORM_TOKEN
+  const int32_t* cu_seqlens;
+  const int32_t* seqused;
+  const int32_t* tile_prefix;  // [B+1] (from launch_schedule)
+  WsHeader* hdr;
+  const float* lse;            // PROTO [T,H] (natural log); TOKEN [B,H,k]
+  const float* sketch;         // TOKEN: forward output [B,H,k,d] (for D_j = dO_j . O_j)
+  const __nv_bfloat16* dsketch;// [B,H,k,d] (TOKEN: D_j)
+  float* dk;                   // [T,H,d]
+  float* dv;                   // [T,H,d]
+  float* dq_partial;           // [(B*H + ctas) * k * d]
+  int B, H, k, total_tokens, q_per_user;
+  float scale;
+  uint64_t budget_ns;
+};
+
+bool sa_bwd_supported(int head_dim, int num_protos);
+size_t sa_bwd_smem_bytes(int head_dim, int num_protos);
+cudaError_t launch_sa_bwd(int head_dim, int num_ctas, const CUtensorMap& mapQ, const CUtensorMap& mapDO,
+                          const CUtensorMap& mapK, const CUtensorMap& mapV, const SaBwdParams& p,
+                          cudaStream_t stream);
+// dq = scale * sum of the partial slots of every segment with head h (shared prototypes) or of
+// segment (b, h) (per-user queries), in a fixed order; also zeroes dK/dV rows of padding tokens.
+cudaError_t launch_sa_bwd_finish(const SaBwdParams& p, int head_dim, float* dq, cudaStream_t stream);
 
 // Small kernels (ska_small.cu).
 cudaError_t launch_schedule(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,
