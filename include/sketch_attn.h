@@ -172,6 +172,10 @@ ska_status stca_forward(const ska_stca_desc* desc, const void* q, const int32_t*
 /* Human-readable name of a status code (static string). */
 const char* ska_status_string(ska_status status);
 
+/* Text of the last failure this host thread's calls recorded (the CUDA error behind an
+ * SKA_ERR_CUDA return, or the step that failed); an empty string if none. Static, per thread. */
+const char* ska_last_error_string(void);
+
 /* Reads the device status word of a workspace after synchronising `stream`; returns SKA_OK or
  * the first device-side error a kernel recorded there (e.g. SKA_ERR_DEVICE_TIMEOUT), and
  * clears it. Test and debug helper: it blocks the host. */

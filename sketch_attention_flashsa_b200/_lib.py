@@ -22,7 +22,7 @@ SKA_NORM_TOKEN = 1
 EXPORTED = ("sa_forward_workspace_size", "sa_forward", "sa_backward_workspace_size", "sa_backward",
             "stca_forward_workspace_size", "stca_forward", "ska_status_string",
             "ska_read_device_status", "ska_set_debug", "ska_set_timing_events",
-            "sa_forward_noalloc", "sa_forward_noalloc_scratch_bytes")
+            "sa_forward_noalloc", "sa_forward_noalloc_scratch_bytes", "ska_last_error_string")
 
 
 class SaDesc(ctypes.Structure):
@@ -44,7 +44,10 @@ class StcaDesc(ctypes.Structure):
 class SkaError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
-        super().__init__(f"{what}: {status_string(code)} ({code})")
+        detail = ""
+        if code == SKA_ERR_CUDA and _lib is not None:
+            detail = " [" + _lib.ska_last_error_string().decode() + "]"
+        super().__init__(f"{what}: {status_string(code)} ({code}){detail}")
 
 
 _lib = None
@@ -72,6 +75,8 @@ def lib() -> ctypes.CDLL:
     L.stca_forward_workspace_size.restype = sz
     L.stca_forward.argtypes = [ctypes.POINTER(StcaDesc), vp, i32p, vp, vp, i32p, i32p, vp, vp, vp, vp, vp, sz, vp]
     L.stca_forward.restype = ctypes.c_int
+    L.ska_last_error_string.argtypes = []
+    L.ska_last_error_string.restype = ctypes.c_char_p
     L.ska_status_string.argtypes = [ctypes.c_int]
     L.ska_status_string.restype = ctypes.c_char_p
     L.ska_read_device_status.argtypes = [vp, vp]

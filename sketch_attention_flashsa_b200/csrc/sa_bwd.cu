@@ -32,7 +32,7 @@ constexpr int kBwdWarps = 8;
 constexpr int kBlk = 16384;  // [128 rows x 64 bf16] swizzled block
 
 struct BwdLayout {
-  uint32_t q_off, do_off, k_off, v_off, a_off, lo_off, lse_off, d_off, total;
+  uint32_t q_off, do_off, k_off, v_off, a_off, lo_off, lse_off, d_off, bar_off, total;
 };
 
 // Q, dO: ceil(d/64) blocks of k rows x 128 B (k padded to a multiple of 8);
@@ -58,6 +58,8 @@ __host__ __device__ inline BwdLayout bwd_layout(int D, int k) {
   off += 256 * 4;
   L.d_off = off;
   off += 256 * 4;
+  L.bar_off = off;
+  off += 128;  // mbarriers, TMEM base, abort flag
   L.total = off;
   return L;
 }
@@ -65,7 +67,7 @@ __host__ __device__ inline BwdLayout bwd_layout(int D, int k) {
 __host__ __device__ inline int bwd_tmem_cols(int D, int k) { return k + 2 * D + ((k + 127) / 128) * D; }
 
 struct BwdBars {
-  uint64_t ld, qd, m1, a, m2, ds, m3, out, drain;
+  uint64_t ld, qd, m1, a, m2, ds, m3, out, drain, dready;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -141,11 +143,16 @@ __global__ void __maxnreg__(224)
   constexpr int QBLOCKS = (KP + 127) / 128;
   static_assert(CQ + QBLOCKS * D <= 512, "TMEM");
   static_assert(NCOL % 8 == 0, "columns");
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ BwdBars bars;
-  __shared__ uint64_t dready;
+  // No static shared memory: the dynamic region starts on a 1024-byte boundary (checked below)
+  // and holds the barriers too, so that k = 256, d = 64 fits without alignment slack.
+  extern __shared__ __align__(1024) uint8_t smem[];
   const BwdLayout L = bwd_layout(D, KP);
+  BwdBars& bars = *reinterpret_cast<BwdBars*>(smem + L.bar_off);
+  uint64_t& dready = bars.dready;
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicCAS(&p.hdr->status, 0, (int)SKA_ERR_UNSUPPORTED);
+    return;
+  }
   uint8_t* sQ = smem + L.q_off;
   uint8_t* sDO = smem + L.do_off;
   uint8_t* sK = smem + L.k_off;
@@ -478,7 +485,7 @@ template <int D, int KP>
 cudaError_t bwd_launch_t(int num_ctas, const CUtensorMap& mQ, const CUtensorMap& mDO, const CUtensorMap& mK,
                          const CUtensorMap& mV, const SaBwdParams& p, cudaStream_t stream) {
   auto kern = sa_bwd_kernel<D, KP>;
-  const size_t smem = bwd_layout(D, KP).total + 1024;
+  const size_t smem = bwd_layout(D, KP).total;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<num_ctas, kBwdThreads, smem, stream>>>(mQ, mDO, mK, mV, p);
@@ -491,10 +498,10 @@ bool sa_bwd_supported(int D, int k) {
   if (D != 64 && D != 128) return false;
   if (!(k == 16 || k == 32 || k == 64 || k == 128 || k == 256)) return false;
   if (bwd_tmem_cols(D, k) + ((k + 31) / 32 * 32 - k) > 512) return false;
-  return bwd_layout(D, k).total + 1024 <= 227 * 1024 - 512;
+  return bwd_layout(D, k).total <= 227 * 1024;
 }
 
-size_t sa_bwd_smem_bytes(int D, int k) { return bwd_layout(D, k).total + 1024; }
+size_t sa_bwd_smem_bytes(int D, int k) { return bwd_layout(D, k).total; }
 
 cudaError_t launch_sa_bwd(int D, int num_ctas, const CUtensorMap& mQ, const CUtensorMap& mDO,
                           const CUtensorMap& mK, const CUtensorMap& mV, const SaBwdParams& p,

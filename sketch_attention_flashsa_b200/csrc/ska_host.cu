@@ -16,6 +16,13 @@ using namespace ska;
 
 namespace {
 
+thread_local char g_last_error[256] = "";
+
+void record_error(const char* what, cudaError_t e) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what,
+                e == cudaSuccess ? "failed" : cudaGetErrorString(e));
+}
+
 std::atomic<uint64_t> g_budget_ns{0};
 std::atomic<uint32_t> g_debug_flags{0};
 std::atomic<void*> g_ev_start{nullptr};
@@ -73,7 +80,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_elems,
                uint32_t box_inner, uint32_t box_rows) {
   auto fn = encode_fn();
-  if (!fn) return false;
+  if (!fn) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled: driver entry point not found");
+    return false;
+  }
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {row_stride_elems * 2};
   cuuint32_t box[2] = {box_inner, box_rows};
@@ -81,6 +91,9 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled: CUresult %d (inner %llu, rows %llu, box %u x %u)",
+                  int(r), (unsigned long long)inner, (unsigned long long)rows, box_inner, box_rows);
   return r == CUDA_SUCCESS;
 }
 
@@ -244,7 +257,7 @@ ska_status sa_forward_token(const ska_sa_desc* d, const void* q, const void* k, 
   p.scale_log2 = d->scale * 1.4426950408889634f;
   p.budget_ns = wait_budget();
   p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
-  if (launch_fa_schedule(p, ctas, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (cudaError_t e_ = launch_fa_schedule(p, ctas, s); e_ != cudaSuccess) { record_error("launch_fa_schedule", e_); return SKA_ERR_CUDA; }
   if (T > 0) {
     CUtensorMap mQ, mK, mV;
     const uint64_t qrows = uint64_t(d->q_per_user ? B : 1) * H * kp;
@@ -256,9 +269,12 @@ ska_status sa_forward_token(const ska_sa_desc* d, const void* q, const void* k, 
       TimedRegion tr(s);
       e = launch_fa_fwd(D, ctas, smem, mQ, mK, mV, mK, mV, p, s);
     }
-    if (e != cudaSuccess) return SKA_ERR_CUDA;
+    if (e != cudaSuccess) {
+      record_error("fused kernel launch", e);
+      return SKA_ERR_CUDA;
+    }
   }
-  if (launch_fa_combine(p, D, B * H * p.group, sketch, lse, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (cudaError_t e_ = launch_fa_combine(p, D, B * H * p.group, sketch, lse, s); e_ != cudaSuccess) { record_error("launch_fa_combine", e_); return SKA_ERR_CUDA; }
   return SKA_OK;
 }
 
@@ -292,6 +308,8 @@ size_t stca_ws_size(const ska_stca_desc* d, FaWs* w, int* ctas, size_t* smem, in
 }  // namespace
 
 extern "C" {
+
+const char* ska_last_error_string(void) { return g_last_error; }
 
 const char* ska_status_string(ska_status s) {
   switch (s) {
@@ -406,7 +424,7 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
     vb = wsb + w.vb;
   }
 
-  if (launch_schedule(cu_seqlens, seqused, B, H, L.num_clusters, prefix, hdr, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (cudaError_t e_ = launch_schedule(cu_seqlens, seqused, B, H, L.num_clusters, prefix, hdr, s); e_ != cudaSuccess) { record_error("launch_schedule", e_); return SKA_ERR_CUDA; }
   if (T > 0) {
     CUtensorMap mQ, mK, mV;
     const uint64_t qrows = uint64_t(d->q_per_user ? B : 1) * H * kp;
@@ -436,12 +454,15 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
       TimedRegion tr(s);
       e = launch_proto_fwd(D, L, mQ, mK, mV, p, s);
     }
-    if (e != cudaSuccess) return SKA_ERR_CUDA;
+    if (e != cudaSuccess) {
+      record_error("fused kernel launch", e);
+      return SKA_ERR_CUDA;
+    }
   }
   if (launch_proto_combine(prefix, hdr, partial, nullptr, B, H, kp, D, sketch, nullptr, s) != cudaSuccess)
     return SKA_ERR_CUDA;
   if (lse && T > 0) {
-    if (launch_fill_padding_lse(cu_seqlens, seqused, B, H, T, lse, s) != cudaSuccess) return SKA_ERR_CUDA;
+    if (cudaError_t e_ = launch_fill_padding_lse(cu_seqlens, seqused, B, H, T, lse, s); e_ != cudaSuccess) { record_error("launch_fill_padding_lse", e_); return SKA_ERR_CUDA; }
   }
   return SKA_OK;
 }
@@ -499,7 +520,7 @@ ska_status sa_backward(const ska_sa_desc* d, const void* q, const void* k, const
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
   int32_t* prefix = reinterpret_cast<int32_t*>(wsb + sizeof(WsHeader));
   float* dqp = reinterpret_cast<float*>(wsb + align256(sizeof(WsHeader) + size_t(B + 1) * 4));
-  if (launch_schedule(cu_seqlens, seqused, B, H, sms, prefix, hdr, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (cudaError_t e_ = launch_schedule(cu_seqlens, seqused, B, H, sms, prefix, hdr, s); e_ != cudaSuccess) { record_error("launch_schedule", e_); return SKA_ERR_CUDA; }
   SaBwdParams p{};
   p.norm = d->norm;
   p.cu_seqlens = cu_seqlens;
@@ -531,9 +552,12 @@ ska_status sa_backward(const ska_sa_desc* d, const void* q, const void* k, const
       TimedRegion tr(s);
       e = launch_sa_bwd(D, sms, mQ, mDO, mK, mV, p, s);
     }
-    if (e != cudaSuccess) return SKA_ERR_CUDA;
+    if (e != cudaSuccess) {
+      record_error("fused kernel launch", e);
+      return SKA_ERR_CUDA;
+    }
   }
-  if (launch_sa_bwd_finish(p, D, dq, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (cudaError_t e_ = launch_sa_bwd_finish(p, D, dq, s); e_ != cudaSuccess) { record_error("launch_sa_bwd_finish", e_); return SKA_ERR_CUDA; }
   return SKA_OK;
 }
 
@@ -601,7 +625,7 @@ ska_status stca_forward(const ska_stca_desc* d, const void* q, const int32_t* cu
   p.scale_log2 = d->scale * 1.4426950408889634f;
   p.budget_ns = wait_budget();
   p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
-  if (launch_fa_schedule(p, ctas, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (cudaError_t e_ = launch_fa_schedule(p, ctas, s); e_ != cudaSuccess) { record_error("launch_fa_schedule", e_); return SKA_ERR_CUDA; }
   CUtensorMap mQ, mK, mV, mKs, mVs;
   if (!encode_2d(&mQ, q, uint64_t(H) * D, Tq, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
   // maps over absent segments point at q with one row; no tile of theirs is ever loaded
@@ -626,7 +650,7 @@ ska_status stca_forward(const ska_stca_desc* d, const void* q, const int32_t* cu
     e = launch_fa_fwd(D, ctas, smem, mQ, mK, mV, mKs, mVs, p, s);
   }
   if (e != cudaSuccess) return SKA_ERR_CUDA;
-  if (launch_fa_combine(p, D, B * H * p.group, out, lse, s) != cudaSuccess) return SKA_ERR_CUDA;
+  if (cudaError_t e_ = launch_fa_combine(p, D, B * H * p.group, out, lse, s); e_ != cudaSuccess) { record_error("launch_fa_combine", e_); return SKA_ERR_CUDA; }
   return SKA_OK;
 }
 
