@@ -15,7 +15,7 @@
 //   MMA  dQ  += dS . K          (M=proto, N=d) -> TMEM, accumulated over the CTA's tiles of one
 //        segment with both halves of the pair; written to a partial slot at segment end.
 // Warps 0-7 (two warpgroups, each owning half of the prototype columns) do the elementwise
-// work; warp 8 issues TMA loads and MMAs. The phases of a tile run one after another.
+// work; thread 0 also issues the TMA loads and MMAs. The phases of a tile run one after another.
 #include <algorithm>
 #include <cmath>
 
@@ -26,10 +26,10 @@ namespace ska {
 
 namespace {
 
-constexpr int kBwdWorkers = 256;
-constexpr int kBwdThreads = 288;
+constexpr int kBwdThreads = 256;
 constexpr int kBwdWarps = 8;
 constexpr int kBlk = 16384;  // [128 rows x 64 bf16] swizzled block
+constexpr int kDqFlush = 8;  // tiles per dQ accumulation chain in TMEM
 
 struct BwdLayout {
   uint32_t q_off, do_off, k_off, v_off, a_off, lo_off, lse_off, d_off, bar_off, total;
@@ -67,10 +67,12 @@ __host__ __device__ inline BwdLayout bwd_layout(int D, int k) {
 __host__ __device__ inline int bwd_tmem_cols(int D, int k) { return k + 2 * D + ((k + 127) / 128) * D; }
 
 struct BwdBars {
-  uint64_t ld, qd, m1, a, m2, ds, m3, out, drain, dready;
+  uint64_t ld, qd, m1, a, m2, ds, m3, out, drain, dready, dl;
   uint32_t tmem_base;
   int abort_flag;
 };
+
+static_assert(sizeof(BwdBars) <= 128, "barrier area");
 
 struct BwdPos {
   int b, h, j, nb;
@@ -129,7 +131,7 @@ struct BwdWaiter {
 
 
 template <int D, int KP>
-__global__ void __maxnreg__(224)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     sa_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapDO,
                   const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                   const SaBwdParams p) {
@@ -157,9 +159,10 @@ __global__ void __maxnreg__(224)
   uint8_t* sDO = smem + L.do_off;
   uint8_t* sK = smem + L.k_off;
   uint8_t* sV = smem + L.v_off;
-  uint8_t* sA = smem + L.a_off;    // A, then dS hi
-  uint8_t* sLo = smem + L.lo_off;  // dS lo
+  uint8_t* sA = smem + L.a_off;    // A hi, then dS hi
+  uint8_t* sLo = smem + L.lo_off;  // A lo, then dS lo
   float* sLse = reinterpret_cast<float*>(smem + L.lse_off);
+  float* sDl = sLse;  // PROTO (no per-prototype lse): each warpgroup's partial delta per token
   float* sDj = reinterpret_cast<float*>(smem + L.d_off);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -172,11 +175,12 @@ __global__ void __maxnreg__(224)
     mbar_init(&bars.ds, kBwdWarps);
     mbar_init(&bars.out, kBwdWarps);
     mbar_init(&dready, kBwdWarps);
+    mbar_init(&bars.dl, kBwdWarps);
     mbar_init(&bars.drain, 1);
     bars.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 0) {
     tmem_alloc(&bars.tmem_base, 512);
     tmem_relinquish();
   }
@@ -190,64 +194,191 @@ __global__ void __maxnreg__(224)
   const int g0 = blockIdx.x * W;
   const int ntiles = (W > 0 && g0 < total) ? (min(total, g0 + W) - g0) : 0;
 
-  if (warp == 8) {
-    // ---------------------------------------------------------------- control: TMA + MMA
-    if (lane == 0 && ntiles > 0) {
-      constexpr uint32_t i1 = idesc_bf16_f32(128, KP, false, false);
-      constexpr uint32_t iV = idesc_bf16_f32(128, D, false, true);
-      constexpr uint32_t iQ = idesc_bf16_f32(128, D, true, true);
-      BwdPos t;
-      bwd_seek(p, g0, t);
-      int nseg = 0;
-      bool ok = true;
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const bool first = (t.j == 0) || (i == 0);
-        if (first) {
-          const int qrow = (p.q_per_user ? t.b * p.H * p.k : 0) + t.h * p.k;
-          const int orow = (t.b * p.H + t.h) * p.k;
-          mbar_expect_tx(&bars.qd, 2 * KB * KP * 128);
-          for (int kb = 0; kb < KB; ++kb) {
-            tma_load_2d(sQ + kb * QBLK, &mapQ, &bars.qd, kb * 64, qrow);
-            tma_load_2d(sDO + kb * QBLK, &mapDO, &bars.qd, kb * 64, orow);
-          }
-        }
-        const int tok0 = p.cu_seqlens[t.b] + t.j * 128;
-        mbar_expect_tx(&bars.ld, 2 * KB * kBlk);
+  // One program for all 256 threads; thread 0 also issues the TMA loads and the MMAs of each
+  // phase (the phases of a tile are sequential, so no separate control warp is needed).
+  constexpr uint32_t i1 = idesc_bf16_f32(128, KP, false, false);
+  constexpr uint32_t iV = idesc_bf16_f32(128, D, false, true);
+  constexpr uint32_t iQ = idesc_bf16_f32(128, D, true, true);
+  const bool ctl = (threadIdx.x == 0);
+  const int wg = warp >> 2, q4 = warp & 3;
+  const int r = q4 * 32 + lane;
+  const int col0 = wg * NCOL;
+  const uint32_t loff = static_cast<uint32_t>(q4 * 32) << 16;
+  const float L2E = 1.4426950408889634f;
+  const float c2 = p.scale * L2E;
+  BwdPos t;
+  if (ntiles > 0) bwd_seek(p, g0, t);
+  int nseg = 0;
+  int segt = 0;  // tile index inside this CTA's part of the current (user, head) segment
+  bool ok = true;
+  for (int i = 0; i < ntiles && ok; ++i) {
+    const bool first = (t.j == 0) || (i == 0);
+    const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
+    segt = first ? 0 : segt + 1;
+    // dQ restarts in TMEM every kDqFlush tiles and is added into the partial slot: the tensor
+    // core's fp32 accumulation is not round-to-nearest, so long chains would drift
+    const bool fresh = (segt % kDqFlush) == 0;
+    const bool flush = last || (segt % kDqFlush) == kDqFlush - 1;
+    const int used = bwd_used(p, t.b);
+    const int tok0 = p.cu_seqlens[t.b] + t.j * 128;
+    const int tok = tok0 + r;
+    const bool valid = (t.j * 128 + r) < used;
+    if (ctl) {
+      if (first) {
+        const int qrow = (p.q_per_user ? t.b * p.H * p.k : 0) + t.h * p.k;
+        const int orow = (t.b * p.H + t.h) * p.k;
+        mbar_expect_tx(&bars.qd, 2 * KB * KP * 128);
         for (int kb = 0; kb < KB; ++kb) {
-          tma_load_2d(sK + kb * kBlk, &mapK, &bars.ld, t.h * D + kb * 64, tok0);
-          tma_load_2d(sV + kb * kBlk, &mapV, &bars.ld, t.h * D + kb * 64, tok0);
+          tma_load_2d(sQ + kb * QBLK, &mapQ, &bars.qd, kb * 64, qrow);
+          tma_load_2d(sDO + kb * QBLK, &mapDO, &bars.qd, kb * 64, orow);
         }
-        ok = wait(&bars.ld, i & 1);
-        if (ok && first) ok = wait(&bars.qd, nseg & 1);
-        if (!ok) break;
-        tc_fence_after();
-        // S^T = K . Q^T
+      }
+      mbar_expect_tx(&bars.ld, 2 * KB * kBlk);
+      for (int kb = 0; kb < KB; ++kb) {
+        tma_load_2d(sK + kb * kBlk, &mapK, &bars.ld, t.h * D + kb * 64, tok0);
+        tma_load_2d(sV + kb * kBlk, &mapV, &bars.ld, t.h * D + kb * 64, tok0);
+      }
+    }
+    if (first && p.norm == SKA_NORM_TOKEN) {
+      // per-prototype lse (log2 units) and D_j = dO_j . O_j of this (user, head)
+      const int jj = threadIdx.x;
+      if (jj < p.k) {
+        const int64_t row = (static_cast<int64_t>(t.b) * p.H + t.h) * p.k + jj;
+        sLse[jj] = p.lse[row] * L2E;
+        float acc = 0.f;
+        for (int dd = 0; dd < D; ++dd) acc += __bfloat162float(p.dsketch[row * D + dd]) * p.sketch[row * D + dd];
+        sDj[jj] = acc;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dready);
+      ok = __all_sync(0xffffffffu, wait(&dready, nseg & 1));
+      if (!ok) break;
+    }
+    ok = __all_sync(0xffffffffu, wait(&bars.ld, i & 1) && (!first || wait(&bars.qd, nseg & 1)));
+    if (!ok) break;
+    if (ctl) {
+      tc_fence_after();
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s)
-          umma_bf16(tb, sw128_desc(smem_u32(sK) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
-                    sw128_desc(smem_u32(sQ) + (s / 4) * QBLK + (s % 4) * 32, 16, 1024), i1, s > 0);
-        umma_commit(&bars.m1);
-        ok = wait(&bars.a, i & 1);
-        if (!ok) break;
-        tc_fence_after();
-        // dV = A^T . dO ; dA^T = V . dO^T (over S^T)
+      for (int s = 0; s < D / 16; ++s)
+        umma_bf16(tb, sw128_desc(smem_u32(sK) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                  sw128_desc(smem_u32(sQ) + (s / 4) * QBLK + (s % 4) * 32, 16, 1024), i1, s > 0);
+      umma_commit(&bars.m1);
+    }
+    ok = __all_sync(0xffffffffu, wait(&bars.m1, i & 1));
+    if (!ok) break;
+    tc_fence_after();
+    // A = exp(scale s - lse): PROTO per token row, TOKEN per prototype column
+    float a[NCOL];
+    {
+      uint32_t sv[NCOL];
 #pragma unroll
-        for (int s = 0; s < KP / 16; ++s)
-          umma_bf16(tb + CV, sw128_desc(smem_u32(sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
-                    sw128_desc(smem_u32(sDO) + s * 2048, QBLK, 1024), iV, s > 0);
+      for (int c = 0; c < NCOL; c += 8) tmem_ld8(tb + loff + col0 + c, sv + c);
+      tmem_ld_wait();
+      const float lrow = (p.norm == SKA_NORM_PROTO && valid) ? p.lse[static_cast<int64_t>(tok) * p.H + t.h] * L2E : 0.f;
+#pragma unroll
+      for (int c = 0; c < NCOL; ++c) {
+        const float l2 = (p.norm == SKA_NORM_PROTO) ? lrow : sLse[col0 + c];
+        a[c] = valid ? ex2_approx(__uint_as_float(sv[c]) * c2 - l2) : 0.f;
+      }
+    }
+    // A as a bf16 pair hi + lo, so that dV carries no bf16 rounding of A
+#pragma unroll
+    for (int c = 0; c < NCOL; c += 8) {
+      float hi[8], lo[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        hi[u] = __bfloat162float(__float2bfloat16_rn(a[c + u]));
+        lo[u] = a[c + u] - hi[u];
+      }
+      const int jj = col0 + c;
+      const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
+      *reinterpret_cast<uint4*>(sA + off) = make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]),
+                                                       pack_bf16x2(hi[4], hi[5]), pack_bf16x2(hi[6], hi[7]));
+      *reinterpret_cast<uint4*>(sLo + off) = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]),
+                                                        pack_bf16x2(lo[4], lo[5]), pack_bf16x2(lo[6], lo[7]));
+    }
+    fence_async_shared();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.a);
+    if (ctl) {
+      ok = wait(&bars.a, i & 1);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+          for (int s = 0; s < KP / 16; ++s)
+            umma_bf16(tb + CV, sw128_desc(smem_u32(half ? sLo : sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                      sw128_desc(smem_u32(sDO) + s * 2048, QBLK, 1024), iV, (half | s) > 0);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
           umma_bf16(tb, sw128_desc(smem_u32(sV) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
                     sw128_desc(smem_u32(sDO) + (s / 4) * QBLK + (s % 4) * 32, 16, 1024), i1, s > 0);
         umma_commit(&bars.m2);
-        ok = wait(&bars.ds, i & 1);
-        if (!ok) break;
-        tc_fence_after();
-        // dK = dS^T . Q ; dQ += dS . K (hi and lo halves of dS)
+      }
+    }
+    ok = __all_sync(0xffffffffu, wait(&bars.m2, i & 1));
+    if (!ok) break;
+    tc_fence_after();
+    // PROTO: delta_i = sum_j A_ij dA_ij in fp32; each warpgroup sums its half of the
+    // prototypes and the two halves are added in a fixed order
+    float delta = 0.f;
+    if (p.norm == SKA_NORM_PROTO) {
+      float part = 0.f;
 #pragma unroll
-        for (int s = 0; s < KP / 16; ++s)
-          umma_bf16(tb + CK, sw128_desc(smem_u32(sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
-                    sw128_desc(smem_u32(sQ) + s * 2048, QBLK, 1024), iV, s > 0);
+      for (int c = 0; c < NCOL; c += 8) {
+        uint32_t da[8];
+        tmem_ld8(tb + loff + col0 + c, da);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) part = fmaf(a[c + u], __uint_as_float(da[u]), part);
+      }
+      sDl[wg * 128 + r] = part;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.dl);
+      ok = __all_sync(0xffffffffu, wait(&bars.dl, i & 1));
+      if (!ok) break;
+      delta = sDl[r] + sDl[128 + r];
+    }
+    // dS = A (dA - delta) as a bf16 pair hi + lo
+#pragma unroll
+    for (int c = 0; c < NCOL; c += 8) {
+      uint32_t da[8];
+      tmem_ld8(tb + loff + col0 + c, da);
+      tmem_ld_wait();
+      float hi[8], lo[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float sub = (p.norm == SKA_NORM_PROTO) ? delta : sDj[col0 + c + u];
+        const float ds = a[c + u] * (__uint_as_float(da[u]) - sub);
+        hi[u] = __bfloat162float(__float2bfloat16_rn(ds));
+        lo[u] = ds - hi[u];
+      }
+      const int jj = col0 + c;
+      uint4 wh, wl;
+      wh.x = pack_bf16x2(hi[0], hi[1]); wh.y = pack_bf16x2(hi[2], hi[3]);
+      wh.z = pack_bf16x2(hi[4], hi[5]); wh.w = pack_bf16x2(hi[6], hi[7]);
+      wl.x = pack_bf16x2(lo[0], lo[1]); wl.y = pack_bf16x2(lo[2], lo[3]);
+      wl.z = pack_bf16x2(lo[4], lo[5]); wl.w = pack_bf16x2(lo[6], lo[7]);
+      const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
+      *reinterpret_cast<uint4*>(sA + off) = wh;
+      *reinterpret_cast<uint4*>(sLo + off) = wl;
+    }
+    fence_async_shared();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.ds);
+    if (ctl) {
+      ok = wait(&bars.ds, i & 1);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+          for (int s = 0; s < KP / 16; ++s)
+            umma_bf16(tb + CK, sw128_desc(smem_u32(half ? sLo : sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                      sw128_desc(smem_u32(sQ) + s * 2048, QBLK, 1024), iV, (half | s) > 0);
 #pragma unroll
         for (int g = 0; g < QBLOCKS; ++g)
 #pragma unroll
@@ -257,187 +388,80 @@ __global__ void __maxnreg__(224)
               const uint32_t abase = smem_u32(half == 0 ? sA : sLo) + 2 * g * kBlk;
               umma_bf16(tb + CQ + g * D, sw128_desc(abase + s * 2048, kBlk, 1024),
                         sw128_desc(smem_u32(sK) + s * 2048, kBlk, 1024), iQ,
-                        (first && half == 0 && s == 0) ? 0u : 1u);
+                        (fresh && half == 0 && s == 0) ? 0u : 1u);
             }
         umma_commit(&bars.m3);
-        ok = wait(&bars.out, i & 1);
-        if (!ok) break;
-        if (first) ++nseg;
-        bwd_next(p, t);
       }
-      umma_commit(&bars.drain);  // completes when every MMA issued above has
-      wait(&bars.drain, 0, true);
     }
-  } else {
-    // ---------------------------------------------------------------- workers
-    const int wg = warp >> 2, q4 = warp & 3;
-    const int r = q4 * 32 + lane;
-    const int col0 = wg * NCOL;
-    const uint32_t loff = static_cast<uint32_t>(q4 * 32) << 16;
-    const float L2E = 1.4426950408889634f;
-    const float c2 = p.scale * L2E;
-    BwdPos t;
-    if (ntiles > 0) bwd_seek(p, g0, t);
-    int nseg = 0;
-    bool ok = true;
-    for (int i = 0; i < ntiles && ok; ++i) {
-      const bool first = (t.j == 0) || (i == 0);
-      const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
-      const int used = bwd_used(p, t.b);
-      const int tok = p.cu_seqlens[t.b] + t.j * 128 + r;
-      const bool valid = (t.j * 128 + r) < used;
-      if (first && p.norm == SKA_NORM_TOKEN) {
-        // per-prototype lse (log2 units) and D_j = dO_j . O_j of this (user, head)
-        const int jj = threadIdx.x;
-        if (jj < p.k) {
-          const int64_t row = (static_cast<int64_t>(t.b) * p.H + t.h) * p.k + jj;
-          sLse[jj] = p.lse[row] * L2E;
-          float acc = 0.f;
-          for (int dd = 0; dd < D; ++dd)
-            acc += __bfloat162float(p.dsketch[row * D + dd]) * p.sketch[row * D + dd];
-          sDj[jj] = acc;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&dready);
-        ok = __all_sync(0xffffffffu, wait(&dready, nseg & 1));
-        if (!ok) break;
-      }
-      ok = __all_sync(0xffffffffu, wait(&bars.m1, i & 1));
-      if (!ok) break;
-      tc_fence_after();
-      // A = exp(scale s - lse): PROTO per token row, TOKEN per prototype column
-      float a[NCOL];
-      {
-        uint32_t sv[NCOL];
+    ok = __all_sync(0xffffffffu, wait(&bars.m3, i & 1));
+    if (!ok) break;
+    tc_fence_after();
+    // dK (scaled) and dV rows: warpgroup wg writes channels [wg D/2, (wg+1) D/2)
 #pragma unroll
-        for (int c = 0; c < NCOL; c += 8) tmem_ld8(tb + loff + col0 + c, sv + c);
+    for (int c = 0; c < D / 2; c += 32) {
+      const int cc = wg * (D / 2) + c;
+      uint32_t kr[32], vr[32];
+      tmem_ld32(tb + loff + CK + cc, kr);
+      tmem_ld32(tb + loff + CV + cc, vr);
+      tmem_ld_wait();
+      if (tok < p.total_tokens && (t.j * 128 + r) < (p.cu_seqlens[t.b + 1] - p.cu_seqlens[t.b])) {
+        float* dk = p.dk + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
+        float* dv = p.dv + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
+#pragma unroll
+        for (int u = 0; u < 32; u += 4) {
+          *reinterpret_cast<float4*>(dk + u) =
+              make_float4(p.scale * __uint_as_float(kr[u]), p.scale * __uint_as_float(kr[u + 1]),
+                          p.scale * __uint_as_float(kr[u + 2]), p.scale * __uint_as_float(kr[u + 3]));
+          *reinterpret_cast<float4*>(dv + u) = make_float4(__uint_as_float(vr[u]), __uint_as_float(vr[u + 1]),
+                                                           __uint_as_float(vr[u + 2]), __uint_as_float(vr[u + 3]));
+        }
+      }
+    }
+    if (flush && wg < QBLOCKS) {
+      // dQ block wg (prototypes 128 wg + r) of this segment, scaled, into its partial slot;
+      // only this CTA writes the slot, and each element always by the same thread
+      const int jrow = wg * 128 + r;
+      const int slot = (t.b * p.H + t.h) + static_cast<int>(blockIdx.x);
+      const bool add = segt >= kDqFlush;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t qr[32];
+        tmem_ld32(tb + loff + CQ + wg * D + c, qr);
         tmem_ld_wait();
-        const float lrow = (p.norm == SKA_NORM_PROTO && valid) ? p.lse[static_cast<int64_t>(tok) * p.H + t.h] * L2E : 0.f;
-#pragma unroll
-        for (int c = 0; c < NCOL; ++c) {
-          const float l2 = (p.norm == SKA_NORM_PROTO) ? lrow : sLse[col0 + c];
-          a[c] = valid ? ex2_approx(__uint_as_float(sv[c]) * c2 - l2) : 0.f;
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < NCOL; c += 8) {
-        uint4 w;
-        w.x = pack_bf16x2(a[c + 0], a[c + 1]);
-        w.y = pack_bf16x2(a[c + 2], a[c + 3]);
-        w.z = pack_bf16x2(a[c + 4], a[c + 5]);
-        w.w = pack_bf16x2(a[c + 6], a[c + 7]);
-        const int jj = col0 + c;
-        *reinterpret_cast<uint4*>(sA + (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2)) = w;
-      }
-      fence_async_shared();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.a);
-      ok = __all_sync(0xffffffffu, wait(&bars.m2, i & 1));
-      if (!ok) break;
-      tc_fence_after();
-      // PROTO: delta_i = dV_i . v_i
-      float delta = 0.f;
-      if (p.norm == SKA_NORM_PROTO) {
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t dvr[32];
-          tmem_ld32(tb + loff + CV + c, dvr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int u = 0; u < 32; u += 8) {
-            const int dd = c + u;
-            const uint4 w = *reinterpret_cast<const uint4*>(sV + (dd >> 6) * kBlk + sw128_offset(r, (dd & 63) * 2));
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              delta = fmaf(__uint_as_float(dvr[u + 2 * e]), __uint_as_float(ww[e] << 16), delta);
-              delta = fmaf(__uint_as_float(dvr[u + 2 * e + 1]), __uint_as_float(ww[e] & 0xFFFF0000u), delta);
-            }
-          }
-        }
-      }
-      // dS = A (dA - delta) as a bf16 pair hi + lo
-#pragma unroll
-      for (int c = 0; c < NCOL; c += 8) {
-        uint32_t da[8];
-        tmem_ld8(tb + loff + col0 + c, da);
-        tmem_ld_wait();
-        float hi[8], lo[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float sub = (p.norm == SKA_NORM_PROTO) ? delta : sDj[col0 + c + u];
-          const float ds = a[c + u] * (__uint_as_float(da[u]) - sub);
-          hi[u] = __bfloat162float(__float2bfloat16_rn(ds));
-          lo[u] = ds - hi[u];
-        }
-        const int jj = col0 + c;
-        uint4 wh, wl;
-        wh.x = pack_bf16x2(hi[0], hi[1]); wh.y = pack_bf16x2(hi[2], hi[3]);
-        wh.z = pack_bf16x2(hi[4], hi[5]); wh.w = pack_bf16x2(hi[6], hi[7]);
-        wl.x = pack_bf16x2(lo[0], lo[1]); wl.y = pack_bf16x2(lo[2], lo[3]);
-        wl.z = pack_bf16x2(lo[4], lo[5]); wl.w = pack_bf16x2(lo[6], lo[7]);
-        const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
-        *reinterpret_cast<uint4*>(sA + off) = wh;
-        *reinterpret_cast<uint4*>(sLo + off) = wl;
-      }
-      fence_async_shared();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.ds);
-      ok = __all_sync(0xffffffffu, wait(&bars.m3, i & 1));
-      if (!ok) break;
-      tc_fence_after();
-      // dK (scaled) and dV rows: warpgroup wg writes channels [wg D/2, (wg+1) D/2)
-#pragma unroll
-      for (int c = 0; c < D / 2; c += 32) {
-        const int cc = wg * (D / 2) + c;
-        uint32_t kr[32], vr[32];
-        tmem_ld32(tb + loff + CK + cc, kr);
-        tmem_ld32(tb + loff + CV + cc, vr);
-        tmem_ld_wait();
-        if (tok < p.total_tokens && (t.j * 128 + r) < (p.cu_seqlens[t.b + 1] - p.cu_seqlens[t.b])) {
-          float* dk = p.dk + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
-          float* dv = p.dv + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
+        if (jrow < p.k) {
+          float* dst = p.dq_partial + (static_cast<int64_t>(slot) * p.k + jrow) * D + c;
 #pragma unroll
           for (int u = 0; u < 32; u += 4) {
-            *reinterpret_cast<float4*>(dk + u) =
-                make_float4(p.scale * __uint_as_float(kr[u]), p.scale * __uint_as_float(kr[u + 1]),
-                            p.scale * __uint_as_float(kr[u + 2]), p.scale * __uint_as_float(kr[u + 3]));
-            *reinterpret_cast<float4*>(dv + u) = make_float4(__uint_as_float(vr[u]), __uint_as_float(vr[u + 1]),
-                                                             __uint_as_float(vr[u + 2]), __uint_as_float(vr[u + 3]));
+            float4 o = make_float4(p.scale * __uint_as_float(qr[u]), p.scale * __uint_as_float(qr[u + 1]),
+                                   p.scale * __uint_as_float(qr[u + 2]), p.scale * __uint_as_float(qr[u + 3]));
+            if (add) {
+              const float4 prev = *reinterpret_cast<const float4*>(dst + u);
+              o.x += prev.x;
+              o.y += prev.y;
+              o.z += prev.z;
+              o.w += prev.w;
+            }
+            *reinterpret_cast<float4*>(dst + u) = o;
           }
         }
       }
-      if (last && wg < QBLOCKS) {
-        // dQ block wg (prototypes 128 wg + r) of this segment -> partial slot (scaled)
-        const int jrow = wg * 128 + r;
-        const int slot = (t.b * p.H + t.h) + static_cast<int>(blockIdx.x);
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t qr[32];
-          tmem_ld32(tb + loff + CQ + wg * D + c, qr);
-          tmem_ld_wait();
-          if (jrow < p.k) {
-            float* dst = p.dq_partial + (static_cast<int64_t>(slot) * p.k + jrow) * D + c;
-#pragma unroll
-            for (int u = 0; u < 32; u += 4)
-              *reinterpret_cast<float4*>(dst + u) =
-                  make_float4(p.scale * __uint_as_float(qr[u]), p.scale * __uint_as_float(qr[u + 1]),
-                              p.scale * __uint_as_float(qr[u + 2]), p.scale * __uint_as_float(qr[u + 3]));
-          }
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.out);
-      if (first) ++nseg;
-      bwd_next(p, t);
     }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.out);
+    // the next tile's loads overwrite K, V (and Q, dO): every role must be done with them
+    ok = __all_sync(0xffffffffu, wait(&bars.out, i & 1));
+    if (!ok) break;
+    if (first) ++nseg;
+    bwd_next(p, t);
+  }
+  if (ctl) {
+    umma_commit(&bars.drain);  // completes when every MMA issued above has
+    wait(&bars.drain, 0, true);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tb, 512);
   }

@@ -80,6 +80,14 @@ def test_backward_deterministic(norm):
         assert np.array_equal(x, y)
 
 
+@pytest.mark.parametrize("norm", ["proto", "token"])
+def test_backward_long_chains(norm):
+    """240K tokens x 2 heads = 3752 tiles over the SMs: every CTA walks dozens of tiles of one
+    (user, head), so dQ is restarted and added into its partial slot several times."""
+    inp = W.make_sa([150_000, 90_000], 2, 64, 128, seed=53, with_dsketch=True, dsketch_seed=10)
+    check_bwd(inp, norm)
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("norm", ["proto", "token"])
 def test_backward_config4_full(norm):
