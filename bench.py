@@ -229,7 +229,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    from sketch_attention_flashsa_b200 import api, flops
+    from sketch_attention_flashsa_b200 import api, dp, flops
 
     inp = make_device_inputs(args.workload, rank, dev)
     H, d, kp, B = inp["H"], inp["d"], inp["k_protos"], inp["users"]
@@ -279,10 +279,7 @@ def main():
     clocks = sampler.stop()
     ms_total = e0.elapsed_time(e1)
     kern_ms = [a.elapsed_time(b) for a, b in kev]
-    t = torch.tensor([ms_total, statistics.mean(kern_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, kern_mean = float(t[0]), float(t[1])
+    ms_total, kern_mean = dp.max_over_ranks([ms_total, statistics.mean(kern_ms)], device=dev)
     ms_per_step = ms_total / args.steps
     valid = inp["valid"]
     total_tokens_all = valid * world
@@ -349,9 +346,7 @@ def main():
         e2e_step()
     f1.record()
     torch.cuda.synchronize()
-    te = torch.tensor([f0.elapsed_time(f1) / args.e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    te = dp.max_over_ranks([f0.elapsed_time(f1) / args.e2e_steps], device=dev)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hcu) + ((hsu,) if hsu is not None else ()))
     d2h = hout.numel() * hout.element_size()
     e2e = {"value": total_tokens_all / (float(te[0]) / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,

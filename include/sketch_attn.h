@@ -51,6 +51,13 @@
 #include <stddef.h>
 #include <stdint.h>
 
+/* The library is built with hidden visibility; only the calls below are exported. */
+#if defined(__GNUC__)
+#define SKA_API __attribute__((visibility("default")))
+#else
+#define SKA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -98,7 +105,7 @@ typedef struct {
 } ska_sa_desc;
 
 /* Bytes of workspace sa_forward needs for this descriptor (0 if the descriptor is invalid). */
-size_t sa_forward_workspace_size(const ska_sa_desc* desc);
+SKA_API size_t sa_forward_workspace_size(const ska_sa_desc* desc);
 
 /* SA forward (FlashSA), §3.1 Eq. (7)-(9) and §4.4.
  *   q           [H,k,d] or [B,H,k,d] (q_per_user), in_dtype
@@ -111,12 +118,12 @@ size_t sa_forward_workspace_size(const ska_sa_desc* desc);
  *               log-sum-exp over the valid tokens (-inf for an empty user). The backward pass
  *               needs it.
  *   mass        out, fp32 [B, H, k] or NULL: sum_i A[j,i], the mass each prototype received.  */
-ska_status sa_forward(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
+SKA_API ska_status sa_forward(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
                       const int32_t* cu_seqlens, const int32_t* seqused, float* sketch, float* lse,
                       float* mass, void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of workspace sa_backward needs (0 if the descriptor is invalid). */
-size_t sa_backward_workspace_size(const ska_sa_desc* desc);
+SKA_API size_t sa_backward_workspace_size(const ska_sa_desc* desc);
 
 /* SA backward: gradients of <dsketch, sketch> through Eq. (7)-(9) (SA is trained end to end,
  * App. A.4). Inputs as in sa_forward (bf16 only), plus:
@@ -130,7 +137,7 @@ size_t sa_backward_workspace_size(const ska_sa_desc* desc);
  * Supported: num_protos in {16, 32, 64, 128, 256} for head_dim 64, up to 128 for head_dim 128
  * (SKA_ERR_UNSUPPORTED otherwise). dQ is formed from a two-term bf16 split of dS (16
  * significant bits) and reduced over users in a fixed order.                                  */
-ska_status sa_backward(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
+SKA_API ska_status sa_backward(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
                        const int32_t* cu_seqlens, const int32_t* seqused, const float* sketch,
                        const float* lse, const void* dsketch, float* dq, float* dk, float* dv, void* ws,
                        size_t ws_bytes, void* stream);
@@ -155,7 +162,7 @@ typedef struct {
   int32_t reserved;
 } ska_stca_desc;
 
-size_t stca_forward_workspace_size(const ska_stca_desc* desc);
+SKA_API size_t stca_forward_workspace_size(const ska_stca_desc* desc);
 
 /* STCA forward. All bf16 except the fp32 outputs.
  *   q              [total_targets, H, d]; targets of user b are rows [cu_targets[b], cu_targets[b+1])
@@ -164,28 +171,28 @@ size_t stca_forward_workspace_size(const ska_stca_desc* desc);
  *                  suffix rows of its user (request-aware masking, §4.2)
  *   k_sk, v_sk     [B, H, num_sketch, d] (NULL when num_sketch == 0)
  *   out            fp32 [total_targets, H, d];  lse  fp32 [total_targets, H] or NULL          */
-ska_status stca_forward(const ska_stca_desc* desc, const void* q, const int32_t* cu_targets,
+SKA_API ska_status stca_forward(const ska_stca_desc* desc, const void* q, const int32_t* cu_targets,
                         const void* k_hist, const void* v_hist, const int32_t* cu_hist,
                         const int32_t* target_kv_len, const void* k_sk, const void* v_sk, float* out,
                         float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* Human-readable name of a status code (static string). */
-const char* ska_status_string(ska_status status);
+SKA_API const char* ska_status_string(ska_status status);
 
 /* Text of the last failure this host thread's calls recorded (the CUDA error behind an
  * SKA_ERR_CUDA return, or the step that failed); an empty string if none. Static, per thread. */
-const char* ska_last_error_string(void);
+SKA_API const char* ska_last_error_string(void);
 
 /* Reads the device status word of a workspace after synchronising `stream`; returns SKA_OK or
  * the first device-side error a kernel recorded there (e.g. SKA_ERR_DEVICE_TIMEOUT), and
  * clears it. Test and debug helper: it blocks the host. */
-ska_status ska_read_device_status(void* ws, void* stream);
+SKA_API ska_status ska_read_device_status(void* ws, void* stream);
 
 /* Test hook (process-wide, not synchronised with concurrent calls): the time budget in ns of
  * every barrier wait in later launches (0 restores the default of 4 s), and debug flags
  * (1 = the load producer of later SA forward launches withholds its first arrival, so that
  * the consumers' bounded waits must run out and report SKA_ERR_DEVICE_TIMEOUT). */
-void ska_set_debug(uint64_t wait_budget_ns, uint32_t flags);
+SKA_API void ska_set_debug(uint64_t wait_budget_ns, uint32_t flags);
 
 /* SA forward for callers that cannot allocate device memory (code running inside a memory
  * pool it does not own, plugins that only receive input and output pointers, service paths
@@ -199,18 +206,18 @@ void ska_set_debug(uint64_t wait_budget_ns, uint32_t flags);
  *   The first call on a device looks up the array's address (cudaGetSymbolAddress); make it
  *   before any stream capture. All calls on a device share the array: calls that overlap on
  *   the GPU (other streams, other host threads) race and must be serialised by the caller.   */
-ska_status sa_forward_noalloc(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
+SKA_API ska_status sa_forward_noalloc(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
                               const int32_t* cu_seqlens, const int32_t* seqused, float* sketch,
                               float* lse, float* mass, void* stream);
 
 /* Size in bytes of the device array that sa_forward_noalloc uses as scratch. */
-size_t sa_forward_noalloc_scratch_bytes(void);
+SKA_API size_t sa_forward_noalloc_scratch_bytes(void);
 
 /* Bench hook (process-wide): while both handles are non-NULL, every later call records
  * `start_event` on its stream immediately before its fused main kernel and `stop_event`
  * immediately after it (cudaEvent_t handles created by the caller), so that the main kernel
  * can be timed on its own stream with CUDA events. Pass NULL, NULL to stop recording. */
-void ska_set_timing_events(void* start_event, void* stop_event);
+SKA_API void ska_set_timing_events(void* start_event, void* stop_event);
 
 #ifdef __cplusplus
 }

@@ -63,6 +63,21 @@ int device_sm_count() {
   return cache[dev];
 }
 
+// True (and the reason recorded) when no CUDA device is usable from this thread.
+bool no_device() {
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) {
+    cudaGetLastError();
+    record_error("cudaGetDevice", e);
+    return true;
+  }
+  if (device_sm_count() == 0) {
+    record_error("cudaDeviceGetAttribute(multiProcessorCount)", cudaErrorInvalidDevice);
+    return true;
+  }
+  return false;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -379,6 +394,7 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
       !aligned16(mass) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
       (reinterpret_cast<uintptr_t>(seqused) & 3u))
     return SKA_ERR_INVALID_VALUE;
+  if (no_device()) return SKA_ERR_CUDA;
   const size_t ws_need = sa_forward_workspace_size(d);
   if (ws_need == 0) return SKA_ERR_UNSUPPORTED;
   if (ws_bytes < ws_need) return SKA_ERR_WORKSPACE_TOO_SMALL;
@@ -495,6 +511,7 @@ ska_status sa_backward(const ska_sa_desc* d, const void* q, const void* k, const
       (reinterpret_cast<uintptr_t>(ws) & 255u) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
       (reinterpret_cast<uintptr_t>(seqused) & 3u))
     return SKA_ERR_INVALID_VALUE;
+  if (no_device()) return SKA_ERR_CUDA;
   const size_t need = sa_backward_workspace_size(d);
   if (need == 0) return SKA_ERR_UNSUPPORTED;
   if (ws_bytes < need) return SKA_ERR_WORKSPACE_TOO_SMALL;
@@ -585,6 +602,7 @@ ska_status stca_forward(const ska_stca_desc* d, const void* q, const int32_t* cu
       (reinterpret_cast<uintptr_t>(cu_targets) & 3u) || (reinterpret_cast<uintptr_t>(cu_hist) & 3u) ||
       (reinterpret_cast<uintptr_t>(target_kv_len) & 3u))
     return SKA_ERR_INVALID_VALUE;
+  if (no_device()) return SKA_ERR_CUDA;
   FaWs w;
   int ctas, nk, nv;
   size_t smem;

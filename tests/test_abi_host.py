@@ -1,0 +1,174 @@
+"""The C ABI without a GPU: libska.so loads, exports exactly the calls the header declares, and
+rejects bad arguments on the host before it touches a device (the header's error contract:
+invalid arguments are reported before anything is launched). Fake, never-dereferenced
+addresses stand in for device pointers."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from sketch_attention_flashsa_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sketch_attn.h")
+
+A = 0x10000  # a 64 KB-aligned fake address; any multiple of it is 256-byte aligned
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"^SKA_API\s+[\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M))
+
+
+def exported_symbols():
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True, check=True)
+    return {ln.split()[-1] for ln in out.stdout.splitlines() if len(ln.split()) == 3 and ln.split()[1] == "T"}
+
+
+def test_header_declares_the_boundary():
+    names = header_functions()
+    assert {"sa_forward", "sa_backward", "stca_forward", "sa_forward_workspace_size",
+            "sa_backward_workspace_size", "stca_forward_workspace_size", "ska_status_string"} <= names
+
+
+def test_library_loads_and_exports_every_declared_call():
+    lib = L.lib()
+    names = header_functions()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert exported_symbols() == names, "libska.so exports exactly the header's calls"
+    assert set(L.EXPORTED) == names, "the binding wraps every declared call"
+
+
+def test_status_strings():
+    want = {L.SKA_OK: "SKA_OK", L.SKA_ERR_INVALID_VALUE: "SKA_ERR_INVALID_VALUE",
+            L.SKA_ERR_UNSUPPORTED: "SKA_ERR_UNSUPPORTED", L.SKA_ERR_WORKSPACE_TOO_SMALL: "SKA_ERR_WORKSPACE_TOO_SMALL",
+            L.SKA_ERR_CUDA: "SKA_ERR_CUDA", L.SKA_ERR_DEVICE_TIMEOUT: "SKA_ERR_DEVICE_TIMEOUT"}
+    for code, name in want.items():
+        assert L.status_string(code) == name
+    assert L.status_string(99) not in want.values()
+
+
+def sa_desc(**kw):
+    f = dict(num_users=2, num_heads=2, head_dim=64, num_protos=256, total_tokens=1000, max_seqlen=600, scale=1.0,
+             norm=L.SKA_NORM_PROTO, in_dtype=L.SKA_BF16, q_per_user=0, reserved=0)
+    f.update(kw)
+    return L.SaDesc(*[f[n] for n, _ in L.SaDesc._fields_])
+
+
+def stca_desc(**kw):
+    f = dict(num_users=2, num_heads=2, head_dim=64, num_sketch=256, total_targets=100, total_hist=1000,
+             max_targets=60, max_hist=600, scale=0.125, reserved=0)
+    f.update(kw)
+    return L.StcaDesc(*[f[n] for n, _ in L.StcaDesc._fields_])
+
+
+def fwd(desc, q=A, k=2 * A, v=3 * A, cu=4 * A, su=None, sk=5 * A, lse=6 * A, mass=None, ws=256 * A,
+        ws_bytes=1 << 30):
+    return L.lib().sa_forward(ctypes.byref(desc) if desc is not None else None, q, k, v, cu, su, sk, lse, mass, ws,
+                              ws_bytes, None)
+
+
+def bwd(desc, q=A, k=2 * A, v=3 * A, cu=4 * A, su=None, sk=5 * A, lse=6 * A, dsk=7 * A, dq=8 * A, dk=9 * A,
+        dv=10 * A, ws=256 * A, ws_bytes=1 << 30):
+    return L.lib().sa_backward(ctypes.byref(desc) if desc is not None else None, q, k, v, cu, su, sk, lse, dsk, dq,
+                               dk, dv, ws, ws_bytes, None)
+
+
+def stca(desc, q=A, cut=2 * A, kh=3 * A, vh=4 * A, cuh=5 * A, kvl=None, ks=6 * A, vs=7 * A, out=8 * A, lse=9 * A,
+         ws=256 * A, ws_bytes=1 << 30):
+    return L.lib().stca_forward(ctypes.byref(desc) if desc is not None else None, q, cut, kh, vh, cuh, kvl, ks, vs,
+                                out, lse, ws, ws_bytes, None)
+
+
+INVALID, UNSUP = L.SKA_ERR_INVALID_VALUE, L.SKA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw,code", [
+    ({"num_heads": 0}, INVALID), ({"num_users": -1}, INVALID), ({"total_tokens": -5}, INVALID),
+    ({"total_tokens": 1 << 31}, INVALID), ({"scale": 0.0}, INVALID), ({"scale": -1.0}, INVALID),
+    ({"scale": float("nan")}, INVALID), ({"scale": float("inf")}, INVALID), ({"norm": 7}, INVALID),
+    ({"in_dtype": 5}, INVALID), ({"q_per_user": 2}, INVALID), ({"num_protos": 0}, INVALID),
+    ({"head_dim": 96}, UNSUP), ({"head_dim": 256}, UNSUP),
+])
+def test_sa_forward_rejects_bad_descriptors(kw, code):
+    assert fwd(sa_desc(**kw)) == code
+
+
+def test_sa_forward_pointer_checks():
+    d = sa_desc()
+    assert fwd(None) == INVALID
+    assert fwd(d, mass=11 * A) == UNSUP  # the per-prototype mass output is not produced
+    assert fwd(d, q=None) == INVALID
+    assert fwd(d, k=None) == INVALID
+    assert fwd(d, sk=None) == INVALID
+    assert fwd(d, cu=None) == INVALID
+    assert fwd(d, ws=None) == INVALID
+    assert fwd(d, q=A + 8) == INVALID  # 16-byte alignment
+    assert fwd(d, ws=256 * A + 128) == INVALID  # 256-byte workspace alignment
+    assert fwd(d, cu=4 * A + 2) == INVALID
+
+
+def test_empty_batch_is_a_no_op_on_the_host():
+    # nothing to do: the call returns before any pointer or device check
+    assert fwd(sa_desc(num_users=0, total_tokens=0), q=None, k=None, v=None, cu=None, sk=None, ws=None) == L.SKA_OK
+    assert stca(stca_desc(total_targets=0), q=None, out=None, ws=None) == L.SKA_OK
+
+
+@pytest.mark.parametrize("kw,code", [
+    ({"in_dtype": L.SKA_F32}, UNSUP), ({"num_protos": 512}, UNSUP), ({"num_protos": 48}, UNSUP),
+    ({"head_dim": 128, "num_protos": 256}, UNSUP), ({"scale": 0.0}, INVALID), ({"norm": 3}, INVALID),
+])
+def test_sa_backward_rejects(kw, code):
+    assert bwd(sa_desc(**kw)) == code
+
+
+def test_sa_backward_pointer_checks():
+    d = sa_desc()
+    assert bwd(d, dq=None) == INVALID
+    assert bwd(d, dsk=None) == INVALID
+    assert bwd(d, lse=None) == INVALID
+    assert bwd(d, dk=None) == INVALID
+    assert bwd(sa_desc(norm=L.SKA_NORM_TOKEN), sk=None) == INVALID  # D_j needs the sketch
+    assert bwd(d, dv=10 * A + 4) == INVALID
+
+
+@pytest.mark.parametrize("kw,code", [
+    ({"num_heads": 0}, INVALID), ({"num_sketch": -1}, INVALID), ({"total_hist": -1}, INVALID),
+    ({"scale": 0.0}, INVALID), ({"head_dim": 32}, UNSUP),
+])
+def test_stca_rejects_bad_descriptors(kw, code):
+    assert stca(stca_desc(**kw)) == code
+
+
+def test_stca_pointer_checks():
+    d = stca_desc()
+    assert stca(None) == INVALID
+    assert stca(d, q=None) == INVALID
+    assert stca(d, kh=None) == INVALID
+    assert stca(d, ks=None) == INVALID
+    assert stca(stca_desc(num_sketch=0), ks=None, vs=None) != INVALID  # no sketch rows: no sketch pointers needed
+    assert stca(d, out=8 * A + 4) == INVALID
+    assert stca(d, kvl=2 * A + 2) == INVALID
+
+
+def test_valid_call_without_a_device_reports_cuda_error():
+    """Arguments that pass every host check reach the device query, which fails loudly here."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert fwd(sa_desc()) == L.SKA_ERR_CUDA
+    assert b"cudaGetDevice" in L.lib().ska_last_error_string()
+    assert bwd(sa_desc()) == L.SKA_ERR_CUDA
+    assert stca(stca_desc()) == L.SKA_ERR_CUDA
+    assert L.lib().sa_forward_workspace_size(ctypes.byref(sa_desc())) == 0
+
+
+def test_debug_and_timing_hooks_are_host_only():
+    lib = L.lib()
+    lib.ska_set_debug(1_000_000, 0)
+    lib.ska_set_debug(0, 0)  # back to the default budget
+    lib.ska_set_timing_events(None, None)
