@@ -25,6 +25,7 @@
 #include <cstdio>
 
 #include "ska_internal.h"
+#include "ska_proto_common.cuh"
 #include "ska_ptx.cuh"
 
 namespace ska {
@@ -40,10 +41,10 @@ constexpr int kSlotBytes = 16384;  // one [128 rows x 64 bf16] swizzled block
 constexpr int kMaxRing = 8;
 
 // Groups of four exponentials (out of every eight) computed on the FMA pipe by exp2_fma_pair
-// instead of MUFU. At d = 128 the MUFU time of a tile equals its MMA time, but in the present
-// pipeline the softmax is bound by its dependency chain, not by MUFU throughput: measured on
-// the 8 x 100K x 8-head workload, moving 3/8 of the exponentials to the FMA pipe made the
-// kernel slower (3.01 ms against 2.64 ms), so the split is off.
+// instead of MUFU. At d = 128 the MUFU time of a tile equals its MMA time, but in this pipeline
+// the softmax is bound by its dependency chain, not by MUFU throughput, and the longer unrolled
+// loop costs instruction fetches: on the 8 x 100K x 8-head workload the fused kernel took
+// 2.45 ms with no group on the FMA pipe, 2.65 ms with one and 2.77 ms with two, so it is off.
 constexpr int kExpFmaGroups = 0;
 __host__ __device__ constexpr bool exp_on_fma(int group4) { return (group4 & 7) < kExpFmaGroups; }
 
@@ -78,71 +79,26 @@ struct Bars {
   int abort_flag;
 };
 
-// Position in the concatenated tile stream: segment (b, h), tile j of user b.
-struct TilePos {
-  int b, h, j, nb;  // nb = tiles of user b
-  int g;            // global tile index
-};
-
-__device__ __forceinline__ int user_used(const ProtoFwdParams& p, int b) {
-  int len = p.cu_seqlens[b + 1] - p.cu_seqlens[b];
-  if (p.seqused) len = min(len, p.seqused[b]);
-  return max(len, 0);
-}
-
-__device__ __forceinline__ void tile_seek(const ProtoFwdParams& p, int g, TilePos& t) {
-  // largest b in [0, B) with H * prefix[b] <= g
-  int lo = 0, hi = p.B - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (p.H * p.tile_prefix[mid] <= g) lo = mid; else hi = mid - 1;
-  }
-  t.b = lo;
-  t.nb = p.tile_prefix[lo + 1] - p.tile_prefix[lo];
-  int off = g - p.H * p.tile_prefix[lo];
-  t.h = off / t.nb;
-  t.j = off - t.h * t.nb;
-  t.g = g;
-}
-
-__device__ __forceinline__ void tile_next(const ProtoFwdParams& p, TilePos& t) {
-  t.g++;
-  if (++t.j < t.nb) return;
-  t.j = 0;
-  if (++t.h < p.H) return;
-  t.h = 0;
-  do {
-    t.b++;
-    if (t.b >= p.B) return;
-    t.nb = p.tile_prefix[t.b + 1] - p.tile_prefix[t.b];
-  } while (t.nb == 0);
-}
-
-struct Waiter {
-  Bars* bars;
-  int* status;
-  uint64_t budget;
-  // Bounded wait; on timeout records the error and raises the CTA's abort flag. Unless
-  // `drain` is set, a raised abort flag ends the wait early; drains (waiting for this
-  // thread's own copies and MMAs in flight before exit) only end on completion or budget.
-  __device__ __forceinline__ bool operator()(uint64_t* bar, uint32_t parity, bool cluster_scope = false,
-                                             bool drain = false) {
-    volatile int* ab = &bars->abort_flag;
-    bool ok = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
-    if (ok) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-      ok = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
-      if (ok) return true;
-      if (!drain && *ab) return false;
-      if (globaltimer_ns() - t0 > budget) {
-        atomicCAS(status, 0, (int)SKA_ERR_DEVICE_TIMEOUT);
-        *ab = 1;
-        return false;
-      }
+// Segment epilogue (once per segment, kept out of line so that it does not crowd the softmax
+// loop's instructions): this warp's rows of O^T, NCOL prototype columns of TMEM starting at tO,
+// into the partial sketch dst[j * D + dd]. D = 128: lane row = channel; D = 64: lanes 0-15 of
+// each quarter hold the channels (M = 64 accumulator layout).
+template <int D, int NCOL>
+__device__ __noinline__ void drain_o(uint32_t tO, float* dst, int q4, int lane) {
+  tc_fence_after();
+  const int dd = (D == 128) ? q4 * 32 + lane : ((lane < 16) ? q4 * 16 + lane : -1);
+  for (int c = 0; c < NCOL; c += 8) {
+    float ov[8];
+    tmem_ld8(tO + c, reinterpret_cast<uint32_t*>(ov));
+    tmem_ld_wait();
+    if (dd >= 0) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) dst[(c + u) * D + dd] = ov[u];
     }
   }
-};
+  tc_fence_before();
+  __syncwarp();
+}
 
 template <int D, int KC>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -205,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tS = tbase;        // S^T: 128 lanes x KC columns
   const uint32_t tO = tbase + KC;   // O^T: D rows x KC columns
 
-  Waiter wait{&bars, &p.hdr->status, p.budget_ns};
+  Waiter wait{&bars.abort_flag, &p.hdr->status, p.budget_ns};
 
   const int total = p.hdr->total_tiles;
   const int W = p.hdr->tiles_per_cluster;
@@ -385,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       uint4* base = reinterpret_cast<uint4*>(sV + vent * KB * kSlotBytes);
       constexpr int kChunks = KB * kSlotBytes / 16;
-#pragma unroll 4
+#pragma unroll 8
       for (int c = ct; c < kChunks; c += kConvThreads) {
         uint4 w = base[c];
         w.x = bf16x2_to_f16x2(w.x);
@@ -494,14 +450,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         st_async_f32x2(mapa_shared(xbase + xoff, c), m2, lsum, mapa_shared(xbar_local[par], c));
       ok = __all_sync(0xffffffffu, wait(&bars.xbar[par], (i >> 1) & 1, true));
       if (!ok) break;
+      // (unrolled so that the loads of a row's entries are in flight together)
       float M = -INFINITY;
+#pragma unroll 4
       for (int c = 0; c < CS * 2; ++c) M = fmaxf(M, sX[(par * CS * 2 + c) * 128 + r].x);
       float Lsum = 0.f;
+#pragma unroll 4
       for (int c = 0; c < CS * 2; ++c) {
         const float2 e = sX[(par * CS * 2 + c) * 128 + r];
-        Lsum += e.y * ex2_approx(e.x - M);
+        Lsum = fmaf(e.y, ex2_approx(e.x - M), Lsum);
       }
-      const float f = valid ? ex2_approx(m2 - M) / Lsum : 0.f;
+      const float f = valid ? __fdividef(ex2_approx(m2 - M), Lsum) : 0.f;
       const uint64_t f2 = f2_pack(f, f);
 
       // P[tok, j] = A_{j,tok} as fp16 into the swizzled MN-major operand of MMA2.
@@ -531,28 +490,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&bars.pfull);
 
       if (p.lse && valid && g == 0 && rank == 0 && tok < p.total_tokens)
-        p.lse[static_cast<int64_t>(tok) * p.H + t.h] = (M + log2f(Lsum)) * 0.69314718055994531f;
+        p.lse[static_cast<int64_t>(tok) * p.H + t.h] = (M + __log2f(Lsum)) * 0.69314718055994531f;
 
       if (last) {
         // Segment epilogue: O^T (this CTA's KC prototypes) -> partial sketch slot.
         ok = __all_sync(0xffffffffu, wait(&bars.ofull, nseg & 1));
         if (!ok) break;
-        tc_fence_after();
         const int slot = (t.b * p.H + t.h) + cid;
-        float* dst = p.partial + (static_cast<int64_t>(slot) * p.k + rank * KC + col0) * D;
-        const int dd = (D == 128) ? r : ((lane < 16) ? q4 * 16 + lane : -1);
-#pragma unroll
-        for (int c = 0; c < NCOL; c += 8) {
-          float ov[8];
-          tmem_ld8(tO + lane_off + col0 + c, reinterpret_cast<uint32_t*>(ov));
-          tmem_ld_wait();
-          if (dd >= 0) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) dst[(c + u) * D + dd] = ov[u];
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
+        drain_o<D, NCOL>(tO + lane_off + col0, p.partial + (static_cast<int64_t>(slot) * p.k + rank * KC + col0) * D,
+                         q4, lane);
         if (lane == 0) mbar_arrive(&bars.ofree);
         ++nseg;
       }
