@@ -1,9 +1,16 @@
 #!/usr/bin/env python
-"""Benchmark of the FlashSA forward (Sketch Attention, SequenceO1 §3.1 / §4.4) on B200.
+"""Benchmark of the Sketch Attention hot path on B200 (SequenceO1 §3.1 SA, §4.4 FlashSA, §2.3 STCA).
 
-Default workload: 8 users x 100,000 history tokens, H=8 heads, d=128, k=512 prototypes,
-prototype-wise normalisation (the paper's Eq. (8)), bf16 inputs, fp32 sketch and per-token lse.
-One step = one sa_forward call (schedule, fused kernel, partial combine, lse padding fill).
+Default workload (the headline): the FlashSA forward on 8 users x 100,000 history tokens, H=8
+heads, d=128, k=512 prototypes, prototype-wise normalisation (the paper's Eq. (8)), bf16 inputs,
+fp32 sketch and per-token lse. One step = one sa_forward call (schedule, fused kernel, partial
+combine, lse fill). The other rows of the path run with --workload (same JSON contract):
+
+  sa_fwd_*                          one step = one sa_forward call (--norm proto|token)
+  sa_bwd_b64_ragged_h4_d64_k256     one step = one sa_backward call: 64 ragged users (1.45M
+                                    tokens), H=4, d=64, k=256 -> dQ, dK, dV (--norm proto|token)
+  stca_b16_t512_h4_d64_l10k_s256    one step = one stca_forward call: 16 users x 512 targets over
+                                    [10,000 suffix ; 256 sketch] keys, H=4, d=64
 
   python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--norm proto|token]
   python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
@@ -16,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import math
 import os
@@ -29,17 +37,27 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = "SA fwd history-tokens/s and TFLOP/s (fraction of B200 bf16 peak) at L=100K"
-UNIT = "history-tokens/s"
+METRICS = {
+    "sa_fwd": ("SA fwd history-tokens/s and TFLOP/s (fraction of B200 bf16 peak) at L=100K", "history-tokens/s"),
+    "sa_bwd": ("SA bwd history-tokens/s (dQ, dK, dV with A recomputed) and TFLOP/s", "history-tokens/s"),
+    "stca": ("STCA targets/s over [10K suffix ; 256 sketch] keys and TFLOP/s", "targets/s"),
+}
 
-# name -> (lengths or "ragged64", H, d, k, seqused, q_sigma_is_inv_sqrt_d)
+# name -> kind and shapes. lens: list, "ragged64" (64 users, log-uniform in [1K, 100K], seed 1) or
+# "paper" (8 users, N(85K, 10K) clipped to [1K, 100K], seed 5).
 WORKLOADS = {
-    "sa_fwd_b8_l100k_h8_d128_k512": ([100_000] * 8, 8, 128, 512, None),
-    "sa_fwd_b8_l100k_h8_d128_k512_masked": ([100_000] * 8, 8, 128, 512, [70_000] + [100_000] * 7),
-    "sa_fwd_b64_ragged_h4_d64_k256": ("ragged64", 4, 64, 256, None),
-    "sa_fwd_paper_h1_d128_k1024": ("paper", 1, 128, 1024, None),
+    "sa_fwd_b8_l100k_h8_d128_k512": dict(kind="sa_fwd", lens=[100_000] * 8, H=8, d=128, k=512, seqused=None),
+    "sa_fwd_b8_l100k_h8_d128_k512_masked": dict(kind="sa_fwd", lens=[100_000] * 8, H=8, d=128, k=512,
+                                                seqused=[70_000] + [100_000] * 7),
+    "sa_fwd_b64_ragged_h4_d64_k256": dict(kind="sa_fwd", lens="ragged64", H=4, d=64, k=256, seqused=None),
+    "sa_fwd_paper_h1_d128_k1024": dict(kind="sa_fwd", lens="paper", H=1, d=128, k=1024, seqused=None),
     # profiling size: same per-tile work as the headline, 205 MB of K+V (> L2), ~0.25 ms
-    "sa_fwd_b2_l100k_h2_d128_k512": ([100_000] * 2, 2, 128, 512, None),
+    "sa_fwd_b2_l100k_h2_d128_k512": dict(kind="sa_fwd", lens=[100_000] * 2, H=2, d=128, k=512, seqused=None),
+    "sa_bwd_b64_ragged_h4_d64_k256": dict(kind="sa_bwd", lens="ragged64", H=4, d=64, k=256, seqused=None),
+    # profiling size for the backward: 2 x 100K, one head, same per-tile work
+    "sa_bwd_b2_l100k_h1_d64_k256": dict(kind="sa_bwd", lens=[100_000] * 2, H=1, d=64, k=256, seqused=None),
+    "stca_b16_t512_h4_d64_l10k_s256": dict(kind="stca", users=16, targets=512, hist=10_000, ks=256, H=4, d=64,
+                                           scale=0.125),
 }
 DEFAULT_WORKLOAD = "sa_fwd_b8_l100k_h8_d128_k512"
 
@@ -54,7 +72,7 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def lengths_for(spec, rank):
+def lengths_for(spec):
     if isinstance(spec, list):
         return spec
     rng = np.random.default_rng(1 if spec == "ragged64" else 5)
@@ -64,22 +82,13 @@ def lengths_for(spec, rank):
     return [int(v) for v in np.clip(np.round(rng.normal(85_000, 10_000, 8)), 1000, 100_000)]
 
 
-def make_device_inputs(name, rank, device):
-    """Seeded synthetic inputs drawn on the device: K, V ~ N(0,1), Q ~ N(0,1)/sqrt(d), bf16."""
-    import torch
-    spec, H, d, kp, su = WORKLOADS[name]
-    lens = lengths_for(spec, rank)
-    T = sum(lens)
-    gen = torch.Generator(device=device)
-    gen.manual_seed(1000 + rank)
-    q = (torch.randn((H, kp, d), generator=gen, device=device) / math.sqrt(d)).bfloat16()
-    k = torch.randn((T, H, d), generator=gen, device=device, dtype=torch.bfloat16)
-    v = torch.randn((T, H, d), generator=gen, device=device, dtype=torch.bfloat16)
-    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=device)
-    seqused = torch.tensor(np.array(su, dtype=np.int32), device=device) if su else None
-    valid = sum(min(a, b) for a, b in zip(lens, su)) if su else T
-    return dict(q=q, k=k, v=v, cu=cu, seqused=seqused, lens=lens, H=H, d=d, k_protos=kp, valid=valid,
-                users=len(lens), scale=1.0)
+def oracle_threads():
+    from threadpoolctl import threadpool_info
+    return max([p.get("num_threads", 0) for p in threadpool_info()] or [0]) or os.cpu_count()
+
+
+def f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
 
 
 class ClockSampler:
@@ -124,78 +133,263 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(mine)}
 
 
-def cpu_baseline(inp, budget_s=12.0):
-    """The fp64 oracle (oracle/sa.py, as it stands) on whole (user, head) problems of the same
-    workload until about budget_s seconds of CPU work; returns history-tokens/s equivalents."""
-    import torch
-    import oracle
-    from threadpoolctl import threadpool_info
-    H = inp["H"]
-    cu = inp["cu"].cpu().numpy()
-    q = inp["q"].float().cpu().numpy().astype(np.float64)
-    done_tok = 0.0
-    pairs = 0
-    t0 = time.perf_counter()
-    b = 0
-    while True:
-        lo, hi = int(cu[b]), int(cu[b + 1])
-        h = pairs % H
-        kk = inp["k"][lo:hi, h].float().cpu().numpy().astype(np.float64)
-        vv = inp["v"][lo:hi, h].float().cpu().numpy().astype(np.float64)
-        ts = time.perf_counter()
-        oracle.sa_problem(q[h], kk, vv, inp["scale"], 0)
-        t_pair = time.perf_counter() - ts
-        done_tok += (hi - lo) / H
-        pairs += 1
-        b = (b + 1) % inp["users"]
-        if time.perf_counter() - t0 > budget_s or pairs >= 64:
-            break
-    elapsed_compute = time.perf_counter() - t0
-    threads = 0
-    for pool in threadpool_info():
-        threads = max(threads, pool.get("num_threads", 0))
-    return {"value": done_tok / elapsed_compute, "unit": UNIT, "cores": threads or os.cpu_count(),
-            "kind": "oracle",
-            "sample": f"{pairs} whole (user, head) problems of the workload, {done_tok:.0f} history-token "
-                      f"equivalents (tokens x heads done / H), fp64 numpy, {elapsed_compute:.1f} s incl. "
-                      f"host copies of the slices"}
+# ---------------------------------------------------------------------------------------- jobs
+# A job draws its seeded synthetic inputs on the device, runs one step through the public API on a
+# dict of device tensors (so that the end-to-end leg can run the same call on freshly copied
+# inputs), and states the step's units, algorithmic FLOPs and bytes, and its fused kernel.
+
+class SaFwdJob:
+    def __init__(self, spec, norm, rank, dev):
+        import torch
+        from sketch_attention_flashsa_b200 import api, flops
+        self.api, self.norm = api, norm
+        lens = lengths_for(spec["lens"])
+        H, d, kp = spec["H"], spec["d"], spec["k"]
+        T, B = sum(lens), len(lens)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1000 + rank)
+        su = spec["seqused"]
+        self.inputs = {
+            "q": (torch.randn((H, kp, d), generator=gen, device=dev) / math.sqrt(d)).bfloat16(),
+            "k": torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
+            "v": torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
+            "cu": torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=dev),
+        }
+        if su:
+            self.inputs["seqused"] = torch.tensor(np.array(su, dtype=np.int32), device=dev)
+        self.valid = sum(min(a, b) for a, b in zip(lens, su)) if su else T
+        self.B, self.H, self.d, self.kp = B, H, d, kp
+        desc = api.sa_desc(self.inputs["q"], self.inputs["k"], self.inputs["cu"], scale=1.0, norm=norm)
+        self.ws = torch.empty(api.sa_forward_workspace_size(desc), dtype=torch.uint8, device=dev)
+        self.sketch = torch.empty((B, H, kp, d), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((T, H) if norm == "proto" else (B, H, kp), dtype=torch.float32, device=dev)
+        self.units = self.valid
+        self.flops = flops.sa_forward_flops(self.valid, H, kp, d)
+        self.bytes = flops.sa_forward_bytes(self.valid, H, kp, d, B, norm=0 if norm == "proto" else 1)
+        self.kernel = "sa_proto_fwd_kernel" if norm == "proto" else "fa_fwd_kernel"
+        self.launches = 4 if norm == "proto" else 3
+        self.config = {"users_per_gpu": B, "heads": H, "head_dim": d, "protos": kp, "norm": norm,
+                       "valid_tokens_per_gpu": self.valid,
+                       "l2": "inputs larger than L2 (K and V are %.2f GB each per GPU)" % (T * H * d * 2 / 1e9)}
+
+    def run(self, x):
+        self.api.sa_forward(x["q"], x["k"], x["v"], x["cu"], x.get("seqused"), scale=1.0, norm=self.norm,
+                            workspace=self.ws, out=self.sketch, lse_out=self.lse)
+        return self.sketch
+
+    def oracle_sample(self, budget_s):
+        """Whole (user, head) problems of this workload through the oracle until about budget_s
+        seconds; returns (history-token equivalents done, seconds, description)."""
+        import oracle
+        cu = self.inputs["cu"].cpu().numpy()
+        q = f64(self.inputs["q"])
+        done, pairs, b, t0 = 0.0, 0, 0, time.perf_counter()
+        while time.perf_counter() - t0 < budget_s and pairs < 64:
+            lo, hi = int(cu[b]), int(cu[b + 1])
+            h = pairs % self.H
+            oracle.sa_problem(q[h], f64(self.inputs["k"][lo:hi, h]), f64(self.inputs["v"][lo:hi, h]), 1.0,
+                              0 if self.norm == "proto" else 1)
+            done += (hi - lo) / self.H
+            pairs += 1
+            b = (b + 1) % self.B
+        return done, time.perf_counter() - t0, f"{pairs} whole (user, head) problems, fp64 numpy"
+
+
+class SaBwdJob:
+    def __init__(self, spec, norm, rank, dev):
+        import torch
+        from sketch_attention_flashsa_b200 import api, flops
+        self.api, self.norm = api, norm
+        lens = lengths_for(spec["lens"])
+        H, d, kp = spec["H"], spec["d"], spec["k"]
+        T, B = sum(lens), len(lens)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(2000 + rank)
+        x = {
+            "q": (torch.randn((H, kp, d), generator=gen, device=dev) / math.sqrt(d)).bfloat16(),
+            "k": torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
+            "v": torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
+            "cu": torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=dev),
+            "dsketch": torch.randn((B, H, kp, d), generator=gen, device=dev, dtype=torch.bfloat16),
+        }
+        # the forward's saved statistics (and, token-wise, its sketch) are inputs of the backward
+        sk, lse, _ = api.sa_forward(x["q"], x["k"], x["v"], x["cu"], None, scale=1.0, norm=norm)
+        x["lse"] = lse
+        if norm == "token":
+            x["sketch"] = sk
+        self.inputs = x
+        self.valid, self.B, self.H, self.d, self.kp = T, B, H, d, kp
+        self.outs = (torch.empty_like(x["q"], dtype=torch.float32), torch.empty_like(x["k"], dtype=torch.float32),
+                     torch.empty_like(x["v"], dtype=torch.float32))
+        desc = api.sa_desc(x["q"], x["k"], x["cu"], scale=1.0, norm=norm)
+        self.ws = torch.empty(api.sa_backward_workspace_size(desc), dtype=torch.uint8, device=dev)
+        self.units = T
+        self.flops = flops.sa_backward_flops(T, H, kp, d)
+        # K, V read (bf16), dK, dV written (fp32), saved statistics, dSketch (and sketch), Q and dQ
+        self.bytes = (T * H * d * (2 + 2 + 4 + 4) + (T * H * 4 if norm == "proto" else B * H * kp * 4)
+                      + B * H * kp * d * (2 + (4 if norm == "token" else 0)) + H * kp * d * (2 + 4))
+        self.kernel = "sa_bwd_kernel"
+        self.launches = 4
+        self.config = {"users_per_gpu": B, "heads": H, "head_dim": d, "protos": kp, "norm": norm,
+                       "tokens_per_gpu": T, "outputs": "dQ, dK, dV fp32",
+                       "l2": "inputs larger than L2 (K and V are %.2f GB each per GPU)" % (T * H * d * 2 / 1e9)}
+
+    def run(self, x):
+        dq, _, _ = self.api.sa_backward(x["q"], x["k"], x["v"], x["cu"], None, x["lse"], x["dsketch"],
+                                        x.get("sketch"), scale=1.0, norm=self.norm, workspace=self.ws,
+                                        outs=self.outs)
+        return dq
+
+    def oracle_sample(self, budget_s):
+        import oracle
+        cu = self.inputs["cu"].cpu().numpy()
+        q, do = f64(self.inputs["q"]), f64(self.inputs["dsketch"])
+        nid = 0 if self.norm == "proto" else 1
+        done, users, t0 = 0.0, 0, time.perf_counter()
+        order = np.argsort(np.diff(cu))  # shortest users first, so that the sample stays bounded
+        for b in order:
+            if time.perf_counter() - t0 > budget_s or users >= 16:
+                break
+            lo, hi = int(cu[b]), int(cu[b + 1])
+            oracle.sa_backward(q, f64(self.inputs["k"][lo:hi]), f64(self.inputs["v"][lo:hi]), np.array([0, hi - lo]),
+                               None, do[b:b + 1], 1.0, nid)
+            done += hi - lo
+            users += 1
+        return done, time.perf_counter() - t0, f"{users} whole users (all heads, dQ dK dV), fp64 numpy"
+
+
+class StcaJob:
+    def __init__(self, spec, norm, rank, dev):
+        import torch
+        from sketch_attention_flashsa_b200 import api, flops
+        self.api = api
+        B, Tq, L, ks, H, d = spec["users"], spec["targets"], spec["hist"], spec["ks"], spec["H"], spec["d"]
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(3000 + rank)
+        x = {
+            "q": torch.randn((B * Tq, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
+            "cu_t": torch.arange(0, B * Tq + 1, Tq, dtype=torch.int32, device=dev),
+            "k_hist": torch.randn((B * L, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
+            "v_hist": torch.randn((B * L, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
+            "cu_h": torch.arange(0, B * L + 1, L, dtype=torch.int32, device=dev),
+            "k_sk": torch.randn((B, H, ks, d), generator=gen, device=dev, dtype=torch.bfloat16),
+            "v_sk": torch.randn((B, H, ks, d), generator=gen, device=dev, dtype=torch.bfloat16),
+        }
+        self.inputs, self.scale, self.Tq, self.B, self.H = x, spec["scale"], Tq, B, H
+        self.out = torch.empty((B * Tq, H, d), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((B * Tq, H), dtype=torch.float32, device=dev)
+        desc = api.stca_desc(x["q"], x["k_hist"], x["k_sk"], x["cu_t"], x["cu_h"], scale=self.scale, max_targets=Tq)
+        self.ws = torch.empty(max(api.stca_forward_workspace_size(desc), 256), dtype=torch.uint8, device=dev)
+        self.units = B * Tq
+        self.flops = flops.stca_forward_flops(B * Tq, L + ks, H, d)
+        self.bytes = B * Tq * H * d * (2 + 4) + B * Tq * H * 4 + 2 * B * L * H * d * 2 + 2 * B * H * ks * d * 2
+        self.kernel = "fa_fwd_kernel"
+        self.launches = 3
+        self.config = {"users_per_gpu": B, "targets_per_user": Tq, "suffix_keys": L, "sketch_keys": ks, "heads": H,
+                       "head_dim": d, "scale": self.scale,
+                       "l2": "inputs larger than L2 (suffix K and V are %.0f MB together per GPU)" % (
+                           2 * B * L * H * d * 2 / 1e6)}
+
+    def run(self, x):
+        out, _ = self.api.stca_forward(x["q"], x["cu_t"], x["k_hist"], x["v_hist"], x["cu_h"], x["k_sk"], x["v_sk"],
+                                       scale=self.scale, max_targets=self.Tq, workspace=self.ws, out=self.out,
+                                       lse_out=self.lse)
+        return out
+
+    def oracle_sample(self, budget_s):
+        import oracle
+        x = self.inputs
+        cut, cuh = x["cu_t"].cpu().numpy(), x["cu_h"].cpu().numpy()
+        done, users, t0 = 0.0, 0, time.perf_counter()
+        per_user = 64
+        while time.perf_counter() - t0 < budget_s and users < self.B:
+            b = users
+            rows = slice(int(cut[b]), int(cut[b]) + per_user)
+            oracle.stca_forward(f64(x["q"][rows]), np.array([0, per_user]), f64(x["k_hist"][cuh[b]:cuh[b + 1]]),
+                                f64(x["v_hist"][cuh[b]:cuh[b + 1]]), np.array([0, cuh[b + 1] - cuh[b]]),
+                                f64(x["k_sk"][b:b + 1]), f64(x["v_sk"][b:b + 1]), self.scale, None)
+            done += per_user
+            users += 1
+        return done, time.perf_counter() - t0, f"{per_user} targets of each of {users} users (all heads), fp64 numpy"
+
+
+JOBS = {"sa_fwd": SaFwdJob, "sa_bwd": SaBwdJob, "stca": StcaJob}
+
+
+def traffic_for(workload, norm):
+    """DRAM bytes per launch of the fused kernel from a committed ncu capture, or None when the
+    kernel source has changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        tr = json.load(f).get(workload, {}).get(norm)
+    if not tr:
+        return None
+    with open(os.path.join(ROOT, tr["source"]), "rb") as f:
+        cur = hashlib.sha256(f.read()).hexdigest()[:16]
+    return tr["bytes"] if cur == tr["source_sha256"] else None
 
 
 def run_reference(args, rank, world):
-    """--impl reference: the fp64 CPU oracle on the host cores, bounded samples per step."""
+    """--impl reference: the fp64 CPU oracle on the host cores, a bounded sample per step."""
     if rank != 0:
         return
-    import torch
-    name = args.workload
-    spec, H, d, kp, su = WORKLOADS[name]
-    lens = lengths_for(spec, 0)
-    rng = np.random.default_rng(2)
-    q = (rng.standard_normal((H, kp, d), dtype=np.float32) / math.sqrt(d))
-    q = torch.from_numpy(q).bfloat16().float().numpy().astype(np.float64)
-    import oracle
-    n = min(lens[0], 100_000)
-    kk = torch.from_numpy(rng.standard_normal((n, d), dtype=np.float32)).bfloat16().float().numpy().astype(np.float64)
-    vv = torch.from_numpy(rng.standard_normal((n, d), dtype=np.float32)).bfloat16().float().numpy().astype(np.float64)
-    for _ in range(args.warmup if args.warmup < 1 else 1):
-        oracle.sa_problem(q[0], kk[:1000], vv[:1000], 1.0, 0 if args.norm == "proto" else 1)
-    times = []
+    spec = WORKLOADS[args.workload]
+    metric, unit = METRICS[spec["kind"]]
+    job = _host_job(spec, args.norm)
+    budget = 4.0 if args.steps > 5 else 10.0
+    job.oracle_sample(0.01)  # warm-up: imports and first calls
+    times, units, desc = [], [], ""
     for _ in range(args.steps):
-        t0 = time.perf_counter()
-        oracle.sa_problem(q[0], kk, vv, 1.0, 0 if args.norm == "proto" else 1)
-        times.append(time.perf_counter() - t0)
-    tok_equiv = n / H
+        u, t, desc = job.oracle_sample(budget)
+        times.append(t)
+        units.append(u)
+    value = sum(units) / sum(times)
     ms = 1e3 * statistics.mean(times)
-    value = tok_equiv / (ms / 1e3)
-    from threadpoolctl import threadpool_info
-    threads = max([p.get("num_threads", 0) for p in threadpool_info()] or [os.cpu_count()])
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+    cores = oracle_threads()
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": name, "norm": args.norm, "sample": f"one (user, head) problem of {n} tokens per step"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": f"one whole (user, head) problem ({n} tokens, k={kp}, d={d}) per step"},
-            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "config": {"workload": args.workload, "norm": args.norm, "sample": desc},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": f"per step: {desc}, about {budget:.0f} s"},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def _host_job(spec, norm):
+    """A job's inputs drawn on the host, the same distributions, for the oracle alone (the
+    reference arm touches neither the GPU nor libska.so)."""
+    import types
+    import torch
+    g = torch.Generator().manual_seed(7)
+    job = types.SimpleNamespace()
+    if spec["kind"] == "stca":
+        B, Tq, L, ks, H, d = 2, 64, spec["hist"], spec["ks"], spec["H"], spec["d"]
+        job.inputs = {"q": torch.randn((B * Tq, H, d), generator=g).bfloat16(),
+                      "cu_t": torch.arange(0, B * Tq + 1, Tq, dtype=torch.int32),
+                      "k_hist": torch.randn((B * L, H, d), generator=g).bfloat16(),
+                      "v_hist": torch.randn((B * L, H, d), generator=g).bfloat16(),
+                      "cu_h": torch.arange(0, B * L + 1, L, dtype=torch.int32),
+                      "k_sk": torch.randn((B, H, ks, d), generator=g).bfloat16(),
+                      "v_sk": torch.randn((B, H, ks, d), generator=g).bfloat16()}
+        job.scale, job.B = spec["scale"], B
+        job.oracle_sample = types.MethodType(StcaJob.oracle_sample, job)
+        return job
+    lens = lengths_for(spec["lens"])
+    H, d, kp = spec["H"], spec["d"], spec["k"]
+    # a bounded sample: the shortest users of the workload, up to 4 of them
+    take = sorted(lens)[:4]
+    T = sum(take)
+    job.inputs = {"q": (torch.randn((H, kp, d), generator=g) / math.sqrt(d)).bfloat16(),
+                  "k": torch.randn((T, H, d), generator=g).bfloat16(), "v": torch.randn((T, H, d), generator=g).bfloat16(),
+                  "cu": torch.tensor(np.concatenate([[0], np.cumsum(take)]).astype(np.int32)),
+                  "dsketch": torch.randn((len(take), H, kp, d), generator=g).bfloat16()}
+    job.norm, job.H, job.B = norm, H, len(take)
+    cls = SaFwdJob if spec["kind"] == "sa_fwd" else SaBwdJob
+    job.oracle_sample = types.MethodType(cls.oracle_sample, job)
+    return job
 
 
 def main():
@@ -229,24 +423,19 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    from sketch_attention_flashsa_b200 import api, dp, flops
+    from sketch_attention_flashsa_b200 import api, dp
 
-    inp = make_device_inputs(args.workload, rank, dev)
-    H, d, kp, B = inp["H"], inp["d"], inp["k_protos"], inp["users"]
-    T = inp["k"].shape[0]
-    desc = api.sa_desc(inp["q"], inp["k"], inp["cu"], scale=inp["scale"], norm=args.norm)
-    ws = torch.empty(api.sa_forward_workspace_size(desc), dtype=torch.uint8, device=dev)
-    sketch = torch.empty((B, H, kp, d), dtype=torch.float32, device=dev)
-    lse = torch.empty((T, H) if args.norm == "proto" else (B, H, kp), dtype=torch.float32, device=dev)
+    spec = WORKLOADS[args.workload]
+    metric, unit = METRICS[spec["kind"]]
+    job = JOBS[spec["kind"]](spec, args.norm, rank, dev)
 
     def step():
-        api.sa_forward(inp["q"], inp["k"], inp["v"], inp["cu"], inp["seqused"], scale=inp["scale"],
-                       norm=args.norm, workspace=ws, out=sketch, lse_out=lse)
+        job.run(job.inputs)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    st = api.read_device_status(ws)
+    st = api.read_device_status(job.ws)
     if st != 0:
         raise SystemExit(f"device status {st} after warm-up")
 
@@ -277,64 +466,40 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms_total = e0.elapsed_time(e1)
     kern_ms = [a.elapsed_time(b) for a, b in kev]
-    ms_total, kern_mean = dp.max_over_ranks([ms_total, statistics.mean(kern_ms)], device=dev)
+    ms_total, kern_mean = dp.max_over_ranks([e0.elapsed_time(e1), statistics.mean(kern_ms)], device=dev)
     ms_per_step = ms_total / args.steps
-    valid = inp["valid"]
-    total_tokens_all = valid * world
-    value = total_tokens_all / (ms_per_step / 1e3)
-    fl = flops.sa_forward_flops(valid, H, kp, d)
-    by = flops.sa_forward_bytes(valid, H, kp, d, B, norm=0 if args.norm == "proto" else 1)
-    tflops = fl / (ms_per_step / 1e3) / 1e12
+    units_all = job.units * world
+    value = units_all / (ms_per_step / 1e3)
+    tflops = job.flops / (ms_per_step / 1e3) / 1e12
 
     peaks = load_peaks()
-    kname = "sa_proto_fwd_kernel" if args.norm == "proto" else "fa_fwd_kernel"
-    t_tensor = fl / (peaks["bf16_tflops"] * 1e12)
-    t_hbm = by / (peaks["hbm_gbs"] * 1e9)
-    bound = "tensor" if t_tensor >= t_hbm else "hbm"
-    if bound == "tensor":
-        achieved = fl / (kern_mean / 1e3) / 1e12
+    t_tensor = job.flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = job.bytes / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        achieved = job.flops / (kern_mean / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                "peak_source": f"{peaks['source']} bf16 dense (burst); sustained {peaks['bf16_tflops_sustained']}",
-                "kernel": kname, "kernel_ms": kern_mean}
+                "peak_source": f"{peaks['source']} bf16 dense (burst); sustained {peaks['bf16_tflops_sustained']}"}
     else:
-        achieved = by / (kern_mean / 1e3) / 1e9
+        achieved = job.bytes / (kern_mean / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
-                "kernel": kname, "kernel_ms": kern_mean}
-    traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(traffic_file):
-        import hashlib
-        with open(traffic_file) as f:
-            tr = json.load(f).get(args.workload, {}).get(args.norm)
-        if tr:
-            with open(os.path.join(ROOT, tr["source"]), "rb") as f:
-                cur = hashlib.sha256(f.read()).hexdigest()[:16]
-            # counters are only valid for the kernel source they were taken on
-            roof["traffic"] = tr["bytes"] if cur == tr["source_sha256"] else None
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"]}
+    roof.update({"kernel": job.kernel, "kernel_ms": kern_mean, "algorithmic_flops": job.flops,
+                 "algorithmic_bytes": job.bytes})
+    roof["traffic"] = traffic_for(args.workload, args.norm if spec["kind"] != "stca" else "stca")
 
-    # End to end through the public API: pinned host inputs -> device, forward, sketch -> host.
-    hq = inp["q"].cpu().pin_memory()
-    hk = inp["k"].cpu().pin_memory()
-    hv = inp["v"].cpu().pin_memory()
-    hcu = inp["cu"].cpu().pin_memory()
-    hsu = inp["seqused"].cpu().pin_memory() if inp["seqused"] is not None else None
-    hout = torch.empty(sketch.shape, dtype=torch.float32).pin_memory()
-    dq, dk, dv, dcu = (torch.empty_like(x) for x in (inp["q"], inp["k"], inp["v"], inp["cu"]))
-    dsu = torch.empty_like(inp["seqused"]) if hsu is not None else None
+    # End to end through the public API: pinned host inputs -> device, the call, result -> host.
+    host = {n: t.cpu().pin_memory() for n, t in job.inputs.items()}
+    devx = {n: torch.empty_like(t) for n, t in job.inputs.items()}
+    res = job.run(job.inputs)
+    hout = torch.empty(res.shape, dtype=res.dtype).pin_memory()
 
     def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        dcu.copy_(hcu, non_blocking=True)
-        if dsu is not None:
-            dsu.copy_(hsu, non_blocking=True)
-        api.sa_forward(dq, dk, dv, dcu, dsu, scale=inp["scale"], norm=args.norm, workspace=ws, out=sketch,
-                       lse_out=lse)
-        hout.copy_(sketch, non_blocking=True)
+        for n in host:
+            devx[n].copy_(host[n], non_blocking=True)
+        r = job.run(devx)
+        hout.copy_(r, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -347,27 +512,25 @@ def main():
     f1.record()
     torch.cuda.synchronize()
     te = dp.max_over_ranks([f0.elapsed_time(f1) / args.e2e_steps], device=dev)
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hcu) + ((hsu,) if hsu is not None else ()))
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = hout.numel() * hout.element_size()
-    e2e = {"value": total_tokens_all / (float(te[0]) / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": float(te[0])}
+    e2e = {"value": units_all / (te[0] / 1e3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": te[0], "result_read_back": list(hout.shape)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(inp)
+        done, secs, desc = job.oracle_sample(12.0)
+        cpu = {"value": done / secs, "unit": unit, "cores": oracle_threads(), "kind": "oracle",
+               "sample": f"{desc}, {secs:.1f} s incl. host copies of the slices"}
 
-    launches_per_step = 3 + (1 if lse is not None else 0)
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": args.workload, "norm": args.norm, "users_per_gpu": B, "heads": H,
-                           "head_dim": d, "protos": kp, "valid_tokens_per_gpu": valid,
-                           "l2": "inputs larger than L2 (K and V are %.2f GB each per GPU)" % (
-                               inp["k"].numel() * 2 / 1e9),
+                "config": {"workload": args.workload, **job.config,
                            "parallelism": f"dp{world} (independent users per rank)"},
                 "tflops": tflops, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
+                "gpu_launches": job.launches * args.steps, "clocks": clocks}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -134,12 +134,14 @@ def stca_forward_workspace_size(desc: StcaDesc) -> int:
 def stca_forward(q: torch.Tensor, cu_targets: torch.Tensor, k_hist: torch.Tensor, v_hist: torch.Tensor,
                  cu_hist: torch.Tensor, k_sk: Optional[torch.Tensor], v_sk: Optional[torch.Tensor], *,
                  scale: float, target_kv_len: Optional[torch.Tensor] = None, want_lse: bool = True,
-                 max_targets: Optional[int] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+                 max_targets: Optional[int] = None, workspace: Optional[torch.Tensor] = None, stream=None,
+                 out: Optional[torch.Tensor] = None, lse_out: Optional[torch.Tensor] = None):
     """STCA forward (SequenceO1 §2.3; the suffix and sketch branches of §3.4; MRLB §4.2).
 
     q [Tq,H,d] bf16 with cu_targets int32 [B+1]; k_hist, v_hist [Th,H,d] bf16 with cu_hist;
     k_sk, v_sk [B,H,ks,d] bf16 or None; target_kv_len int32 [Tq] or None; max_targets: an upper
-    bound on any user's target count (read from cu_targets when None).
+    bound on any user's target count (read from cu_targets when None, which synchronises);
+    out / lse_out: preallocated outputs (fp32 [Tq,H,d] / [Tq,H]).
     Returns (out fp32 [Tq,H,d], lse fp32 [Tq,H] or None).
     """
     if max_targets is None:
@@ -155,8 +157,13 @@ def stca_forward(q: torch.Tensor, cu_targets: torch.Tensor, k_hist: torch.Tensor
         raise SkaError(_lib.SKA_ERR_UNSUPPORTED, "stca_forward_workspace_size")
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
-    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev) if want_lse else None
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev) if out is None else out
+    if want_lse:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev) if lse_out is None else lse_out
+    else:
+        lse = None
+    _dev_tensor("out", out, (torch.float32,))
+    _dev_tensor("lse_out", lse, (torch.float32,))
     rc = _lib.lib().stca_forward(ctypes.byref(desc), _ptr(q), _ptr(cu_targets), _ptr(k_hist), _ptr(v_hist),
                                  _ptr(cu_hist), _ptr(target_kv_len), _ptr(k_sk), _ptr(v_sk), _ptr(out),
                                  _ptr(lse), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
@@ -164,13 +171,18 @@ def stca_forward(q: torch.Tensor, cu_targets: torch.Tensor, k_hist: torch.Tensor
     return out, lse
 
 
+def sa_backward_workspace_size(desc: SaDesc) -> int:
+    return int(_lib.lib().sa_backward_workspace_size(ctypes.byref(desc)))
+
+
 def sa_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
                 seqused: Optional[torch.Tensor], lse: torch.Tensor, dsketch: torch.Tensor,
                 sketch: Optional[torch.Tensor] = None, *, scale: float = 1.0, norm="proto",
-                workspace: Optional[torch.Tensor] = None, stream=None):
+                workspace: Optional[torch.Tensor] = None, stream=None, outs=None):
     """SA backward (gradients of <dsketch, sketch> through SequenceO1 §3.1 Eq. (7)-(9)).
 
-    bf16 q, k, v, dsketch; the forward's lse (and, for norm="token", its sketch).
+    bf16 q, k, v, dsketch; the forward's lse (and, for norm="token", its sketch); outs: an
+    optional preallocated (dq, dk, dv).
     Returns (dq fp32 shaped like q, dk fp32 [T,H,d], dv fp32 [T,H,d]).
     """
     for name, t in (("q", q), ("k", k), ("v", v), ("dsketch", dsketch)):
@@ -181,14 +193,19 @@ def sa_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: t
     _dev_tensor("seqused", seqused, (torch.int32,))
     desc = sa_desc(q, k, cu_seqlens, scale=scale, norm=norm)
     dev = k.device
-    need = int(_lib.lib().sa_backward_workspace_size(ctypes.byref(desc)))
+    need = sa_backward_workspace_size(desc)
     if need == 0:
         raise SkaError(_lib.SKA_ERR_UNSUPPORTED, "sa_backward_workspace_size")
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
-    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
-    dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    if outs is None:
+        outs = (torch.empty(q.shape, dtype=torch.float32, device=dev), torch.empty(k.shape, dtype=torch.float32,
+                device=dev), torch.empty(v.shape, dtype=torch.float32, device=dev))
+    dq, dk, dv = outs
+    for name, t, like in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        _dev_tensor(name, t, (torch.float32,))
+        if t.shape != like.shape:
+            raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(like.shape)}")
     rc = _lib.lib().sa_backward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(seqused),
                                 _ptr(sketch), _ptr(lse), _ptr(dsketch), _ptr(dq), _ptr(dk), _ptr(dv),
                                 _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
