@@ -4,16 +4,19 @@
 // Per 128-token tile of one (user, head), one CTA holding all k <= 256 prototypes, tokens on
 // TMEM lanes (S^T orientation):
 //   MMA  S^T  = K . Q^T                        -> A = exp(scale s - lse) (PROTO: per-token lse;
-//                                                 TOKEN: per-prototype lse), A as bf16 to smem
-//   MMA  dV   = A^T . dO        (M=tok, N=d)   -> TMEM
+//                                                 TOKEN: per-prototype lse), to smem as a bf16
+//                                                 pair hi + lo (16 significant bits)
+//   MMA  dV   = A^T . dO        (M=tok, N=d)   -> TMEM, both halves of the pair
 //   MMA  dA^T = V . dO^T        (M=tok, N=k)   -> TMEM (over S^T)
-//   softmax-gradient: PROTO dS = A (dA - delta_i) with delta_i = dV_i . v_i (equal to
-//        sum_j A_ji dA_ji, so no reduction over prototypes is needed); TOKEN dS = A (dA - D_j)
-//        with D_j = dO_j . O_j from the forward sketch. dS goes to smem as a bf16 pair
-//        hi + lo (hi = bf16(dS), lo = bf16(dS - hi)), 16 significant bits.
-//   MMA  dK   = dS^T . Q        (M=tok, N=d)   -> TMEM, scaled by `scale` on the way out
-//   MMA  dQ  += dS . K          (M=proto, N=d) -> TMEM, accumulated over the CTA's tiles of one
-//        segment with both halves of the pair; written to a partial slot at segment end.
+//   softmax-gradient: PROTO dS = A (dA - delta_i) with delta_i = sum_j A_ji dA_ji in fp32 (each
+//        warpgroup sums its half of the prototypes, the halves are added in a fixed order);
+//        TOKEN dS = A (dA - D_j) with D_j = dO_j . O_j from the forward sketch. dS goes to smem
+//        as a bf16 pair hi + lo.
+//   MMA  dK   = dS^T . Q        (M=tok, N=d)   -> TMEM, both halves, scaled on the way out
+//   MMA  dQ  += dS . K          (M=proto, N=d) -> TMEM, both halves; restarted every 8 tiles and
+//        added into the CTA's partial slot (the tensor core's fp32 accumulation is not
+//        round-to-nearest, so one chain over a whole segment would drift); a second kernel sums
+//        the partial slots of every prototype set in a fixed order.
 // Warps 0-7 (two warpgroups, each owning half of the prototype columns) do the elementwise
 // work; thread 0 also issues the TMA loads and MMAs. The phases of a tile run one after another.
 #include <algorithm>
