@@ -70,7 +70,7 @@ __host__ __device__ inline BwdLayout bwd_layout(int D, int k) {
 __host__ __device__ inline int bwd_tmem_cols(int D, int k) { return k + 2 * D + ((k + 127) / 128) * D; }
 
 struct BwdBars {
-  uint64_t ld, qd, m1, a, m2, ds, m3, out, drain, dready, dl;
+  uint64_t ldk, ldv, qd, m1, a, m2, ds, m3, drain, dready, dl;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -169,14 +169,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* sDj = reinterpret_cast<float*>(smem + L.d_off);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(&bars.ld, 1);
+    mbar_init(&bars.ldk, 1);
+    mbar_init(&bars.ldv, 1);
     mbar_init(&bars.qd, 1);
     mbar_init(&bars.m1, 1);
     mbar_init(&bars.m2, 1);
     mbar_init(&bars.m3, 1);
     mbar_init(&bars.a, kBwdWarps);
     mbar_init(&bars.ds, kBwdWarps);
-    mbar_init(&bars.out, kBwdWarps);
     mbar_init(&dready, kBwdWarps);
     mbar_init(&bars.dl, kBwdWarps);
     mbar_init(&bars.drain, 1);
@@ -209,6 +209,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t loff = static_cast<uint32_t>(q4 * 32) << 16;
   const float L2E = 1.4426950408889634f;
   const float c2 = p.scale * L2E;
+  int nk_issued = 0, nv_issued = 0, nq_issued = 0;  // fills requested (thread 0)
+  int nk_seen = 0, nv_seen = 0;                        // fills waited for
+  auto load_qdo = [&](const BwdPos& u) {
+    ++nq_issued;
+    const int qrow = (p.q_per_user ? u.b * p.H * p.k : 0) + u.h * p.k;
+    const int orow = (u.b * p.H + u.h) * p.k;
+    mbar_expect_tx(&bars.qd, 2 * KB * KP * 128);
+    for (int kb = 0; kb < KB; ++kb) {
+      tma_load_2d(sQ + kb * QBLK, &mapQ, &bars.qd, kb * 64, qrow);
+      tma_load_2d(sDO + kb * QBLK, &mapDO, &bars.qd, kb * 64, orow);
+    }
+  };
+  auto load_k = [&](const BwdPos& u) {
+    ++nk_issued;
+    const int row = p.cu_seqlens[u.b] + u.j * 128;
+    mbar_expect_tx(&bars.ldk, KB * kBlk);
+    for (int kb = 0; kb < KB; ++kb) tma_load_2d(sK + kb * kBlk, &mapK, &bars.ldk, u.h * D + kb * 64, row);
+  };
+  auto load_v = [&](const BwdPos& u) {
+    ++nv_issued;
+    const int row = p.cu_seqlens[u.b] + u.j * 128;
+    mbar_expect_tx(&bars.ldv, KB * kBlk);
+    for (int kb = 0; kb < KB; ++kb) tma_load_2d(sV + kb * kBlk, &mapV, &bars.ldv, u.h * D + kb * 64, row);
+  };
   BwdPos t;
   if (ntiles > 0) bwd_seek(p, g0, t);
   int nseg = 0;
@@ -226,21 +250,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int tok0 = p.cu_seqlens[t.b] + t.j * 128;
     const int tok = tok0 + r;
     const bool valid = (t.j * 128 + r) < used;
-    if (ctl) {
-      if (first) {
-        const int qrow = (p.q_per_user ? t.b * p.H * p.k : 0) + t.h * p.k;
-        const int orow = (t.b * p.H + t.h) * p.k;
-        mbar_expect_tx(&bars.qd, 2 * KB * KP * 128);
-        for (int kb = 0; kb < KB; ++kb) {
-          tma_load_2d(sQ + kb * QBLK, &mapQ, &bars.qd, kb * 64, qrow);
-          tma_load_2d(sDO + kb * QBLK, &mapDO, &bars.qd, kb * 64, orow);
-        }
-      }
-      mbar_expect_tx(&bars.ld, 2 * KB * kBlk);
-      for (int kb = 0; kb < KB; ++kb) {
-        tma_load_2d(sK + kb * kBlk, &mapK, &bars.ld, t.h * D + kb * 64, tok0);
-        tma_load_2d(sV + kb * kBlk, &mapV, &bars.ld, t.h * D + kb * 64, tok0);
-      }
+    // this row's lse, requested before the waits (PROTO)
+    const float lrow = (p.norm == SKA_NORM_PROTO && valid) ? p.lse[static_cast<int64_t>(tok) * p.H + t.h] * L2E : 0.f;
+    if (ctl && i == 0) {  // later tiles' loads are issued as soon as the previous tile frees the buffers
+      load_qdo(t);
+      load_v(t);
+      load_k(t);
     }
     if (first && p.norm == SKA_NORM_TOKEN) {
       // per-prototype lse (log2 units) and D_j = dO_j . O_j of this (user, head)
@@ -257,7 +272,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, wait(&dready, nseg & 1));
       if (!ok) break;
     }
-    ok = __all_sync(0xffffffffu, wait(&bars.ld, i & 1) && (!first || wait(&bars.qd, nseg & 1)));
+    ok = __all_sync(0xffffffffu, wait(&bars.ldk, i & 1) && wait(&bars.ldv, i & 1) &&
+                                     (!first || wait(&bars.qd, nseg & 1)));
+    nk_seen = nv_seen = i + 1;
     if (!ok) break;
     if (ctl) {
       tc_fence_after();
@@ -277,7 +294,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int c = 0; c < NCOL; c += 8) tmem_ld8(tb + loff + col0 + c, sv + c);
       tmem_ld_wait();
-      const float lrow = (p.norm == SKA_NORM_PROTO && valid) ? p.lse[static_cast<int64_t>(tok) * p.H + t.h] * L2E : 0.f;
 #pragma unroll
       for (int c = 0; c < NCOL; ++c) {
         const float l2 = (p.norm == SKA_NORM_PROTO) ? lrow : sLse[col0 + c];
@@ -324,18 +340,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     ok = __all_sync(0xffffffffu, wait(&bars.m2, i & 1));
     if (!ok) break;
     tc_fence_after();
+    BwdPos tn = t;  // the next tile of this CTA
+    if (i + 1 < ntiles) bwd_next(p, tn);
+    if (ctl && i + 1 < ntiles) load_v(tn);  // the MMAs reading V are complete
     // PROTO: delta_i = sum_j A_ij dA_ij in fp32; each warpgroup sums its half of the
     // prototypes and the two halves are added in a fixed order
     float delta = 0.f;
     if (p.norm == SKA_NORM_PROTO) {
       float part = 0.f;
 #pragma unroll
-      for (int c = 0; c < NCOL; c += 8) {
-        uint32_t da[8];
-        tmem_ld8(tb + loff + col0 + c, da);
+      for (int c = 0; c < NCOL; c += 16) {
+        uint32_t da[16];
+        if constexpr (NCOL >= 16) {
+          tmem_ld16(tb + loff + col0 + c, da);
+        } else {
+          tmem_ld8(tb + loff + col0 + c, da);
+        }
         tmem_ld_wait();
 #pragma unroll
-        for (int u = 0; u < 8; ++u) part = fmaf(a[c + u], __uint_as_float(da[u]), part);
+        for (int u = 0; u < (NCOL >= 16 ? 16 : 8); ++u) part = fmaf(a[c + u], __uint_as_float(da[u]), part);
       }
       sDl[wg * 128 + r] = part;
       __syncwarp();
@@ -345,28 +368,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       delta = sDl[r] + sDl[128 + r];
     }
     // dS = A (dA - delta) as a bf16 pair hi + lo
+    constexpr int DC = (NCOL >= 16) ? 16 : 8;  // columns per TMEM round trip
 #pragma unroll
-    for (int c = 0; c < NCOL; c += 8) {
-      uint32_t da[8];
-      tmem_ld8(tb + loff + col0 + c, da);
-      tmem_ld_wait();
-      float hi[8], lo[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float sub = (p.norm == SKA_NORM_PROTO) ? delta : sDj[col0 + c + u];
-        const float ds = a[c + u] * (__uint_as_float(da[u]) - sub);
-        hi[u] = __bfloat162float(__float2bfloat16_rn(ds));
-        lo[u] = ds - hi[u];
+    for (int c0 = 0; c0 < NCOL; c0 += DC) {
+      uint32_t da[DC];
+      if constexpr (DC == 16) {
+        tmem_ld16(tb + loff + col0 + c0, da);
+      } else {
+        tmem_ld8(tb + loff + col0 + c0, da);
       }
-      const int jj = col0 + c;
-      uint4 wh, wl;
-      wh.x = pack_bf16x2(hi[0], hi[1]); wh.y = pack_bf16x2(hi[2], hi[3]);
-      wh.z = pack_bf16x2(hi[4], hi[5]); wh.w = pack_bf16x2(hi[6], hi[7]);
-      wl.x = pack_bf16x2(lo[0], lo[1]); wl.y = pack_bf16x2(lo[2], lo[3]);
-      wl.z = pack_bf16x2(lo[4], lo[5]); wl.w = pack_bf16x2(lo[6], lo[7]);
-      const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
-      *reinterpret_cast<uint4*>(sA + off) = wh;
-      *reinterpret_cast<uint4*>(sLo + off) = wl;
+      tmem_ld_wait();
+#pragma unroll
+      for (int h8 = 0; h8 < DC; h8 += 8) {
+        const int c = c0 + h8;
+        float hi[8], lo[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float sub = (p.norm == SKA_NORM_PROTO) ? delta : sDj[col0 + c + u];
+          const float ds = a[c + u] * (__uint_as_float(da[h8 + u]) - sub);
+          hi[u] = __bfloat162float(__float2bfloat16_rn(ds));
+          lo[u] = ds - hi[u];
+        }
+        const int jj = col0 + c;
+        uint4 wh, wl;
+        wh.x = pack_bf16x2(hi[0], hi[1]); wh.y = pack_bf16x2(hi[2], hi[3]);
+        wh.z = pack_bf16x2(hi[4], hi[5]); wh.w = pack_bf16x2(hi[6], hi[7]);
+        wl.x = pack_bf16x2(lo[0], lo[1]); wl.y = pack_bf16x2(lo[2], lo[3]);
+        wl.z = pack_bf16x2(lo[4], lo[5]); wl.w = pack_bf16x2(lo[6], lo[7]);
+        const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
+        *reinterpret_cast<uint4*>(sA + off) = wh;
+        *reinterpret_cast<uint4*>(sLo + off) = wl;
+      }
     }
     fence_async_shared();
     tc_fence_before();
@@ -399,7 +431,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     ok = __all_sync(0xffffffffu, wait(&bars.m3, i & 1));
     if (!ok) break;
     tc_fence_after();
-    // dK (scaled) and dV rows: warpgroup wg writes channels [wg D/2, (wg+1) D/2)
+    if (ctl && i + 1 < ntiles) {  // every MMA of this tile is complete: K, Q and dO are free
+      if (tn.j == 0) load_qdo(tn);
+      load_k(tn);
+    }
+    // dK (scaled) and dV rows: warpgroup wg holds channels [wg D/2, (wg+1) D/2) of token row r.
+    // With 64 or more prototype columns per warpgroup the rows go out coalesced: each warp stages
+    // its 32 rows x 32 channels (128 B a row) in the part of A hi / A lo that only it writes, and
+    // reads them back so that one store covers four whole 128-byte rows.
+    const int urows = (p.cu_seqlens[t.b + 1] - p.cu_seqlens[t.b]) - t.j * 128;  // this user's rows in the tile
+    uint8_t* stk = sA + wg * (NCOL / 64) * kBlk + q4 * 32 * 128;   // this warp's staging (dK)
+    uint8_t* stv = sLo + wg * (NCOL / 64) * kBlk + q4 * 32 * 128;  // (dV)
+    auto stage_row = [&](uint8_t* st, const uint32_t* v, float mul) {  // lane's 32 floats -> row `lane`
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<float4*>(st + lane * 128 + ((ch ^ (lane & 7)) << 4)) =
+            make_float4(mul * __uint_as_float(v[4 * ch]), mul * __uint_as_float(v[4 * ch + 1]),
+                        mul * __uint_as_float(v[4 * ch + 2]), mul * __uint_as_float(v[4 * ch + 3]));
+    };
+    auto staged = [&](const uint8_t* st, int u) -> float4 {  // row 4u + lane/8, chunk lane%8
+      const int rho = 4 * u + (lane >> 3);
+      return *reinterpret_cast<const float4*>(st + rho * 128 + (((lane & 7) ^ (rho & 7)) << 4));
+    };
 #pragma unroll
     for (int c = 0; c < D / 2; c += 32) {
       const int cc = wg * (D / 2) + c;
@@ -407,60 +460,100 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_ld32(tb + loff + CK + cc, kr);
       tmem_ld32(tb + loff + CV + cc, vr);
       tmem_ld_wait();
-      if (tok < p.total_tokens && (t.j * 128 + r) < (p.cu_seqlens[t.b + 1] - p.cu_seqlens[t.b])) {
-        float* dk = p.dk + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
-        float* dv = p.dv + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
+      if constexpr (NCOL >= 64) {
+        stage_row(stk, kr, p.scale);
+        stage_row(stv, vr, 1.f);
+        __syncwarp();
 #pragma unroll
-        for (int u = 0; u < 32; u += 4) {
-          *reinterpret_cast<float4*>(dk + u) =
-              make_float4(p.scale * __uint_as_float(kr[u]), p.scale * __uint_as_float(kr[u + 1]),
-                          p.scale * __uint_as_float(kr[u + 2]), p.scale * __uint_as_float(kr[u + 3]));
-          *reinterpret_cast<float4*>(dv + u) = make_float4(__uint_as_float(vr[u]), __uint_as_float(vr[u + 1]),
-                                                           __uint_as_float(vr[u + 2]), __uint_as_float(vr[u + 3]));
+        for (int u = 0; u < 8; ++u) {
+          const int row = q4 * 32 + 4 * u + (lane >> 3);  // token row in the tile
+          const int64_t tk = static_cast<int64_t>(tok0) + row;
+          if (row < urows && tk < p.total_tokens) {
+            const int64_t off = (tk * p.H + t.h) * D + cc + (lane & 7) * 4;
+            *reinterpret_cast<float4*>(p.dk + off) = staged(stk, u);
+            *reinterpret_cast<float4*>(p.dv + off) = staged(stv, u);
+          }
+        }
+        __syncwarp();
+      } else {
+        if (tok < p.total_tokens && (t.j * 128 + r) < (p.cu_seqlens[t.b + 1] - p.cu_seqlens[t.b])) {
+          float* dk = p.dk + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
+          float* dv = p.dv + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) {
+            *reinterpret_cast<float4*>(dk + u) =
+                make_float4(p.scale * __uint_as_float(kr[u]), p.scale * __uint_as_float(kr[u + 1]),
+                            p.scale * __uint_as_float(kr[u + 2]), p.scale * __uint_as_float(kr[u + 3]));
+            *reinterpret_cast<float4*>(dv + u) = make_float4(__uint_as_float(vr[u]), __uint_as_float(vr[u + 1]),
+                                                             __uint_as_float(vr[u + 2]), __uint_as_float(vr[u + 3]));
+          }
         }
       }
     }
     if (flush && wg < QBLOCKS) {
-      // dQ block wg (prototypes 128 wg + r) of this segment, scaled, into its partial slot;
-      // only this CTA writes the slot, and each element always by the same thread
-      const int jrow = wg * 128 + r;
+      // dQ block wg (prototypes 128 wg + r) of this segment, scaled, into its partial slot; only
+      // this CTA writes the slot, and each element always by the same warp. Staged like dK.
       const int slot = (t.b * p.H + t.h) + static_cast<int>(blockIdx.x);
       const bool add = segt >= kDqFlush;
+      float* qbase = p.dq_partial + (static_cast<int64_t>(slot) * p.k + wg * 128) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t qr[32];
         tmem_ld32(tb + loff + CQ + wg * D + c, qr);
         tmem_ld_wait();
-        if (jrow < p.k) {
-          float* dst = p.dq_partial + (static_cast<int64_t>(slot) * p.k + jrow) * D + c;
+        if constexpr (NCOL >= 64) {
+          stage_row(stk, qr, p.scale);
+          __syncwarp();
 #pragma unroll
-          for (int u = 0; u < 32; u += 4) {
-            float4 o = make_float4(p.scale * __uint_as_float(qr[u]), p.scale * __uint_as_float(qr[u + 1]),
-                                   p.scale * __uint_as_float(qr[u + 2]), p.scale * __uint_as_float(qr[u + 3]));
-            if (add) {
-              const float4 prev = *reinterpret_cast<const float4*>(dst + u);
-              o.x += prev.x;
-              o.y += prev.y;
-              o.z += prev.z;
-              o.w += prev.w;
+          for (int u = 0; u < 8; ++u) {
+            const int row = q4 * 32 + 4 * u + (lane >> 3);  // prototype within the block
+            if (wg * 128 + row < p.k) {
+              float4* dst = reinterpret_cast<float4*>(qbase + static_cast<int64_t>(row) * D + c + (lane & 7) * 4);
+              float4 o = staged(stk, u);
+              if (add) {
+                const float4 prev = *dst;
+                o.x += prev.x;
+                o.y += prev.y;
+                o.z += prev.z;
+                o.w += prev.w;
+              }
+              *dst = o;
             }
-            *reinterpret_cast<float4*>(dst + u) = o;
+          }
+          __syncwarp();
+        } else {
+          const int jrow = wg * 128 + r;
+          if (jrow < p.k) {
+            float* dst = qbase + static_cast<int64_t>(r) * D + c;
+#pragma unroll
+            for (int u = 0; u < 32; u += 4) {
+              float4 o = make_float4(p.scale * __uint_as_float(qr[u]), p.scale * __uint_as_float(qr[u + 1]),
+                                     p.scale * __uint_as_float(qr[u + 2]), p.scale * __uint_as_float(qr[u + 3]));
+              if (add) {
+                const float4 prev = *reinterpret_cast<const float4*>(dst + u);
+                o.x += prev.x;
+                o.y += prev.y;
+                o.z += prev.z;
+                o.w += prev.w;
+              }
+              *reinterpret_cast<float4*>(dst + u) = o;
+            }
           }
         }
       }
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars.out);
-    // the next tile's loads overwrite K, V (and Q, dO): every role must be done with them
-    ok = __all_sync(0xffffffffu, wait(&bars.out, i & 1));
-    if (!ok) break;
     if (first) ++nseg;
-    bwd_next(p, t);
+    t = tn;
   }
   if (ctl) {
     umma_commit(&bars.drain);  // completes when every MMA issued above has
     wait(&bars.drain, 0, true);
+    // on an early exit, loads issued for a tile that was not reached must land first
+    if (nk_issued > nk_seen) wait(&bars.ldk, (nk_issued - 1) & 1, true);
+    if (nv_issued > nv_seen) wait(&bars.ldv, (nv_issued - 1) & 1, true);
+    if (nq_issued > nseg) wait(&bars.qd, (nq_issued - 1) & 1, true);
   }
   tc_fence_before();
   __syncthreads();
