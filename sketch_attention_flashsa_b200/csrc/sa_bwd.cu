@@ -32,7 +32,7 @@ namespace {
 constexpr int kBwdThreads = 256;
 constexpr int kBwdWarps = 8;
 constexpr int kBlk = 16384;  // [128 rows x 64 bf16] swizzled block
-constexpr int kDqFlush = 8;  // tiles per dQ accumulation chain in TMEM
+constexpr int kDqFlush = 16;  // tiles per dQ accumulation chain in TMEM
 
 struct BwdLayout {
   uint32_t q_off, do_off, k_off, v_off, a_off, lo_off, lse_off, d_off, bar_off, total;
@@ -256,6 +256,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       load_qdo(t);
       load_v(t);
       load_k(t);
+    }
+    if (ctl && i + 2 < ntiles) {  // K and V two tiles ahead into L2
+      BwdPos t2 = t;
+      bwd_next(p, t2);
+      bwd_next(p, t2);
+      const int row = p.cu_seqlens[t2.b] + t2.j * 128;
+      for (int kb = 0; kb < KB; ++kb) {
+        tma_prefetch_l2_2d(&mapK, t2.h * D + kb * 64, row);
+        tma_prefetch_l2_2d(&mapV, t2.h * D + kb * 64, row);
+      }
     }
     if (first && p.norm == SKA_NORM_TOKEN) {
       // per-prototype lse (log2 units) and D_j = dO_j . O_j of this (user, head)
@@ -504,20 +514,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if constexpr (NCOL >= 64) {
           stage_row(stk, qr, p.scale);
           __syncwarp();
+          float4 prev[8];  // all the slot's previous values in flight together
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const int row = q4 * 32 + 4 * u + (lane >> 3);  // prototype within the block
+            prev[u] = (add && wg * 128 + row < p.k)
+                          ? *reinterpret_cast<const float4*>(qbase + static_cast<int64_t>(row) * D + c + (lane & 7) * 4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int row = q4 * 32 + 4 * u + (lane >> 3);
             if (wg * 128 + row < p.k) {
-              float4* dst = reinterpret_cast<float4*>(qbase + static_cast<int64_t>(row) * D + c + (lane & 7) * 4);
               float4 o = staged(stk, u);
-              if (add) {
-                const float4 prev = *dst;
-                o.x += prev.x;
-                o.y += prev.y;
-                o.z += prev.z;
-                o.w += prev.w;
-              }
-              *dst = o;
+              o.x += prev[u].x;
+              o.y += prev[u].y;
+              o.z += prev[u].z;
+              o.w += prev[u].w;
+              *reinterpret_cast<float4*>(qbase + static_cast<int64_t>(row) * D + c + (lane & 7) * 4) = o;
             }
           }
           __syncwarp();
