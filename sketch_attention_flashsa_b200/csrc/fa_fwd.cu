@@ -495,29 +495,24 @@ __global__ void __launch_bounds__(kFaThreads, 1)
     float m = -INFINITY, l = 0.f;
     int nseg = 0;
     bool ok = true;
+    int nh = 0, hlen = 0;  // this segment's history tiles and this row's valid history keys
     for (int i = 0; i < ntiles && ok; ++i) {
       const bool first = (t.j == 0) || (i == 0);
       const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
       if (first) {
         m = -INFINITY;
         l = 0.f;
-      }
-      // valid keys of this tile for this row
-      const int nh = fa_hist_tiles(p, t.b);
-      int kk0, vlen;
-      if (t.j < nh) {
-        kk0 = t.j * 128;
-        vlen = fa_used(p, t.b);
+        // constant over the key tiles of a segment: read once
+        hlen = fa_used(p, t.b);
+        nh = (hlen + 127) / 128;
         if (p.mode == 1 && p.kv_len) {
           const int q = qt * 128 + r;
           const int nq = p.cu_q[t.b + 1] - p.cu_q[t.b];
-          if (q < nq) vlen = min(vlen, max(p.kv_len[p.cu_q[t.b] + q], 0));
+          if (q < nq) hlen = min(hlen, max(p.kv_len[p.cu_q[t.b] + q], 0));
         }
-      } else {
-        kk0 = (t.j - nh) * 128;
-        vlen = p.ks;
       }
-      const int nvalid = vlen - kk0;  // keys [0, nvalid) of this tile count
+      // valid keys of this tile for this row
+      const int nvalid = (t.j < nh) ? hlen - t.j * 128 : p.ks - (t.j - nh) * 128;  // keys [0, nvalid) count
 
       const int sb = i & 1;
       ok = __all_sync(0xffffffffu, wait(&bars.sfull[sb], (i >> 1) & 1));
@@ -533,9 +528,11 @@ __global__ void __launch_bounds__(kFaThreads, 1)
 
       // mask and tile max
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      if (nvalid < 128) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c)
-        if (c >= nvalid) sv[c] = __float_as_uint(-INFINITY);
+        for (int c = 0; c < 128; ++c)
+          if (c >= nvalid) sv[c] = __float_as_uint(-INFINITY);
+      }
 #pragma unroll
       for (int c = 0; c < 128; c += 8) {
         mx0 = max3f(mx0, __uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
