@@ -13,12 +13,19 @@
 // CTAs, each CTA writes an unnormalised partial (O, max, sum) per stream it touches, and a
 // combine kernel merges the partials of a stream by their log-sum-exp weights.
 //
-// Per key tile (one CTA, 256 threads):
-//   MMA1  S[q, key] = Q_tile . K_tile^T       M=128, N=128, K=d   -> TMEM (two buffers)
-//   softmax warpgroup (thread = query row): mask, running max (rescaling O in TMEM only when
-//         the max grows by more than 2^8), P = 2^(s c - m) as bf16 into shared memory
-//   MMA2  O[q, dd] += P . V_tile              M=128, N=d, K=128   -> TMEM
-// Warp 0: TMA producer; warp 1: TMEM owner + MMA issuer; warps 4-7: softmax.
+// Per key tile, one CTA (384 threads) holds two query tiles Q_0, Q_1 (query tiles 2u, 2u+1 of a
+// stream pair) and, for w = 0, 1:
+//   MMA1  S_w = Q_w . K_tile^T        M=128, N=128, K=d   -> TMEM columns [128 w, 128 w + 128)
+//   softmax warpgroup w (thread = query row of Q_w): mask, running max (O_w rescaled in TMEM only
+//         when the max grows by more than 2^8), P_w = 2^(s c - m) as bf16 pairs written back over
+//         the first 64 columns of S_w
+//   MMA2  O_w += P_w . V_tile         M=128, N=d, K=128 keys, A read from TMEM  -> TMEM
+// The MMA issuer orders MMA2(P_w, tile) before MMA1(Q_w, next tile) into the same columns, and
+// tcgen05 MMAs of one thread run in issue order, so S_w is only overwritten once P_w has been
+// read. The two warpgroups settle half a tile apart: while one computes its exponentials, the
+// tensor core runs the other's two MMAs.
+// Warp 0: TMA producer of Q and K; warp 1: TMEM owner + MMA issuer; warp 2: TMA producer of V;
+// warps 4-7 and 8-11: softmax warpgroups 0 and 1.
 #include <algorithm>
 #include <cmath>
 
@@ -29,8 +36,7 @@ namespace ska {
 
 namespace {
 
-constexpr int kFaThreads = 256;
-constexpr int kFaSoftmaxWarps = 4;
+constexpr int kFaThreads = 384;
 constexpr int kFaSlot = 16384;         // one [128 rows x 64 bf16] swizzled block
 constexpr int kFaMaxRing = 8;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
@@ -38,16 +44,14 @@ constexpr float kRescaleThreshold = 8.f;  // log2 units
 __host__ __device__ constexpr int fa_q_bytes(int D) { return 128 * D * 2; }
 
 struct FaLayout {
-  uint32_t q_off, p_off, k_off, v_off, total;
+  uint32_t q_off, k_off, v_off, total;
 };
 
 __host__ __device__ inline FaLayout fa_layout(int D, int nk, int nv) {
   FaLayout L;
   uint32_t off = 0;
   L.q_off = off;
-  off += fa_q_bytes(D);
-  L.p_off = off;
-  off += 2 * kFaSlot;                 // P: 128 rows x 128 keys bf16, two 64-key blocks
+  off += 2 * fa_q_bytes(D);           // Q_0, Q_1
   L.k_off = off;
   off += nk * (D / 64) * kFaSlot;     // K ring: tile entries
   L.v_off = off;
@@ -76,11 +80,12 @@ __device__ __forceinline__ int fa_ktiles(const FaFwdParams& p, int b) {
 }
 
 // Work layout. Columns are the key tiles of every (user, head): user b contributes H * n_b
-// columns (n_b key tiles per head), in order (b, h, j). Persistent CTAs form groups of G (G =
-// the largest number of 128-row query tiles of any user); the CTAs of group g walk the same
-// contiguous column range together, CTA (g, qt) with query tile qt, so a K/V tile is read from
-// DRAM once and from L2 by the other G - 1 CTAs. Columns of users with fewer than qt + 1 query
-// tiles are skipped by that CTA.
+// columns (n_b key tiles per head), in order (b, h, j). G is the largest number of 128-row
+// query tiles of any user; persistent CTAs form groups of (G + 1) / 2, and the CTAs of group g
+// walk the same contiguous column range together, CTA (g, u) with query tiles 2u and 2u + 1, so
+// a K/V tile is read from DRAM once and from L2 by the other CTAs of the group. Columns of users
+// with fewer than 2u + 1 query tiles are skipped by that CTA; a user with exactly 2u + 1 leaves
+// its second query tile (and second softmax warpgroup) idle.
 struct FaPos {
   int b, h, j;   // user, head, key tile
   int nb, qtn;   // key tiles per head of user b, query tiles of user b
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(128) fa_combine_kernel(const FaFwdParams p, in
 
 struct FaBars {
   uint64_t kfull[kFaMaxRing], kempty[kFaMaxRing], vfull[kFaMaxRing], vempty[kFaMaxRing];
-  uint64_t qfull, qfree, sfull[2], sfree[2], pfull, pfree, ofull, ofree, drain;
+  uint64_t qfull, qfree, sfull[2], pfull[2], ofull[2], ofree[2], drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -269,7 +274,7 @@ struct FaWaiter {
   }
 };
 
-// Q tile row (in the Q map) and column base for stream `seg` of user b.
+// Q tile row (in the Q map) and column base for query tile qt of the stream at t.
 __device__ __forceinline__ void fa_q_coord(const FaFwdParams& p, const FaPos& t, int qt, int D, int& c0,
                                            int& row) {
   const int h = t.h;
@@ -282,6 +287,27 @@ __device__ __forceinline__ void fa_q_coord(const FaFwdParams& p, const FaPos& t,
   }
 }
 
+// K / V tile coordinates of the key tile at t: [history or suffix rows ; sketch rows (STCA)].
+__device__ __forceinline__ bool fa_kv_coord(const FaFwdParams& p, const FaPos& t, int D, int& c0, int& row) {
+  const int nh = fa_hist_tiles(p, t.b);
+  if (t.j < nh) {
+    c0 = t.h * D;
+    row = p.cu_keys[t.b] + t.j * 128;
+    return false;
+  }
+  c0 = 0;
+  row = (t.b * p.H + t.h) * p.ks + (t.j - nh) * 128;
+  return true;
+}
+
+// Waits of the producers at exit for their loads still in flight (none may land after exit).
+__device__ __forceinline__ void fa_drain_ring(FaWaiter& wait, uint64_t* full, int slots, int uses) {
+  for (int e = 0; e < slots; ++e) {
+    const int fills = (uses > e) ? (uses - e - 1) / slots + 1 : 0;
+    if (fills > 0) wait(&full[e], (fills - 1) & 1, true);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kFaThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
@@ -289,27 +315,29 @@ __global__ void __launch_bounds__(kFaThreads, 1)
                   const __grid_constant__ CUtensorMap mapVs, const FaFwdParams p) {
   constexpr int KB = D / 64;
   constexpr int kTileBytes = KB * kFaSlot;
+  constexpr int kQBytes = fa_q_bytes(D);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ FaBars bars;
   const FaLayout L = fa_layout(D, p.nk_slots, p.nv_entries);
   uint8_t* sQ = smem + L.q_off;
-  uint8_t* sP = smem + L.p_off;
   uint8_t* sK = smem + L.k_off;
   uint8_t* sV = smem + L.v_off;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int nk = p.nk_slots, nv = p.nv_entries;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < p.nk_slots; ++i) { mbar_init(&bars.kfull[i], 1); mbar_init(&bars.kempty[i], 1); }
-    for (int i = 0; i < p.nv_entries; ++i) { mbar_init(&bars.vfull[i], 1); mbar_init(&bars.vempty[i], 1); }
+    for (int i = 0; i < nk; ++i) { mbar_init(&bars.kfull[i], 1); mbar_init(&bars.kempty[i], 1); }
+    for (int i = 0; i < nv; ++i) { mbar_init(&bars.vfull[i], 1); mbar_init(&bars.vempty[i], 1); }
     mbar_init(&bars.qfull, 1);
     mbar_init(&bars.qfree, 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(&bars.sfull[i], 1); mbar_init(&bars.sfree[i], kFaSoftmaxWarps); }
-    mbar_init(&bars.pfull, kFaSoftmaxWarps);
-    mbar_init(&bars.pfree, 1);
-    mbar_init(&bars.ofull, 1);
-    mbar_init(&bars.ofree, kFaSoftmaxWarps);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bars.sfull[w], 1);
+      mbar_init(&bars.pfull[w], 4);  // the four warps of softmax warpgroup w
+      mbar_init(&bars.ofull[w], 1);
+      mbar_init(&bars.ofree[w], 4);
+    }
     mbar_init(&bars.drain, 1);
     bars.abort_flag = 0;
     fence_mbar_init();
@@ -321,311 +349,325 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // TMEM columns: S_0 [0, 128), S_1 [128, 256), O_0 [256, 256 + D), O_1 [256 + D, 256 + 2 D)
   const uint32_t tbase = bars.tmem_base;
-  const uint32_t tO = tbase + 256;   // O: 128 lanes x D columns; S buffers at columns 0 and 128
   FaWaiter wait{&bars, &p.hdr->status, p.budget_ns};
-  // group of G CTAs walking one column range; this CTA's query tile
+  // group of (G + 1) / 2 CTAs walking one column range; this CTA's query tiles qt0, qt0 + 1
   const int G = p.group;
-  const int grp = blockIdx.x / G, qt = blockIdx.x % G;
-  const int ngroups = gridDim.x / G;
+  const int Gc = (G + 1) >> 1;
+  const int grp = blockIdx.x / Gc;
+  const int qt0 = 2 * (blockIdx.x % Gc);
+  const int ngroups = gridDim.x / Gc;
   const int total = p.hdr->total_tiles;
   const int W = p.hdr->tiles_per_cluster;
   const int c0 = grp * W, c1 = min(total, c0 + W);
-  const int ntiles = (grp < ngroups && W > 0 && c0 < total && p.hdr->status == 0) ? fa_count(p, qt, c0, c1) : 0;
+  const int ntiles = (grp < ngroups && W > 0 && c0 < total && p.hdr->status == 0) ? fa_count(p, qt0, c0, c1) : 0;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer: Q pairs and K
     if (lane == 0 && ntiles > 0) {
-      FaPos tk, tv;
-      fa_seek(p, c0, qt, tk);
-      tv = tk;
-      int kent = 0, kuse = 0, vent = 0, vuse = 0, nq = 0;
+      FaPos t;
+      fa_seek(p, c0, qt0, t);
+      int kent = 0, kuse = 0, nq = 0;
       bool ok = true;
       bool skip_first = (p.debug_flags & 1u) != 0;
-      auto kv_coord = [&](const FaPos& t, int& c0, int& row, const CUtensorMap*& mk, const CUtensorMap*& mv) {
-        const int h = t.h;
-        const int nh = fa_hist_tiles(p, t.b);
-        if (t.j < nh) {
-          c0 = h * D;
-          row = p.cu_keys[t.b] + t.j * 128;
-          mk = &mapK;
-          mv = &mapV;
-        } else {
-          c0 = 0;
-          row = (t.b * p.H + h) * p.ks + (t.j - nh) * 128;
-          mk = &mapKs;
-          mv = &mapVs;
-        }
-      };
-      for (int i = 0; i <= ntiles && ok; ++i) {
-        if (i < ntiles) {
-          if (tk.j == 0 || i == 0) {
-            if (nq > 0) ok = wait(&bars.qfree, (nq - 1) & 1);
-            if (!ok) break;
-            int qc0, qrow;
-            fa_q_coord(p, tk, qt, D, qc0, qrow);
-            mbar_expect_tx(&bars.qfull, fa_q_bytes(D));
-            for (int kb = 0; kb < KB; ++kb) tma_load_2d(sQ + kb * kFaSlot, &mapQ, &bars.qfull, qc0 + kb * 64, qrow);
-            ++nq;
-          }
-          ok = wait(&bars.kempty[kent], ((kuse / p.nk_slots) & 1) ^ 1);
+      for (int i = 0; i < ntiles && ok; ++i) {
+        if (t.j == 0 || i == 0) {
+          // the stream's query tiles, once the previous stream's last MMA1 has read sQ
+          if (nq > 0) ok = wait(&bars.qfree, (nq - 1) & 1);
           if (!ok) break;
-          int c0, row;
-          const CUtensorMap *mk, *mv;
-          kv_coord(tk, c0, row, mk, mv);
-          if (skip_first) {
-            skip_first = false;  // withhold this arrival: the MMA warp's wait must run out
-          } else {
-            mbar_expect_tx(&bars.kfull[kent], kTileBytes);
+          const int nqt = (qt0 + 1 < t.qtn) ? 2 : 1;
+          int qc0, qrow;
+          fa_q_coord(p, t, qt0, D, qc0, qrow);
+          mbar_expect_tx(&bars.qfull, kQBytes * nqt);
+          for (int w = 0; w < nqt; ++w)
             for (int kb = 0; kb < KB; ++kb)
-              tma_load_2d(sK + kent * kTileBytes + kb * kFaSlot, mk, &bars.kfull[kent], c0 + kb * 64, row);
-          }
-          kent = (kent + 1 == p.nk_slots) ? 0 : kent + 1;
-          ++kuse;
-          fa_next(p, qt, tk);
+              tma_load_2d(sQ + w * kQBytes + kb * kFaSlot, &mapQ, &bars.qfull, qc0 + kb * 64, qrow + w * 128);
+          ++nq;
         }
-        if (i >= 1) {
-          ok = wait(&bars.vempty[vent], ((vuse / p.nv_entries) & 1) ^ 1);
-          if (!ok) break;
-          int c0, row;
-          const CUtensorMap *mk, *mv;
-          kv_coord(tv, c0, row, mk, mv);
-          mbar_expect_tx(&bars.vfull[vent], kTileBytes);
+        ok = wait(&bars.kempty[kent], ((kuse / nk) & 1) ^ 1);
+        if (!ok) break;
+        int kc0, krow;
+        const CUtensorMap* mk = fa_kv_coord(p, t, D, kc0, krow) ? &mapKs : &mapK;
+        if (skip_first) {
+          skip_first = false;  // withhold this arrival: the MMA warp's wait must run out
+        } else {
+          mbar_expect_tx(&bars.kfull[kent], kTileBytes);
           for (int kb = 0; kb < KB; ++kb)
-            tma_load_2d(sV + vent * kTileBytes + kb * kFaSlot, mv, &bars.vfull[vent], c0 + kb * 64, row);
-          vent = (vent + 1 == p.nv_entries) ? 0 : vent + 1;
-          ++vuse;
-          fa_next(p, qt, tv);
+            tma_load_2d(sK + kent * kTileBytes + kb * kFaSlot, mk, &bars.kfull[kent], kc0 + kb * 64, krow);
         }
+        kent = (kent + 1 == nk) ? 0 : kent + 1;
+        ++kuse;
+        fa_next(p, qt0, t);
       }
-      for (int e = 0; e < p.nk_slots; ++e) {
-        const int fills = (kuse > e) ? (kuse - e - 1) / p.nk_slots + 1 : 0;
-        if (fills > 0) wait(&bars.kfull[e], (fills - 1) & 1, true);
-      }
-      for (int e = 0; e < p.nv_entries; ++e) {
-        const int fills = (vuse > e) ? (vuse - e - 1) / p.nv_entries + 1 : 0;
-        if (fills > 0) wait(&bars.vfull[e], (fills - 1) & 1, true);
-      }
+      fa_drain_ring(wait, bars.kfull, nk, kuse);
       if (nq > 0) wait(&bars.qfull, (nq - 1) & 1, true);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ TMA producer: V
+    if (lane == 0 && ntiles > 0) {
+      FaPos t;
+      fa_seek(p, c0, qt0, t);
+      int vent = 0, vuse = 0;
+      bool ok = true;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        ok = wait(&bars.vempty[vent], ((vuse / nv) & 1) ^ 1);
+        if (!ok) break;
+        int vc0, vrow;
+        const CUtensorMap* mv = fa_kv_coord(p, t, D, vc0, vrow) ? &mapVs : &mapV;
+        mbar_expect_tx(&bars.vfull[vent], kTileBytes);
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_2d(sV + vent * kTileBytes + kb * kFaSlot, mv, &bars.vfull[vent], vc0 + kb * 64, vrow);
+        vent = (vent + 1 == nv) ? 0 : vent + 1;
+        ++vuse;
+        fa_next(p, qt0, t);
+      }
+      fa_drain_ring(wait, bars.vfull, nv, vuse);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Order per key tile i: for w = 0, 1: MMA2(P_w, V_i) -> O_w, then MMA1(Q_w, K_{i+1}) -> S_w.
     if (lane == 0 && ntiles > 0) {
       constexpr uint32_t idesc1 = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
-      FaPos t1, t2;
-      fa_seek(p, c0, qt, t1);
-      t2 = t1;
-      int kent = 0, kuse = 0, vent = 0, vuse = 0, nq = 0, nseg2 = 0;
+      auto mma1 = [&](int w, uint32_t kbase) {
+        const uint32_t qbase = smem_u32(sQ + w * kQBytes);
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+          const uint64_t ad = sw128_desc(qbase + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(kbase + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
+          umma_bf16(tbase + w * 128, ad, bd, idesc1, s > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars.sfull[w]);
+      };
+      auto mma2 = [&](int w, uint32_t vbase, bool fresh) {
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const uint64_t bd = sw128_desc(vbase + s * 2048, kFaSlot, 1024);
+          umma_bf16_ts(tbase + 256 + w * D, tbase + w * 128 + s * 8, bd, idesc2, (fresh && s == 0) ? 0u : 1u);
+        }
+      };
+      FaPos t;
+      fa_seek(p, c0, qt0, t);
+      int kent = 0, kuse = 0, vent = 0, vuse = 0, nq = 0;
+      int np[2] = {0, 0}, nseg[2] = {0, 0};
       bool ok = true;
-      for (int i = 0; i <= ntiles && ok; ++i) {
-        if (i < ntiles) {
-          const bool first = (t1.j == 0) || (i == 0);
-          const bool last = (t1.j == t1.nb - 1) || (i == ntiles - 1);
-          if (first) {
-            ok = wait(&bars.qfull, nq & 1);
-            if (!ok) break;
+      {
+        // MMA1 of the first tile
+        ok = wait(&bars.qfull, 0) && wait(&bars.kfull[0], 0);
+        if (ok) {
+          ++nq;
+          tc_fence_after();
+          const uint32_t kbase = smem_u32(sK);
+          mma1(0, kbase);
+          if (qt0 + 1 < t.qtn) mma1(1, kbase);
+          umma_commit(&bars.kempty[0]);
+          if (t.j == t.nb - 1 || ntiles == 1) umma_commit(&bars.qfree);
+          kent = (nk == 1) ? 0 : 1;
+          ++kuse;
+        }
+      }
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const bool first = (t.j == 0) || (i == 0);
+        const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
+        const bool q1 = qt0 + 1 < t.qtn;
+        const bool more = i + 1 < ntiles;
+        FaPos tn = t;
+        if (more) fa_next(p, qt0, tn);
+        const bool nq1 = more && (qt0 + 1 < tn.qtn);
+        const bool nfirst = more && (tn.j == 0);
+        const bool nlast = more && ((tn.j == tn.nb - 1) || (i + 1 == ntiles - 1));
+        ok = wait(&bars.vfull[vent], (vuse / nv) & 1);
+        if (!ok) break;
+        const uint32_t vbase = smem_u32(sV + vent * kTileBytes);
+        const uint32_t knext = smem_u32(sK + kent * kTileBytes);
+        bool next_in = false;
+        // Q (first tile of a stream) and K of tile i + 1 resident
+        auto next_ready = [&]() -> bool {
+          if (next_in) return true;
+          if (nfirst) {
+            if (!wait(&bars.qfull, nq & 1)) return false;
             ++nq;
           }
-          const int sb = i & 1;
-          if (i >= 2) {
-            ok = wait(&bars.sfree[sb], ((i >> 1) - 1) & 1);
-            if (!ok) break;
-          }
-          ok = wait(&bars.kfull[kent], (kuse / p.nk_slots) & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t kbase = smem_u32(sK + kent * kTileBytes);
+          if (!wait(&bars.kfull[kent], (kuse / nk) & 1)) return false;
+          next_in = true;
+          return true;
+        };
 #pragma unroll
-          for (int s = 0; s < D / 16; ++s) {
-            const uint64_t ad = sw128_desc(smem_u32(sQ) + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(kbase + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
-            umma_bf16(tbase + sb * 128, ad, bd, idesc1, s > 0 ? 1u : 0u);
-          }
-          umma_commit(&bars.kempty[kent]);
-          umma_commit(&bars.sfull[sb]);
-          if (last) umma_commit(&bars.qfree);
-          kent = (kent + 1 == p.nk_slots) ? 0 : kent + 1;
-          ++kuse;
-          fa_next(p, qt, t1);
-        }
-        if (i >= 1) {
-          const bool first = (t2.j == 0) || (i == 1);
-          const bool last = (t2.j == t2.nb - 1) || (i == ntiles);
-          ok = wait(&bars.pfull, (i - 1) & 1);
+        for (int w = 0; w < 2; ++w) {
+          if (w == 1 && !q1) break;
+          ok = wait(&bars.pfull[w], np[w] & 1);
           if (!ok) break;
-          ok = wait(&bars.vfull[vent], (vuse / p.nv_entries) & 1);
-          if (!ok) break;
-          if (first && nseg2 > 0) {
-            ok = wait(&bars.ofree, (nseg2 - 1) & 1);
+          ++np[w];
+          if (first && nseg[w] > 0) {
+            ok = wait(&bars.ofree[w], (nseg[w] - 1) & 1);
             if (!ok) break;
           }
           tc_fence_after();
-          const uint32_t vbase = smem_u32(sV + vent * kTileBytes);
-#pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            const uint64_t ad = sw128_desc(smem_u32(sP) + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(vbase + s * 2048, kFaSlot, 1024);
-            umma_bf16(tO, ad, bd, idesc2, (first && s == 0) ? 0u : 1u);
-          }
-          umma_commit(&bars.vempty[vent]);
-          umma_commit(&bars.pfree);
+          mma2(w, vbase, first);
           if (last) {
-            umma_commit(&bars.ofull);
-            ++nseg2;
+            umma_commit(&bars.ofull[w]);
+            ++nseg[w];
           }
-          vent = (vent + 1 == p.nv_entries) ? 0 : vent + 1;
-          ++vuse;
-          fa_next(p, qt, t2);
+          if (more && (w == 0 || nq1)) {
+            ok = next_ready();
+            if (!ok) break;
+            tc_fence_after();
+            mma1(w, knext);
+          }
         }
+        if (!ok) break;
+        if (nq1 && !q1) {
+          // a stream with two query tiles after one with a single tile
+          ok = next_ready();
+          if (!ok) break;
+          tc_fence_after();
+          mma1(1, knext);
+        }
+        umma_commit(&bars.vempty[vent]);
+        vent = (vent + 1 == nv) ? 0 : vent + 1;
+        ++vuse;
+        if (more) {
+          umma_commit(&bars.kempty[kent]);
+          if (nlast) umma_commit(&bars.qfree);
+          kent = (kent + 1 == nk) ? 0 : kent + 1;
+          ++kuse;
+        }
+        t = tn;
       }
       umma_commit(&bars.drain);
       wait(&bars.drain, 0, true);
     }
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax warpgroup
-    // (continued below)
-    const int q4 = warp - 4;
+    // ------------------------------------------------------------ softmax warpgroups
+    // Warpgroup w (warps 4-7, 8-11) owns query tile qt0 + w: thread r holds query row r, its
+    // running maximum m (the reference P is scaled against) and its running sum l.
+    const int w = (warp - 4) >> 2;
+    const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    const uint32_t tS = tbase + w * 128 + lane_off;
+    const uint32_t tO = tbase + 256 + w * D + lane_off;
     const float c2 = p.scale_log2;
     const uint64_t c2x2 = f2_pack(c2, c2);
     FaPos t;
-    if (ntiles > 0) fa_seek(p, c0, qt, t);
+    if (ntiles > 0) fa_seek(p, c0, qt0, t);
     float m = -INFINITY, l = 0.f;
-    int nseg = 0;
+    int ns = 0, nseg = 0;
     bool ok = true;
-    int nh = 0, hlen = 0;  // this segment's history tiles and this row's valid history keys
+    int nh = 0, hlen = 0;  // this stream's history tiles and this row's valid history keys
     for (int i = 0; i < ntiles && ok; ++i) {
-      const bool first = (t.j == 0) || (i == 0);
-      const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
-      if (first) {
-        m = -INFINITY;
-        l = 0.f;
-        // constant over the key tiles of a segment: read once
-        hlen = fa_used(p, t.b);
-        nh = (hlen + 127) / 128;
-        if (p.mode == 1 && p.kv_len) {
-          const int q = qt * 128 + r;
-          const int nq = p.cu_q[t.b + 1] - p.cu_q[t.b];
-          if (q < nq) hlen = min(hlen, max(p.kv_len[p.cu_q[t.b] + q], 0));
+      if (w == 0 || qt0 + 1 < t.qtn) {
+        const bool first = (t.j == 0) || (i == 0);
+        const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
+        if (first) {
+          m = -INFINITY;
+          l = 0.f;
+          // constant over the key tiles of a stream: read once
+          hlen = fa_used(p, t.b);
+          nh = (hlen + 127) / 128;
+          if (p.mode == 1 && p.kv_len) {
+            const int q = (qt0 + w) * 128 + r;
+            const int nq = p.cu_q[t.b + 1] - p.cu_q[t.b];
+            if (q < nq) hlen = min(hlen, max(p.kv_len[p.cu_q[t.b] + q], 0));
+          }
         }
-      }
-      // valid keys of this tile for this row
-      const int nvalid = (t.j < nh) ? hlen - t.j * 128 : p.ks - (t.j - nh) * 128;  // keys [0, nvalid) count
+        // valid keys of this tile for this row
+        const int nvalid = (t.j < nh) ? hlen - t.j * 128 : p.ks - (t.j - nh) * 128;
 
-      const int sb = i & 1;
-      ok = __all_sync(0xffffffffu, wait(&bars.sfull[sb], (i >> 1) & 1));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sv[128];
-#pragma unroll
-      for (int c = 0; c < 128; c += 32) tmem_ld32(tbase + sb * 128 + lane_off + c, sv + c);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.sfree[sb]);
-
-      // mask and tile max
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-      if (nvalid < 128) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= nvalid) sv[c] = __float_as_uint(-INFINITY);
-      }
-#pragma unroll
-      for (int c = 0; c < 128; c += 8) {
-        mx0 = max3f(mx0, __uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
-        mx1 = max3f(mx1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
-        mx2 = max3f(mx2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
-        mx3 = max3f(mx3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
-      }
-      const float mt = fmaxf(max3f(mx0, mx1, mx2), mx3) * c2;
-      // lazy rescale: move the reference only when the max grows by more than 2^8
-      float factor = 1.f;
-      if (mt > m + kRescaleThreshold || (m == -INFINITY && mt > -INFINITY)) {
-        factor = (m == -INFINITY) ? 0.f : ex2_approx(m - mt);
-        m = mt;
-      }
-      const float mref = (m == -INFINITY) ? 0.f : m;
-      const uint64_t negm = f2_pack(-mref, -mref);
-      uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
-#pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        float x0, x1, x2, x3;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), c2x2, negm), x0, x1);
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), c2x2, negm), x2, x3);
-        const float e0 = ex2_approx(x0), e1 = ex2_approx(x1), e2 = ex2_approx(x2), e3 = ex2_approx(x3);
-        sv[c] = __float_as_uint(e0);
-        sv[c + 1] = __float_as_uint(e1);
-        sv[c + 2] = __float_as_uint(e2);
-        sv[c + 3] = __float_as_uint(e3);
-        acc0 = f2_add(acc0, f2_pack(e0, e1));
-        acc1 = f2_add(acc1, f2_pack(e2, e3));
-      }
-      float a0, a1, b0, b1;
-      f2_unpack(acc0, a0, a1);
-      f2_unpack(acc1, b0, b1);
-      l = l * factor + ((a0 + a1) + (b0 + b1));
-
-      if (i > 0) {
-        ok = __all_sync(0xffffffffu, wait(&bars.pfree, (i - 1) & 1));
+        ok = __all_sync(0xffffffffu, wait(&bars.sfull[w], ns & 1));
         if (!ok) break;
-      }
-      // O rows whose reference moved are rescaled in TMEM (MMA2 of the previous tile is done)
-      if (!first && __any_sync(0xffffffffu, factor != 1.f)) {
+        ++ns;
         tc_fence_after();
+        uint32_t sv[128];
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t ov[32];
-          tmem_ld32(tO + lane_off + c, ov);
-          tmem_ld_wait();
+        for (int c = 0; c < 128; c += 32) tmem_ld32(tS + c, sv + c);
+        tmem_ld_wait();
+        if (nvalid < 128) {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * factor);
-          tmem_st32(tO + lane_off + c, ov);
+          for (int c = 0; c < 128; ++c)
+            if (c >= nvalid) sv[c] = __float_as_uint(-INFINITY);
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 8) {
+          mx0 = max3f(mx0, __uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
+          mx1 = max3f(mx1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
+          mx2 = max3f(mx2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
+          mx3 = max3f(mx3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
+        }
+        const float mt = fmaxf(max3f(mx0, mx1, mx2), mx3) * c2;
+        // lazy rescale: move the reference only when the max grows by more than 2^8
+        float factor = 1.f;
+        if (mt > m + kRescaleThreshold || (m == -INFINITY && mt > -INFINITY)) {
+          factor = (m == -INFINITY) ? 0.f : ex2_approx(m - mt);
+          m = mt;
+        }
+        const float mref = (m == -INFINITY) ? 0.f : m;
+        const uint64_t negm = f2_pack(-mref, -mref);
+        uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+        // P as bf16 pairs, packed in place: word c / 2 holds columns c, c + 1
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), c2x2, negm), x0, x1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), c2x2, negm), x2, x3);
+          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1), e2 = ex2_approx(x2), e3 = ex2_approx(x3);
+          acc0 = f2_add(acc0, f2_pack(e0, e1));
+          acc1 = f2_add(acc1, f2_pack(e2, e3));
+          sv[c / 2] = pack_bf16x2(e0, e1);
+          sv[c / 2 + 1] = pack_bf16x2(e2, e3);
+        }
+        float a0, a1, b0, b1;
+        f2_unpack(acc0, a0, a1);
+        f2_unpack(acc1, b0, b1);
+        l = l * factor + ((a0 + a1) + (b0 + b1));
+        tmem_st32(tS, sv);
+        tmem_st32(tS + 32, sv + 32);
+        // O_w rows whose reference moved are rescaled in TMEM: MMA2 of this warpgroup's previous
+        // tile completed before S_w was written (sfull)
+        if (!first && __any_sync(0xffffffffu, factor != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < D; c += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * factor);
+            tmem_st32(tO + c, ov);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
-      }
-      // P row as bf16 into the K-major A operand of MMA2
-#pragma unroll
-      for (int c = 0; c < 128; c += 8) {
-        uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
-        w.y = pack_bf16x2(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
-        w.z = pack_bf16x2(__uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
-        w.w = pack_bf16x2(__uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
-        *reinterpret_cast<uint4*>(sP + (c >> 6) * kFaSlot + sw128_offset(r, (c & 63) * 2)) = w;
-      }
-      fence_async_shared();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.pfull);
-
-      if (last) {
-        ok = __all_sync(0xffffffffu, wait(&bars.ofull, nseg & 1));
-        if (!ok) break;
-        tc_fence_after();
-        // slot of (column stream (b, h), group, query tile): unique along the column staircase
-        const int slot = ((t.b * p.H + t.h) + grp) * G + qt;
-        float* dst = p.part_o + (static_cast<int64_t>(slot) * 128 + r) * D;
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t ov[32];
-          tmem_ld32(tO + lane_off + c, ov);
-          tmem_ld_wait();
-#pragma unroll
-          for (int u = 0; u < 32; u += 4)
-            *reinterpret_cast<float4*>(dst + c + u) = make_float4(__uint_as_float(ov[u]), __uint_as_float(ov[u + 1]),
-                                                                  __uint_as_float(ov[u + 2]), __uint_as_float(ov[u + 3]));
-        }
-        p.part_ml[(static_cast<int64_t>(slot) * 128 + r) * 2] = m;
-        p.part_ml[(static_cast<int64_t>(slot) * 128 + r) * 2 + 1] = l;
-        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.ofree);
-        ++nseg;
+        if (lane == 0) mbar_arrive(&bars.pfull[w]);
+
+        if (last) {
+          ok = __all_sync(0xffffffffu, wait(&bars.ofull[w], nseg & 1));
+          if (!ok) break;
+          tc_fence_after();
+          // slot of (column stream (b, h), group, query tile): unique along the column staircase
+          const int slot = ((t.b * p.H + t.h) + grp) * G + qt0 + w;
+          float* dst = p.part_o + (static_cast<int64_t>(slot) * 128 + r) * D;
+#pragma unroll 1
+          for (int c = 0; c < D; c += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 32; u += 4)
+              *reinterpret_cast<float4*>(dst + c + u) = make_float4(__uint_as_float(ov[u]), __uint_as_float(ov[u + 1]),
+                                                                    __uint_as_float(ov[u + 2]), __uint_as_float(ov[u + 3]));
+          }
+          p.part_ml[(static_cast<int64_t>(slot) * 128 + r) * 2] = m;
+          p.part_ml[(static_cast<int64_t>(slot) * 128 + r) * 2 + 1] = l;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.ofree[w]);
+          ++nseg;
+        }
       }
-      fa_next(p, qt, t);
+      fa_next(p, qt0, t);
     }
   }
 
@@ -657,8 +699,9 @@ bool fa_fwd_plan(int D, int num_sms, int* num_ctas, size_t* smem_bytes, int* nk,
   for (int v = 1; v <= kFaMaxRing; ++v)
     for (int k = 1; k <= kFaMaxRing; ++k) {
       if (fa_layout(D, k, v).total > budget) continue;
-      const int score = std::min(k, v) * 100 + k + v;
-      if (best_k == 0 || score > std::min(best_k, best_v) * 100 + best_k + best_v) {
+      // the deeper ring goes to V: a V entry is held from its load until the second MMA2 of the tile
+      const int score = std::min(k, v) * 100 + k + 2 * v;
+      if (best_k == 0 || score > std::min(best_k, best_v) * 100 + best_k + 2 * best_v) {
         best_k = k;
         best_v = v;
       }
@@ -680,7 +723,7 @@ cudaError_t launch_fa_fwd(int D, int num_ctas, size_t smem, const CUtensorMap& m
 }
 
 cudaError_t launch_fa_schedule(const FaFwdParams& p, int num_ctas, cudaStream_t stream) {
-  fa_schedule_kernel<<<1, 1024, 0, stream>>>(p, num_ctas / p.group, p.group);
+  fa_schedule_kernel<<<1, 1024, 0, stream>>>(p, num_ctas / ((p.group + 1) / 2), p.group);
   return cudaGetLastError();
 }
 

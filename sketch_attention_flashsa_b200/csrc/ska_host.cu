@@ -203,11 +203,13 @@ void fa_ws_layout(int B, int H, int D, int G, int ngroups, size_t cast_q, size_t
   w->total = off;
 }
 
-// Group size (query tiles walked together) and CTA count of the row-softmax engine.
+// CTA count of the row-softmax engine for G query tiles walked together: groups of (G + 1) / 2
+// CTAs, each CTA holding two query tiles.
 bool fa_groups(int G, int sms, int* ctas, int* ngroups) {
-  if (G < 1 || G > sms) return false;
-  *ngroups = sms / G;
-  *ctas = *ngroups * G;
+  const int Gc = (G + 1) / 2;
+  if (G < 1 || Gc > sms) return false;
+  *ngroups = sms / Gc;
+  *ctas = *ngroups * Gc;
   return true;
 }
 

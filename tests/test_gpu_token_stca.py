@@ -34,6 +34,8 @@ TOKEN_CASES = {
     "d64_k16": ([1000, 5], 1, 64, 16),
     "d128_k192": ([640, 33], 3, 128, 192),
     "d64_k1024": ([257], 1, 64, 1024),
+    # three query tiles: the second CTA of a group holds one query tile (second warpgroup idle)
+    "d128_k384": ([520, 1, 129], 2, 128, 384),
 }
 
 
@@ -122,6 +124,9 @@ STCA_CASES = {
     "no_sketch": ([129, 40], [500, 1], 0, 4, 64, False),
     "kv_len_mask": ([150, 60], [700, 300], 100, 2, 64, True),
     "only_sketch": ([64], [0], 256, 1, 128, False),
+    # users with 3, 1 and 3 query tiles: pairs with and without a second query tile alternate
+    # along one CTA's key columns
+    "odd_tiles_mixed": ([300, 100, 257], [400, 900, 130], 64, 2, 128, True),
 }
 
 
