@@ -13,7 +13,7 @@
 //        TOKEN dS = A (dA - D_j) with D_j = dO_j . O_j from the forward sketch. dS goes to smem
 //        as a bf16 pair hi + lo.
 //   MMA  dK   = dS^T . Q        (M=tok, N=d)   -> TMEM, both halves, scaled on the way out
-//   MMA  dQ  += dS . K          (M=proto, N=d) -> TMEM, both halves; restarted every 8 tiles and
+//   MMA  dQ  += dS . K          (M=proto, N=d) -> TMEM, both halves; restarted every 16 tiles and
 //        added into the CTA's partial slot (the tensor core's fp32 accumulation is not
 //        round-to-nearest, so one chain over a whole segment would drift); a second kernel sums
 //        the partial slots of every prototype set in a fixed order.
