@@ -37,6 +37,12 @@ namespace ska {
 namespace {
 
 constexpr int kFaThreads = 384;
+// Registers per thread after the split: the launch gives every thread 168 (three warps per
+// sub-partition); warpgroup 0 drops to 96 and the two softmax warpgroups rise to 200
+// (96 x 128 + 200 x 256 <= 168 x 384, and 32 x (96 + 2 x 200) registers per sub-partition fit in
+// its 16,384). With this split neither instantiation spills; with 168 for all they spill 72-88 bytes.
+constexpr uint32_t kFaRoleRegs = 96;
+constexpr uint32_t kFaSoftmaxRegs = 200;
 constexpr int kFaSlot = 16384;         // one [128 rows x 64 bf16] swizzled block
 constexpr int kFaMaxRing = 8;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
@@ -363,182 +369,187 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   const int c0 = grp * W, c1 = min(total, c0 + W);
   const int ntiles = (grp < ngroups && W > 0 && c0 < total && p.hdr->status == 0) ? fa_count(p, qt0, c0, c1) : 0;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer: Q pairs and K
-    if (lane == 0 && ntiles > 0) {
-      FaPos t;
-      fa_seek(p, c0, qt0, t);
-      int kent = 0, kuse = 0, nq = 0;
-      bool ok = true;
-      bool skip_first = (p.debug_flags & 1u) != 0;
-      for (int i = 0; i < ntiles && ok; ++i) {
-        if (t.j == 0 || i == 0) {
-          // the stream's query tiles, once the previous stream's last MMA1 has read sQ
-          if (nq > 0) ok = wait(&bars.qfree, (nq - 1) & 1);
-          if (!ok) break;
-          const int nqt = (qt0 + 1 < t.qtn) ? 2 : 1;
-          int qc0, qrow;
-          fa_q_coord(p, t, qt0, D, qc0, qrow);
-          mbar_expect_tx(&bars.qfull, kQBytes * nqt);
-          for (int w = 0; w < nqt; ++w)
-            for (int kb = 0; kb < KB; ++kb)
-              tma_load_2d(sQ + w * kQBytes + kb * kFaSlot, &mapQ, &bars.qfull, qc0 + kb * 64, qrow + w * 128);
-          ++nq;
-        }
-        ok = wait(&bars.kempty[kent], ((kuse / nk) & 1) ^ 1);
-        if (!ok) break;
-        int kc0, krow;
-        const CUtensorMap* mk = fa_kv_coord(p, t, D, kc0, krow) ? &mapKs : &mapK;
-        if (skip_first) {
-          skip_first = false;  // withhold this arrival: the MMA warp's wait must run out
-        } else {
-          mbar_expect_tx(&bars.kfull[kent], kTileBytes);
-          for (int kb = 0; kb < KB; ++kb)
-            tma_load_2d(sK + kent * kTileBytes + kb * kFaSlot, mk, &bars.kfull[kent], kc0 + kb * 64, krow);
-        }
-        kent = (kent + 1 == nk) ? 0 : kent + 1;
-        ++kuse;
-        fa_next(p, qt0, t);
-      }
-      fa_drain_ring(wait, bars.kfull, nk, kuse);
-      if (nq > 0) wait(&bars.qfull, (nq - 1) & 1, true);
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ TMA producer: V
-    if (lane == 0 && ntiles > 0) {
-      FaPos t;
-      fa_seek(p, c0, qt0, t);
-      int vent = 0, vuse = 0;
-      bool ok = true;
-      for (int i = 0; i < ntiles && ok; ++i) {
-        ok = wait(&bars.vempty[vent], ((vuse / nv) & 1) ^ 1);
-        if (!ok) break;
-        int vc0, vrow;
-        const CUtensorMap* mv = fa_kv_coord(p, t, D, vc0, vrow) ? &mapVs : &mapV;
-        mbar_expect_tx(&bars.vfull[vent], kTileBytes);
-        for (int kb = 0; kb < KB; ++kb)
-          tma_load_2d(sV + vent * kTileBytes + kb * kFaSlot, mv, &bars.vfull[vent], vc0 + kb * 64, vrow);
-        vent = (vent + 1 == nv) ? 0 : vent + 1;
-        ++vuse;
-        fa_next(p, qt0, t);
-      }
-      fa_drain_ring(wait, bars.vfull, nv, vuse);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // Order per key tile i: for w = 0, 1: MMA2(P_w, V_i) -> O_w, then MMA1(Q_w, K_{i+1}) -> S_w.
-    if (lane == 0 && ntiles > 0) {
-      constexpr uint32_t idesc1 = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
-      auto mma1 = [&](int w, uint32_t kbase) {
-        const uint32_t qbase = smem_u32(sQ + w * kQBytes);
-#pragma unroll
-        for (int s = 0; s < D / 16; ++s) {
-          const uint64_t ad = sw128_desc(qbase + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
-          const uint64_t bd = sw128_desc(kbase + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
-          umma_bf16(tbase + w * 128, ad, bd, idesc1, s > 0 ? 1u : 0u);
-        }
-        umma_commit(&bars.sfull[w]);
-      };
-      auto mma2 = [&](int w, uint32_t vbase, bool fresh) {
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const uint64_t bd = sw128_desc(vbase + s * 2048, kFaSlot, 1024);
-          umma_bf16_ts(tbase + 256 + w * D, tbase + w * 128 + s * 8, bd, idesc2, (fresh && s == 0) ? 0u : 1u);
-        }
-      };
-      FaPos t;
-      fa_seek(p, c0, qt0, t);
-      int kent = 0, kuse = 0, vent = 0, vuse = 0, nq = 0;
-      int np[2] = {0, 0}, nseg[2] = {0, 0};
-      bool ok = true;
-      {
-        // MMA1 of the first tile
-        ok = wait(&bars.qfull, 0) && wait(&bars.kfull[0], 0);
-        if (ok) {
-          ++nq;
-          tc_fence_after();
-          const uint32_t kbase = smem_u32(sK);
-          mma1(0, kbase);
-          if (qt0 + 1 < t.qtn) mma1(1, kbase);
-          umma_commit(&bars.kempty[0]);
-          if (t.j == t.nb - 1 || ntiles == 1) umma_commit(&bars.qfree);
-          kent = (nk == 1) ? 0 : 1;
-          ++kuse;
-        }
-      }
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const bool first = (t.j == 0) || (i == 0);
-        const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
-        const bool q1 = qt0 + 1 < t.qtn;
-        const bool more = i + 1 < ntiles;
-        FaPos tn = t;
-        if (more) fa_next(p, qt0, tn);
-        const bool nq1 = more && (qt0 + 1 < tn.qtn);
-        const bool nfirst = more && (tn.j == 0);
-        const bool nlast = more && ((tn.j == tn.nb - 1) || (i + 1 == ntiles - 1));
-        ok = wait(&bars.vfull[vent], (vuse / nv) & 1);
-        if (!ok) break;
-        const uint32_t vbase = smem_u32(sV + vent * kTileBytes);
-        const uint32_t knext = smem_u32(sK + kent * kTileBytes);
-        bool next_in = false;
-        // Q (first tile of a stream) and K of tile i + 1 resident
-        auto next_ready = [&]() -> bool {
-          if (next_in) return true;
-          if (nfirst) {
-            if (!wait(&bars.qfull, nq & 1)) return false;
+  if (warp < 4) {
+    // warps 0-3 (producers, MMA issuer, one idle warp) give registers to the softmax warpgroups
+    setmaxnreg_dec<kFaRoleRegs>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer: Q pairs and K
+      if (lane == 0 && ntiles > 0) {
+        FaPos t;
+        fa_seek(p, c0, qt0, t);
+        int kent = 0, kuse = 0, nq = 0;
+        bool ok = true;
+        bool skip_first = (p.debug_flags & 1u) != 0;
+        for (int i = 0; i < ntiles && ok; ++i) {
+          if (t.j == 0 || i == 0) {
+            // the stream's query tiles, once the previous stream's last MMA1 has read sQ
+            if (nq > 0) ok = wait(&bars.qfree, (nq - 1) & 1);
+            if (!ok) break;
+            const int nqt = (qt0 + 1 < t.qtn) ? 2 : 1;
+            int qc0, qrow;
+            fa_q_coord(p, t, qt0, D, qc0, qrow);
+            mbar_expect_tx(&bars.qfull, kQBytes * nqt);
+            for (int w = 0; w < nqt; ++w)
+              for (int kb = 0; kb < KB; ++kb)
+                tma_load_2d(sQ + w * kQBytes + kb * kFaSlot, &mapQ, &bars.qfull, qc0 + kb * 64, qrow + w * 128);
             ++nq;
           }
-          if (!wait(&bars.kfull[kent], (kuse / nk) & 1)) return false;
-          next_in = true;
-          return true;
-        };
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          if (w == 1 && !q1) break;
-          ok = wait(&bars.pfull[w], np[w] & 1);
+          ok = wait(&bars.kempty[kent], ((kuse / nk) & 1) ^ 1);
           if (!ok) break;
-          ++np[w];
-          if (first && nseg[w] > 0) {
-            ok = wait(&bars.ofree[w], (nseg[w] - 1) & 1);
+          int kc0, krow;
+          const CUtensorMap* mk = fa_kv_coord(p, t, D, kc0, krow) ? &mapKs : &mapK;
+          if (skip_first) {
+            skip_first = false;  // withhold this arrival: the MMA warp's wait must run out
+          } else {
+            mbar_expect_tx(&bars.kfull[kent], kTileBytes);
+            for (int kb = 0; kb < KB; ++kb)
+              tma_load_2d(sK + kent * kTileBytes + kb * kFaSlot, mk, &bars.kfull[kent], kc0 + kb * 64, krow);
+          }
+          kent = (kent + 1 == nk) ? 0 : kent + 1;
+          ++kuse;
+          fa_next(p, qt0, t);
+        }
+        fa_drain_ring(wait, bars.kfull, nk, kuse);
+        if (nq > 0) wait(&bars.qfull, (nq - 1) & 1, true);
+      }
+    } else if (warp == 2) {
+      // ------------------------------------------------------------ TMA producer: V
+      if (lane == 0 && ntiles > 0) {
+        FaPos t;
+        fa_seek(p, c0, qt0, t);
+        int vent = 0, vuse = 0;
+        bool ok = true;
+        for (int i = 0; i < ntiles && ok; ++i) {
+          ok = wait(&bars.vempty[vent], ((vuse / nv) & 1) ^ 1);
+          if (!ok) break;
+          int vc0, vrow;
+          const CUtensorMap* mv = fa_kv_coord(p, t, D, vc0, vrow) ? &mapVs : &mapV;
+          mbar_expect_tx(&bars.vfull[vent], kTileBytes);
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_2d(sV + vent * kTileBytes + kb * kFaSlot, mv, &bars.vfull[vent], vc0 + kb * 64, vrow);
+          vent = (vent + 1 == nv) ? 0 : vent + 1;
+          ++vuse;
+          fa_next(p, qt0, t);
+        }
+        fa_drain_ring(wait, bars.vfull, nv, vuse);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      // Order per key tile i: for w = 0, 1: MMA2(P_w, V_i) -> O_w, then MMA1(Q_w, K_{i+1}) -> S_w.
+      if (lane == 0 && ntiles > 0) {
+        constexpr uint32_t idesc1 = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
+        auto mma1 = [&](int w, uint32_t kbase) {
+          const uint32_t qbase = smem_u32(sQ + w * kQBytes);
+  #pragma unroll
+          for (int s = 0; s < D / 16; ++s) {
+            const uint64_t ad = sw128_desc(qbase + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(kbase + (s / 4) * kFaSlot + (s % 4) * 32, 16, 1024);
+            umma_bf16(tbase + w * 128, ad, bd, idesc1, s > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars.sfull[w]);
+        };
+        auto mma2 = [&](int w, uint32_t vbase, bool fresh) {
+  #pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint64_t bd = sw128_desc(vbase + s * 2048, kFaSlot, 1024);
+            umma_bf16_ts(tbase + 256 + w * D, tbase + w * 128 + s * 8, bd, idesc2, (fresh && s == 0) ? 0u : 1u);
+          }
+        };
+        FaPos t;
+        fa_seek(p, c0, qt0, t);
+        int kent = 0, kuse = 0, vent = 0, vuse = 0, nq = 0;
+        int np[2] = {0, 0}, nseg[2] = {0, 0};
+        bool ok = true;
+        {
+          // MMA1 of the first tile
+          ok = wait(&bars.qfull, 0) && wait(&bars.kfull[0], 0);
+          if (ok) {
+            ++nq;
+            tc_fence_after();
+            const uint32_t kbase = smem_u32(sK);
+            mma1(0, kbase);
+            if (qt0 + 1 < t.qtn) mma1(1, kbase);
+            umma_commit(&bars.kempty[0]);
+            if (t.j == t.nb - 1 || ntiles == 1) umma_commit(&bars.qfree);
+            kent = (nk == 1) ? 0 : 1;
+            ++kuse;
+          }
+        }
+        for (int i = 0; i < ntiles && ok; ++i) {
+          const bool first = (t.j == 0) || (i == 0);
+          const bool last = (t.j == t.nb - 1) || (i == ntiles - 1);
+          const bool q1 = qt0 + 1 < t.qtn;
+          const bool more = i + 1 < ntiles;
+          FaPos tn = t;
+          if (more) fa_next(p, qt0, tn);
+          const bool nq1 = more && (qt0 + 1 < tn.qtn);
+          const bool nfirst = more && (tn.j == 0);
+          const bool nlast = more && ((tn.j == tn.nb - 1) || (i + 1 == ntiles - 1));
+          ok = wait(&bars.vfull[vent], (vuse / nv) & 1);
+          if (!ok) break;
+          const uint32_t vbase = smem_u32(sV + vent * kTileBytes);
+          const uint32_t knext = smem_u32(sK + kent * kTileBytes);
+          bool next_in = false;
+          // Q (first tile of a stream) and K of tile i + 1 resident
+          auto next_ready = [&]() -> bool {
+            if (next_in) return true;
+            if (nfirst) {
+              if (!wait(&bars.qfull, nq & 1)) return false;
+              ++nq;
+            }
+            if (!wait(&bars.kfull[kent], (kuse / nk) & 1)) return false;
+            next_in = true;
+            return true;
+          };
+  #pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            if (w == 1 && !q1) break;
+            ok = wait(&bars.pfull[w], np[w] & 1);
             if (!ok) break;
+            ++np[w];
+            if (first && nseg[w] > 0) {
+              ok = wait(&bars.ofree[w], (nseg[w] - 1) & 1);
+              if (!ok) break;
+            }
+            tc_fence_after();
+            mma2(w, vbase, first);
+            if (last) {
+              umma_commit(&bars.ofull[w]);
+              ++nseg[w];
+            }
+            if (more && (w == 0 || nq1)) {
+              ok = next_ready();
+              if (!ok) break;
+              tc_fence_after();
+              mma1(w, knext);
+            }
           }
-          tc_fence_after();
-          mma2(w, vbase, first);
-          if (last) {
-            umma_commit(&bars.ofull[w]);
-            ++nseg[w];
-          }
-          if (more && (w == 0 || nq1)) {
+          if (!ok) break;
+          if (nq1 && !q1) {
+            // a stream with two query tiles after one with a single tile
             ok = next_ready();
             if (!ok) break;
             tc_fence_after();
-            mma1(w, knext);
+            mma1(1, knext);
           }
+          umma_commit(&bars.vempty[vent]);
+          vent = (vent + 1 == nv) ? 0 : vent + 1;
+          ++vuse;
+          if (more) {
+            umma_commit(&bars.kempty[kent]);
+            if (nlast) umma_commit(&bars.qfree);
+            kent = (kent + 1 == nk) ? 0 : kent + 1;
+            ++kuse;
+          }
+          t = tn;
         }
-        if (!ok) break;
-        if (nq1 && !q1) {
-          // a stream with two query tiles after one with a single tile
-          ok = next_ready();
-          if (!ok) break;
-          tc_fence_after();
-          mma1(1, knext);
-        }
-        umma_commit(&bars.vempty[vent]);
-        vent = (vent + 1 == nv) ? 0 : vent + 1;
-        ++vuse;
-        if (more) {
-          umma_commit(&bars.kempty[kent]);
-          if (nlast) umma_commit(&bars.qfree);
-          kent = (kent + 1 == nk) ? 0 : kent + 1;
-          ++kuse;
-        }
-        t = tn;
+        umma_commit(&bars.drain);
+        wait(&bars.drain, 0, true);
       }
-      umma_commit(&bars.drain);
-      wait(&bars.drain, 0, true);
     }
-  } else if (warp >= 4) {
+  } else {
+    setmaxnreg_inc<kFaSoftmaxRegs>();
     // ------------------------------------------------------------ softmax warpgroups
     // Warpgroup w (warps 4-7, 8-11) owns query tile qt0 + w: thread r holds query row r, its
     // running maximum m (the reference P is scaled against) and its running sum l.
