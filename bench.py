@@ -15,9 +15,14 @@ combine, lse fill). The other rows of the path run with --workload (same JSON co
   python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--norm proto|token]
   python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
 
-Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of the workload
-(independent users, no collective on the data path) -> weak scaling; the reported time is the
-max over ranks of the device-timed region.
+Multi-GPU (one process per GPU): `--gpus N` outside a launcher re-executes this script under
+torch.distributed.run with N ranks. The global batch is N copies of the workload's users (ragged
+lengths drawn for all N x B users at once); dp.partition_users assigns them to ranks balanced by
+length, so each rank holds about one workload's worth (weak scaling) and computes its users with
+no collective on the data path. The reported time is the max over ranks of the device-timed region.
+
+The headline (default) line also carries the token-wise normalisation of the same workload on the
+same inputs under "token", so that one run reports the forward in both normalisations.
 """
 from __future__ import annotations
 
@@ -72,14 +77,27 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def lengths_for(spec):
+def lengths_for(spec, copies=1):
+    """Packed lengths of `copies` workloads' worth of users (one draw for all of them)."""
     if isinstance(spec, list):
-        return spec
+        return spec * copies
     rng = np.random.default_rng(1 if spec == "ragged64" else 5)
     if spec == "ragged64":
-        x = np.exp(rng.uniform(math.log(1000), math.log(100_000), 64))
+        x = np.exp(rng.uniform(math.log(1000), math.log(100_000), 64 * copies))
         return [int(v) for v in np.clip(np.round(x), 1000, 100_000)]
-    return [int(v) for v in np.clip(np.round(rng.normal(85_000, 10_000, 8)), 1000, 100_000)]
+    return [int(v) for v in np.clip(np.round(rng.normal(85_000, 10_000, 8 * copies)), 1000, 100_000)]
+
+
+def rank_users(spec, rank, world):
+    """This rank's users of the global batch (world copies of the workload), assigned by
+    dp.partition_users (balanced by valid length): returns (lengths, seqused or None)."""
+    from sketch_attention_flashsa_b200 import dp
+    lens = lengths_for(spec["lens"], world)
+    su = spec.get("seqused")
+    su_all = (su * world) if su else None
+    valid = [min(a, b) for a, b in zip(lens, su_all)] if su_all else lens
+    mine = dp.partition_users(valid, world)[rank]
+    return [lens[u] for u in mine], ([su_all[u] for u in mine] if su_all else None)
 
 
 def oracle_threads():
@@ -139,24 +157,26 @@ class ClockSampler:
 # inputs), and states the step's units, algorithmic FLOPs and bytes, and its fused kernel.
 
 class SaFwdJob:
-    def __init__(self, spec, norm, rank, dev):
+    def __init__(self, spec, norm, rank, world, dev, inputs=None):
         import torch
         from sketch_attention_flashsa_b200 import api, flops
         self.api, self.norm = api, norm
-        lens = lengths_for(spec["lens"])
+        lens, su = rank_users(spec, rank, world)
         H, d, kp = spec["H"], spec["d"], spec["k"]
         T, B = sum(lens), len(lens)
-        gen = torch.Generator(device=dev)
-        gen.manual_seed(1000 + rank)
-        su = spec["seqused"]
-        self.inputs = {
-            "q": (torch.randn((H, kp, d), generator=gen, device=dev) / math.sqrt(d)).bfloat16(),
-            "k": torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
-            "v": torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
-            "cu": torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=dev),
-        }
-        if su:
-            self.inputs["seqused"] = torch.tensor(np.array(su, dtype=np.int32), device=dev)
+        if inputs is not None:
+            self.inputs = inputs  # the same tensors as another job (the headline's token-wise line)
+        else:
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(1000 + rank)
+            self.inputs = {
+                "q": (torch.randn((H, kp, d), generator=gen, device=dev) / math.sqrt(d)).bfloat16(),
+                "k": torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
+                "v": torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
+                "cu": torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=dev),
+            }
+            if su:
+                self.inputs["seqused"] = torch.tensor(np.array(su, dtype=np.int32), device=dev)
         self.valid = sum(min(a, b) for a, b in zip(lens, su)) if su else T
         self.B, self.H, self.d, self.kp = B, H, d, kp
         desc = api.sa_desc(self.inputs["q"], self.inputs["k"], self.inputs["cu"], scale=1.0, norm=norm)
@@ -196,11 +216,11 @@ class SaFwdJob:
 
 
 class SaBwdJob:
-    def __init__(self, spec, norm, rank, dev):
+    def __init__(self, spec, norm, rank, world, dev):
         import torch
         from sketch_attention_flashsa_b200 import api, flops
         self.api, self.norm = api, norm
-        lens = lengths_for(spec["lens"])
+        lens, _ = rank_users(spec, rank, world)
         H, d, kp = spec["H"], spec["d"], spec["k"]
         T, B = sum(lens), len(lens)
         gen = torch.Generator(device=dev)
@@ -259,7 +279,7 @@ class SaBwdJob:
 
 
 class StcaJob:
-    def __init__(self, spec, norm, rank, dev):
+    def __init__(self, spec, norm, rank, world, dev):
         import torch
         from sketch_attention_flashsa_b200 import api, flops
         self.api = api
@@ -338,7 +358,7 @@ def run_reference(args, rank, world):
     spec = WORKLOADS[args.workload]
     metric, unit = METRICS[spec["kind"]]
     job = _host_job(spec, args.norm)
-    budget = 4.0 if args.steps > 5 else 10.0
+    budget = args.ref_seconds if args.ref_seconds is not None else (4.0 if args.steps > 5 else 10.0)
     job.oracle_sample(0.01)  # warm-up: imports and first calls
     times, units, desc = [], [], ""
     for _ in range(args.steps):
@@ -402,6 +422,9 @@ def main():
     ap.add_argument("--norm", default="proto", choices=["proto", "token"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-token", action="store_true", help="headline: skip the token-wise line")
+    ap.add_argument("--ref-seconds", type=float, default=None,
+                    help="--impl reference: seconds of oracle work per step (default 4, or 10 for <= 5 steps)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -409,6 +432,12 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # not under a launcher: start one process per GPU and pass this run's exit status through
+        sys.exit(subprocess.call(launcher_command(args.gpus, sys.argv[1:])))
+    if "WORLD_SIZE" in os.environ and world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
 
     if args.impl == "reference":
         run_reference(args, rank, world)
@@ -427,73 +456,16 @@ def main():
 
     spec = WORKLOADS[args.workload]
     metric, unit = METRICS[spec["kind"]]
-    job = JOBS[spec["kind"]](spec, args.norm, rank, dev)
-
-    def step():
-        job.run(job.inputs)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    st = api.read_device_status(job.ws)
-    if st != 0:
-        raise SystemExit(f"device status {st} after warm-up")
-
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for a, b in kev:  # materialise the event handles
-        a.record()
-        b.record()
-    torch.cuda.synchronize()
-    uuid = None
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        pass
-    sampler = ClockSampler(uuid)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.3)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(args.steps):
-        api.set_timing_events(*kev[i])
-        step()
-    e1.record()
-    api.set_timing_events(None, None)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop()
-    kern_ms = [a.elapsed_time(b) for a, b in kev]
-    ms_total, kern_mean = dp.max_over_ranks([e0.elapsed_time(e1), statistics.mean(kern_ms)], device=dev)
-    ms_per_step = ms_total / args.steps
-    units_all = job.units * world
-    value = units_all / (ms_per_step / 1e3)
-    tflops = job.flops / (ms_per_step / 1e3) / 1e12
-
+    job = JOBS[spec["kind"]](spec, args.norm, rank, world, dev)
     peaks = load_peaks()
-    t_tensor = job.flops / (peaks["bf16_tflops"] * 1e12)
-    t_hbm = job.bytes / (peaks["hbm_gbs"] * 1e9)
-    if t_tensor >= t_hbm:
-        achieved = job.flops / (kern_mean / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                "peak_source": f"{peaks['source']} bf16 dense (burst); sustained {peaks['bf16_tflops_sustained']}"}
-    else:
-        achieved = job.bytes / (kern_mean / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"]}
-    roof.update({"kernel": job.kernel, "kernel_ms": kern_mean, "algorithmic_flops": job.flops,
-                 "algorithmic_bytes": job.bytes})
-    roof["traffic"] = traffic_for(args.workload, args.norm if spec["kind"] != "stca" else "stca")
+    res = time_job(job, args, world, dev, peaks)
+    res["roofline"]["traffic"] = traffic_for(args.workload, args.norm if spec["kind"] != "stca" else "stca")
 
     # End to end through the public API: pinned host inputs -> device, the call, result -> host.
     host = {n: t.cpu().pin_memory() for n, t in job.inputs.items()}
     devx = {n: torch.empty_like(t) for n, t in job.inputs.items()}
-    res = job.run(job.inputs)
-    hout = torch.empty(res.shape, dtype=res.dtype).pin_memory()
+    out = job.run(job.inputs)
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
 
     def e2e_step():
         for n in host:
@@ -514,8 +486,18 @@ def main():
     te = dp.max_over_ranks([f0.elapsed_time(f1) / args.e2e_steps], device=dev)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = hout.numel() * hout.element_size()
-    e2e = {"value": units_all / (te[0] / 1e3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "ms_per_step": te[0], "result_read_back": list(hout.shape)}
+    e2e = {"value": res["units_all"] / (te[0] / 1e3), "unit": unit, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": te[0], "result_read_back": list(hout.shape)}
+    del host, devx
+
+    # The headline also reports the token-wise normalisation on the same inputs.
+    token = None
+    if spec["kind"] == "sa_fwd" and args.norm == "proto" and not args.no_token:
+        tjob = SaFwdJob(spec, "token", rank, world, dev, inputs=job.inputs)
+        tres = time_job(tjob, args, world, dev, peaks)
+        tres["roofline"]["traffic"] = traffic_for(args.workload, "token")
+        token = {"value": tres["value"], "unit": unit, "ms_per_step": tres["ms_per_step"], "tflops": tres["tflops"],
+                 "roofline": tres["roofline"], "gpu_launches": tjob.launches * args.steps, "clocks": tres["clocks"]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -524,16 +506,92 @@ def main():
                "sample": f"{desc}, {secs:.1f} s incl. host copies of the slices"}
 
     if rank == 0:
-        line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        line = {"metric": metric, "value": res["value"], "unit": unit, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": args.workload, **job.config,
-                           "parallelism": f"dp{world} (independent users per rank)"},
-                "tflops": tflops, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": job.launches * args.steps, "clocks": clocks}
+                           "parallelism": f"dp{world} (users partitioned over ranks by length, no collective)"},
+                "tflops": res["tflops"], "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": job.launches * args.steps, "clocks": res["clocks"]}
+        if token is not None:
+            line["token"] = token
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def launcher_command(gpus, argv):
+    """torch.distributed.run with one process per GPU on this node (rendezvous on 127.0.0.1)."""
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
+def time_job(job, args, world, dev, peaks):
+    """W warm-up steps, then K steps between a barrier and a synchronize on both sides, timed with
+    CUDA events on the launching stream (the whole step and, through the library's timing hook,
+    its fused kernel); clocks sampled meanwhile; times are the max over ranks."""
+    import torch
+    import torch.distributed as dist
+    from sketch_attention_flashsa_b200 import api, dp
+
+    for _ in range(args.warmup):
+        job.run(job.inputs)
+    torch.cuda.synchronize()
+    st = api.read_device_status(job.ws)
+    if st != 0:
+        raise SystemExit(f"device status {st} after warm-up")
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in kev:  # materialise the event handles
+        a.record()
+        b.record()
+    torch.cuda.synchronize()
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        api.set_timing_events(*kev[i])
+        job.run(job.inputs)
+    e1.record()
+    api.set_timing_events(None, None)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    kern_mean = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    ms_total, kern_max = dp.max_over_ranks([e0.elapsed_time(e1), kern_mean], device=dev)
+    units_all, flops_all = dp.sum_over_ranks([job.units, job.flops], device=dev)
+    ms_per_step = ms_total / args.steps
+    t_tensor = job.flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = job.bytes / (peaks["hbm_gbs"] * 1e9)
+    # the dominant kernel's rate on each rank (its own work over its own kernel time), slowest rank
+    if t_tensor >= t_hbm:
+        achieved = -dp.max_over_ranks([-(job.flops / (kern_mean / 1e3) / 1e12)], device=dev)[0]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": f"{peaks['source']} bf16 dense (burst); sustained {peaks['bf16_tflops_sustained']}"}
+    else:
+        achieved = -dp.max_over_ranks([-(job.bytes / (kern_mean / 1e3) / 1e9)], device=dev)[0]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"]}
+    roof.update({"kernel": job.kernel, "kernel_ms": kern_max, "algorithmic_flops": job.flops,
+                 "algorithmic_bytes": job.bytes})
+    return {"ms_per_step": ms_per_step, "value": units_all / (ms_per_step / 1e3),
+            "tflops": flops_all / (ms_per_step / 1e3) / 1e12, "roofline": roof, "clocks": clocks,
+            "units_all": units_all}
 
 
 if __name__ == "__main__":

@@ -34,15 +34,19 @@
  *              SKA_ERR_UNSUPPORTED, SKA_ERR_WORKSPACE_TOO_SMALL); a failed launch returns
  *              SKA_ERR_CUDA. A kernel that waits longer than its time budget on a pipeline
  *              barrier stops, records SKA_ERR_DEVICE_TIMEOUT in the workspace status word and
- *              exits; ska_read_device_status() reports it.
+ *              exits; ska_read_device_status() reports it. Whenever a call's status word holds
+ *              an error, that call's outputs are NaN, never plausible-looking values.
  *   Outputs    Outputs are fully overwritten (zeros for empty users). No output may alias an
  *              input. k and v may alias each other (the paper's V = X).
  *   Padding    Tokens of user b at positions >= seqused[b] take no part in the result, but their
  *              rows must hold finite numbers (a zero weight times a non-finite value is NaN).
  *   Precision  Scores S = scale Q K^T are exact products of the bf16 inputs summed in fp32; the
- *              softmax runs in fp32; the aggregation A V multiplies fp16-rounded weights A with
- *              the values converted to fp16 (exact for |v| in [2^-14, 65504]; larger magnitudes
- *              saturate to 65504) and accumulates in fp32.
+ *              softmax runs in fp32. SKA_NORM_PROTO aggregates in fp16 with fp32 accumulation:
+ *              each value row v_i enters as fp16(w_i v_i), w_i the largest weight of token i
+ *              among the prototypes of one CTA, times fp16 weights A / w_i in (0, 1]; this needs
+ *              |w_i v_i| < 65520, else the product is infinite, the call records
+ *              SKA_ERR_RANGE in the device status word and its outputs are NaN. SKA_NORM_TOKEN
+ *              and STCA aggregate bf16 weights with the bf16 values in fp32.
  *   Determinism  Results are bitwise reproducible run to run (fixed-order reductions).
  */
 #ifndef SKETCH_ATTN_H_
@@ -68,7 +72,8 @@ typedef enum {
   SKA_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. head_dim not 64/128) */
   SKA_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < *_workspace_size(desc) */
   SKA_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
-  SKA_ERR_DEVICE_TIMEOUT = 5       /* a kernel gave up waiting on a pipeline barrier */
+  SKA_ERR_DEVICE_TIMEOUT = 5,      /* a kernel gave up waiting on a pipeline barrier */
+  SKA_ERR_RANGE = 6                /* a value is outside the range the kernel represents */
 } ska_status;
 
 typedef enum { SKA_BF16 = 0, SKA_F32 = 1 } ska_dtype;
@@ -81,8 +86,11 @@ typedef enum {
 /* One batched SA problem: num_users ragged users, each with its own history.
  *   num_heads    H >= 1
  *   head_dim     d, 64 or 128
- *   num_protos   k: a multiple of 16 in [16, 256], or 512, 1024, 2048 (k/ceil(k/256) a
- *                multiple of 16)
+ *   num_protos   k >= 1. SKA_NORM_TOKEN: any k. SKA_NORM_PROTO: k / ceil(k / 256) in
+ *                {16, 32, 64, 96, 128, 192, 256}, e.g. 16, 32, 64, 96, 128, 192, 256, 384, 512,
+ *                576, 768, 1024; also 1536 and 2048 with head_dim 64 (with d = 128 the cluster
+ *                exchange of k/256 CTAs does not fit shared memory); other k give
+ *                SKA_ERR_UNSUPPORTED
  *   total_tokens rows of k and v (= cu_seqlens[num_users]); < 2^31
  *   max_seqlen   an upper bound on any user's length (informational; may be 0)
  *   scale        multiplies Q K^T; must be > 0 and finite (1/sqrt(d) in Eq. (7))
@@ -117,7 +125,11 @@ SKA_API size_t sa_forward_workspace_size(const ska_sa_desc* desc);
  *               the k prototypes (-inf on padding rows). TOKEN: [B, H, k], the per-prototype
  *               log-sum-exp over the valid tokens (-inf for an empty user). The backward pass
  *               needs it.
- *   mass        out, fp32 [B, H, k] or NULL: sum_i A[j,i], the mass each prototype received.  */
+ *   mass        out, fp32 [B, H, k] or NULL: sum_i A[j,i] over the valid tokens, the mass each
+ *               prototype received (PROTO: sum_j mass = the user's valid length; TOKEN: 1, or 0
+ *               for an empty user). In PROTO mode a CTA then holds at most 128 prototypes,
+ *               which limits k to 1024 and makes the call slower; without it (NULL) the call
+ *               runs at full speed.                                                          */
 SKA_API ska_status sa_forward(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
                       const int32_t* cu_seqlens, const int32_t* seqused, float* sketch, float* lse,
                       float* mass, void* ws, size_t ws_bytes, void* stream);
@@ -212,6 +224,13 @@ SKA_API ska_status sa_forward_noalloc(const ska_sa_desc* desc, const void* q, co
 
 /* Size in bytes of the device array that sa_forward_noalloc uses as scratch. */
 SKA_API size_t sa_forward_noalloc_scratch_bytes(void);
+
+/* Device status of the sa_forward_noalloc calls on the current device: synchronises `stream`,
+ * then returns SKA_OK or the first device-side error the last call recorded in the shared
+ * array's status word (e.g. SKA_ERR_DEVICE_TIMEOUT, SKA_ERR_RANGE) and clears it. The next
+ * sa_forward_noalloc call clears the word itself, so read it before that call. Blocks the host.
+ * Returns SKA_ERR_CUDA when the array cannot be reached (no usable device).                  */
+SKA_API ska_status sa_forward_noalloc_read_status(void* stream);
 
 /* Bench hook (process-wide): while both handles are non-NULL, every later call records
  * `start_event` on its stream immediately before its fused main kernel and `stop_event`

@@ -13,6 +13,7 @@ SKA_ERR_UNSUPPORTED = 2
 SKA_ERR_WORKSPACE_TOO_SMALL = 3
 SKA_ERR_CUDA = 4
 SKA_ERR_DEVICE_TIMEOUT = 5
+SKA_ERR_RANGE = 6
 
 SKA_BF16 = 0
 SKA_F32 = 1
@@ -22,7 +23,8 @@ SKA_NORM_TOKEN = 1
 EXPORTED = ("sa_forward_workspace_size", "sa_forward", "sa_backward_workspace_size", "sa_backward",
             "stca_forward_workspace_size", "stca_forward", "ska_status_string",
             "ska_read_device_status", "ska_set_debug", "ska_set_timing_events",
-            "sa_forward_noalloc", "sa_forward_noalloc_scratch_bytes", "ska_last_error_string")
+            "sa_forward_noalloc", "sa_forward_noalloc_scratch_bytes", "sa_forward_noalloc_read_status",
+            "ska_last_error_string")
 
 
 class SaDesc(ctypes.Structure):
@@ -87,6 +89,8 @@ def lib() -> ctypes.CDLL:
     L.sa_forward_noalloc.restype = ctypes.c_int
     L.sa_forward_noalloc_scratch_bytes.argtypes = []
     L.sa_forward_noalloc_scratch_bytes.restype = sz
+    L.sa_forward_noalloc_read_status.argtypes = [vp]
+    L.sa_forward_noalloc_read_status.restype = ctypes.c_int
     L.ska_set_timing_events.argtypes = [vp, vp]
     L.ska_set_timing_events.restype = None
     _lib = L

@@ -27,12 +27,44 @@ def _stream(stream) -> ctypes.c_void_p:
 def _dev_tensor(name, t, dtypes):
     if t is None:
         return
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if t.dtype not in dtypes:
-        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+
+
+def _shape(name, t, want):
+    if t is not None and tuple(t.shape) != tuple(want):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(want)}")
+
+
+def _check_sa_inputs(q, k, v, cu_seqlens, seqused, dtypes):
+    """Shapes and dtypes of an SA call's inputs, checked against one another on the host (the C ABI
+    takes the sizes from the descriptor and cannot see a mismatched buffer)."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype not in dtypes:
+            raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError(f"q, k and v must share one dtype (got {q.dtype}, {k.dtype}, {v.dtype})")
+    if k.dim() != 3:
+        raise ValueError(f"k must be [T, H, d], got shape {tuple(k.shape)}")
+    _shape("v", v, k.shape)
+    if q.dim() not in (3, 4):
+        raise ValueError(f"q must be [H, k, d] or [B, H, k, d], got shape {tuple(q.shape)}")
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1 or cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor of B + 1 offsets")
+    B = cu_seqlens.numel() - 1
+    H, d = k.shape[1], k.shape[2]
+    if q.shape[-3] != H or q.shape[-1] != d:
+        raise ValueError(f"q {tuple(q.shape)} does not match k's heads {H} and head_dim {d}")
+    if q.dim() == 4 and q.shape[0] != B:
+        raise ValueError(f"per-user q has {q.shape[0]} users, cu_seqlens describes {B}")
+    if seqused is not None:
+        if seqused.dtype != torch.int32 or tuple(seqused.shape) != (B,):
+            raise ValueError(f"seqused must be int32 of shape ({B},)")
+    return B, H, q.shape[-2], d
 
 
 def _check(rc: int, what: str):
@@ -64,20 +96,28 @@ def sa_forward_workspace_size(desc: SaDesc) -> int:
 def sa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
                seqused: Optional[torch.Tensor] = None, *, scale: float = 1.0, norm="proto",
                want_lse: bool = True, want_mass: bool = False, workspace: Optional[torch.Tensor] = None,
-               out: Optional[torch.Tensor] = None, lse_out: Optional[torch.Tensor] = None, stream=None):
+               out: Optional[torch.Tensor] = None, lse_out: Optional[torch.Tensor] = None,
+               mass_out: Optional[torch.Tensor] = None, stream=None):
     """Sketch Attention forward (SequenceO1 §3.1 Eq. (7)-(9), FlashSA §4.4).
 
-    q [H,k,d] or [B,H,k,d]; k, v [T,H,d] (bf16, or fp32 rounded to bf16 on the device);
-    cu_seqlens int32 [B+1]; seqused int32 [B] or None. Returns (sketch fp32 [B,H,k,d],
-    lse or None, mass or None).
+    q [H,k,d] or [B,H,k,d]; k, v [T,H,d] (bf16, or fp32 rounded to bf16 on the device; all three
+    of one dtype); cu_seqlens int32 [B+1]; seqused int32 [B] or None. out / lse_out / mass_out:
+    optional preallocated outputs. Returns (sketch fp32 [B,H,k,d], lse or None, mass or None):
+    lse is [T,H] (prototype-wise) or [B,H,k] (token-wise); mass [B,H,k] = sum_i A[j,i].
     """
-    dts = (torch.bfloat16, torch.float32)
+    B, H, kp, D = _check_sa_inputs(q, k, v, cu_seqlens, seqused, (torch.bfloat16, torch.float32))
+    nid = _NORMS[norm]
+    T = k.shape[0]
+    _shape("out", out, (B, H, kp, D))
+    _shape("lse_out", lse_out, (T, H) if nid == _lib.SKA_NORM_PROTO else (B, H, kp))
+    _shape("mass_out", mass_out, (B, H, kp))
+    for name, t in (("out", out), ("lse_out", lse_out), ("mass_out", mass_out)):
+        _dev_tensor(name, t, (torch.float32,))
     for name, t in (("q", q), ("k", k), ("v", v)):
-        _dev_tensor(name, t, dts)
+        _dev_tensor(name, t, (torch.bfloat16, torch.float32))
     _dev_tensor("cu_seqlens", cu_seqlens, (torch.int32,))
     _dev_tensor("seqused", seqused, (torch.int32,))
     desc = sa_desc(q, k, cu_seqlens, scale=scale, norm=norm)
-    B, H, D, kp, T = desc.num_users, desc.num_heads, desc.head_dim, desc.num_protos, desc.total_tokens
     dev = k.device
     need = sa_forward_workspace_size(desc)
     if need == 0 and B > 0:
@@ -86,15 +126,46 @@ def sa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: to
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     sketch = out if out is not None else torch.empty((B, H, kp, D), dtype=torch.float32, device=dev)
     lse = None
-    if want_lse:
+    if want_lse or lse_out is not None:
         shape = (T, H) if desc.norm == _lib.SKA_NORM_PROTO else (B, H, kp)
         lse = lse_out if lse_out is not None else torch.empty(shape, dtype=torch.float32, device=dev)
-    mass = torch.empty((B, H, kp), dtype=torch.float32, device=dev) if want_mass else None
+    mass = None
+    if want_mass or mass_out is not None:
+        mass = mass_out if mass_out is not None else torch.empty((B, H, kp), dtype=torch.float32, device=dev)
     rc = _lib.lib().sa_forward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
                                _ptr(seqused), _ptr(sketch), _ptr(lse), _ptr(mass), _ptr(workspace),
                                ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check(rc, "sa_forward")
     return sketch, lse, mass
+
+
+def sa_forward_noalloc(q, k, v, cu_seqlens, seqused=None, *, scale: float = 1.0, norm="proto", out=None,
+                       lse_out=None, mass_out=None, stream=None):
+    """sa_forward for callers that cannot allocate device memory: scratch comes from a fixed array
+    inside libska.so (sa_forward_noalloc_scratch_bytes()). The outputs must be preallocated."""
+    B, H, kp, D = _check_sa_inputs(q, k, v, cu_seqlens, seqused, (torch.bfloat16, torch.float32))
+    nid = _NORMS[norm]
+    if out is None:
+        raise ValueError("sa_forward_noalloc writes into a preallocated out")
+    _shape("out", out, (B, H, kp, D))
+    _shape("lse_out", lse_out, (k.shape[0], H) if nid == _lib.SKA_NORM_PROTO else (B, H, kp))
+    _shape("mass_out", mass_out, (B, H, kp))
+    for name, t in (("out", out), ("lse_out", lse_out), ("mass_out", mass_out)):
+        _dev_tensor(name, t, (torch.float32,))
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _dev_tensor(name, t, (torch.bfloat16, torch.float32))
+    _dev_tensor("cu_seqlens", cu_seqlens, (torch.int32,))
+    _dev_tensor("seqused", seqused, (torch.int32,))
+    desc = sa_desc(q, k, cu_seqlens, scale=scale, norm=norm)
+    rc = _lib.lib().sa_forward_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                                       _ptr(seqused), _ptr(out), _ptr(lse_out), _ptr(mass_out), _stream(stream))
+    _check(rc, "sa_forward_noalloc")
+    return out, lse_out, mass_out
+
+
+def read_noalloc_status(stream=None) -> int:
+    """Device status of the last sa_forward_noalloc call on this device (synchronises, then clears)."""
+    return int(_lib.lib().sa_forward_noalloc_read_status(_stream(stream)))
 
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:
@@ -141,9 +212,36 @@ def stca_forward(q: torch.Tensor, cu_targets: torch.Tensor, k_hist: torch.Tensor
     q [Tq,H,d] bf16 with cu_targets int32 [B+1]; k_hist, v_hist [Th,H,d] bf16 with cu_hist;
     k_sk, v_sk [B,H,ks,d] bf16 or None; target_kv_len int32 [Tq] or None; max_targets: an upper
     bound on any user's target count (read from cu_targets when None, which synchronises);
-    out / lse_out: preallocated outputs (fp32 [Tq,H,d] / [Tq,H]).
+    out / lse_out: preallocated outputs (fp32 [Tq,H,d] / [Tq,H]). A max_targets below a user's
+    real target count is recorded in the device status word and makes every output NaN.
     Returns (out fp32 [Tq,H,d], lse fp32 [Tq,H] or None).
     """
+    for name, t in (("q", q), ("k_hist", k_hist), ("v_hist", v_hist), ("k_sk", k_sk), ("v_sk", v_sk)):
+        if t is not None and t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} has dtype {t.dtype}, expected torch.bfloat16")
+    if q.dim() != 3:
+        raise ValueError(f"q must be [Tq, H, d], got shape {tuple(q.shape)}")
+    Tq, H, D = q.shape
+    for name, t in (("cu_targets", cu_targets), ("cu_hist", cu_hist)):
+        if t.dtype != torch.int32 or t.dim() != 1 or t.numel() < 1:
+            raise ValueError(f"{name} must be a 1-D int32 tensor of B + 1 offsets")
+    B = cu_targets.numel() - 1
+    if cu_hist.numel() != B + 1:
+        raise ValueError(f"cu_hist has {cu_hist.numel()} entries, cu_targets {B + 1}")
+    if k_hist is not None:
+        if k_hist.dim() != 3 or k_hist.shape[1:] != (H, D):
+            raise ValueError(f"k_hist {tuple(k_hist.shape)} does not match q's heads and head_dim")
+        _shape("v_hist", v_hist, k_hist.shape)
+    if (k_sk is None) != (v_sk is None):
+        raise ValueError("k_sk and v_sk come together")
+    if k_sk is not None:
+        if k_sk.dim() != 4 or k_sk.shape[0] != B or k_sk.shape[1] != H or k_sk.shape[3] != D:
+            raise ValueError(f"k_sk must be [{B}, {H}, ks, {D}], got {tuple(k_sk.shape)}")
+        _shape("v_sk", v_sk, k_sk.shape)
+    if target_kv_len is not None and (target_kv_len.dtype != torch.int32 or tuple(target_kv_len.shape) != (Tq,)):
+        raise ValueError(f"target_kv_len must be int32 of shape ({Tq},)")
+    _shape("out", out, (Tq, H, D))
+    _shape("lse_out", lse_out, (Tq, H))
     if max_targets is None:
         max_targets = int((cu_targets[1:] - cu_targets[:-1]).max().item()) if cu_targets.numel() > 1 else 0
     for name, t in (("q", q), ("k_hist", k_hist), ("v_hist", v_hist), ("k_sk", k_sk), ("v_sk", v_sk)):
@@ -185,6 +283,19 @@ def sa_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: t
     optional preallocated (dq, dk, dv).
     Returns (dq fp32 shaped like q, dk fp32 [T,H,d], dv fp32 [T,H,d]).
     """
+    B, H, kp, D = _check_sa_inputs(q, k, v, cu_seqlens, seqused, (torch.bfloat16,))
+    nid = _NORMS[norm]
+    if dsketch.dtype != torch.bfloat16:
+        raise ValueError(f"dsketch has dtype {dsketch.dtype}, expected torch.bfloat16")
+    _shape("dsketch", dsketch, (B, H, kp, D))
+    if lse.dtype != torch.float32:
+        raise ValueError(f"lse has dtype {lse.dtype}, expected torch.float32")
+    _shape("lse", lse, (k.shape[0], H) if nid == _lib.SKA_NORM_PROTO else (B, H, kp))
+    if nid == _lib.SKA_NORM_TOKEN and sketch is None:
+        raise ValueError("the token-wise backward needs the forward sketch (D_j = dO_j . O_j)")
+    if sketch is not None and sketch.dtype != torch.float32:
+        raise ValueError(f"sketch has dtype {sketch.dtype}, expected torch.float32")
+    _shape("sketch", sketch, (B, H, kp, D))
     for name, t in (("q", q), ("k", k), ("v", v), ("dsketch", dsketch)):
         _dev_tensor(name, t, (torch.bfloat16,))
     _dev_tensor("lse", lse, (torch.float32,))

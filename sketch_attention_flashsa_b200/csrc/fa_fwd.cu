@@ -205,9 +205,14 @@ __global__ void __launch_bounds__(1024) fa_schedule_kernel(const FaFwdParams p, 
 
 // ---------------------------------------------------------------- combine
 // One block per (user, head, query tile) up to B * H * G; thread r merges row r of the stream
-// over the partial slots ((b H + h) + g) G + qt of the groups g that walked its columns.
+// over the partial slots ((b H + h) + g) G + qt of the groups g that walked its columns. When an
+// earlier kernel of the call recorded an error (a bounded wait that ran out, a user with more
+// targets than max_targets) every output of the call is NaN. Token-wise SA also writes the
+// mass of each prototype, sum_i A[j, i], which the softmax over tokens makes 1 (0 for a user
+// without valid tokens).
 __global__ void __launch_bounds__(128) fa_combine_kernel(const FaFwdParams p, int D, int G, float* __restrict__ out,
-                                                         float* __restrict__ lse) {
+                                                         float* __restrict__ lse, float* __restrict__ mass) {
+  const bool failed = *reinterpret_cast<const volatile int32_t*>(&p.hdr->status) != 0;
   const int qt = blockIdx.x % G;
   const int bh = blockIdx.x / G;
   const int b = bh / p.H, h = bh - b * p.H;
@@ -222,35 +227,45 @@ __global__ void __launch_bounds__(128) fa_combine_kernel(const FaFwdParams p, in
     g1 = (c0 + nb - 1) / W;
   }
   const int r = threadIdx.x;
-  const int q = qt * 128 + r;
   const int nq = (p.mode == 0) ? p.k : (p.cu_q[b + 1] - p.cu_q[b]);
-  if (q >= nq) return;
-  auto slot = [&](int g) { return (static_cast<int64_t>(bh + g) * G + qt) * 128 + r; };
-  float M = -INFINITY;
-  for (int g = g0; g <= g1; ++g) M = fmaxf(M, p.part_ml[slot(g) * 2]);
-  float L = 0.f;
-  for (int g = g0; g <= g1; ++g) {
-    const float mg = p.part_ml[slot(g) * 2];
-    if (mg != -INFINITY) L += p.part_ml[slot(g) * 2 + 1] * exp2f(mg - M);
-  }
-  const float inv = (L > 0.f) ? 1.f / L : 0.f;
-  int64_t orow;
-  if (p.mode == 0) orow = (static_cast<int64_t>(b) * p.H + h) * p.k + q;
-  else orow = static_cast<int64_t>(p.cu_q[b] + q) * p.H + h;
-  float* dst = out + orow * D;
-  for (int dd = 0; dd < D; dd += 4) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int g = g0; g <= g1; ++g) {
-      const float mg = p.part_ml[slot(g) * 2];
-      if (mg == -INFINITY) continue;
-      const float wg = exp2f(mg - M);
-      const float4 v = *reinterpret_cast<const float4*>(p.part_o + slot(g) * D + dd);
-      acc.x += wg * v.x; acc.y += wg * v.y; acc.z += wg * v.z; acc.w += wg * v.w;
+  auto slot = [&](int g, int q) { return (static_cast<int64_t>(bh + g) * G + qt) * 128 + (q & 127); };
+  // Rows qt*128 + r, then G*128 further on: the second and later rows exist only when a user has
+  // more query tiles than G, which the schedule records as an error; they are written as NaN.
+  for (int q = qt * 128 + r; q < nq; q += G * 128) {
+    const bool bad = failed || q >= G * 128;
+    float M = -INFINITY;
+    float L = 0.f;
+    if (!bad) {
+      for (int g = g0; g <= g1; ++g) M = fmaxf(M, p.part_ml[slot(g, q) * 2]);
+      for (int g = g0; g <= g1; ++g) {
+        const float mg = p.part_ml[slot(g, q) * 2];
+        if (mg != -INFINITY) L += p.part_ml[slot(g, q) * 2 + 1] * exp2f(mg - M);
+      }
     }
-    acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
-    *reinterpret_cast<float4*>(dst + dd) = acc;
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    int64_t orow;
+    if (p.mode == 0) orow = (static_cast<int64_t>(b) * p.H + h) * p.k + q;
+    else orow = static_cast<int64_t>(p.cu_q[b] + q) * p.H + h;
+    float* dst = out + orow * D;
+    for (int dd = 0; dd < D; dd += 4) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (!bad) {
+        for (int g = g0; g <= g1; ++g) {
+          const float mg = p.part_ml[slot(g, q) * 2];
+          if (mg == -INFINITY) continue;
+          const float wg = exp2f(mg - M);
+          const float4 v = *reinterpret_cast<const float4*>(p.part_o + slot(g, q) * D + dd);
+          acc.x += wg * v.x; acc.y += wg * v.y; acc.z += wg * v.z; acc.w += wg * v.w;
+        }
+        acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+      } else {
+        acc = make_float4(NAN, NAN, NAN, NAN);
+      }
+      *reinterpret_cast<float4*>(dst + dd) = acc;
+    }
+    if (lse) lse[orow] = bad ? NAN : (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    if (mass) mass[orow] = bad ? NAN : (L > 0.f) ? 1.f : 0.f;
   }
-  if (lse) lse[orow] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 struct FaBars {
@@ -738,10 +753,10 @@ cudaError_t launch_fa_schedule(const FaFwdParams& p, int num_ctas, cudaStream_t 
   return cudaGetLastError();
 }
 
-cudaError_t launch_fa_combine(const FaFwdParams& p, int D, int max_streams, float* out, float* lse,
+cudaError_t launch_fa_combine(const FaFwdParams& p, int D, int max_streams, float* out, float* lse, float* mass,
                               cudaStream_t stream) {
   if (max_streams <= 0) return cudaSuccess;
-  fa_combine_kernel<<<max_streams, 128, 0, stream>>>(p, D, p.group, out, lse);
+  fa_combine_kernel<<<max_streams, 128, 0, stream>>>(p, D, p.group, out, lse, mass);
   return cudaGetLastError();
 }
 

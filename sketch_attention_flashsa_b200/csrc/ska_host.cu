@@ -134,6 +134,10 @@ ska_status check_sa_desc(const ska_sa_desc* d) {
   if (d->num_protos < 1) return SKA_ERR_INVALID_VALUE;
   if (d->head_dim != 64 && d->head_dim != 128) return SKA_ERR_UNSUPPORTED;
   if (int64_t(d->num_users) * d->num_heads >= (int64_t(1) << 30)) return SKA_ERR_INVALID_VALUE;
+  // The concatenated tile stream (H * sum_b ceil(len_b / 128) <= H * (T / 128 + B)) is indexed
+  // with 32-bit integers on the device.
+  if (int64_t(d->num_heads) * (d->total_tokens / 128 + d->num_users + 1) >= (int64_t(1) << 31))
+    return SKA_ERR_INVALID_VALUE;
   return SKA_OK;
 }
 
@@ -168,10 +172,14 @@ bool fwd_ws_layout(const ska_sa_desc* d, const ProtoFwdLaunch& L, FwdWs* w) {
   return true;
 }
 
-bool plan_forward(const ska_sa_desc* d, ProtoFwdLaunch* L, int* nk, int* nv) {
+bool plan_forward(const ska_sa_desc* d, bool mass, ProtoFwdLaunch* L, int* nk, int* nv) {
   const int sms = device_sm_count();
   if (sms <= 0) return false;
-  return proto_fwd_plan(d->head_dim, d->num_protos, sms, L, nk, nv);
+  if (!proto_fwd_plan(d->head_dim, d->num_protos, sms, mass, L, nk, nv)) return false;
+  // persistent clusters: no more than the device holds at once (a second wave would double the time)
+  const int resident = proto_fwd_max_clusters(d->head_dim, *L);
+  if (resident > 0 && resident < L->num_clusters) L->num_clusters = resident;
+  return true;
 }
 
 // ---------------------------------------------------------------- row-softmax engine (token SA, STCA)
@@ -230,7 +238,7 @@ size_t sa_token_ws_size(const ska_sa_desc* d, FaWs* w, int* ctas, size_t* smem, 
 
 ska_status sa_forward_token(const ska_sa_desc* d, const void* q, const void* k, const void* v,
                             const int32_t* cu_seqlens, const int32_t* seqused, float* sketch, float* lse,
-                            void* ws, size_t ws_bytes, cudaStream_t s) {
+                            float* mass, void* ws, size_t ws_bytes, cudaStream_t s) {
   const int B = d->num_users, H = d->num_heads, D = d->head_dim, kp = d->num_protos;
   const int64_t T = d->total_tokens;
   FaWs w;
@@ -291,7 +299,7 @@ ska_status sa_forward_token(const ska_sa_desc* d, const void* q, const void* k, 
       return SKA_ERR_CUDA;
     }
   }
-  if (cudaError_t e_ = launch_fa_combine(p, D, B * H * p.group, sketch, lse, s); e_ != cudaSuccess) { record_error("launch_fa_combine", e_); return SKA_ERR_CUDA; }
+  if (cudaError_t e_ = launch_fa_combine(p, D, B * H * p.group, sketch, lse, mass, s); e_ != cudaSuccess) { record_error("launch_fa_combine", e_); return SKA_ERR_CUDA; }
   return SKA_OK;
 }
 
@@ -303,6 +311,10 @@ ska_status check_stca_desc(const ska_stca_desc* d) {
   if (!(d->scale > 0.f) || !std::isfinite(d->scale)) return SKA_ERR_INVALID_VALUE;
   if (d->head_dim != 64 && d->head_dim != 128) return SKA_ERR_UNSUPPORTED;
   if (int64_t(d->num_users) * d->num_heads * std::max(d->num_sketch, 1) >= (int64_t(1) << 31))
+    return SKA_ERR_INVALID_VALUE;
+  // key-tile columns: H * sum_b (ceil(hist_b / 128) + ceil(ks / 128)), 32-bit on the device
+  if (int64_t(d->num_heads) * (d->total_hist / 128 + int64_t(d->num_users) * (d->num_sketch / 128 + 2) + 1) >=
+      (int64_t(1) << 31))
     return SKA_ERR_INVALID_VALUE;
   return SKA_OK;
 }
@@ -336,6 +348,7 @@ const char* ska_status_string(ska_status s) {
     case SKA_ERR_WORKSPACE_TOO_SMALL: return "SKA_ERR_WORKSPACE_TOO_SMALL";
     case SKA_ERR_CUDA: return "SKA_ERR_CUDA";
     case SKA_ERR_DEVICE_TIMEOUT: return "SKA_ERR_DEVICE_TIMEOUT";
+    case SKA_ERR_RANGE: return "SKA_ERR_RANGE";
   }
   return "SKA_ERR_UNKNOWN";
 }
@@ -372,12 +385,19 @@ size_t sa_forward_workspace_size(const ska_sa_desc* d) {
     size_t sm;
     return sa_token_ws_size(d, &w, &c, &sm, &nk, &nv);
   }
+  // Enough for the call with or without the mass output (their plans differ in cluster count,
+  // hence in partial slots).
   ProtoFwdLaunch L;
   int nk, nv;
-  if (!plan_forward(d, &L, &nk, &nv)) return 0;
+  if (!plan_forward(d, false, &L, &nk, &nv)) return 0;
   FwdWs w;
   fwd_ws_layout(d, L, &w);
-  return w.total;
+  size_t total = w.total;
+  if (plan_forward(d, true, &L, &nk, &nv)) {
+    fwd_ws_layout(d, L, &w);
+    total = std::max(total, w.total);
+  }
+  return total;
 }
 
 ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
@@ -385,7 +405,6 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
                       void* stream) {
   ska_status st = check_sa_desc(d);
   if (st != SKA_OK) return st;
-  if (mass) return SKA_ERR_UNSUPPORTED;
   const int B = d->num_users, H = d->num_heads, D = d->head_dim, kp = d->num_protos;
   const int64_t T = d->total_tokens;
   if (B == 0) return SKA_OK;
@@ -396,31 +415,38 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
       !aligned16(mass) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
       (reinterpret_cast<uintptr_t>(seqused) & 3u))
     return SKA_ERR_INVALID_VALUE;
-  if (no_device()) return SKA_ERR_CUDA;
-  const size_t ws_need = sa_forward_workspace_size(d);
-  if (ws_need == 0) return SKA_ERR_UNSUPPORTED;
-  if (ws_bytes < ws_need) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  // outputs against inputs and each other (host-only checks, before any device query)
   const size_t esz = d->in_dtype == SKA_F32 ? 4 : 2;
   const size_t qn = size_t(d->q_per_user ? B : 1) * H * kp * D;
   const size_t kvn = size_t(T) * H * D;
   const size_t sk_bytes = size_t(B) * H * kp * D * 4;
   const size_t lse_bytes = (d->norm == SKA_NORM_PROTO ? size_t(T) : size_t(B) * kp) * H * 4;
+  const size_t mass_bytes = size_t(B) * H * kp * 4;
   if (overlaps(sketch, sk_bytes, q, qn * esz) || overlaps(sketch, sk_bytes, k, kvn * esz) ||
       overlaps(sketch, sk_bytes, v, kvn * esz) || overlaps(lse, lse_bytes, q, qn * esz) ||
       overlaps(lse, lse_bytes, k, kvn * esz) || overlaps(lse, lse_bytes, v, kvn * esz) ||
-      overlaps(lse, lse_bytes, sketch, sk_bytes) || overlaps(ws, ws_need, sketch, sk_bytes) ||
-      overlaps(ws, ws_need, lse, lse_bytes) || overlaps(ws, ws_need, q, qn * esz) ||
-      overlaps(ws, ws_need, k, kvn * esz) || overlaps(ws, ws_need, v, kvn * esz))
+      overlaps(lse, lse_bytes, sketch, sk_bytes) || overlaps(mass, mass_bytes, q, qn * esz) ||
+      overlaps(mass, mass_bytes, k, kvn * esz) || overlaps(mass, mass_bytes, v, kvn * esz) ||
+      overlaps(mass, mass_bytes, sketch, sk_bytes) || overlaps(mass, mass_bytes, lse, lse_bytes))
+    return SKA_ERR_INVALID_VALUE;
+  if (no_device()) return SKA_ERR_CUDA;
+  const size_t ws_need = sa_forward_workspace_size(d);
+  if (ws_need == 0) return SKA_ERR_UNSUPPORTED;
+  if (ws_bytes < ws_need) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  if (overlaps(ws, ws_need, sketch, sk_bytes) || overlaps(ws, ws_need, lse, lse_bytes) ||
+      overlaps(ws, ws_need, q, qn * esz) || overlaps(ws, ws_need, k, kvn * esz) ||
+      overlaps(ws, ws_need, v, kvn * esz) || overlaps(mass, mass_bytes, ws, ws_need))
     return SKA_ERR_INVALID_VALUE;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d->norm == SKA_NORM_TOKEN)
-    return sa_forward_token(d, q, k, v, cu_seqlens, seqused, sketch, lse, ws, ws_bytes, s);
+    return sa_forward_token(d, q, k, v, cu_seqlens, seqused, sketch, lse, mass, ws, ws_bytes, s);
   ProtoFwdLaunch L;
   int nk = 0, nv = 0;
-  if (!plan_forward(d, &L, &nk, &nv)) return SKA_ERR_UNSUPPORTED;
+  if (!plan_forward(d, mass != nullptr, &L, &nk, &nv)) return SKA_ERR_UNSUPPORTED;
   FwdWs w;
   fwd_ws_layout(d, L, &w);
+  if (w.total > ws_bytes) return SKA_ERR_WORKSPACE_TOO_SMALL;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb + w.hdr);
   int32_t* prefix = reinterpret_cast<int32_t*>(wsb + w.prefix);
@@ -456,7 +482,7 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
     p.hdr = hdr;
     p.partial = partial;
     p.lse = lse;
-    p.mass_partial = nullptr;
+    p.mass_partial = mass ? mass_partial : nullptr;
     p.B = B;
     p.H = H;
     p.k = kp;
@@ -477,8 +503,12 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
       return SKA_ERR_CUDA;
     }
   }
-  if (launch_proto_combine(prefix, hdr, partial, nullptr, B, H, kp, D, sketch, nullptr, s) != cudaSuccess)
+  if (cudaError_t e_ = launch_proto_combine(prefix, hdr, partial, mass ? mass_partial : nullptr, B, H, kp, D, sketch,
+                                            mass, s);
+      e_ != cudaSuccess) {
+    record_error("launch_proto_combine", e_);
     return SKA_ERR_CUDA;
+  }
   if (lse && T > 0) {
     if (cudaError_t e_ = launch_fill_padding_lse(cu_seqlens, seqused, B, H, T, lse, s); e_ != cudaSuccess) { record_error("launch_fill_padding_lse", e_); return SKA_ERR_CUDA; }
   }
@@ -669,8 +699,11 @@ ska_status stca_forward(const ska_stca_desc* d, const void* q, const int32_t* cu
     TimedRegion tr(s);
     e = launch_fa_fwd(D, ctas, smem, mQ, mK, mV, mKs, mVs, p, s);
   }
-  if (e != cudaSuccess) return SKA_ERR_CUDA;
-  if (cudaError_t e_ = launch_fa_combine(p, D, B * H * p.group, out, lse, s); e_ != cudaSuccess) { record_error("launch_fa_combine", e_); return SKA_ERR_CUDA; }
+  if (e != cudaSuccess) {
+    record_error("fused kernel launch", e);
+    return SKA_ERR_CUDA;
+  }
+  if (cudaError_t e_ = launch_fa_combine(p, D, B * H * p.group, out, lse, nullptr, s); e_ != cudaSuccess) { record_error("launch_fa_combine", e_); return SKA_ERR_CUDA; }
   return SKA_OK;
 }
 

@@ -45,12 +45,17 @@ struct ProtoFwdLaunch {
   int cluster;          // CTAs per cluster (prototype groups)
   int kc;               // prototypes per CTA
   int num_clusters;     // persistent clusters
+  bool mass;            // the kernel also accumulates the per-prototype mass
   size_t smem_bytes;
 };
 
-// Host-side planning (no device access).
-bool proto_fwd_plan(int head_dim, int num_protos, int num_sms, ProtoFwdLaunch* out, int* nk_slots,
+// Host-side planning (no device access). With `mass` the CTAs hold at most 128 prototypes each,
+// which leaves tensor memory for the mass accumulator.
+bool proto_fwd_plan(int head_dim, int num_protos, int num_sms, bool mass, ProtoFwdLaunch* out, int* nk_slots,
                     int* nv_entries);
+
+// Clusters of the planned configuration resident at once on the current device (0 if unknown).
+int proto_fwd_max_clusters(int head_dim, const ProtoFwdLaunch& L);
 
 cudaError_t launch_proto_fwd(int head_dim, const ProtoFwdLaunch& L, const CUtensorMap& mapQ,
                              const CUtensorMap& mapK, const CUtensorMap& mapV, const ProtoFwdParams& p,
@@ -89,9 +94,10 @@ cudaError_t launch_fa_fwd(int head_dim, int num_ctas, size_t smem_bytes, const C
 cudaError_t launch_fa_schedule(const FaFwdParams& p, int num_ctas, cudaStream_t stream);
 
 // LSE merge of the partials into the outputs (max_streams = B * H * group blocks).
-// SA: out = sketch [B,H,k,D], lse [B,H,k]. STCA: out [total_targets, H, D], lse [total_targets, H].
+// SA: out = sketch [B,H,k,D], lse [B,H,k], mass [B,H,k] (nullable). STCA: out [total_targets, H, D],
+// lse [total_targets, H], mass null.
 cudaError_t launch_fa_combine(const FaFwdParams& p, int head_dim, int max_streams, float* out, float* lse,
-                              cudaStream_t stream);
+                              float* mass, cudaStream_t stream);
 
 // Parameters of the SA backward (both normalisations).
 struct SaBwdParams {
@@ -123,7 +129,9 @@ cudaError_t launch_sa_bwd_finish(const SaBwdParams& p, int head_dim, float* dq, 
 // Small kernels (ska_small.cu).
 cudaError_t launch_schedule(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,
                             int num_clusters, int32_t* tile_prefix, WsHeader* hdr, cudaStream_t stream);
-cudaError_t launch_proto_combine(const int32_t* tile_prefix, const WsHeader* hdr, const float* partial,
+// Also marks the call SKA_ERR_RANGE in hdr->status when a summed sketch value is not finite (an
+// fp16 overflow of a scaled value row), and writes NaN when hdr->status reports an error.
+cudaError_t launch_proto_combine(const int32_t* tile_prefix, WsHeader* hdr, const float* partial,
                                  const float* mass_partial, int B, int H, int k, int D, float* sketch,
                                  float* mass, cudaStream_t stream);
 cudaError_t launch_fill_padding_lse(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,

@@ -18,6 +18,8 @@
 //   or from several host threads) race on the array: serialise them.
 // * The first call on each device looks up the array's device address with
 //   cudaGetSymbolAddress; make that first call before any stream capture.
+// * Device-side errors (a bounded wait that ran out, an fp16 overflow) land in the array's
+//   status word; sa_forward_noalloc_read_status reads and clears it.
 #include <mutex>
 
 #include "ska_internal.h"
@@ -65,4 +67,11 @@ extern "C" ska_status sa_forward_noalloc(const ska_sa_desc* desc, const void* q,
   void* scratch = scratch_address(&err);
   if (!scratch || err != cudaSuccess) return SKA_ERR_CUDA;
   return sa_forward(desc, q, k, v, cu_seqlens, seqused, sketch, lse, mass, scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" ska_status sa_forward_noalloc_read_status(void* stream) {
+  cudaError_t err = cudaSuccess;
+  void* scratch = scratch_address(&err);
+  if (!scratch || err != cudaSuccess) return SKA_ERR_CUDA;
+  return ska_read_device_status(scratch, stream);
 }

@@ -329,16 +329,6 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return d;
 }
 
-// Two bf16 in one word -> two fp16 in one word. Exact inside the fp16 normal range; values
-// beyond +-65504 saturate to +-65504, values below 2^-14 become fp16 subnormals.
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
-  const float lo = __uint_as_float(w << 16);
-  const float hi = __uint_as_float(w & 0xFFFF0000u);
-  uint32_t d;
-  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-  return d;
-}
-
 // ---- packed fp32 pairs (Blackwell f32x2 arithmetic)
 __device__ __forceinline__ uint64_t f2_pack(float a, float b) {
   uint64_t r;
@@ -380,16 +370,17 @@ __device__ __forceinline__ void st_async_f32x2(uint32_t dst_cluster_addr, float 
                : "memory");
 }
 
-// Two bf16 in one word, each multiplied by a fp32 pair `f2` (both halves equal), rounded once to
-// two fp16 (saturating at +-65504).
-__device__ __forceinline__ uint32_t scale_bf16x2_to_f16x2(uint32_t w, uint64_t f2) {
+// Two bf16 in one word, each multiplied by the fp32 pair `f2` (both halves equal) and rounded
+// once to fp16 (round to nearest even). Products beyond the fp16 range become +-inf, so that an
+// overflow shows in the result instead of being clamped.
+__device__ __forceinline__ uint32_t scale_bf16x2_to_f16x2_rn(uint32_t w, uint64_t f2) {
   uint64_t v;
   asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(w << 16), "r"(w & 0xFFFF0000u));
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(v) : "l"(v), "l"(f2));
   float lo, hi;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
   uint32_t d;
-  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
 }
 
@@ -397,42 +388,6 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
-}
-
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
-// Two bf16 in one word -> two fp16 in one word (unscaled; saturating at +-65504).
-__device__ __forceinline__ uint32_t bf16x2_as_f16x2(uint32_t w) {
-  uint32_t d;
-  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(__uint_as_float(w & 0xFFFF0000u)),
-      "f"(__uint_as_float(w << 16)));
-  return d;
-}
-
-// 2^x for a pair of fp32 values on the FMA and integer pipes instead of the MUFU unit.
-// x is clamped to >= -126; n = round(x) by the 1.5 * 2^23 addition trick, f = x - n in
-// [-1/2, 1/2], 2^f by the degree-3 minimax polynomial fitted in exp2_poly_fit.py (Remez,
-// max relative error 7.5e-5), and 2^n added into the exponent field of the result.
-__device__ __forceinline__ void exp2_fma_pair(float x0, float x1, float& y0, float& y1) {
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t t = f2_add(x, magic);
-  const uint64_t fr = f2_sub(x, f2_sub(t, magic));
-  uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), fr,
-                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
-  p = f2_fma(p, fr, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-  p = f2_fma(p, fr, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -45,20 +45,26 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restric
   }
   if (t == 1023) {
     prefix[B] = part[1023];
-    const int total = H * part[1023];
-    hdr->total_tiles = total;
-    hdr->tiles_per_cluster = (total + num_clusters - 1) / num_clusters;
+    // the host bounds H * (tiles) below 2^31 (descriptor check); 64-bit here all the same
+    const long long total = static_cast<long long>(H) * part[1023];
+    hdr->total_tiles = static_cast<int>(total);
+    hdr->tiles_per_cluster = static_cast<int>((total + num_clusters - 1) / num_clusters);
     hdr->status = 0;
   }
 }
 
 // sketch[s, :, :] = sum over the clusters p that touched segment s of partial[s + p, :, :],
 // in increasing p. Segment s = b*H + h covers global tiles [H*prefix[b] + h*n_b, ... + n_b).
-__global__ void proto_combine_kernel(const int32_t* __restrict__ prefix, const WsHeader* __restrict__ hdr,
+// When an earlier kernel of the call recorded an error the outputs are NaN; a sum that is not
+// finite (a value row that overflowed fp16 once scaled by its weight) is recorded as
+// SKA_ERR_RANGE.
+__global__ void proto_combine_kernel(const int32_t* __restrict__ prefix, WsHeader* __restrict__ hdr,
                                      const float* __restrict__ partial, const float* __restrict__ mass_partial,
                                      int B, int H, int k, int D, float* __restrict__ sketch,
                                      float* __restrict__ mass) {
   const int s = blockIdx.x;
+  const bool failed = *reinterpret_cast<volatile int32_t*>(&hdr->status) != 0;
+  bool finite = true;
   const int b = s / H, h = s - b * H;
   const int nb = prefix[b + 1] - prefix[b];
   const int W = hdr->tiles_per_cluster;
@@ -76,15 +82,19 @@ __global__ void proto_combine_kernel(const int32_t* __restrict__ prefix, const W
       const float4 v = *reinterpret_cast<const float4*>(partial + (static_cast<int64_t>(s + pc) * per + e));
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
+    finite = finite && isfinite(acc.x) && isfinite(acc.y) && isfinite(acc.z) && isfinite(acc.w);
+    if (failed) acc = make_float4(NAN, NAN, NAN, NAN);
     *reinterpret_cast<float4*>(sketch + static_cast<int64_t>(s) * per + e) = acc;
   }
   if (mass && blockIdx.y == 0) {
     for (int j = threadIdx.x; j < k; j += blockDim.x) {
       float acc = 0.f;
       for (int pc = p0; pc <= p1; ++pc) acc += mass_partial[static_cast<int64_t>(s + pc) * k + j];
-      mass[static_cast<int64_t>(s) * k + j] = acc;
+      finite = finite && isfinite(acc);
+      mass[static_cast<int64_t>(s) * k + j] = failed ? NAN : acc;
     }
   }
+  if (!finite && !failed) atomicCAS(&hdr->status, 0, static_cast<int>(SKA_ERR_RANGE));
 }
 
 // lse rows of padding tokens (positions >= seqused[b] inside user b) are -inf.
@@ -113,7 +123,7 @@ cudaError_t launch_schedule(const int32_t* cu, const int32_t* seqused, int B, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_proto_combine(const int32_t* prefix, const WsHeader* hdr, const float* partial,
+cudaError_t launch_proto_combine(const int32_t* prefix, WsHeader* hdr, const float* partial,
                                  const float* mass_partial, int B, int H, int k, int D, float* sketch,
                                  float* mass, cudaStream_t stream) {
   const int per4 = (k * D) / 4;

@@ -54,6 +54,16 @@ def max_over_ranks(values, device=None, group=None):
     return [float(x) for x in t.cpu()]
 
 
+def sum_over_ranks(values, device=None, group=None):
+    """Element-wise sum of a list of floats over ranks (whole-job totals of per-rank work)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+    return [float(x) for x in t.cpu()]
+
+
 def sa_backward_data_parallel(q, k, v, cu_seqlens, seqused, lse, dsketch, sketch=None, *, scale=1.0,
                               norm="proto", group=None, **kw):
     """Backward of this rank's users followed by the dQ all-reduce when the prototypes are shared

@@ -14,7 +14,8 @@ from sketch_attention_flashsa_b200 import _lib as L
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "sketch_attn.h")
 
-A = 0x10000  # a 64 KB-aligned fake address; any multiple of it is 256-byte aligned
+A = 1 << 32  # a fake address: multiples of it are 256-byte aligned and 4 GiB apart, so no
+#               two fake buffers overlap
 
 
 def header_functions():
@@ -46,7 +47,8 @@ def test_library_loads_and_exports_every_declared_call():
 def test_status_strings():
     want = {L.SKA_OK: "SKA_OK", L.SKA_ERR_INVALID_VALUE: "SKA_ERR_INVALID_VALUE",
             L.SKA_ERR_UNSUPPORTED: "SKA_ERR_UNSUPPORTED", L.SKA_ERR_WORKSPACE_TOO_SMALL: "SKA_ERR_WORKSPACE_TOO_SMALL",
-            L.SKA_ERR_CUDA: "SKA_ERR_CUDA", L.SKA_ERR_DEVICE_TIMEOUT: "SKA_ERR_DEVICE_TIMEOUT"}
+            L.SKA_ERR_CUDA: "SKA_ERR_CUDA", L.SKA_ERR_DEVICE_TIMEOUT: "SKA_ERR_DEVICE_TIMEOUT",
+            L.SKA_ERR_RANGE: "SKA_ERR_RANGE"}
     for code, name in want.items():
         assert L.status_string(code) == name
     assert L.status_string(99) not in want.values()
@@ -93,6 +95,8 @@ INVALID, UNSUP = L.SKA_ERR_INVALID_VALUE, L.SKA_ERR_UNSUPPORTED
     ({"scale": float("nan")}, INVALID), ({"scale": float("inf")}, INVALID), ({"norm": 7}, INVALID),
     ({"in_dtype": 5}, INVALID), ({"q_per_user": 2}, INVALID), ({"num_protos": 0}, INVALID),
     ({"head_dim": 96}, UNSUP), ({"head_dim": 256}, UNSUP),
+    # the tile stream H * (T / 128 + B) must stay below 2^31 (32-bit tile indices on the device)
+    ({"num_heads": 1 << 16, "total_tokens": (1 << 31) - 1}, INVALID),
 ])
 def test_sa_forward_rejects_bad_descriptors(kw, code):
     assert fwd(sa_desc(**kw)) == code
@@ -101,7 +105,8 @@ def test_sa_forward_rejects_bad_descriptors(kw, code):
 def test_sa_forward_pointer_checks():
     d = sa_desc()
     assert fwd(None) == INVALID
-    assert fwd(d, mass=11 * A) == UNSUP  # the per-prototype mass output is not produced
+    assert fwd(d, mass=11 * A + 4) == INVALID  # 16-byte alignment of the mass output
+    assert fwd(d, mass=5 * A) == INVALID  # the mass output may not overlap the sketch
     assert fwd(d, q=None) == INVALID
     assert fwd(d, k=None) == INVALID
     assert fwd(d, sk=None) == INVALID
@@ -139,6 +144,7 @@ def test_sa_backward_pointer_checks():
 @pytest.mark.parametrize("kw,code", [
     ({"num_heads": 0}, INVALID), ({"num_sketch": -1}, INVALID), ({"total_hist": -1}, INVALID),
     ({"scale": 0.0}, INVALID), ({"head_dim": 32}, UNSUP),
+    ({"num_heads": 1 << 16, "total_hist": (1 << 31) - 1}, INVALID),
 ])
 def test_stca_rejects_bad_descriptors(kw, code):
     assert stca(stca_desc(**kw)) == code
@@ -162,6 +168,8 @@ def test_valid_call_without_a_device_reports_cuda_error():
         pytest.skip("a device is present")
     assert fwd(sa_desc()) == L.SKA_ERR_CUDA
     assert b"cudaGetDevice" in L.lib().ska_last_error_string()
+    assert fwd(sa_desc(), mass=11 * A) == L.SKA_ERR_CUDA  # the mass output passes the host checks
+    assert L.lib().sa_forward_noalloc_read_status(None) == L.SKA_ERR_CUDA
     assert bwd(sa_desc()) == L.SKA_ERR_CUDA
     assert stca(stca_desc()) == L.SKA_ERR_CUDA
     assert L.lib().sa_forward_workspace_size(ctypes.byref(sa_desc())) == 0

@@ -47,3 +47,41 @@ def test_traffic_gate_follows_the_source_hash(tmp_path, monkeypatch):
 def test_traffic_gate_without_captures(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.traffic_for(bench.DEFAULT_WORKLOAD, "proto") is None
+
+
+def test_launcher_command_starts_one_process_per_gpu():
+    cmd = bench.launcher_command(4, ["--gpus", "4", "--steps", "3"])
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd
+    assert cmd[-5:] == [os.path.join(bench.ROOT, "bench.py"), "--gpus", "4", "--steps", "3"]
+
+
+def test_rank_users_partition_the_global_batch():
+    """Weak scaling: N ranks split N copies of the workload's users, balanced by valid length, and
+    one rank alone gets exactly the workload."""
+    for name in ("sa_fwd_b64_ragged_h4_d64_k256", "sa_fwd_b8_l100k_h8_d128_k512_masked", "sa_fwd_paper_h1_d128_k1024"):
+        spec = bench.WORKLOADS[name]
+        one, su1 = bench.rank_users(spec, 0, 1)
+        assert one == bench.lengths_for(spec["lens"]) and su1 == spec["seqused"]
+        for world in (2, 4, 8):
+            parts = [bench.rank_users(spec, r, world) for r in range(world)]
+            lens = [x for p, _ in parts for x in p]
+            assert sorted(lens) == sorted(bench.lengths_for(spec["lens"], world))
+            valid = [sum(min(a, b) for a, b in zip(p, su)) if su else sum(p) for p, su in parts]
+            assert max(valid) - min(valid) <= max(bench.lengths_for(spec["lens"], world)), (name, world, valid)
+            per_rank = sum(valid) / world
+            assert max(valid) <= 1.15 * per_rank, (name, world, valid)
+
+
+def test_gpus_flag_launches_ranks_on_the_cpu():
+    """`bench.py --gpus 2` outside a launcher re-executes itself under torch.distributed.run; the
+    reference arm (the oracle, no GPU) then prints one line from rank 0 with n_gpus 2."""
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                          "--steps", "1", "--warmup", "3", "--ref-seconds", "0.2",
+                          "--workload", "stca_b16_t512_h4_d64_l10k_s256"],
+                         capture_output=True, text=True, timeout=600, cwd=bench.ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(x) for x in out.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1 and lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"

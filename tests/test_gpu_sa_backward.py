@@ -92,7 +92,7 @@ def test_backward_long_chains(norm):
 @pytest.mark.parametrize("norm", ["proto", "token"])
 def test_backward_config4_full(norm):
     """Config 4: config-2 shapes (64 ragged users up to 91K tokens, H=4, d=64, k=256), dQ reduced
-    over all 1.45M tokens; dQ compared in full, dK and dV on three users."""
+    over all 1.45M tokens; dQ, dK and dV of every user compared with the oracle."""
     inp = W.config4(W.NORM_PROTO if norm == "proto" else W.NORM_TOKEN)
     nid = inp.norm
     cu = inp.cu_seqlens.numpy()
@@ -100,8 +100,6 @@ def test_backward_config4_full(norm):
     B, H = inp.num_users, inp.num_heads
     osk = np.zeros((B, H, inp.num_protos, inp.head_dim))
     olse = np.full((inp.total_tokens, H), -np.inf) if nid == W.NORM_PROTO else np.zeros((B, H, inp.num_protos))
-    odq = np.zeros_like(q)
-    sampled = {0: None, 37: None, int(np.argmax(inp.valid_lengths())): None}
     for b in range(B):
         lo, hi = int(cu[b]), int(cu[b + 1])
         kb, vb = f64(k[lo:hi]), f64(v[lo:hi])
@@ -112,13 +110,16 @@ def test_backward_config4_full(norm):
                 olse[lo:hi, h] = ls
             else:
                 olse[b, h] = ls
-        gq, gk, gv = oracle.sa_backward(q, kb, vb, np.array([0, hi - lo]), None, do[b:b + 1], inp.scale, nid)
-        odq += gq
-        if b in sampled:
-            sampled[b] = (gk, gv)
     dq, dk, dv = run_bwd(inp, norm, osk, olse)
-    assert_close(dq, odq, f"{norm} dq (all users)")
-    for b, (gk, gv) in sampled.items():
+    odq = np.zeros_like(q)
+    worst = 0.0
+    for b in range(B):
         lo, hi = int(cu[b]), int(cu[b + 1])
-        assert_close(dk[lo:hi], gk, f"{norm} dk user {b}")
-        assert_close(dv[lo:hi], gv, f"{norm} dv user {b}")
+        gq, gk, gv = oracle.sa_backward(q, f64(k[lo:hi]), f64(v[lo:hi]), np.array([0, hi - lo]), None, do[b:b + 1],
+                                        inp.scale, nid)
+        odq += gq
+        mk, _ = assert_close(dk[lo:hi], gk, f"{norm} dk user {b}")
+        mv, _ = assert_close(dv[lo:hi], gv, f"{norm} dv user {b}")
+        worst = max(worst, mk, mv)
+    assert_close(dq, odq, f"{norm} dq (all users)")
+    print(f"[parity] dK, dV of all {B} users, worst max abs {worst:.3e}")

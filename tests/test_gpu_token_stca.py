@@ -10,7 +10,7 @@ import torch
 import oracle
 from sketch_attention_flashsa_b200 import workloads as W
 
-from test_gpu_sa_forward import assert_close, f64, run_gpu, run_oracle
+from test_gpu_sa_forward import _full_parity, assert_close, f64, run_gpu, run_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -70,51 +70,78 @@ def test_token_padding_bitwise_and_deterministic():
     assert np.array_equal(a, c) and np.array_equal(la, lc)
 
 
-@pytest.mark.slow
-def test_token_config2_full_sampled():
-    inp = W.config2(W.NORM_TOKEN)
-    sk, lse = run_gpu(inp, norm="token")
-    cu = inp.cu_seqlens.numpy()
-    lens = inp.valid_lengths()
-    q = f64(inp.q)
-    for b, h in [(0, 0), (int(np.argmax(lens)), 3), (63, 1)]:
-        lo, n = int(cu[b]), int(lens[b])
-        osk, olse, _, _ = oracle.sa_problem(q[h], f64(inp.k[lo:lo + n, h]), f64(inp.v[lo:lo + n, h]), inp.scale,
-                                            W.NORM_TOKEN)
-        assert_close(sk[b, h], osk, f"token sketch[{b},{h}]")
-        assert_close(lse[b, h], olse, f"token lse[{b},{h}]")
+def test_token_mass_is_one_per_prototype():
+    """Token-wise: each prototype's weights sum to 1 over its user's valid tokens (0 for an empty
+    user), so mass is exactly that."""
+    inp = W.make_sa([300, 0, 129, 50], 2, 64, 256, seed=33, seqused=[300, 0, 100, 0], norm=W.NORM_TOKEN)
+    sk, lse, ms = run_gpu(inp, norm="token", mass=True)
+    osk, olse, oms = run_oracle(inp, W.NORM_TOKEN)
+    assert_close(sk, osk, "token sketch")
+    assert_close(ms, oms, "token mass")
+    assert (ms[[0, 2]] == 1.0).all() and (ms[[1, 3]] == 0.0).all()
+
+
+@pytest.mark.parametrize("d,k", [(64, 256), (128, 512)])
+def test_token_keys_alias_values(d, k):
+    inp = W.make_sa([700, 129, 1], 2, d, k, seed=34 + d, norm=W.NORM_TOKEN)
+    sk, lse = run_gpu(inp, norm="token", alias=True)
+    osk, olse, _ = run_oracle(inp, W.NORM_TOKEN, alias=True)
+    assert_close(sk, osk, "token sketch (k is v)")
+    assert_close(lse, olse, "token lse (k is v)")
+
+
+def test_token_large_values_match():
+    """bf16 weights times bf16 values accumulate in fp32: |v| beyond the fp16 range is fine."""
+    inp = W.make_sa([900, 300], 2, 128, 256, seed=35, norm=W.NORM_TOKEN)
+    s = 3.0e4
+    big = W.SAInputs(inp.q, inp.k, (inp.v.float() * s).bfloat16(), inp.cu_seqlens, None, inp.scale, inp.norm)
+    sk, lse = run_gpu(big, norm="token")
+    osk, olse, _ = run_oracle(big, W.NORM_TOKEN)
+    assert_close(sk, osk, "token sketch (|v| > 65504)", scale=s)
+    assert_close(lse, olse, "token lse")
 
 
 @pytest.mark.slow
-def test_token_config3_full_sampled():
-    inp = W.config3(W.NORM_TOKEN)
-    sk, lse = run_gpu(inp, norm="token")
-    q = f64(inp.q)
-    for b, h in [(0, 0), (7, 5)]:
-        lo = b * 100_000
-        osk, olse, _, _ = oracle.sa_problem(q[h], f64(inp.k[lo:lo + 100_000, h]), f64(inp.v[lo:lo + 100_000, h]),
-                                            inp.scale, W.NORM_TOKEN)
-        assert_close(sk[b, h], osk, f"token sketch[{b},{h}]")
-        assert_close(lse[b, h], olse, f"token lse[{b},{h}]")
+def test_token_config2_full():
+    _full_parity(W.config2(W.NORM_TOKEN), W.NORM_TOKEN)
+
+
+@pytest.mark.slow
+def test_token_config3_full():
+    _full_parity(W.config3(W.NORM_TOKEN), W.NORM_TOKEN)
+
+
+@pytest.mark.slow
+def test_token_config3_masked_full():
+    _full_parity(W.config3(W.NORM_TOKEN, masked=True), W.NORM_TOKEN)
 
 
 # ---------------------------------------------------------------------------------- STCA
-def run_stca(inp: W.STCAInputs):
+def run_stca(inp: W.STCAInputs, alias=False, max_targets=None, status=False):
+    """alias: one device tensor for k_hist and v_hist and one for k_sk and v_sk (keys = values)."""
     api = _api()
     dev = "cuda"
     ks = inp.k_sk.to(dev) if inp.k_sk.shape[2] > 0 else None
-    vs = inp.v_sk.to(dev) if inp.v_sk.shape[2] > 0 else None
+    vs = (ks if alias else inp.v_sk.to(dev)) if inp.v_sk.shape[2] > 0 else None
     kvl = inp.target_kv_len.to(dev) if inp.target_kv_len is not None else None
-    out, lse = api.stca_forward(inp.q.to(dev), inp.cu_targets.to(dev), inp.k_hist.to(dev), inp.v_hist.to(dev),
-                                inp.cu_hist.to(dev), ks, vs, scale=inp.scale, target_kv_len=kvl)
+    kh = inp.k_hist.to(dev)
+    vh = kh if alias else inp.v_hist.to(dev)
+    cut = inp.cu_targets.to(dev)
+    desc = api.stca_desc(inp.q, inp.k_hist, ks, cut, inp.cu_hist, scale=inp.scale,
+                         max_targets=max_targets if max_targets is not None else int(inp.q.shape[0]))
+    ws = torch.empty(max(api.stca_forward_workspace_size(desc), 256), dtype=torch.uint8, device=dev)
+    out, lse = api.stca_forward(inp.q.to(dev), cut, kh, vh, inp.cu_hist.to(dev), ks, vs, scale=inp.scale,
+                                target_kv_len=kvl, max_targets=max_targets, workspace=ws)
     torch.cuda.synchronize()
-    return out.cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+    res = (out.cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64))
+    return res + (api.read_device_status(ws),) if status else res
 
 
-def oracle_stca(inp: W.STCAInputs):
+def oracle_stca(inp: W.STCAInputs, alias=False):
     kvl = inp.target_kv_len.numpy() if inp.target_kv_len is not None else None
-    return oracle.stca_forward(f64(inp.q), inp.cu_targets.numpy(), f64(inp.k_hist), f64(inp.v_hist),
-                               inp.cu_hist.numpy(), f64(inp.k_sk), f64(inp.v_sk), inp.scale, kvl)
+    vh, vs = (inp.k_hist, inp.k_sk) if alias else (inp.v_hist, inp.v_sk)
+    return oracle.stca_forward(f64(inp.q), inp.cu_targets.numpy(), f64(inp.k_hist), f64(vh),
+                               inp.cu_hist.numpy(), f64(inp.k_sk), f64(vs), inp.scale, kvl)
 
 
 STCA_CASES = {
@@ -140,6 +167,26 @@ def test_stca_parity_small(name):
     assert_close(lse, olse, "stca lse")
 
 
+def test_stca_keys_alias_values():
+    inp = W.make_stca([200, 64], [900, 300], 2, 64, 128, seed=42, with_kv_len=True)
+    out, lse = run_stca(inp, alias=True)
+    oout, olse = oracle_stca(inp, alias=True)
+    assert_close(out, oout, "stca out (k is v)")
+    assert_close(lse, olse, "stca lse (k is v)")
+
+
+def test_stca_too_small_max_targets_gives_nan_and_status():
+    """max_targets below a user's target count: the schedule records SKA_ERR_INVALID_VALUE and the
+    combine writes NaN to every output instead of partial slots that were never written."""
+    inp = W.make_stca([300, 40], [500, 200], 2, 64, 16, seed=43)
+    out, lse, st = run_stca(inp, max_targets=100, status=True)
+    assert st == 1  # SKA_ERR_INVALID_VALUE
+    assert np.isnan(out).all() and np.isnan(lse).all()
+    out, lse = run_stca(inp)  # the next call on the same context is correct
+    oout, olse = oracle_stca(inp)
+    assert_close(out, oout, "stca out after a refused call")
+
+
 def test_stca_merge_law_on_gpu():
     """[suffix ; sketch] in one call equals the lse-weighted merge of the two one-segment calls."""
     inp = W.make_stca([300, 100], [2000, 700], 2, 64, 256, seed=41)
@@ -157,15 +204,15 @@ def test_stca_merge_law_on_gpu():
 
 
 @pytest.mark.slow
-def test_stca_config5_full_sampled():
+def test_stca_config5_full():
+    """Config 5 in full: every target of every user against the oracle."""
     inp = W.config5()
     out, lse = run_stca(inp)
     cut = inp.cu_targets.numpy()
     cuh = inp.cu_hist.numpy()
-    rng = np.random.default_rng(5)
-    for b in (0, 7, 15):
-        rows = np.sort(rng.choice(np.arange(cut[b], cut[b + 1]), size=12, replace=False))
-        sub = W.STCAInputs(inp.q[rows], torch.tensor([0, len(rows)], dtype=torch.int32),
+    for b in range(len(cut) - 1):
+        rows = slice(int(cut[b]), int(cut[b + 1]))
+        sub = W.STCAInputs(inp.q[rows], torch.tensor([0, cut[b + 1] - cut[b]], dtype=torch.int32),
                            inp.k_hist[cuh[b]:cuh[b + 1]], inp.v_hist[cuh[b]:cuh[b + 1]],
                            torch.tensor([0, cuh[b + 1] - cuh[b]], dtype=torch.int32), inp.k_sk[b:b + 1],
                            inp.v_sk[b:b + 1], inp.scale)
