@@ -361,3 +361,82 @@ def test_stca_no_keys():
     q, cut, kh, vh, cuh, ksk, vsk = _stca_problem([2], [0], 0)
     out, lse = oracle.stca_forward(q, cut, kh, vh, cuh, ksk, vsk, 1.0)
     assert (out == 0).all() and np.isneginf(lse).all()
+
+
+# ---------------------------------------------------------------------------------- refinement
+# SequenceO1 §3.3 Eq. (13)-(14) and the SwiGLU FFN of App. G.1: pins that a dropped term, a wrong
+# axis or a transposed weight would break.
+
+def test_layer_norm_rows_have_zero_mean_and_unit_variance():
+    rng = np.random.default_rng(70)
+    x = rng.normal(3.0, 5.0, size=(6, 128))
+    y = oracle.layer_norm(x)
+    assert np.abs(y.mean(axis=-1)).max() < 1e-12
+    var = x.var(axis=-1)
+    assert np.allclose(y.var(axis=-1), var / (var + 1e-5), rtol=1e-12)
+
+
+def test_layer_norm_axis_affine_and_scale_invariance():
+    rng = np.random.default_rng(71)
+    x = rng.normal(size=(4, 16))
+    g, b = rng.normal(size=16), rng.normal(size=16)
+    base = oracle.layer_norm(x)
+    assert np.allclose(oracle.layer_norm(x, g, b), base * g + b, atol=1e-14)
+    # over the features of each row, not over the rows: rows are independent
+    assert np.allclose(oracle.layer_norm(x[1:2]), base[1:2], atol=1e-14)
+    # invariant to a positive scale and a shift of the row (up to the eps term, ~eps / var)
+    assert np.allclose(oracle.layer_norm(7.0 * x + 3.0), base, atol=1e-4)
+    # a constant row normalises to zero (then beta)
+    assert np.allclose(oracle.layer_norm(np.full((1, 8), 2.5), None, np.arange(8.0)), np.arange(8.0))
+
+
+def test_swish_closed_forms():
+    assert oracle.swish(0.0) == 0.0
+    assert abs(oracle.swish(1.0) - 1.0 / (1.0 + math.exp(-1.0))) < 1e-15
+    assert abs(oracle.swish(40.0) - 40.0) < 1e-12 and abs(oracle.swish(-40.0)) < 1e-15
+    assert abs(oracle.swish(-1.0) + math.exp(-1.0) / (1.0 + math.exp(-1.0))) < 1e-15
+
+
+def test_swiglu_ffn_hand_example():
+    """d = 2, intermediate 2: x = [1, 2], W_1 = I, W_g = [[0, 1], [1, 0]], W_2 = I:
+    x W_1 = [1, 2], x W_g = [2, 1], swish(x W_1) * x W_g = [2 swish(1), swish(2)].
+    With W_1 and W_g swapped the activation falls on the other projection: [swish(2), 2 swish(1)]."""
+    s1, s2 = 1.0 / (1.0 + math.exp(-1.0)), 2.0 / (1.0 + math.exp(-2.0))
+    eye, swap = np.eye(2), np.array([[0.0, 1.0], [1.0, 0.0]])
+    x = np.array([[1.0, 2.0]])
+    assert np.allclose(oracle.swiglu_ffn(x, eye, swap, eye), [[2 * s1, s2]], atol=1e-15)
+    assert np.allclose(oracle.swiglu_ffn(x, swap, eye, eye), [[s2, 2 * s1]], atol=1e-15)
+    # the output projection: W_2 = [[1, 0], [1, 1]] sums the two gated features into the second output
+    assert np.allclose(oracle.swiglu_ffn(x, eye, swap, np.array([[1.0, 0.0], [1.0, 1.0]])),
+                       [[2 * s1 + s2, s2]], atol=1e-15)
+
+
+def test_refine_with_zero_ffn_output_is_ln_of_the_residual_twice():
+    """W_2 = 0 makes FFN = 0, so Eq. (14) is LN(LN(X~ + X^)): LayerNorm is idempotent up to eps."""
+    rng = np.random.default_rng(72)
+    B, H, k, d, f = 2, 2, 5, 16, 32
+    xt, xh = rng.normal(size=(B, H, k, d)), rng.normal(size=(B, H, k, d))
+    w1, wg = rng.normal(size=(H, d, f)), rng.normal(size=(H, d, f))
+    w2 = np.zeros((H, f, d))
+    xb, out = oracle.refine(xt, xh, w1, wg, w2)
+    assert np.allclose(xb, oracle.layer_norm(xt + xh), atol=1e-14)
+    assert np.allclose(out, xb, atol=1e-4)
+
+
+def test_refine_heads_rows_and_users_are_independent():
+    rng = np.random.default_rng(73)
+    B, H, k, d, f = 3, 2, 4, 8, 16
+    xt, xh = rng.normal(size=(B, H, k, d)), rng.normal(size=(B, H, k, d))
+    w1, wg, w2 = rng.normal(size=(H, d, f)), rng.normal(size=(H, d, f)), rng.normal(size=(H, f, d)) / 4
+    g1, b1, g2, b2 = (rng.normal(size=(H, d)) for _ in range(4))
+    xb, out = oracle.refine(xt, xh, w1, wg, w2, g1, b1, g2, b2)
+    # head 1 alone with its own parameters
+    xb1, out1 = oracle.refine(xt[:, 1:], xh[:, 1:], w1[1:], wg[1:], w2[1:], g1[1:], b1[1:], g2[1:], b2[1:])
+    assert np.allclose(out[:, 1:], out1, atol=1e-14)
+    # a permutation of the sketch tokens permutes the output rows the same way
+    perm = rng.permutation(k)
+    _, outp = oracle.refine(xt[:, :, perm], xh[:, :, perm], w1, wg, w2, g1, b1, g2, b2)
+    assert np.allclose(outp, out[:, :, perm], atol=1e-12)
+    # the residual: x_bar is LN of the sum, so swapping the two inputs changes nothing
+    xb_s, out_s = oracle.refine(xh, xt, w1, wg, w2, g1, b1, g2, b2)
+    assert np.allclose(out_s, out, atol=1e-12)
