@@ -55,9 +55,14 @@ WORKLOADS = {
     "sa_fwd_b8_l100k_h8_d128_k512_masked": dict(kind="sa_fwd", lens=[100_000] * 8, H=8, d=128, k=512,
                                                 seqused=[70_000] + [100_000] * 7),
     "sa_fwd_b64_ragged_h4_d64_k256": dict(kind="sa_fwd", lens="ragged64", H=4, d=64, k=256, seqused=None),
+    # the paper's V = X (Eq. (9)): one tensor passed as both keys and values
+    "sa_fwd_b8_l100k_h8_d128_k512_kv_alias": dict(kind="sa_fwd", lens=[100_000] * 8, H=8, d=128, k=512, seqused=None,
+                                                  alias=True),
     "sa_fwd_paper_h1_d128_k1024": dict(kind="sa_fwd", lens="paper", H=1, d=128, k=1024, seqused=None),
     # profiling size: same per-tile work as the headline, 205 MB of K+V (> L2), ~0.25 ms
     "sa_fwd_b2_l100k_h2_d128_k512": dict(kind="sa_fwd", lens=[100_000] * 2, H=2, d=128, k=512, seqused=None),
+    "sa_fwd_b2_l100k_h2_d128_k512_kv_alias": dict(kind="sa_fwd", lens=[100_000] * 2, H=2, d=128, k=512,
+                                                  seqused=None, alias=True),
     "sa_bwd_b64_ragged_h4_d64_k256": dict(kind="sa_bwd", lens="ragged64", H=4, d=64, k=256, seqused=None),
     # profiling size for the backward: 2 x 100K, one head, same per-tile work
     "sa_bwd_b2_l100k_h1_d64_k256": dict(kind="sa_bwd", lens=[100_000] * 2, H=1, d=64, k=256, seqused=None),
@@ -172,9 +177,10 @@ class SaFwdJob:
             self.inputs = {
                 "q": (torch.randn((H, kp, d), generator=gen, device=dev) / math.sqrt(d)).bfloat16(),
                 "k": torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
-                "v": torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16),
                 "cu": torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=dev),
             }
+            if not spec.get("alias"):
+                self.inputs["v"] = torch.randn((T, H, d), generator=gen, device=dev, dtype=torch.bfloat16)
             if su:
                 self.inputs["seqused"] = torch.tensor(np.array(su, dtype=np.int32), device=dev)
         self.valid = sum(min(a, b) for a, b in zip(lens, su)) if su else T
@@ -185,7 +191,8 @@ class SaFwdJob:
         self.lse = torch.empty((T, H) if norm == "proto" else (B, H, kp), dtype=torch.float32, device=dev)
         self.units = self.valid
         self.flops = flops.sa_forward_flops(self.valid, H, kp, d)
-        self.bytes = flops.sa_forward_bytes(self.valid, H, kp, d, B, norm=0 if norm == "proto" else 1)
+        self.bytes = flops.sa_forward_bytes(self.valid, H, kp, d, B, norm=0 if norm == "proto" else 1,
+                                            kv_alias=bool(spec.get("alias")))
         self.kernel = "sa_proto_fwd_kernel" if norm == "proto" else "fa_fwd_kernel"
         self.launches = 4 if norm == "proto" else 3
         self.config = {"users_per_gpu": B, "heads": H, "head_dim": d, "protos": kp, "norm": norm,
@@ -193,7 +200,8 @@ class SaFwdJob:
                        "l2": "inputs larger than L2 (K and V are %.2f GB each per GPU)" % (T * H * d * 2 / 1e9)}
 
     def run(self, x):
-        self.api.sa_forward(x["q"], x["k"], x["v"], x["cu"], x.get("seqused"), scale=1.0, norm=self.norm,
+        v = x["v"] if "v" in x else x["k"]  # no "v": the values are the keys (V = X)
+        self.api.sa_forward(x["q"], x["k"], v, x["cu"], x.get("seqused"), scale=1.0, norm=self.norm,
                             workspace=self.ws, out=self.sketch, lse_out=self.lse)
         return self.sketch
 
@@ -207,7 +215,8 @@ class SaFwdJob:
         while time.perf_counter() - t0 < budget_s and pairs < 64:
             lo, hi = int(cu[b]), int(cu[b + 1])
             h = pairs % self.H
-            oracle.sa_problem(q[h], f64(self.inputs["k"][lo:hi, h]), f64(self.inputs["v"][lo:hi, h]), 1.0,
+            vv = self.inputs.get("v", self.inputs["k"])
+            oracle.sa_problem(q[h], f64(self.inputs["k"][lo:hi, h]), f64(vv[lo:hi, h]), 1.0,
                               0 if self.norm == "proto" else 1)
             done += (hi - lo) / self.H
             pairs += 1

@@ -4,15 +4,14 @@
 // Per 128-token tile of one (user, head), one CTA holding all k <= 256 prototypes, tokens on
 // TMEM lanes (S^T orientation):
 //   MMA  S^T  = K . Q^T                        -> A = exp(scale s - lse) (PROTO: per-token lse;
-//                                                 TOKEN: per-prototype lse), to smem as a bf16
-//                                                 pair hi + lo (16 significant bits)
-//   MMA  dV   = A^T . dO        (M=tok, N=d)   -> TMEM, both halves of the pair
+//                                                 TOKEN: per-prototype lse), to smem in bf16
+//   MMA  dV   = A^T . dO        (M=tok, N=d)   -> TMEM
 //   MMA  dA^T = V . dO^T        (M=tok, N=k)   -> TMEM (over S^T)
 //   softmax-gradient: PROTO dS = A (dA - delta_i) with delta_i = sum_j A_ji dA_ji in fp32 (each
 //        warpgroup sums its half of the prototypes, the halves are added in a fixed order);
 //        TOKEN dS = A (dA - D_j) with D_j = dO_j . O_j from the forward sketch. dS goes to smem
 //        as a bf16 pair hi + lo.
-//   MMA  dK   = dS^T . Q        (M=tok, N=d)   -> TMEM, both halves, scaled on the way out
+//   MMA  dK   = dS^T . Q        (M=tok, N=d)   -> TMEM from the hi half, scaled on the way out
 //   MMA  dQ  += dS . K          (M=proto, N=d) -> TMEM, both halves; restarted every 16 tiles and
 //        added into the CTA's partial slot (the tensor core's fp32 accumulation is not
 //        round-to-nearest, so one chain over a whole segment would drift); a second kernel sums
@@ -310,21 +309,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         a[c] = valid ? ex2_approx(__uint_as_float(sv[c]) * c2 - l2) : 0.f;
       }
     }
-    // A as a bf16 pair hi + lo, so that dV carries no bf16 rounding of A
+    // A in bf16 for dV = A^T dO (fp32 A stays in registers for dS): dV_i is a weighted mean of
+    // dO rows, so rounding the weights to 8 significant bits leaves ~1e-3 relative error in dV
 #pragma unroll
     for (int c = 0; c < NCOL; c += 8) {
-      float hi[8], lo[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        hi[u] = __bfloat162float(__float2bfloat16_rn(a[c + u]));
-        lo[u] = a[c + u] - hi[u];
-      }
       const int jj = col0 + c;
       const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
-      *reinterpret_cast<uint4*>(sA + off) = make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]),
-                                                       pack_bf16x2(hi[4], hi[5]), pack_bf16x2(hi[6], hi[7]));
-      *reinterpret_cast<uint4*>(sLo + off) = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]),
-                                                        pack_bf16x2(lo[4], lo[5]), pack_bf16x2(lo[6], lo[7]));
+      *reinterpret_cast<uint4*>(sA + off) = make_uint4(pack_bf16x2(a[c], a[c + 1]), pack_bf16x2(a[c + 2], a[c + 3]),
+                                                       pack_bf16x2(a[c + 4], a[c + 5]), pack_bf16x2(a[c + 6], a[c + 7]));
     }
     fence_async_shared();
     tc_fence_before();
@@ -335,11 +327,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int half = 0; half < 2; ++half)
-#pragma unroll
-          for (int s = 0; s < KP / 16; ++s)
-            umma_bf16(tb + CV, sw128_desc(smem_u32(half ? sLo : sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
-                      sw128_desc(smem_u32(sDO) + s * 2048, QBLK, 1024), iV, (half | s) > 0);
+        for (int s = 0; s < KP / 16; ++s)
+          umma_bf16(tb + CV, sw128_desc(smem_u32(sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                    sw128_desc(smem_u32(sDO) + s * 2048, QBLK, 1024), iV, s > 0);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
           umma_bf16(tb, sw128_desc(smem_u32(sV) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
@@ -418,12 +408,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = wait(&bars.ds, i & 1);
       if (ok) {
         tc_fence_after();
+        // dK from the hi half of dS alone (~1e-3 relative); dQ, a sum over every token of every
+        // user, takes both halves
 #pragma unroll
-        for (int half = 0; half < 2; ++half)
-#pragma unroll
-          for (int s = 0; s < KP / 16; ++s)
-            umma_bf16(tb + CK, sw128_desc(smem_u32(half ? sLo : sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
-                      sw128_desc(smem_u32(sQ) + s * 2048, QBLK, 1024), iV, (half | s) > 0);
+        for (int s = 0; s < KP / 16; ++s)
+          umma_bf16(tb + CK, sw128_desc(smem_u32(sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                    sw128_desc(smem_u32(sQ) + s * 2048, QBLK, 1024), iV, s > 0);
 #pragma unroll
         for (int g = 0; g < QBLOCKS; ++g)
 #pragma unroll

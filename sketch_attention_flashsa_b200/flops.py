@@ -112,9 +112,10 @@ def sa_backward_flops(valid_tokens: int, heads: int, protos: int, head_dim: int,
 
 
 def sa_forward_bytes(valid_tokens: int, heads: int, protos: int, head_dim: int, users: int,
-                     in_bytes: int = 2, norm: int = 0, q_users: int = 1) -> float:
-    """K and V read once, Q read once, sketch written once (fp32), plus the saved lse."""
-    kv = 2.0 * valid_tokens * heads * head_dim * in_bytes
+                     in_bytes: int = 2, norm: int = 0, q_users: int = 1, kv_alias: bool = False) -> float:
+    """K and V read once (one tensor when the values are the keys, the paper's V = X), Q read once,
+    sketch written once (fp32), plus the saved lse."""
+    kv = (1.0 if kv_alias else 2.0) * valid_tokens * heads * head_dim * in_bytes
     q = float(q_users) * heads * protos * head_dim * in_bytes
     out = 4.0 * users * heads * protos * head_dim
     lse = 4.0 * valid_tokens * heads if norm == 0 else 4.0 * users * heads * protos
