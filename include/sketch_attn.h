@@ -19,6 +19,9 @@
  *   §4.2): out_t = softmax(scale * q_t K^T) V over the keys [suffix rows of the target's user ;
  *   that user's sketch rows], one softmax per (target, head).
  *
+ *   Stacked refinement (§3.3, Eq. (13)-(14)): after a layer's SA aggregation X^ the sketch is
+ *   updated as LN(X~ + X^), then LN(. + FFN(.)) with a SwiGLU FFN (sa_refine).
+ *
  * Heads: H heads are H independent problems on d-wide slices (the paper's SA is single-head).
  *
  * Conventions shared by every entry point
@@ -188,6 +191,46 @@ SKA_API ska_status stca_forward(const ska_stca_desc* desc, const void* q, const 
                         const int32_t* target_kv_len, const void* k_sk, const void* v_sk, float* out,
                         float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* Stacked refinement of the sketch (§3.3, Eq. (13)-(14)): one layer's update of the per-user
+ * sketch after its SA aggregation,
+ *   x_bar  = LN1(x_tilde + x_hat)                               Eq. (13)
+ *   x_next = LN2(x_bar + FFN(x_bar)),  FFN(U) = (swish(U W_1) * (U W_g)) W_2     Eq. (14)
+ * with the SwiGLU FFN of App. G.1 (swish(u) = u sigmoid(u)) at the intermediate width ffn_dim =
+ * 2 head_dim of App. G.3. Each LayerNorm normalises one row over its head_dim features with the
+ * biased variance and eps, then applies gamma and beta. Head h uses its own weights and LayerNorm
+ * vectors, as the SA call treats heads as independent problems.
+ *   num_users B >= 0, num_heads H >= 1, num_protos k >= 1 (the sketch rows of one user and head;
+ *   any k), head_dim 64 or 128, ffn_dim = 2 head_dim (other pairs: SKA_ERR_UNSUPPORTED), eps > 0
+ *   and finite. B * H * k * head_dim < 2^31.                                                    */
+typedef struct {
+  int32_t num_users;
+  int32_t num_heads;
+  int32_t num_protos;
+  int32_t head_dim;
+  int32_t ffn_dim;
+  float eps;
+} ska_refine_desc;
+
+/* Bytes of workspace sa_refine needs: 256, the status word (0 if the descriptor is invalid). */
+SKA_API size_t sa_refine_workspace_size(const ska_refine_desc* desc);
+
+/* Refinement layer. Device pointers; shapes for B users, H heads, k rows, d = head_dim, F = ffn_dim:
+ *   x_tilde, x_hat   fp32 [B, H, k, d]: the layer's input sketch and its SA output (sa_forward's
+ *                    sketch)
+ *   w1, wg           bf16 [H, d, F];  w2  bf16 [H, F, d]
+ *   gamma1, beta1, gamma2, beta2   fp32 [H, d] or NULL (NULL: gamma = 1, beta = 0)
+ *   x_next           out, fp32 [B, H, k, d]
+ *   x_bar            out, fp32 [B, H, k, d], or NULL when not wanted
+ *   x_next_bf16      out, bf16 [B, H, k, d], or NULL: a bf16 copy of x_next for the next
+ *                    layer's projections
+ * The LayerNorms, the residual sums and swish run in fp32. The FFN products take their
+ * activations as a two-term bf16 split (16 significant bits) against the bf16 weights, with
+ * fp32 accumulation. B = 0 returns SKA_OK without launching anything.                           */
+SKA_API ska_status sa_refine(const ska_refine_desc* desc, const float* x_tilde, const float* x_hat,
+                             const void* w1, const void* wg, const void* w2, const float* gamma1,
+                             const float* beta1, const float* gamma2, const float* beta2, float* x_next,
+                             float* x_bar, void* x_next_bf16, void* ws, size_t ws_bytes, void* stream);
+
 /* Human-readable name of a status code (static string). */
 SKA_API const char* ska_status_string(ska_status status);
 
@@ -202,8 +245,9 @@ SKA_API ska_status ska_read_device_status(void* ws, void* stream);
 
 /* Test hook (process-wide, not synchronised with concurrent calls): the time budget in ns of
  * every barrier wait in later launches (0 restores the default of 4 s), and debug flags
- * (1 = the load producer of later SA forward launches withholds its first arrival, so that
- * the consumers' bounded waits must run out and report SKA_ERR_DEVICE_TIMEOUT). */
+ * (1 = the load producer of later SA forward launches withholds its first arrival; 2 = later
+ * sa_refine launches never signal that their first matrix products are done; either way the
+ * kernels' bounded waits must run out and report SKA_ERR_DEVICE_TIMEOUT). */
 SKA_API void ska_set_debug(uint64_t wait_budget_ns, uint32_t flags);
 
 /* SA forward for callers that cannot allocate device memory (code running inside a memory

@@ -24,7 +24,7 @@ EXPORTED = ("sa_forward_workspace_size", "sa_forward", "sa_backward_workspace_si
             "stca_forward_workspace_size", "stca_forward", "ska_status_string",
             "ska_read_device_status", "ska_set_debug", "ska_set_timing_events",
             "sa_forward_noalloc", "sa_forward_noalloc_scratch_bytes", "sa_forward_noalloc_read_status",
-            "ska_last_error_string")
+            "ska_last_error_string", "sa_refine_workspace_size", "sa_refine")
 
 
 class SaDesc(ctypes.Structure):
@@ -41,6 +41,12 @@ class StcaDesc(ctypes.Structure):
                 ("total_targets", ctypes.c_int64), ("total_hist", ctypes.c_int64),
                 ("max_targets", ctypes.c_int32), ("max_hist", ctypes.c_int32),
                 ("scale", ctypes.c_float), ("reserved", ctypes.c_int32)]
+
+
+class RefineDesc(ctypes.Structure):
+    _fields_ = [("num_users", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+                ("num_protos", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("ffn_dim", ctypes.c_int32), ("eps", ctypes.c_float)]
 
 
 class SkaError(RuntimeError):
@@ -91,6 +97,10 @@ def lib() -> ctypes.CDLL:
     L.sa_forward_noalloc_scratch_bytes.restype = sz
     L.sa_forward_noalloc_read_status.argtypes = [vp]
     L.sa_forward_noalloc_read_status.restype = ctypes.c_int
+    L.sa_refine_workspace_size.argtypes = [ctypes.POINTER(RefineDesc)]
+    L.sa_refine_workspace_size.restype = sz
+    L.sa_refine.argtypes = [ctypes.POINTER(RefineDesc)] + [vp] * 13 + [sz, vp]
+    L.sa_refine.restype = ctypes.c_int
     L.ska_set_timing_events.argtypes = [vp, vp]
     L.ska_set_timing_events.restype = None
     _lib = L

@@ -1,0 +1,367 @@
+// Stacked refinement of the sketch on sm_100a (SequenceO1 §3.3, Eq. (13)-(14)):
+//   X- = LN1(X~ + X^),   X~' = LN2(X- + FFN(X-)),   FFN(U) = (swish(U W_1) * (U W_g)) W_2.
+// The FFN is the SwiGLU of App. G.1 with intermediate width F = 2d (App. G.3). It is applied to
+// every sketch row (b, h, j), using the weights and LayerNorm parameters of head h.
+//
+// One CTA of 128 threads takes 128 rows of one (user, head) at a time, one thread per row:
+//   1. X- = LN1(x_tilde + x_hat) in fp32. The result stays in registers for the residual. It is
+//      also written to shared memory as a bf16 pair hi + lo (16 significant bits) in the
+//      K-major A-operand layout.
+//   2. MMA: H1 = X- W_1 and Hg = X- W_g (M = 128, N = F, K = d; one pass for hi, one for lo),
+//      accumulated in TMEM.
+//   3. G = swish(H1) * Hg, again as a bf16 hi + lo pair in shared memory.
+//   4. MMA: Y = G W_2 (M = 128, N = d, K = F; hi and lo passes) into the TMEM columns H1 held.
+//   5. X~' = LN2(X- + Y) in fp32, written to global memory (plus a bf16 copy when asked for).
+// The weights are bf16 inputs. Multiplying them with the hi + lo pairs leaves about 2^-17 relative
+// error per product, and the fp32 accumulation does the rest. Thread 0 issues the TMA weight
+// loads and the MMAs. The phases of one tile run in sequence. The kernel is memory-bound at its
+// sizes: a row reads 2d fp32 values and writes d.
+//
+// Weight tiles in shared memory are MN-major B operands. W_1 and W_g ([d, F], F contiguous) load
+// as F/64 blocks of [d rows x 64 columns]; W_2 ([F, d], d contiguous) as d/64 blocks of
+// [F rows x 64 columns].
+#include <cmath>
+
+#include "ska_internal.h"
+#include "ska_ptx.cuh"
+
+namespace ska {
+
+namespace {
+
+constexpr int kRefThreads = 128;
+constexpr uint32_t kRefBlk = 16384;  // [128 rows x 64 bf16] swizzled block
+
+template <int D, int F>
+struct RefLayout {
+  // Region A holds X hi | X lo during MMA1, then W_2.
+  // Region B holds W_1 | W_g during MMA1, then G hi | G lo.
+  static constexpr uint32_t x_bytes = (D / 64) * kRefBlk;
+  static constexpr uint32_t g_bytes = (F / 64) * kRefBlk;
+  static constexpr uint32_t w_bytes = D * F * 2;
+  static constexpr uint32_t a_bytes = (2 * x_bytes > w_bytes) ? 2 * x_bytes : w_bytes;
+  static constexpr uint32_t b_bytes = (2 * g_bytes > 2 * w_bytes) ? 2 * g_bytes : 2 * w_bytes;
+  static constexpr uint32_t x_hi = 0;
+  static constexpr uint32_t x_lo = x_bytes;
+  static constexpr uint32_t w2 = 0;
+  static constexpr uint32_t w1 = a_bytes;
+  static constexpr uint32_t wg = a_bytes + w_bytes;
+  static constexpr uint32_t g_hi = a_bytes;
+  static constexpr uint32_t g_lo = a_bytes + g_bytes;
+  static constexpr uint32_t bars = a_bytes + b_bytes;
+  static constexpr uint32_t total = bars + 128;
+  static_assert(a_bytes % 1024 == 0 && w_bytes % 1024 == 0 && g_bytes % 1024 == 0, "1024-byte aligned blocks");
+  static_assert(total <= 227 * 1024, "fits in shared memory");
+};
+
+struct RefBars {
+  uint64_t w1g, w2, x, m1, g, m2, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct RefWaiter {
+  RefBars* bars;
+  int* status;
+  uint64_t budget;
+  // Bounded wait. A wait that runs out records SKA_ERR_DEVICE_TIMEOUT and raises the CTA's abort
+  // flag, after which the other waits give up at once (drain waits still run to their limit).
+  __device__ __forceinline__ bool operator()(uint64_t* bar, uint32_t parity, bool drain = false) {
+    volatile int* ab = &bars->abort_flag;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (!drain && *ab) return false;
+      if (globaltimer_ns() - t0 > budget) {
+        atomicCAS(status, 0, (int)SKA_ERR_DEVICE_TIMEOUT);
+        *ab = 1;
+        return false;
+      }
+    }
+  }
+};
+
+// Splits 8 fp32 values into a bf16 hi + lo pair (lo = bf16(v - hi)) and stores them at row r,
+// columns c .. c + 7, of two swizzled K-major operands.
+__device__ __forceinline__ void store_pair8(uint8_t* hi, uint8_t* lo, int r, int c, const float* v) {
+  float h[8], l[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    h[u] = __bfloat162float(__float2bfloat16_rn(v[u]));
+    l[u] = v[u] - h[u];
+  }
+  const uint32_t off = (c >> 6) * kRefBlk + sw128_offset(r, (c & 63) * 2);
+  *reinterpret_cast<uint4*>(hi + off) =
+      make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+  *reinterpret_cast<uint4*>(lo + off) =
+      make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]), pack_bf16x2(l[4], l[5]), pack_bf16x2(l[6], l[7]));
+}
+
+// LayerNorm of one row held by one thread: mean, biased variance (two passes), then the affine
+// map (gamma, beta may be null: 1 and 0).
+template <int D>
+__device__ __forceinline__ void layer_norm_row(float* x, const float* gamma, const float* beta, float eps) {
+  float mean = 0.f;
+#pragma unroll
+  for (int c = 0; c < D; ++c) mean += x[c];
+  mean *= 1.f / D;
+  float var = 0.f;
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    const float t = x[c] - mean;
+    var = fmaf(t, t, var);
+  }
+  const float rs = rsqrtf(var * (1.f / D) + eps);
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    float y = (x[c] - mean) * rs;
+    if (gamma) y *= __ldg(gamma + c);
+    if (beta) y += __ldg(beta + c);
+    x[c] = y;
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void store_row_f32(float* dst, const float* x) {
+  float4* o = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int u = 0; u < D / 4; ++u) o[u] = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+}
+
+template <int D, int F>
+__global__ void __launch_bounds__(kRefThreads, 1)
+    sa_refine_kernel(const __grid_constant__ CUtensorMap mapW1, const __grid_constant__ CUtensorMap mapWg,
+                     const __grid_constant__ CUtensorMap mapW2, const RefineParams p) {
+  using L = RefLayout<D, F>;
+  constexpr uint32_t kCols = 2 * F;  // H1 | Hg
+  static_assert(kCols <= 512 && (kCols & (kCols - 1)) == 0, "TMEM allocation is a power of two <= 512");
+  extern __shared__ __align__(1024) uint8_t smem[];
+  RefBars& bars = *reinterpret_cast<RefBars*>(smem + L::bars);
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, (int)SKA_ERR_UNSUPPORTED);
+    return;
+  }
+  const int r = threadIdx.x, warp = r >> 5;
+  const bool ctl = (threadIdx.x == 0);
+  if (ctl) {
+    mbar_init(&bars.w1g, 1);
+    mbar_init(&bars.w2, 1);
+    mbar_init(&bars.x, 4);
+    mbar_init(&bars.m1, 1);
+    mbar_init(&bars.g, 4);
+    mbar_init(&bars.m2, 1);
+    mbar_init(&bars.drain, 1);
+    bars.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&bars.tmem_base, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = bars.tmem_base;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  RefWaiter wait{&bars, p.status, p.budget_ns};
+  uint8_t* sXh = smem + L::x_hi;
+  uint8_t* sXl = smem + L::x_lo;
+  uint8_t* sW1 = smem + L::w1;
+  uint8_t* sWg = smem + L::wg;
+  uint8_t* sW2 = smem + L::w2;
+  uint8_t* sGh = smem + L::g_hi;
+  uint8_t* sGl = smem + L::g_lo;
+  constexpr uint32_t i1 = idesc_bf16_f32(128, F, false, true);
+  constexpr uint32_t i2 = idesc_bf16_f32(128, D, false, true);
+  const int tiles_per_bh = (p.k + 127) / 128;
+  const int ntiles = p.B * p.H * tiles_per_bh;
+  int it = 0;
+  bool w1g_pending = false, w2_pending = false;  // thread 0: weight loads not yet waited for
+  // tiles in (h, b, row tile) order
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    const int h = tile / (p.B * tiles_per_bh);
+    const int rem = tile - h * p.B * tiles_per_bh;
+    const int b = rem / tiles_per_bh;
+    const int j = (rem - b * tiles_per_bh) * 128 + r;
+    const bool valid = j < p.k;
+    const int64_t row = (static_cast<int64_t>(b) * p.H + h) * p.k + j;
+    const uint32_t par = it & 1;
+    bool ok = true;
+    if (ctl) {  // W_1, W_g of head h into region B (the previous tile's MMAs have all completed)
+      mbar_expect_tx(&bars.w1g, 2 * L::w_bytes);
+      for (int nb = 0; nb < F / 64; ++nb) {
+        tma_load_2d(sW1 + nb * D * 128, &mapW1, &bars.w1g, nb * 64, h * D);
+        tma_load_2d(sWg + nb * D * 128, &mapWg, &bars.w1g, nb * 64, h * D);
+      }
+      w1g_pending = true;
+    }
+    // 1. X- = LN1(x_tilde + x_hat)
+    float xb[D];
+    if (valid) {
+      const float4* a = reinterpret_cast<const float4*>(p.x_tilde + row * D);
+      const float4* c = reinterpret_cast<const float4*>(p.x_hat + row * D);
+#pragma unroll
+      for (int u = 0; u < D / 4; ++u) {
+        const float4 va = a[u], vc = c[u];
+        xb[4 * u] = va.x + vc.x;
+        xb[4 * u + 1] = va.y + vc.y;
+        xb[4 * u + 2] = va.z + vc.z;
+        xb[4 * u + 3] = va.w + vc.w;
+      }
+      layer_norm_row<D>(xb, p.gamma1 ? p.gamma1 + h * D : nullptr, p.beta1 ? p.beta1 + h * D : nullptr, p.eps);
+      if (p.x_bar) store_row_f32<D>(p.x_bar + row * D, xb);
+    } else {
+#pragma unroll
+      for (int u = 0; u < D; ++u) xb[u] = 0.f;
+    }
+#pragma unroll
+    for (int c = 0; c < D; c += 8) store_pair8(sXh, sXl, r, c, xb + c);
+    fence_async_shared();
+    __syncwarp();
+    if ((r & 31) == 0) mbar_arrive(&bars.x);
+    // 2. H1 = X- W_1, Hg = X- W_g
+    if (ctl) {
+      ok = wait(&bars.x, par) && wait(&bars.w1g, par);
+      if (ok) {
+        w1g_pending = false;
+        tc_fence_after();
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t xa = smem_u32(half ? sXl : sXh);
+#pragma unroll
+          for (int s = 0; s < D / 16; ++s) {
+            const uint64_t ad = sw128_desc(xa + (s / 4) * kRefBlk + (s % 4) * 32, 16, 1024);
+            const uint32_t acc = (half | s) > 0;
+            umma_bf16(tb, ad, sw128_desc(smem_u32(sW1) + s * 2048, D * 128, 1024), i1, acc);
+            umma_bf16(tb + F, ad, sw128_desc(smem_u32(sWg) + s * 2048, D * 128, 1024), i1, acc);
+          }
+        }
+        if (!(p.debug_flags & 2u)) umma_commit(&bars.m1);  // the test hook withholds it
+      }
+    }
+    if (!__syncthreads_and(ok && wait(&bars.m1, par))) break;
+    tc_fence_after();
+    if (ctl) {  // W_2 into region A, whose X hi / lo MMA1 has finished reading
+      mbar_expect_tx(&bars.w2, L::w_bytes);
+      for (int nb = 0; nb < D / 64; ++nb) tma_load_2d(sW2 + nb * F * 128, &mapW2, &bars.w2, nb * 64, h * F);
+      w2_pending = true;
+    }
+    // 3. G = swish(H1) * Hg into region B (W_1 / W_g are no longer read)
+#pragma unroll 1
+    for (int c = 0; c < F; c += 16) {
+      uint32_t v1[16], vg[16];
+      tmem_ld16(tb + lane_off + c, v1);
+      tmem_ld16(tb + lane_off + F + c, vg);
+      tmem_ld_wait();
+      float gv[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float a = __uint_as_float(v1[u]);
+        gv[u] = valid ? a / (1.f + __expf(-a)) * __uint_as_float(vg[u]) : 0.f;
+      }
+      store_pair8(sGh, sGl, r, c, gv);
+      store_pair8(sGh, sGl, r, c + 8, gv + 8);
+    }
+    fence_async_shared();
+    tc_fence_before();
+    __syncwarp();
+    if ((r & 31) == 0) mbar_arrive(&bars.g);
+    // 4. Y = G W_2 into TMEM columns [0, D)
+    if (ctl) {
+      ok = wait(&bars.g, par) && wait(&bars.w2, par);
+      if (ok) {
+        w2_pending = false;
+        tc_fence_after();
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t ga = smem_u32(half ? sGl : sGh);
+#pragma unroll
+          for (int s = 0; s < F / 16; ++s)
+            umma_bf16(tb, sw128_desc(ga + (s / 4) * kRefBlk + (s % 4) * 32, 16, 1024),
+                      sw128_desc(smem_u32(sW2) + s * 2048, F * 128, 1024), i2, (half | s) > 0);
+        }
+        umma_commit(&bars.m2);
+      }
+    }
+    if (!__syncthreads_and(ok && wait(&bars.m2, par))) break;
+    tc_fence_after();
+    // 5. X~' = LN2(X- + Y)
+#pragma unroll
+    for (int c = 0; c < D; c += 32) {
+      uint32_t yv[32];
+      tmem_ld32(tb + lane_off + c, yv);
+      tmem_ld_wait();
+#pragma unroll
+      for (int u = 0; u < 32; ++u) xb[c + u] += __uint_as_float(yv[u]);
+    }
+    tc_fence_before();
+    if (valid) {
+      layer_norm_row<D>(xb, p.gamma2 ? p.gamma2 + h * D : nullptr, p.beta2 ? p.beta2 + h * D : nullptr, p.eps);
+      store_row_f32<D>(p.x_next + row * D, xb);
+      if (p.x_next_bf16) {
+        uint4* ob = reinterpret_cast<uint4*>(p.x_next_bf16 + row * D * 2);
+#pragma unroll
+        for (int u = 0; u < D / 8; ++u)
+          ob[u] = make_uint4(pack_bf16x2(xb[8 * u], xb[8 * u + 1]), pack_bf16x2(xb[8 * u + 2], xb[8 * u + 3]),
+                             pack_bf16x2(xb[8 * u + 4], xb[8 * u + 5]), pack_bf16x2(xb[8 * u + 6], xb[8 * u + 7]));
+      }
+    }
+    __syncthreads();  // every thread is done with this tile's TMEM and shared memory
+  }
+  if (ctl) {
+    // all issued MMAs, and any weight load a stopped tile left in flight, end before the exit
+    umma_commit(&bars.drain);
+    wait(&bars.drain, 0, true);
+    if (w1g_pending) wait(&bars.w1g, it & 1, true);
+    if (w2_pending) wait(&bars.w2, it & 1, true);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tb, kCols);
+  }
+}
+
+// After a device-side error, every output element becomes NaN (the rows the stopped CTAs did not
+// reach would otherwise hold stale values).
+__global__ void refine_poison_kernel(const int* status, float* x_next, float* x_bar, uint16_t* x_next_bf16,
+                                     int64_t n) {
+  if (*reinterpret_cast<const volatile int*>(status) == 0) return;
+  const float nan = __int_as_float(0x7fc00000);
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    x_next[i] = nan;
+    if (x_bar) x_bar[i] = nan;
+    if (x_next_bf16) x_next_bf16[i] = 0x7fc0;
+  }
+}
+
+template <int D, int F>
+cudaError_t refine_launch_t(int num_ctas, const CUtensorMap& m1, const CUtensorMap& mg, const CUtensorMap& m2,
+                            const RefineParams& p, cudaStream_t stream) {
+  auto kern = sa_refine_kernel<D, F>;
+  const size_t smem = RefLayout<D, F>::total;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<num_ctas, kRefThreads, smem, stream>>>(m1, mg, m2, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool sa_refine_supported(int D, int F) { return (D == 64 && F == 128) || (D == 128 && F == 256); }
+
+cudaError_t launch_sa_refine(int D, int F, int num_ctas, const CUtensorMap& m1, const CUtensorMap& mg,
+                             const CUtensorMap& m2, const RefineParams& p, cudaStream_t stream) {
+  cudaError_t e = cudaErrorInvalidValue;
+  if (D == 64 && F == 128) e = refine_launch_t<64, 128>(num_ctas, m1, mg, m2, p, stream);
+  if (D == 128 && F == 256) e = refine_launch_t<128, 256>(num_ctas, m1, mg, m2, p, stream);
+  if (e != cudaSuccess) return e;
+  const int64_t n = int64_t(p.B) * p.H * p.k * D;
+  refine_poison_kernel<<<2 * 148, 256, 0, stream>>>(p.status, p.x_next, p.x_bar,
+                                                    reinterpret_cast<uint16_t*>(p.x_next_bf16), n);
+  return cudaGetLastError();
+}
+
+}  // namespace ska

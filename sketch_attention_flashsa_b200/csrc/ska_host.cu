@@ -336,6 +336,16 @@ size_t stca_ws_size(const ska_stca_desc* d, FaWs* w, int* ctas, size_t* smem, in
 }
 }  // namespace
 
+ska_status check_refine_desc(const ska_refine_desc* d) {
+  if (!d) return SKA_ERR_INVALID_VALUE;
+  if (d->num_users < 0 || d->num_heads < 1 || d->num_protos < 1) return SKA_ERR_INVALID_VALUE;
+  if (!(d->eps > 0.f) || !std::isfinite(d->eps)) return SKA_ERR_INVALID_VALUE;
+  if (!sa_refine_supported(d->head_dim, d->ffn_dim)) return SKA_ERR_UNSUPPORTED;
+  if (int64_t(d->num_users) * d->num_heads * d->num_protos * d->head_dim >= (int64_t(1) << 31))
+    return SKA_ERR_INVALID_VALUE;
+  return SKA_OK;
+}
+
 extern "C" {
 
 const char* ska_last_error_string(void) { return g_last_error; }
@@ -704,6 +714,79 @@ ska_status stca_forward(const ska_stca_desc* d, const void* q, const int32_t* cu
     return SKA_ERR_CUDA;
   }
   if (cudaError_t e_ = launch_fa_combine(p, D, B * H * p.group, out, lse, nullptr, s); e_ != cudaSuccess) { record_error("launch_fa_combine", e_); return SKA_ERR_CUDA; }
+  return SKA_OK;
+}
+
+size_t sa_refine_workspace_size(const ska_refine_desc* d) {
+  if (check_refine_desc(d) != SKA_OK) return 0;
+  return sizeof(WsHeader);
+}
+
+ska_status sa_refine(const ska_refine_desc* d, const float* x_tilde, const float* x_hat, const void* w1,
+                     const void* wg, const void* w2, const float* gamma1, const float* beta1, const float* gamma2,
+                     const float* beta2, float* x_next, float* x_bar, void* x_next_bf16, void* ws, size_t ws_bytes,
+                     void* stream) {
+  ska_status st = check_refine_desc(d);
+  if (st != SKA_OK) return st;
+  const int B = d->num_users, H = d->num_heads, k = d->num_protos, D = d->head_dim, F = d->ffn_dim;
+  if (B == 0) return SKA_OK;
+  if (!x_tilde || !x_hat || !w1 || !wg || !w2 || !x_next || !ws) return SKA_ERR_INVALID_VALUE;
+  const void* al[12] = {x_tilde, x_hat, w1, wg, w2, gamma1, beta1, gamma2, beta2, x_next, x_bar, x_next_bf16};
+  for (int i = 0; i < 12; ++i)
+    if (!aligned16(al[i])) return SKA_ERR_INVALID_VALUE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return SKA_ERR_INVALID_VALUE;
+  if (ws_bytes < sizeof(WsHeader)) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  const size_t xb = size_t(B) * H * k * D * 4, wb = size_t(H) * D * F * 2, vb = size_t(H) * D * 4;
+  const void* ins[9] = {x_tilde, x_hat, w1, wg, w2, gamma1, beta1, gamma2, beta2};
+  const size_t insz[9] = {xb, xb, wb, wb, wb, vb, vb, vb, vb};
+  const void* outs[4] = {x_next, x_bar, x_next_bf16, ws};
+  const size_t outsz[4] = {xb, xb, xb / 2, sizeof(WsHeader)};
+  for (int o = 0; o < 4; ++o) {
+    for (int i = 0; i < 9; ++i)
+      if (overlaps(outs[o], outsz[o], ins[i], insz[i])) return SKA_ERR_INVALID_VALUE;
+    for (int o2 = o + 1; o2 < 4; ++o2)
+      if (overlaps(outs[o], outsz[o], outs[o2], outsz[o2])) return SKA_ERR_INVALID_VALUE;
+  }
+  if (no_device()) return SKA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  if (cudaError_t e = cudaMemsetAsync(&hdr->status, 0, sizeof(int32_t), s); e != cudaSuccess) {
+    record_error("cudaMemsetAsync(status)", e);
+    return SKA_ERR_CUDA;
+  }
+  // W_1, W_g: [H d rows, F] in boxes of 64 columns x d rows; W_2: [H F rows, d] in 64 x F boxes
+  CUtensorMap m1, mg, m2;
+  if (!encode_2d(&m1, w1, F, uint64_t(H) * D, F, 64, D)) return SKA_ERR_CUDA;
+  if (!encode_2d(&mg, wg, F, uint64_t(H) * D, F, 64, D)) return SKA_ERR_CUDA;
+  if (!encode_2d(&m2, w2, D, uint64_t(H) * F, D, 64, F)) return SKA_ERR_CUDA;
+  RefineParams p{};
+  p.x_tilde = x_tilde;
+  p.x_hat = x_hat;
+  p.gamma1 = gamma1;
+  p.beta1 = beta1;
+  p.gamma2 = gamma2;
+  p.beta2 = beta2;
+  p.x_bar = x_bar;
+  p.x_next = x_next;
+  p.x_next_bf16 = static_cast<uint8_t*>(x_next_bf16);
+  p.status = &hdr->status;
+  p.B = B;
+  p.H = H;
+  p.k = k;
+  p.eps = d->eps;
+  p.budget_ns = wait_budget();
+  p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
+  const int64_t tiles = int64_t(B) * H * ((k + 127) / 128);
+  const int ctas = static_cast<int>(std::min<int64_t>(tiles, device_sm_count()));
+  cudaError_t e;
+  {
+    TimedRegion tr(s);
+    e = launch_sa_refine(D, F, ctas, m1, mg, m2, p, s);
+  }
+  if (e != cudaSuccess) {
+    record_error("refinement kernel launch", e);
+    return SKA_ERR_CUDA;
+  }
   return SKA_OK;
 }
 

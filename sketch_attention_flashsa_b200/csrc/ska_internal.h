@@ -126,6 +126,32 @@ cudaError_t launch_sa_bwd(int head_dim, int num_ctas, const CUtensorMap& mapQ, c
 // segment (b, h) (per-user queries), in a fixed order; also zeroes dK/dV rows of padding tokens.
 cudaError_t launch_sa_bwd_finish(const SaBwdParams& p, int head_dim, float* dq, cudaStream_t stream);
 
+// Parameters of the stacked refinement of the sketch (sa_refine.cu): rows (b, h, j) of
+// [B, H, k, D] fp32 tensors; per-head LayerNorm vectors [H, D] (nullable: gamma 1, beta 0).
+struct RefineParams {
+  const float* x_tilde;
+  const float* x_hat;
+  const float* gamma1;
+  const float* beta1;
+  const float* gamma2;
+  const float* beta2;
+  float* x_bar;          // nullable: Eq. (13)'s output
+  float* x_next;
+  uint8_t* x_next_bf16;  // nullable: bf16 copy of x_next
+  int* status;           // the workspace status word
+  int B, H, k;
+  float eps;
+  uint64_t budget_ns;
+  uint32_t debug_flags;  // bit 1 (value 2): never signal MMA1's completion (test hook)
+};
+
+bool sa_refine_supported(int head_dim, int ffn_dim);
+// The fused refinement kernel on num_ctas persistent CTAs, then a kernel that turns the outputs
+// to NaN when the status word holds an error.
+cudaError_t launch_sa_refine(int head_dim, int ffn_dim, int num_ctas, const CUtensorMap& mapW1,
+                             const CUtensorMap& mapWg, const CUtensorMap& mapW2, const RefineParams& p,
+                             cudaStream_t stream);
+
 // Small kernels (ska_small.cu).
 cudaError_t launch_schedule(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,
                             int num_clusters, int32_t* tile_prefix, WsHeader* hdr, cudaStream_t stream);

@@ -238,3 +238,44 @@ def config_paper() -> SAInputs:
     def lens(rng):
         return np.clip(np.round(rng.normal(85_000, 10_000, 8)), 1000, 100_000).astype(np.int64)
     return make_sa(None, 1, 128, 1024, 5, length_fn=lens)
+
+
+@dataclasses.dataclass
+class RefineInputs:
+    """One refinement layer's inputs (SequenceO1 §3.3, Eq. (13)-(14)): [B, H, k, d] sketches and the
+    per-head SwiGLU weights (App. G.1) and LayerNorm vectors."""
+    x_tilde: torch.Tensor   # fp32 [B, H, k, d]
+    x_hat: torch.Tensor     # fp32 [B, H, k, d]
+    w1: torch.Tensor        # bf16 [H, d, F]
+    wg: torch.Tensor        # bf16 [H, d, F]
+    w2: torch.Tensor        # bf16 [H, F, d]
+    gamma1: Optional[torch.Tensor] = None  # fp32 [H, d]
+    beta1: Optional[torch.Tensor] = None
+    gamma2: Optional[torch.Tensor] = None
+    beta2: Optional[torch.Tensor] = None
+
+
+def make_refine(B: int, H: int, k: int, d: int, seed: int, *, affine: bool = True,
+                x_sigma: float = 1.0, hat_sigma: float = 1.0) -> RefineInputs:
+    """Draw order: x_tilde, x_hat (N(0, sigma^2) fp32), W_1, W_g (N(0, 1/d)), W_2 (N(0, 1/F)), each
+    rounded to bf16, F = 2d; with ``affine`` then gamma1, beta1, gamma2, beta2 as 1 + 0.1 N(0,1),
+    0.1 N(0,1), 1 + 0.1 N(0,1), 0.1 N(0,1) in fp32."""
+    rng = np.random.default_rng(seed)
+    F = 2 * d
+    xt = normal(rng, (B, H, k, d), x_sigma)
+    xh = normal(rng, (B, H, k, d), hat_sigma)
+    w1 = normal(rng, (H, d, F), 1.0 / math.sqrt(d))
+    wg = normal(rng, (H, d, F), 1.0 / math.sqrt(d))
+    w2 = normal(rng, (H, F, d), 1.0 / math.sqrt(F))
+    out = RefineInputs(torch.from_numpy(xt), torch.from_numpy(xh), to_bf16(w1), to_bf16(wg), to_bf16(w2))
+    if affine:
+        out.gamma1 = torch.from_numpy(1.0 + normal(rng, (H, d), 0.1))
+        out.beta1 = torch.from_numpy(normal(rng, (H, d), 0.1))
+        out.gamma2 = torch.from_numpy(1.0 + normal(rng, (H, d), 0.1))
+        out.beta2 = torch.from_numpy(normal(rng, (H, d), 0.1))
+    return out
+
+
+def config_refine() -> RefineInputs:
+    """The refinement layer on the sketch of the 8 x 100K, H=8, d=128, k=512 workload; seed 6."""
+    return make_refine(8, 8, 512, 128, 6)

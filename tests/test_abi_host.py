@@ -180,3 +180,57 @@ def test_debug_and_timing_hooks_are_host_only():
     lib.ska_set_debug(1_000_000, 0)
     lib.ska_set_debug(0, 0)  # back to the default budget
     lib.ska_set_timing_events(None, None)
+
+
+def refine_desc(**kw):
+    f = dict(num_users=2, num_heads=2, num_protos=300, head_dim=128, ffn_dim=256, eps=1e-5)
+    f.update(kw)
+    return L.RefineDesc(**f)
+
+
+def refine(d, **kw):
+    # x_tilde, x_hat, w1, wg, w2, gamma1, beta1, gamma2, beta2, x_next, x_bar, x_next_bf16, ws
+    names = ["xt", "xh", "w1", "wg", "w2", "g1", "b1", "g2", "b2", "out", "bar", "bf", "ws"]
+    ptrs = {n: (i + 20) * A for i, n in enumerate(names)}
+    ptrs.update(kw)
+    ws_bytes = kw.pop("ws_bytes", 256) if "ws_bytes" in kw else 256
+    args = [ptrs[n] for n in names]
+    return L.lib().sa_refine(ctypes.byref(d) if d is not None else None, *args, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    ({"num_heads": 0}, INVALID), ({"num_protos": 0}, INVALID), ({"num_users": -1}, INVALID),
+    ({"eps": 0.0}, INVALID), ({"eps": float("inf")}, INVALID), ({"eps": float("nan")}, INVALID),
+    ({"head_dim": 96, "ffn_dim": 192}, UNSUP), ({"ffn_dim": 128}, UNSUP), ({"head_dim": 64, "ffn_dim": 256}, UNSUP),
+    ({"num_users": 1 << 12, "num_heads": 64, "num_protos": 64}, INVALID),  # B H k d >= 2^31
+])
+def test_refine_rejects_bad_descriptors(kw, code):
+    d = refine_desc(**kw)
+    assert refine(d) == code
+    assert L.lib().sa_refine_workspace_size(ctypes.byref(d)) == 0
+
+
+def test_refine_pointer_checks():
+    d = refine_desc()
+    assert L.lib().sa_refine_workspace_size(ctypes.byref(d)) == 256
+    assert refine(None) == INVALID
+    for n in ("xt", "xh", "w1", "wg", "w2", "out", "ws"):
+        assert refine(d, **{n: None}) == INVALID, n
+    assert refine(d, g1=40 * A + 4) == INVALID           # 16-byte alignment
+    assert refine(d, ws=41 * A + 16) == INVALID          # 256-byte workspace alignment
+    assert refine(d, ws_bytes=255) == L.SKA_ERR_WORKSPACE_TOO_SMALL
+    assert refine(d, out=20 * A + 64) == INVALID         # the output overlaps x_tilde
+    assert refine(d, bar=29 * A + 1024) == INVALID       # x_bar overlaps x_next
+    assert refine(d, ws=22 * A) == INVALID               # the workspace overlaps W_1
+    # B = 0: nothing to do, no pointer is looked at
+    assert refine(refine_desc(num_users=0), xt=None, xh=None, out=None, ws=None) == L.SKA_OK
+
+
+def test_refine_without_a_device_reports_cuda_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    d = refine_desc()
+    # optional outputs and LayerNorm vectors may be NULL
+    assert refine(d, g1=None, b1=None, g2=None, b2=None, bar=None, bf=None) == L.SKA_ERR_CUDA
+    assert refine(refine_desc(head_dim=64, ffn_dim=128)) == L.SKA_ERR_CUDA

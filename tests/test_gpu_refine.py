@@ -1,0 +1,134 @@
+"""GPU parity of the refinement layer (SequenceO1 §3.3, Eq. (13)-(14); SwiGLU FFN of App. G.1)
+against the fp64 oracle, through the C ABI (sa_refine).
+
+Tolerance, from the kernel's arithmetic: the FFN products use a two-term bf16 split of the fp32
+activations (relative error 2^-17 per product) against the exact bf16 weights. Sums of up to
+F = 256 terms then accumulate in fp32, and LayerNorm runs in fp32. The expected error on the
+O(1) outputs is about 1e-5. The bounds are max abs <= 1e-3 and relative L2 <= 1e-4. A kernel
+that used plain bf16 activations (2^-9 per product) would miss the L2 bound by an order of
+magnitude.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sketch_attention_flashsa_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 1e-3
+REL_L2 = 1e-4
+
+
+def _api():
+    from sketch_attention_flashsa_b200 import api
+    return api
+
+
+def f64(t):
+    return None if t is None else t.float().numpy().astype(np.float64)
+
+
+def run_gpu(inp: W.RefineInputs, status=False):
+    api = _api()
+    dev = "cuda"
+    g = lambda t: None if t is None else t.to(dev)
+    desc = api.refine_desc(inp.x_tilde, inp.w1)
+    ws = torch.empty(api.sa_refine_workspace_size(desc), dtype=torch.uint8, device=dev)
+    x_next, x_bar, x_bf = api.sa_refine(g(inp.x_tilde), g(inp.x_hat), g(inp.w1), g(inp.wg), g(inp.w2),
+                                        g(inp.gamma1), g(inp.beta1), g(inp.gamma2), g(inp.beta2),
+                                        want_x_bar=True, want_bf16=True, workspace=ws)
+    torch.cuda.synchronize()
+    out = [x_next.cpu(), x_bar.cpu(), x_bf.cpu()]
+    if status:
+        out.append(api.read_device_status(ws))
+    return tuple(out)
+
+
+def run_oracle(inp: W.RefineInputs):
+    return oracle.refine(f64(inp.x_tilde), f64(inp.x_hat), f64(inp.w1), f64(inp.wg), f64(inp.w2),
+                         f64(inp.gamma1), f64(inp.beta1), f64(inp.gamma2), f64(inp.beta2))
+
+
+def assert_close(got, want, what):
+    got = got.numpy().astype(np.float64) if isinstance(got, torch.Tensor) else got
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    err = np.abs(got - want)
+    mx = float(err.max()) if err.size else 0.0
+    denom = float(np.linalg.norm(want))
+    rel = float(np.linalg.norm(got - want) / denom) if denom > 0 else float(np.linalg.norm(got))
+    print(f"[parity] {what}: max abs {mx:.3e}, rel L2 {rel:.3e}")
+    assert mx <= MAX_ABS and rel <= REL_L2, f"{what}: max abs {mx:.3e}, rel L2 {rel:.3e}"
+
+
+def check(inp: W.RefineInputs):
+    x_next, x_bar, x_bf, st = run_gpu(inp, status=True)
+    assert st == 0
+    o_bar, o_next = run_oracle(inp)
+    assert_close(x_bar, o_bar, "x_bar (Eq. 13)")
+    assert_close(x_next, o_next, "x_next (Eq. 14)")
+    # the bf16 copy is the round-to-nearest-even of the fp32 output
+    assert torch.equal(x_bf, x_next.to(torch.bfloat16))
+    return x_next
+
+
+CASES = {
+    # (B, H, k, d, affine): ragged row tails, single rows, exact tiles, many (user, head) pairs
+    "d64_k200_affine": (2, 3, 200, 64, True),
+    "d128_k300_plain": (3, 2, 300, 128, False),
+    "d64_k1": (1, 1, 1, 64, True),
+    "d128_k128": (2, 1, 128, 128, True),
+    "d128_k17": (5, 4, 17, 128, True),
+    "d64_k1000": (1, 2, 1000, 64, True),
+    # more tiles than SMs: every CTA walks several tiles (barrier phases flip)
+    "d64_k700_persistent": (4, 8, 700, 64, True),
+    "d128_k520_persistent": (3, 8, 520, 128, False),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_refine_parity(name):
+    B, H, k, d, affine = CASES[name]
+    check(W.make_refine(B, H, k, d, seed=700 + len(name) + d, affine=affine))
+
+
+def test_refine_full_sketch_config():
+    """Every row of the 8 users x 8 heads x 512 sketch rows, d = 128 (256 tiles)."""
+    check(W.config_refine())
+
+
+def test_refine_constant_rows_and_large_inputs():
+    """Rows whose residual sum is constant have zero variance: LN gives beta exactly (up to the
+    eps-scaled zero). Large input scales leave LN's output unchanged."""
+    inp = W.make_refine(2, 2, 150, 128, seed=91, x_sigma=300.0, hat_sigma=300.0)
+    inp.x_tilde[0, 1, 5:40] = 7.0
+    inp.x_hat[0, 1, 5:40] = -2.5
+    x_next = check(inp)
+    o_bar, _ = run_oracle(inp)
+    np.testing.assert_allclose(o_bar[0, 1, 5:40], np.broadcast_to(inp.beta1[1].double().numpy(), (35, 128)),
+                               atol=1e-12)
+    assert torch.isfinite(x_next).all()
+
+
+def test_refine_deterministic():
+    inp = W.make_refine(2, 4, 333, 64, seed=5)
+    a = run_gpu(inp)[0]
+    b = run_gpu(inp)[0]
+    assert torch.equal(a, b)
+
+
+def test_refine_timeout_reports_and_poisons():
+    """The test hook withholds MMA1's completion: every bounded wait runs out, the call records
+    SKA_ERR_DEVICE_TIMEOUT and all outputs are NaN; the next call is correct again."""
+    api = _api()
+    inp = W.make_refine(2, 2, 256, 64, seed=8)
+    api.set_debug(2_000_000, 2)
+    try:
+        x_next, x_bar, x_bf, st = run_gpu(inp, status=True)
+    finally:
+        api.set_debug(0, 0)
+    assert st == 5
+    assert torch.isnan(x_next).all() and torch.isnan(x_bar).all() and torch.isnan(x_bf.float()).all()
+    check(inp)
