@@ -17,10 +17,16 @@ Readings taken here (the pages name LN and the FFN but not their details):
 * swish(u) = u * sigmoid(u) (swish with beta = 1, i.e. SiLU).
 * H heads are H independent problems on d-wide slices, each with its own LN and FFN parameters
   (the paper's SA is single-head: H = 1).
+* X~^(0) = P^(0): layer 0's input sketch is the prototype matrix itself, the same for every user, so
+  that S^(0) of Eq. (10) is Eq. (7)'s (P^(0) W_Q)(X W_K)^T and its residual in Eq. (13) adds P^(0).
+* The keys K^(l) = X W_K^(l) of each layer are inputs (the key projection of the history is not
+  part of this oracle); the values are X itself (Eq. (9), Eq. (12)).
 """
 from __future__ import annotations
 
 import numpy as np
+
+from .sa import NORM_PROTO, sa_forward
 
 LN_EPS = 1e-5
 
@@ -72,3 +78,39 @@ def refine(x_tilde, x_hat, w1, wg, w2, gamma1=None, beta1=None, gamma2=None, bet
         x_bar[:, h] = xb
         out[:, h] = layer_norm(xb + y, g2, b2)                            # Eq. (14)
     return x_bar, out
+
+
+def project_queries(x, w_q):
+    """Queries of one layer, X~^(l) W_Q^(l) (Eq. (10); Eq. (7) for the prototypes P^(0)), per head.
+
+    x: [H, k, d] or [B, H, k, d]; w_q: [H, d, d]. Returns x's shape.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w_q, dtype=np.float64)
+    out = np.zeros(x.shape)
+    for h in range(w.shape[0]):
+        out[..., h, :, :] = x[..., h, :, :] @ w[h]
+    return out
+
+
+def stacked_sa(p0, w_q, keys, v, cu_seqlens, seqused, scale, ffn):
+    """N_sa stacked SA layers (§3.3, Eq. (10)-(14)), N_sa = len(w_q).
+
+    p0: [H, k, d] prototypes P^(0) (= X~^(0), shared by all users); w_q: N_sa arrays [H, d, d];
+    keys: N_sa arrays [T, H, d], K^(l) = X W_K^(l); v: [T, H, d] the history X (the values);
+    ffn: N_sa tuples (w1, wg, w2, gamma1, beta1, gamma2, beta2) as in `refine`.
+    Layer l: Q = X~^(l) W_Q^(l); X^^(l+1) = A^(l) X with A^(l) the prototype-wise softmax of
+    scale Q K^(l)T (Eq. (10)-(12)); X~^(l+1) from Eq. (13)-(14).
+    Returns X~^(N_sa) as [B, H, k, d] and the per-layer sketches X^^(l+1).
+    """
+    p0 = np.asarray(p0, dtype=np.float64)
+    B = len(cu_seqlens) - 1
+    x_t = np.broadcast_to(p0, (B,) + p0.shape).copy()
+    sketches = []
+    for l in range(len(w_q)):
+        q = project_queries(x_t, w_q[l])
+        x_hat, _, _ = sa_forward(q, keys[l], v, cu_seqlens, seqused, scale, NORM_PROTO)
+        sketches.append(x_hat)
+        _, x_t = refine(x_t, x_hat, *ffn[l])
+    return x_t, sketches
+

@@ -440,3 +440,92 @@ def test_refine_heads_rows_and_users_are_independent():
     # the residual: x_bar is LN of the sum, so swapping the two inputs changes nothing
     xb_s, out_s = oracle.refine(xh, xt, w1, wg, w2, g1, b1, g2, b2)
     assert np.allclose(out_s, out, atol=1e-12)
+
+
+# --------------------------------------------------------------------- stacked layers (§3.3)
+
+def test_project_queries_hand_example():
+    """Per head x W_Q^h, with x on the left: head 0 swaps the two features, head 1 is the upper
+    triangular [[1, 2], [0, 1]] (its transpose would give [3, 1] instead of [1, 3])."""
+    w = np.array([[[0.0, 1.0], [1.0, 0.0]], [[1.0, 2.0], [0.0, 1.0]]])
+    x = np.array([[[1.0, 2.0]], [[1.0, 1.0]]])            # [H=2, k=1, d=2]
+    q = oracle.project_queries(x, w)
+    assert np.array_equal(q, [[[2.0, 1.0]], [[1.0, 3.0]]])
+    # per-user rows [B, H, k, d] use the same weights for every user
+    xb = np.stack([x, 2 * x])
+    assert np.array_equal(oracle.project_queries(xb, w), np.stack([q, 2 * q]))
+
+
+def _ln2(a, b, eps=1e-5):
+    """LayerNorm of the 2-vector [a, b] (no affine): [-c, c] * sign(b - a), c = h / sqrt(h^2 + eps)."""
+    h = (b - a) / 2.0
+    c = h / math.sqrt(h * h + eps)
+    return -c, c
+
+
+def test_stacked_sa_one_prototype_hand_worked():
+    """k = 1: every token gives all its weight to the single prototype, so each layer's sketch is
+    the sum of the values, [1, 2] + [3, 4] = [4, 6], whatever the queries and keys. With W_2 = 0
+    each layer is LN(LN(residual)); layer 0's LN2 has beta = [10, 0]. Layer 0: [1, 0] + [4, 6] ->
+    two LNs -> [-c, c] + [10, 0]; layer 1 adds [4, 6] to that (not to P^(0)), which flips the sign
+    of the normalised difference."""
+    p0 = np.array([[[1.0, 0.0]]])                         # [H=1, k=1, d=2]
+    v = np.array([[[1.0, 2.0]], [[3.0, 4.0]]])            # [T=2, H=1, d=2]
+    rng = np.random.default_rng(80)
+    keys = [rng.normal(size=(2, 1, 2)) for _ in range(2)]
+    w_q = [rng.normal(size=(1, 2, 2)) for _ in range(2)]
+    w1, wg, w2 = rng.normal(size=(1, 2, 4)), rng.normal(size=(1, 2, 4)), np.zeros((1, 4, 2))
+    ffn0 = (w1, wg, w2, None, None, None, np.array([[10.0, 0.0]]))
+    ffn1 = (w1, wg, w2, None, None, None, None)
+    out, sketches = oracle.stacked_sa(p0, w_q, keys, v, np.array([0, 2]), None, 1.0, [ffn0, ffn1])
+    for s in sketches:
+        assert np.allclose(s, [[[[4.0, 6.0]]]], atol=1e-14)
+    a, b = _ln2(1.0 + 4.0, 0.0 + 6.0)
+    a, b = _ln2(a, b)
+    x1 = (a + 10.0, b)
+    a, b = _ln2(x1[0] + 4.0, x1[1] + 6.0)
+    a, b = _ln2(a, b)
+    assert np.allclose(out, [[[[a, b]]]], atol=1e-12)
+    assert a > 0 > b
+
+
+def test_stacked_sa_zero_queries_average_the_values():
+    """W_Q = 0 in every layer: all scores are 0, every token splits its weight evenly over the k
+    prototypes, and each layer's sketch row is (1 / k) sum_i x_i for every prototype."""
+    rng = np.random.default_rng(81)
+    H, k, d, f = 2, 3, 4, 8
+    lens = [5, 2]
+    cu = np.array([0, 5, 7])
+    v = rng.normal(size=(7, H, d))
+    keys = [rng.normal(size=(7, H, d)) for _ in range(2)]
+    w_q = [np.zeros((H, d, d))] * 2
+    ffn = [(rng.normal(size=(H, d, f)), rng.normal(size=(H, d, f)), rng.normal(size=(H, f, d)),
+            None, None, None, None)] * 2
+    _, sketches = oracle.stacked_sa(rng.normal(size=(H, k, d)), w_q, keys, v, cu, None, 1.0, ffn)
+    for s in sketches:
+        for b, (lo, n) in enumerate(zip(cu[:-1], lens)):
+            want = v[lo:lo + n].sum(axis=0) / k                # [H, d]
+            assert np.allclose(s[b], np.broadcast_to(want[:, None, :], (H, k, d)), atol=1e-13)
+
+
+def test_stacked_sa_token_order_and_users():
+    """The stack sees a user's history as a set (the same permutation of keys and values leaves
+    every layer unchanged), and users do not interact."""
+    rng = np.random.default_rng(82)
+    H, k, d, f = 1, 4, 8, 16
+    cu = np.array([0, 6, 9])
+    v = rng.normal(size=(9, H, d))
+    keys = [rng.normal(size=(9, H, d)) for _ in range(2)]
+    w_q = [rng.normal(size=(H, d, d)) / 3 for _ in range(2)]
+    ffn = [(rng.normal(size=(H, d, f)) / 3, rng.normal(size=(H, d, f)) / 3, rng.normal(size=(H, f, d)) / 3,
+            1 + rng.normal(size=(H, d)) / 10, rng.normal(size=(H, d)) / 10,
+            1 + rng.normal(size=(H, d)) / 10, rng.normal(size=(H, d)) / 10) for _ in range(2)]
+    p0 = rng.normal(size=(H, k, d))
+    out, _ = oracle.stacked_sa(p0, w_q, keys, v, cu, None, 0.5, ffn)
+    perm = np.concatenate([rng.permutation(6), 6 + rng.permutation(3)])
+    outp, _ = oracle.stacked_sa(p0, w_q, [kk[perm] for kk in keys], v[perm], cu, None, 0.5, ffn)
+    assert np.allclose(outp, out, atol=1e-12)
+    v2 = v.copy()
+    v2[6:] += rng.normal(size=(3, H, d))  # (a shift equal on every feature would be absorbed by LN)
+    out2, _ = oracle.stacked_sa(p0, w_q, keys, v2, cu, None, 0.5, ffn)
+    assert np.array_equal(out2[0], out[0]) and not np.allclose(out2[1], out[1])
