@@ -201,7 +201,9 @@ SKA_API ska_status stca_forward(const ska_stca_desc* desc, const void* q, const 
  * vectors, as the SA call treats heads as independent problems.
  *   num_users B >= 0, num_heads H >= 1, num_protos k >= 1 (the sketch rows of one user and head;
  *   any k), head_dim 64 or 128, ffn_dim = 2 head_dim (other pairs: SKA_ERR_UNSUPPORTED), eps > 0
- *   and finite. B * H * k * head_dim < 2^31.                                                    */
+ *   and finite. B * H * k * head_dim < 2^31.
+ *   x_tilde_shared  0: x_tilde is [B, H, k, d]; 1: x_tilde is [H, k, d], one set of rows for every
+ *                   user (layer 0, whose X~ is the prototypes P^(0)).                           */
 typedef struct {
   int32_t num_users;
   int32_t num_heads;
@@ -209,27 +211,46 @@ typedef struct {
   int32_t head_dim;
   int32_t ffn_dim;
   float eps;
+  int32_t x_tilde_shared;
+  int32_t reserved;
 } ska_refine_desc;
 
 /* Bytes of workspace sa_refine needs: 256, the status word (0 if the descriptor is invalid). */
 SKA_API size_t sa_refine_workspace_size(const ska_refine_desc* desc);
 
 /* Refinement layer. Device pointers; shapes for B users, H heads, k rows, d = head_dim, F = ffn_dim:
- *   x_tilde, x_hat   fp32 [B, H, k, d]: the layer's input sketch and its SA output (sa_forward's
- *                    sketch)
+ *   x_tilde          fp32 [B, H, k, d] (or [H, k, d] with x_tilde_shared): the layer's input sketch
+ *   x_hat            fp32 [B, H, k, d]: its SA output (sa_forward's sketch)
  *   w1, wg           bf16 [H, d, F];  w2  bf16 [H, F, d]
  *   gamma1, beta1, gamma2, beta2   fp32 [H, d] or NULL (NULL: gamma = 1, beta = 0)
+ *   w_q_next         bf16 [H, d, d] or NULL: the next layer's query weights W_Q^(l+1)
  *   x_next           out, fp32 [B, H, k, d]
  *   x_bar            out, fp32 [B, H, k, d], or NULL when not wanted
- *   x_next_bf16      out, bf16 [B, H, k, d], or NULL: a bf16 copy of x_next for the next
- *                    layer's projections
- * The LayerNorms, the residual sums and swish run in fp32. The FFN products take their
- * activations as a two-term bf16 split (16 significant bits) against the bf16 weights, with
- * fp32 accumulation. B = 0 returns SKA_OK without launching anything.                           */
+ *   x_next_bf16      out, bf16 [B, H, k, d], or NULL: a bf16 copy of x_next
+ *   q_next           out, bf16 [B, H, k, d], or NULL: x_next W_Q^(l+1) for each head, the per-user
+ *                    queries of the next layer (Eq. (10); pass them to sa_forward with
+ *                    q_per_user = 1 and scale 1/sqrt(d)). w_q_next and q_next come together.
+ * The LayerNorms, the residual sums and swish run in fp32. The products with the weights take
+ * their activations as a two-term bf16 split (16 significant bits) against the bf16 weights,
+ * with fp32 accumulation; q_next is rounded to bf16 at the end. B = 0 returns SKA_OK without
+ * launching anything.                                                                           */
 SKA_API ska_status sa_refine(const ska_refine_desc* desc, const float* x_tilde, const float* x_hat,
                              const void* w1, const void* wg, const void* w2, const float* gamma1,
-                             const float* beta1, const float* gamma2, const float* beta2, float* x_next,
-                             float* x_bar, void* x_next_bf16, void* ws, size_t ws_bytes, void* stream);
+                             const float* beta1, const float* gamma2, const float* beta2,
+                             const void* w_q_next, float* x_next, float* x_bar, void* x_next_bf16,
+                             void* q_next, void* ws, size_t ws_bytes, void* stream);
+
+/* Query projection of sketch rows, q = x W_Q per head (Eq. (7)'s P^(0) W_Q for layer 0, Eq. (10)'s
+ * X~^(l) W_Q^(l) otherwise); the same kernel and precision as sa_refine's q_next.
+ *   x      fp32 [num_users, num_heads, num_rows, head_dim]   (num_users = 1 for the prototypes)
+ *   w_q    bf16 [num_heads, head_dim, head_dim]
+ *   q_out  out, bf16, x's shape
+ *   ws     at least 256 bytes (the device status word; ska_read_device_status reads it)
+ * head_dim 64 or 128 (else SKA_ERR_UNSUPPORTED); num_heads, num_rows >= 1; num_users = 0 is a
+ * no-op.                                                                                        */
+SKA_API ska_status sa_project_queries(int32_t num_users, int32_t num_heads, int32_t num_rows, int32_t head_dim,
+                                      const float* x, const void* w_q, void* q_out, void* ws,
+                                      size_t ws_bytes, void* stream);
 
 /* Human-readable name of a status code (static string). */
 SKA_API const char* ska_status_string(ska_status status);

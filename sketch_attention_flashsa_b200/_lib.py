@@ -24,7 +24,7 @@ EXPORTED = ("sa_forward_workspace_size", "sa_forward", "sa_backward_workspace_si
             "stca_forward_workspace_size", "stca_forward", "ska_status_string",
             "ska_read_device_status", "ska_set_debug", "ska_set_timing_events",
             "sa_forward_noalloc", "sa_forward_noalloc_scratch_bytes", "sa_forward_noalloc_read_status",
-            "ska_last_error_string", "sa_refine_workspace_size", "sa_refine")
+            "ska_last_error_string", "sa_refine_workspace_size", "sa_refine", "sa_project_queries")
 
 
 class SaDesc(ctypes.Structure):
@@ -46,7 +46,8 @@ class StcaDesc(ctypes.Structure):
 class RefineDesc(ctypes.Structure):
     _fields_ = [("num_users", ctypes.c_int32), ("num_heads", ctypes.c_int32),
                 ("num_protos", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("ffn_dim", ctypes.c_int32), ("eps", ctypes.c_float)]
+                ("ffn_dim", ctypes.c_int32), ("eps", ctypes.c_float), ("x_tilde_shared", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class SkaError(RuntimeError):
@@ -99,8 +100,10 @@ def lib() -> ctypes.CDLL:
     L.sa_forward_noalloc_read_status.restype = ctypes.c_int
     L.sa_refine_workspace_size.argtypes = [ctypes.POINTER(RefineDesc)]
     L.sa_refine_workspace_size.restype = sz
-    L.sa_refine.argtypes = [ctypes.POINTER(RefineDesc)] + [vp] * 13 + [sz, vp]
+    L.sa_refine.argtypes = [ctypes.POINTER(RefineDesc)] + [vp] * 15 + [sz, vp]
     L.sa_refine.restype = ctypes.c_int
+    L.sa_project_queries.argtypes = [ctypes.c_int32] * 4 + [vp] * 4 + [sz, vp]
+    L.sa_project_queries.restype = ctypes.c_int
     L.ska_set_timing_events.argtypes = [vp, vp]
     L.ska_set_timing_events.restype = None
     _lib = L

@@ -324,11 +324,13 @@ def sa_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: t
     return dq, dk, dv
 
 
-def refine_desc(x_tilde, w1, *, eps: float = 1e-5) -> RefineDesc:
+def refine_desc(x_tilde, x_hat, w1, *, eps: float = 1e-5) -> RefineDesc:
     d = RefineDesc()
-    d.num_users, d.num_heads, d.num_protos, d.head_dim = (int(v) for v in x_tilde.shape)
+    d.num_users, d.num_heads, d.num_protos, d.head_dim = (int(v) for v in x_hat.shape)
     d.ffn_dim = int(w1.shape[-1])
     d.eps = float(eps)
+    d.x_tilde_shared = 1 if x_tilde.dim() == 3 else 0
+    d.reserved = 0
     return d
 
 
@@ -339,46 +341,77 @@ def sa_refine_workspace_size(desc: RefineDesc) -> int:
 def sa_refine(x_tilde: torch.Tensor, x_hat: torch.Tensor, w1: torch.Tensor, wg: torch.Tensor, w2: torch.Tensor,
               gamma1: Optional[torch.Tensor] = None, beta1: Optional[torch.Tensor] = None,
               gamma2: Optional[torch.Tensor] = None, beta2: Optional[torch.Tensor] = None, *, eps: float = 1e-5,
-              want_x_bar: bool = False, want_bf16: bool = False, workspace: Optional[torch.Tensor] = None,
-              out: Optional[torch.Tensor] = None, stream=None):
+              w_q_next: Optional[torch.Tensor] = None, want_x_bar: bool = False, want_bf16: bool = False,
+              workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None):
     """Stacked refinement of the sketch (SequenceO1 §3.3, Eq. (13)-(14)) with the SwiGLU FFN of
     App. G.1: x_bar = LN1(x_tilde + x_hat), x_next = LN2(x_bar + (swish(x_bar W1) * (x_bar Wg)) W2).
 
-    x_tilde, x_hat fp32 [B,H,k,d] (x_hat: this layer's sa_forward sketch); w1, wg bf16 [H,d,F];
-    w2 bf16 [H,F,d] with F = 2d; gamma*, beta* fp32 [H,d] or None. Returns (x_next fp32,
-    x_bar fp32 or None, x_next bf16 or None), each [B,H,k,d].
+    x_hat fp32 [B,H,k,d] (this layer's sa_forward sketch); x_tilde fp32 [B,H,k,d], or [H,k,d] for
+    rows shared by every user (layer 0: the prototypes); w1, wg bf16 [H,d,F]; w2 bf16 [H,F,d] with
+    F = 2d; gamma*, beta* fp32 [H,d] or None; w_q_next bf16 [H,d,d] or None: also return the next
+    layer's per-user queries x_next W_Q (Eq. (10)). Returns (x_next fp32, x_bar fp32 or None,
+    x_next bf16 or None, q_next bf16 or None), each [B,H,k,d].
     """
-    if x_tilde.dim() != 4:
-        raise ValueError(f"x_tilde must be [B, H, k, d], got shape {tuple(x_tilde.shape)}")
-    B, H, k, D = x_tilde.shape
-    _shape("x_hat", x_hat, x_tilde.shape)
+    if x_hat.dim() != 4:
+        raise ValueError(f"x_hat must be [B, H, k, d], got shape {tuple(x_hat.shape)}")
+    B, H, k, D = x_hat.shape
+    if x_tilde.dim() == 3:
+        _shape("x_tilde", x_tilde, (H, k, D))
+    else:
+        _shape("x_tilde", x_tilde, x_hat.shape)
     if w1.dim() != 3 or w1.shape[0] != H or w1.shape[1] != D:
         raise ValueError(f"w1 must be [{H}, {D}, F], got {tuple(w1.shape)}")
     F = w1.shape[2]
     _shape("wg", wg, (H, D, F))
     _shape("w2", w2, (H, F, D))
+    _shape("w_q_next", w_q_next, (H, D, D))
     for name, t in (("gamma1", gamma1), ("beta1", beta1), ("gamma2", gamma2), ("beta2", beta2)):
         _shape(name, t, (H, D))
-    _shape("out", out, x_tilde.shape)
+    _shape("out", out, x_hat.shape)
     for name, t in (("x_tilde", x_tilde), ("x_hat", x_hat), ("gamma1", gamma1), ("beta1", beta1),
                     ("gamma2", gamma2), ("beta2", beta2), ("out", out)):
         _dev_tensor(name, t, (torch.float32,))
-    for name, t in (("w1", w1), ("wg", wg), ("w2", w2)):
+    for name, t in (("w1", w1), ("wg", wg), ("w2", w2), ("w_q_next", w_q_next)):
         _dev_tensor(name, t, (torch.bfloat16,))
-    desc = refine_desc(x_tilde, w1, eps=eps)
+    desc = refine_desc(x_tilde, x_hat, w1, eps=eps)
+    L = _lib.lib()
     need = sa_refine_workspace_size(desc)
     if need == 0:
-        _check(_lib.lib().sa_refine(ctypes.byref(desc), *([ctypes.c_void_p(0)] * 13), ctypes.c_size_t(0),
-                                    ctypes.c_void_p(0)), "sa_refine")
-    dev = x_tilde.device
+        _check(L.sa_refine(ctypes.byref(desc), *([ctypes.c_void_p(0)] * 15), ctypes.c_size_t(0),
+                           ctypes.c_void_p(0)), "sa_refine")
+    dev = x_hat.device
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    out = torch.empty(x_tilde.shape, dtype=torch.float32, device=dev) if out is None else out
-    x_bar = torch.empty(x_tilde.shape, dtype=torch.float32, device=dev) if want_x_bar else None
-    x_bf = torch.empty(x_tilde.shape, dtype=torch.bfloat16, device=dev) if want_bf16 else None
-    rc = _lib.lib().sa_refine(ctypes.byref(desc), _ptr(x_tilde), _ptr(x_hat), _ptr(w1), _ptr(wg), _ptr(w2),
-                              _ptr(gamma1), _ptr(beta1), _ptr(gamma2), _ptr(beta2), _ptr(out), _ptr(x_bar),
-                              _ptr(x_bf), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    out = torch.empty(x_hat.shape, dtype=torch.float32, device=dev) if out is None else out
+    x_bar = torch.empty(x_hat.shape, dtype=torch.float32, device=dev) if want_x_bar else None
+    x_bf = torch.empty(x_hat.shape, dtype=torch.bfloat16, device=dev) if want_bf16 else None
+    q_next = torch.empty(x_hat.shape, dtype=torch.bfloat16, device=dev) if w_q_next is not None else None
+    rc = L.sa_refine(ctypes.byref(desc), _ptr(x_tilde), _ptr(x_hat), _ptr(w1), _ptr(wg), _ptr(w2), _ptr(gamma1),
+                     _ptr(beta1), _ptr(gamma2), _ptr(beta2), _ptr(w_q_next), _ptr(out), _ptr(x_bar), _ptr(x_bf),
+                     _ptr(q_next), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check(rc, "sa_refine")
-    return out, x_bar, x_bf
+    return out, x_bar, x_bf, q_next
 
+
+def project_queries(x: torch.Tensor, w_q: torch.Tensor, *, workspace: Optional[torch.Tensor] = None,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """q = x W_Q for each head (SequenceO1 Eq. (7) P^(0) W_Q; Eq. (10) X~^(l) W_Q^(l)).
+
+    x fp32 [H,k,d] (the prototypes) or [B,H,k,d]; w_q bf16 [H,d,d]. Returns q bf16 of x's shape.
+    """
+    if x.dim() not in (3, 4):
+        raise ValueError(f"x must be [H, k, d] or [B, H, k, d], got shape {tuple(x.shape)}")
+    shape4 = (1,) + tuple(x.shape) if x.dim() == 3 else tuple(x.shape)
+    B, H, k, D = shape4
+    _shape("w_q", w_q, (H, D, D))
+    _shape("out", out, x.shape)
+    _dev_tensor("x", x, (torch.float32,))
+    _dev_tensor("w_q", w_q, (torch.bfloat16,))
+    _dev_tensor("out", out, (torch.bfloat16,))
+    if workspace is None or workspace.numel() < 256:
+        workspace = torch.empty(256, dtype=torch.uint8, device=x.device)
+    out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device) if out is None else out
+    rc = _lib.lib().sa_project_queries(B, H, k, D, _ptr(x), _ptr(w_q), _ptr(out), _ptr(workspace),
+                                       ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check(rc, "sa_project_queries")
+    return out

@@ -4,14 +4,18 @@
 // every sketch row (b, h, j), using the weights and LayerNorm parameters of head h.
 //
 // One CTA of 128 threads takes 128 rows of one (user, head) at a time, one thread per row:
-//   1. X- = LN1(x_tilde + x_hat) in fp32. The result stays in registers for the residual. It is
-//      also written to shared memory as a bf16 pair hi + lo (16 significant bits) in the
-//      K-major A-operand layout.
+//   1. X- = LN1(x_tilde + x_hat) in fp32. The thread parks it in its own row of the output for the
+//      residual of step 5. It is also written to shared memory as a bf16 pair hi + lo
+//      (16 significant bits) in the K-major A-operand layout.
 //   2. MMA: H1 = X- W_1 and Hg = X- W_g (M = 128, N = F, K = d; one pass for hi, one for lo),
 //      accumulated in TMEM.
 //   3. G = swish(H1) * Hg, again as a bf16 hi + lo pair in shared memory.
 //   4. MMA: Y = G W_2 (M = 128, N = d, K = F; hi and lo passes) into the TMEM columns H1 held.
 //   5. X~' = LN2(X- + Y) in fp32, written to global memory (plus a bf16 copy when asked for).
+//   6. (optional) the next layer's queries X~' W_Q (Eq. (10)): X~' as a bf16 hi + lo pair in
+//      shared memory, MMA against W_Q (M = 128, N = d, K = d), rounded to bf16.
+// In projection mode the kernel runs step 6 alone on its input rows: the layer-0 queries
+// P^(0) W_Q of Eq. (7).
 // The weights are bf16 inputs. Multiplying them with the hi + lo pairs leaves about 2^-17 relative
 // error per product, and the fp32 accumulation does the rest. Thread 0 issues the TMA weight
 // loads and the MMAs. The phases of one tile run in sequence. The kernel is memory-bound at its
@@ -39,6 +43,7 @@ struct RefLayout {
   static constexpr uint32_t x_bytes = (D / 64) * kRefBlk;
   static constexpr uint32_t g_bytes = (F / 64) * kRefBlk;
   static constexpr uint32_t w_bytes = D * F * 2;
+  static constexpr uint32_t wq_bytes = D * D * 2;
   static constexpr uint32_t a_bytes = (2 * x_bytes > w_bytes) ? 2 * x_bytes : w_bytes;
   static constexpr uint32_t b_bytes = (2 * g_bytes > 2 * w_bytes) ? 2 * g_bytes : 2 * w_bytes;
   static constexpr uint32_t x_hi = 0;
@@ -52,10 +57,11 @@ struct RefLayout {
   static constexpr uint32_t total = bars + 128;
   static_assert(a_bytes % 1024 == 0 && w_bytes % 1024 == 0 && g_bytes % 1024 == 0, "1024-byte aligned blocks");
   static_assert(total <= 227 * 1024, "fits in shared memory");
+  static_assert(wq_bytes <= b_bytes, "W_Q fits in region B");
 };
 
 struct RefBars {
-  uint64_t w1g, w2, x, m1, g, m2, drain;
+  uint64_t w1g, w2, x, m1, g, m2, wq, xq, m3, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -129,10 +135,20 @@ __device__ __forceinline__ void store_row_f32(float* dst, const float* x) {
   for (int u = 0; u < D / 4; ++u) o[u] = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
 }
 
+template <int D>
+__device__ __forceinline__ void store_row_bf16(uint8_t* dst, const float* x) {
+  uint4* ob = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int u = 0; u < D / 8; ++u)
+    ob[u] = make_uint4(pack_bf16x2(x[8 * u], x[8 * u + 1]), pack_bf16x2(x[8 * u + 2], x[8 * u + 3]),
+                       pack_bf16x2(x[8 * u + 4], x[8 * u + 5]), pack_bf16x2(x[8 * u + 6], x[8 * u + 7]));
+}
+
 template <int D, int F>
 __global__ void __launch_bounds__(kRefThreads, 1)
     sa_refine_kernel(const __grid_constant__ CUtensorMap mapW1, const __grid_constant__ CUtensorMap mapWg,
-                     const __grid_constant__ CUtensorMap mapW2, const RefineParams p) {
+                     const __grid_constant__ CUtensorMap mapW2, const __grid_constant__ CUtensorMap mapWq,
+                     const RefineParams p) {
   using L = RefLayout<D, F>;
   constexpr uint32_t kCols = 2 * F;  // H1 | Hg
   static_assert(kCols <= 512 && (kCols & (kCols - 1)) == 0, "TMEM allocation is a power of two <= 512");
@@ -151,6 +167,9 @@ __global__ void __launch_bounds__(kRefThreads, 1)
     mbar_init(&bars.m1, 1);
     mbar_init(&bars.g, 4);
     mbar_init(&bars.m2, 1);
+    mbar_init(&bars.wq, 1);
+    mbar_init(&bars.xq, 4);
+    mbar_init(&bars.m3, 1);
     mbar_init(&bars.drain, 1);
     bars.abort_flag = 0;
     fence_mbar_init();
@@ -172,12 +191,28 @@ __global__ void __launch_bounds__(kRefThreads, 1)
   uint8_t* sW2 = smem + L::w2;
   uint8_t* sGh = smem + L::g_hi;
   uint8_t* sGl = smem + L::g_lo;
+  uint8_t* sWq = sW1;  // W_Q into region B once G has been read
   constexpr uint32_t i1 = idesc_bf16_f32(128, F, false, true);
   constexpr uint32_t i2 = idesc_bf16_f32(128, D, false, true);
   const int tiles_per_bh = (p.k + 127) / 128;
   const int ntiles = p.B * p.H * tiles_per_bh;
   int it = 0;
-  bool w1g_pending = false, w2_pending = false;  // thread 0: weight loads not yet waited for
+  bool w1g_pending = false, w2_pending = false, wq_pending = false;  // thread 0: loads not yet waited for
+  const bool project_only = p.mode == 1;
+  // the rows to project, as a bf16 hi + lo pair in region A, then the arrival on xq
+  auto stage_x = [&](const float* x) {
+#pragma unroll
+    for (int c = 0; c < D; c += 8) store_pair8(sXh, sXl, r, c, x + c);
+    fence_async_shared();
+    __syncwarp();
+    if ((r & 31) == 0) mbar_arrive(&bars.xq);
+  };
+  // thread 0: W_Q of head h into region B
+  auto load_wq = [&](int h) {
+    mbar_expect_tx(&bars.wq, L::wq_bytes);
+    for (int nb = 0; nb < D / 64; ++nb) tma_load_2d(sWq + nb * D * 128, &mapWq, &bars.wq, nb * 64, h * D);
+    wq_pending = true;
+  };
   // tiles in (h, b, row tile) order
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int h = tile / (p.B * tiles_per_bh);
@@ -186,8 +221,28 @@ __global__ void __launch_bounds__(kRefThreads, 1)
     const int j = (rem - b * tiles_per_bh) * 128 + r;
     const bool valid = j < p.k;
     const int64_t row = (static_cast<int64_t>(b) * p.H + h) * p.k + j;
+    const int64_t xrow = p.x_tilde_shared ? static_cast<int64_t>(h) * p.k + j : row;
     const uint32_t par = it & 1;
     bool ok = true;
+    float xb[D];
+    if (project_only) {
+      if (ctl) load_wq(h);
+      if (valid) {
+        const float4* a = reinterpret_cast<const float4*>(p.x_tilde + xrow * D);
+#pragma unroll
+        for (int u = 0; u < D / 4; ++u) {
+          const float4 va = a[u];
+          xb[4 * u] = va.x;
+          xb[4 * u + 1] = va.y;
+          xb[4 * u + 2] = va.z;
+          xb[4 * u + 3] = va.w;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < D; ++u) xb[u] = 0.f;
+      }
+      stage_x(xb);
+    } else {
     if (ctl) {  // W_1, W_g of head h into region B (the previous tile's MMAs have all completed)
       mbar_expect_tx(&bars.w1g, 2 * L::w_bytes);
       for (int nb = 0; nb < F / 64; ++nb) {
@@ -197,9 +252,8 @@ __global__ void __launch_bounds__(kRefThreads, 1)
       w1g_pending = true;
     }
     // 1. X- = LN1(x_tilde + x_hat)
-    float xb[D];
     if (valid) {
-      const float4* a = reinterpret_cast<const float4*>(p.x_tilde + row * D);
+      const float4* a = reinterpret_cast<const float4*>(p.x_tilde + xrow * D);
       const float4* c = reinterpret_cast<const float4*>(p.x_hat + row * D);
 #pragma unroll
       for (int u = 0; u < D / 4; ++u) {
@@ -211,6 +265,9 @@ __global__ void __launch_bounds__(kRefThreads, 1)
       }
       layer_norm_row<D>(xb, p.gamma1 ? p.gamma1 + h * D : nullptr, p.beta1 ? p.beta1 + h * D : nullptr, p.eps);
       if (p.x_bar) store_row_f32<D>(p.x_bar + row * D, xb);
+      // X- in fp32 waits in this thread's own output row for the residual of step 5, so that it
+      // does not occupy registers across the products
+      store_row_f32<D>(p.x_next + row * D, xb);
     } else {
 #pragma unroll
       for (int u = 0; u < D; ++u) xb[u] = 0.f;
@@ -249,19 +306,18 @@ __global__ void __launch_bounds__(kRefThreads, 1)
     }
     // 3. G = swish(H1) * Hg into region B (W_1 / W_g are no longer read)
 #pragma unroll 1
-    for (int c = 0; c < F; c += 16) {
-      uint32_t v1[16], vg[16];
-      tmem_ld16(tb + lane_off + c, v1);
-      tmem_ld16(tb + lane_off + F + c, vg);
+    for (int c = 0; c < F; c += 8) {
+      uint32_t v1[8], vg[8];
+      tmem_ld8(tb + lane_off + c, v1);
+      tmem_ld8(tb + lane_off + F + c, vg);
       tmem_ld_wait();
-      float gv[16];
+      float gv[8];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const float a = __uint_as_float(v1[u]);
         gv[u] = valid ? a / (1.f + __expf(-a)) * __uint_as_float(vg[u]) : 0.f;
       }
       store_pair8(sGh, sGl, r, c, gv);
-      store_pair8(sGh, sGl, r, c + 8, gv + 8);
     }
     fence_async_shared();
     tc_fence_before();
@@ -286,26 +342,77 @@ __global__ void __launch_bounds__(kRefThreads, 1)
     }
     if (!__syncthreads_and(ok && wait(&bars.m2, par))) break;
     tc_fence_after();
+    if (ctl && p.q_next) load_wq(h);  // region B is free: MMA2 has read G
     // 5. X~' = LN2(X- + Y)
+    if (valid) {
+      const float4* a = reinterpret_cast<const float4*>(p.x_next + row * D);
 #pragma unroll
-    for (int c = 0; c < D; c += 32) {
-      uint32_t yv[32];
-      tmem_ld32(tb + lane_off + c, yv);
+      for (int u = 0; u < D / 4; ++u) {
+        const float4 va = a[u];
+        xb[4 * u] = va.x;
+        xb[4 * u + 1] = va.y;
+        xb[4 * u + 2] = va.z;
+        xb[4 * u + 3] = va.w;
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < D; ++u) xb[u] = 0.f;
+    }
+#pragma unroll
+    for (int c = 0; c < D; c += 16) {
+      uint32_t yv[16];
+      tmem_ld16(tb + lane_off + c, yv);
       tmem_ld_wait();
 #pragma unroll
-      for (int u = 0; u < 32; ++u) xb[c + u] += __uint_as_float(yv[u]);
+      for (int u = 0; u < 16; ++u) xb[c + u] += __uint_as_float(yv[u]);
     }
     tc_fence_before();
     if (valid) {
       layer_norm_row<D>(xb, p.gamma2 ? p.gamma2 + h * D : nullptr, p.beta2 ? p.beta2 + h * D : nullptr, p.eps);
       store_row_f32<D>(p.x_next + row * D, xb);
-      if (p.x_next_bf16) {
-        uint4* ob = reinterpret_cast<uint4*>(p.x_next_bf16 + row * D * 2);
+      if (p.x_next_bf16) store_row_bf16<D>(p.x_next_bf16 + row * D * 2, xb);
+    } else {
 #pragma unroll
-        for (int u = 0; u < D / 8; ++u)
-          ob[u] = make_uint4(pack_bf16x2(xb[8 * u], xb[8 * u + 1]), pack_bf16x2(xb[8 * u + 2], xb[8 * u + 3]),
-                             pack_bf16x2(xb[8 * u + 4], xb[8 * u + 5]), pack_bf16x2(xb[8 * u + 6], xb[8 * u + 7]));
+      for (int u = 0; u < D; ++u) xb[u] = 0.f;
+    }
+    if (p.q_next) stage_x(xb);  // region A: W_2 there has been read by MMA2
+    }  // full refinement
+    if (p.q_next) {
+      // 6. the next layer's queries: X~' W_Q from the hi + lo pair staged in region A
+      if (ctl) {
+        ok = wait(&bars.xq, par) && wait(&bars.wq, par);
+        if (ok) {
+          wq_pending = false;
+          tc_fence_after();
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t xa = smem_u32(half ? sXl : sXh);
+#pragma unroll
+            for (int s = 0; s < D / 16; ++s)
+              umma_bf16(tb, sw128_desc(xa + (s / 4) * kRefBlk + (s % 4) * 32, 16, 1024),
+                        sw128_desc(smem_u32(sWq) + s * 2048, D * 128, 1024), i2, (half | s) > 0);
+          }
+          umma_commit(&bars.m3);
+        }
       }
+      if (!__syncthreads_and(ok && wait(&bars.m3, par))) break;
+      tc_fence_after();
+      uint4* qo = reinterpret_cast<uint4*>(p.q_next + row * D * 2);
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t qv[32];
+        tmem_ld32(tb + lane_off + c, qv);
+        tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int u = 0; u < 32; u += 8)
+            qo[(c + u) / 8] = make_uint4(pack_bf16x2(__uint_as_float(qv[u]), __uint_as_float(qv[u + 1])),
+                                         pack_bf16x2(__uint_as_float(qv[u + 2]), __uint_as_float(qv[u + 3])),
+                                         pack_bf16x2(__uint_as_float(qv[u + 4]), __uint_as_float(qv[u + 5])),
+                                         pack_bf16x2(__uint_as_float(qv[u + 6]), __uint_as_float(qv[u + 7])));
+        }
+      }
+      tc_fence_before();
     }
     __syncthreads();  // every thread is done with this tile's TMEM and shared memory
   }
@@ -315,6 +422,7 @@ __global__ void __launch_bounds__(kRefThreads, 1)
     wait(&bars.drain, 0, true);
     if (w1g_pending) wait(&bars.w1g, it & 1, true);
     if (w2_pending) wait(&bars.w2, it & 1, true);
+    if (wq_pending) wait(&bars.wq, it & 1, true);
   }
   tc_fence_before();
   __syncthreads();
@@ -327,24 +435,25 @@ __global__ void __launch_bounds__(kRefThreads, 1)
 // After a device-side error, every output element becomes NaN (the rows the stopped CTAs did not
 // reach would otherwise hold stale values).
 __global__ void refine_poison_kernel(const int* status, float* x_next, float* x_bar, uint16_t* x_next_bf16,
-                                     int64_t n) {
+                                     uint16_t* q_next, int64_t n) {
   if (*reinterpret_cast<const volatile int*>(status) == 0) return;
   const float nan = __int_as_float(0x7fc00000);
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
-    x_next[i] = nan;
+    if (x_next) x_next[i] = nan;
     if (x_bar) x_bar[i] = nan;
     if (x_next_bf16) x_next_bf16[i] = 0x7fc0;
+    if (q_next) q_next[i] = 0x7fc0;
   }
 }
 
 template <int D, int F>
 cudaError_t refine_launch_t(int num_ctas, const CUtensorMap& m1, const CUtensorMap& mg, const CUtensorMap& m2,
-                            const RefineParams& p, cudaStream_t stream) {
+                            const CUtensorMap& mq, const RefineParams& p, cudaStream_t stream) {
   auto kern = sa_refine_kernel<D, F>;
   const size_t smem = RefLayout<D, F>::total;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<num_ctas, kRefThreads, smem, stream>>>(m1, mg, m2, p);
+  kern<<<num_ctas, kRefThreads, smem, stream>>>(m1, mg, m2, mq, p);
   return cudaGetLastError();
 }
 
@@ -353,14 +462,16 @@ cudaError_t refine_launch_t(int num_ctas, const CUtensorMap& m1, const CUtensorM
 bool sa_refine_supported(int D, int F) { return (D == 64 && F == 128) || (D == 128 && F == 256); }
 
 cudaError_t launch_sa_refine(int D, int F, int num_ctas, const CUtensorMap& m1, const CUtensorMap& mg,
-                             const CUtensorMap& m2, const RefineParams& p, cudaStream_t stream) {
+                             const CUtensorMap& m2, const CUtensorMap& mq, const RefineParams& p,
+                             cudaStream_t stream) {
   cudaError_t e = cudaErrorInvalidValue;
-  if (D == 64 && F == 128) e = refine_launch_t<64, 128>(num_ctas, m1, mg, m2, p, stream);
-  if (D == 128 && F == 256) e = refine_launch_t<128, 256>(num_ctas, m1, mg, m2, p, stream);
+  if (D == 64 && F == 128) e = refine_launch_t<64, 128>(num_ctas, m1, mg, m2, mq, p, stream);
+  if (D == 128 && F == 256) e = refine_launch_t<128, 256>(num_ctas, m1, mg, m2, mq, p, stream);
   if (e != cudaSuccess) return e;
   const int64_t n = int64_t(p.B) * p.H * p.k * D;
   refine_poison_kernel<<<2 * 148, 256, 0, stream>>>(p.status, p.x_next, p.x_bar,
-                                                    reinterpret_cast<uint16_t*>(p.x_next_bf16), n);
+                                                    reinterpret_cast<uint16_t*>(p.x_next_bf16),
+                                                    reinterpret_cast<uint16_t*>(p.q_next), n);
   return cudaGetLastError();
 }
 

@@ -724,27 +724,30 @@ size_t sa_refine_workspace_size(const ska_refine_desc* d) {
 
 ska_status sa_refine(const ska_refine_desc* d, const float* x_tilde, const float* x_hat, const void* w1,
                      const void* wg, const void* w2, const float* gamma1, const float* beta1, const float* gamma2,
-                     const float* beta2, float* x_next, float* x_bar, void* x_next_bf16, void* ws, size_t ws_bytes,
-                     void* stream) {
+                     const float* beta2, const void* w_q_next, float* x_next, float* x_bar, void* x_next_bf16,
+                     void* q_next, void* ws, size_t ws_bytes, void* stream) {
   ska_status st = check_refine_desc(d);
   if (st != SKA_OK) return st;
   const int B = d->num_users, H = d->num_heads, k = d->num_protos, D = d->head_dim, F = d->ffn_dim;
   if (B == 0) return SKA_OK;
   if (!x_tilde || !x_hat || !w1 || !wg || !w2 || !x_next || !ws) return SKA_ERR_INVALID_VALUE;
-  const void* al[12] = {x_tilde, x_hat, w1, wg, w2, gamma1, beta1, gamma2, beta2, x_next, x_bar, x_next_bf16};
-  for (int i = 0; i < 12; ++i)
+  if ((w_q_next == nullptr) != (q_next == nullptr)) return SKA_ERR_INVALID_VALUE;
+  const void* al[14] = {x_tilde, x_hat, w1, wg, w2, gamma1, beta1, gamma2, beta2, w_q_next, x_next, x_bar,
+                        x_next_bf16, q_next};
+  for (int i = 0; i < 14; ++i)
     if (!aligned16(al[i])) return SKA_ERR_INVALID_VALUE;
   if (reinterpret_cast<uintptr_t>(ws) & 255u) return SKA_ERR_INVALID_VALUE;
   if (ws_bytes < sizeof(WsHeader)) return SKA_ERR_WORKSPACE_TOO_SMALL;
   const size_t xb = size_t(B) * H * k * D * 4, wb = size_t(H) * D * F * 2, vb = size_t(H) * D * 4;
-  const void* ins[9] = {x_tilde, x_hat, w1, wg, w2, gamma1, beta1, gamma2, beta2};
-  const size_t insz[9] = {xb, xb, wb, wb, wb, vb, vb, vb, vb};
-  const void* outs[4] = {x_next, x_bar, x_next_bf16, ws};
-  const size_t outsz[4] = {xb, xb, xb / 2, sizeof(WsHeader)};
-  for (int o = 0; o < 4; ++o) {
-    for (int i = 0; i < 9; ++i)
+  const size_t xtb = d->x_tilde_shared ? size_t(H) * k * D * 4 : xb;
+  const void* ins[10] = {x_tilde, x_hat, w1, wg, w2, gamma1, beta1, gamma2, beta2, w_q_next};
+  const size_t insz[10] = {xtb, xb, wb, wb, wb, vb, vb, vb, vb, size_t(H) * D * D * 2};
+  const void* outs[5] = {x_next, x_bar, x_next_bf16, q_next, ws};
+  const size_t outsz[5] = {xb, xb, xb / 2, xb / 2, sizeof(WsHeader)};
+  for (int o = 0; o < 5; ++o) {
+    for (int i = 0; i < 10; ++i)
       if (overlaps(outs[o], outsz[o], ins[i], insz[i])) return SKA_ERR_INVALID_VALUE;
-    for (int o2 = o + 1; o2 < 4; ++o2)
+    for (int o2 = o + 1; o2 < 5; ++o2)
       if (overlaps(outs[o], outsz[o], outs[o2], outsz[o2])) return SKA_ERR_INVALID_VALUE;
   }
   if (no_device()) return SKA_ERR_CUDA;
@@ -754,11 +757,17 @@ ska_status sa_refine(const ska_refine_desc* d, const float* x_tilde, const float
     record_error("cudaMemsetAsync(status)", e);
     return SKA_ERR_CUDA;
   }
-  // W_1, W_g: [H d rows, F] in boxes of 64 columns x d rows; W_2: [H F rows, d] in 64 x F boxes
-  CUtensorMap m1, mg, m2;
+  // W_1, W_g: [H d rows, F] in boxes of 64 columns x d rows; W_2: [H F rows, d] in 64 x F boxes;
+  // W_Q: [H d rows, d] in 64 x d boxes
+  CUtensorMap m1, mg, m2, mq;
   if (!encode_2d(&m1, w1, F, uint64_t(H) * D, F, 64, D)) return SKA_ERR_CUDA;
   if (!encode_2d(&mg, wg, F, uint64_t(H) * D, F, 64, D)) return SKA_ERR_CUDA;
   if (!encode_2d(&m2, w2, D, uint64_t(H) * F, D, 64, F)) return SKA_ERR_CUDA;
+  if (w_q_next) {
+    if (!encode_2d(&mq, w_q_next, D, uint64_t(H) * D, D, 64, D)) return SKA_ERR_CUDA;
+  } else {
+    mq = m1;  // never read
+  }
   RefineParams p{};
   p.x_tilde = x_tilde;
   p.x_hat = x_hat;
@@ -769,10 +778,13 @@ ska_status sa_refine(const ska_refine_desc* d, const float* x_tilde, const float
   p.x_bar = x_bar;
   p.x_next = x_next;
   p.x_next_bf16 = static_cast<uint8_t*>(x_next_bf16);
+  p.q_next = static_cast<uint8_t*>(q_next);
   p.status = &hdr->status;
   p.B = B;
   p.H = H;
   p.k = k;
+  p.x_tilde_shared = d->x_tilde_shared ? 1 : 0;
+  p.mode = 0;
   p.eps = d->eps;
   p.budget_ns = wait_budget();
   p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
@@ -781,10 +793,56 @@ ska_status sa_refine(const ska_refine_desc* d, const float* x_tilde, const float
   cudaError_t e;
   {
     TimedRegion tr(s);
-    e = launch_sa_refine(D, F, ctas, m1, mg, m2, p, s);
+    e = launch_sa_refine(D, F, ctas, m1, mg, m2, mq, p, s);
   }
   if (e != cudaSuccess) {
     record_error("refinement kernel launch", e);
+    return SKA_ERR_CUDA;
+  }
+  return SKA_OK;
+}
+
+ska_status sa_project_queries(int32_t num_users, int32_t num_heads, int32_t num_rows, int32_t head_dim,
+                              const float* x, const void* w_q, void* q_out, void* ws, size_t ws_bytes,
+                              void* stream) {
+  if (num_users < 0 || num_heads < 1 || num_rows < 1) return SKA_ERR_INVALID_VALUE;
+  if (!sa_refine_supported(head_dim, 2 * head_dim)) return SKA_ERR_UNSUPPORTED;
+  const int B = num_users, H = num_heads, k = num_rows, D = head_dim;
+  if (int64_t(B) * H * k * D >= (int64_t(1) << 31)) return SKA_ERR_INVALID_VALUE;
+  if (B == 0) return SKA_OK;
+  if (!x || !w_q || !q_out || !ws) return SKA_ERR_INVALID_VALUE;
+  if (!aligned16(x) || !aligned16(w_q) || !aligned16(q_out) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return SKA_ERR_INVALID_VALUE;
+  if (ws_bytes < sizeof(WsHeader)) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  const size_t xb = size_t(B) * H * k * D * 4, qb = xb / 2, wqb = size_t(H) * D * D * 2;
+  if (overlaps(q_out, qb, x, xb) || overlaps(q_out, qb, w_q, wqb) || overlaps(ws, sizeof(WsHeader), x, xb) ||
+      overlaps(ws, sizeof(WsHeader), w_q, wqb) || overlaps(ws, sizeof(WsHeader), q_out, qb))
+    return SKA_ERR_INVALID_VALUE;
+  if (no_device()) return SKA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  if (cudaError_t e = cudaMemsetAsync(&hdr->status, 0, sizeof(int32_t), s); e != cudaSuccess) {
+    record_error("cudaMemsetAsync(status)", e);
+    return SKA_ERR_CUDA;
+  }
+  CUtensorMap mq;
+  if (!encode_2d(&mq, w_q, D, uint64_t(H) * D, D, 64, D)) return SKA_ERR_CUDA;
+  RefineParams p{};
+  p.x_tilde = x;
+  p.q_next = static_cast<uint8_t*>(q_out);
+  p.status = &hdr->status;
+  p.B = B;
+  p.H = H;
+  p.k = k;
+  p.mode = 1;
+  p.eps = 1.f;
+  p.budget_ns = wait_budget();
+  p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
+  const int64_t tiles = int64_t(B) * H * ((k + 127) / 128);
+  const int ctas = static_cast<int>(std::min<int64_t>(tiles, device_sm_count()));
+  cudaError_t e = launch_sa_refine(D, 2 * D, ctas, mq, mq, mq, mq, p, s);
+  if (e != cudaSuccess) {
+    record_error("projection kernel launch", e);
     return SKA_ERR_CUDA;
   }
   return SKA_OK;

@@ -136,10 +136,13 @@ struct RefineParams {
   const float* gamma2;
   const float* beta2;
   float* x_bar;          // nullable: Eq. (13)'s output
-  float* x_next;
+  float* x_next;         // null in projection mode
   uint8_t* x_next_bf16;  // nullable: bf16 copy of x_next
+  uint8_t* q_next;       // nullable: bf16 [B, H, k, D] = x_next W_Q (projection mode: x_tilde W_Q)
   int* status;           // the workspace status word
   int B, H, k;
+  int x_tilde_shared;    // 1: x_tilde is [H, k, D], the same rows for every user
+  int mode;              // 0: refinement (+ optional projection); 1: projection of x_tilde only
   float eps;
   uint64_t budget_ns;
   uint32_t debug_flags;  // bit 1 (value 2): never signal MMA1's completion (test hook)
@@ -147,10 +150,10 @@ struct RefineParams {
 
 bool sa_refine_supported(int head_dim, int ffn_dim);
 // The fused refinement kernel on num_ctas persistent CTAs, then a kernel that turns the outputs
-// to NaN when the status word holds an error.
+// to NaN when the status word holds an error. mapWq is read only when p.q_next is set.
 cudaError_t launch_sa_refine(int head_dim, int ffn_dim, int num_ctas, const CUtensorMap& mapW1,
-                             const CUtensorMap& mapWg, const CUtensorMap& mapW2, const RefineParams& p,
-                             cudaStream_t stream);
+                             const CUtensorMap& mapWg, const CUtensorMap& mapW2, const CUtensorMap& mapWq,
+                             const RefineParams& p, cudaStream_t stream);
 
 // Small kernels (ska_small.cu).
 cudaError_t launch_schedule(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,

@@ -279,3 +279,43 @@ def make_refine(B: int, H: int, k: int, d: int, seed: int, *, affine: bool = Tru
 def config_refine() -> RefineInputs:
     """The refinement layer on the sketch of the 8 x 100K, H=8, d=128, k=512 workload; seed 6."""
     return make_refine(8, 8, 512, 128, 6)
+
+
+@dataclasses.dataclass
+class StackInputs:
+    """N_sa stacked SA layers (SequenceO1 §3.3): prototypes, per-layer query weights and keys, the
+    history X as values, and per-layer refinement parameters."""
+    p0: torch.Tensor            # fp32 [H, k, d], P^(0)
+    w_q: list                   # N_sa bf16 [H, d, d]
+    keys: list                  # N_sa bf16 [T, H, d], K^(l) = X W_K^(l)
+    v: torch.Tensor             # bf16 [T, H, d], X
+    cu_seqlens: torch.Tensor    # int32 [B + 1]
+    ffn: list                   # N_sa RefineInputs with only the weights and LN vectors set
+    scale: float
+
+
+def make_stack(lengths, num_heads: int, head_dim: int, num_protos: int, n_layers: int, seed: int) -> StackInputs:
+    """Draw order: P^(0) (N(0, 1) fp32); the values X (N(0, 1), bf16); then per layer W_Q
+    (N(0, 1/d), bf16), the keys (N(0, 1), bf16), W_1, W_g (N(0, 1/d)), W_2 (N(0, 1/F)) in bf16 and
+    gamma1, beta1, gamma2, beta2 (1 + 0.1 N, 0.1 N, 1 + 0.1 N, 0.1 N; fp32). Scale 1/sqrt(d)."""
+    rng = np.random.default_rng(seed)
+    H, d, k = num_heads, head_dim, num_protos
+    F = 2 * d
+    T = int(sum(lengths))
+    p0 = torch.from_numpy(normal(rng, (H, k, d)))
+    v = to_bf16(normal(rng, (T, H, d)))
+    w_q, keys, ffn = [], [], []
+    for _ in range(n_layers):
+        w_q.append(to_bf16(normal(rng, (H, d, d), 1.0 / math.sqrt(d))))
+        keys.append(to_bf16(normal(rng, (T, H, d))))
+        w1 = normal(rng, (H, d, F), 1.0 / math.sqrt(d))
+        wg = normal(rng, (H, d, F), 1.0 / math.sqrt(d))
+        w2 = normal(rng, (H, F, d), 1.0 / math.sqrt(F))
+        r = RefineInputs(None, None, to_bf16(w1), to_bf16(wg), to_bf16(w2))
+        r.gamma1 = torch.from_numpy(1.0 + normal(rng, (H, d), 0.1))
+        r.beta1 = torch.from_numpy(normal(rng, (H, d), 0.1))
+        r.gamma2 = torch.from_numpy(1.0 + normal(rng, (H, d), 0.1))
+        r.beta2 = torch.from_numpy(normal(rng, (H, d), 0.1))
+        ffn.append(r)
+    return StackInputs(p0, w_q, keys, v, cu_from_lengths(lengths), ffn, 1.0 / math.sqrt(d))
+

@@ -183,19 +183,21 @@ def test_debug_and_timing_hooks_are_host_only():
 
 
 def refine_desc(**kw):
-    f = dict(num_users=2, num_heads=2, num_protos=300, head_dim=128, ffn_dim=256, eps=1e-5)
+    f = dict(num_users=2, num_heads=2, num_protos=300, head_dim=128, ffn_dim=256, eps=1e-5, x_tilde_shared=0,
+             reserved=0)
     f.update(kw)
     return L.RefineDesc(**f)
 
 
+REFINE_ARGS = ["xt", "xh", "w1", "wg", "w2", "g1", "b1", "g2", "b2", "wq", "out", "bar", "bf", "q", "ws"]
+
+
 def refine(d, **kw):
-    # x_tilde, x_hat, w1, wg, w2, gamma1, beta1, gamma2, beta2, x_next, x_bar, x_next_bf16, ws
-    names = ["xt", "xh", "w1", "wg", "w2", "g1", "b1", "g2", "b2", "out", "bar", "bf", "ws"]
-    ptrs = {n: (i + 20) * A for i, n in enumerate(names)}
+    ptrs = {n: (i + 20) * A for i, n in enumerate(REFINE_ARGS)}
+    ws_bytes = kw.pop("ws_bytes", 256)
     ptrs.update(kw)
-    ws_bytes = kw.pop("ws_bytes", 256) if "ws_bytes" in kw else 256
-    args = [ptrs[n] for n in names]
-    return L.lib().sa_refine(ctypes.byref(d) if d is not None else None, *args, ws_bytes, None)
+    return L.lib().sa_refine(ctypes.byref(d) if d is not None else None, *[ptrs[n] for n in REFINE_ARGS],
+                             ws_bytes, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -216,14 +218,39 @@ def test_refine_pointer_checks():
     assert refine(None) == INVALID
     for n in ("xt", "xh", "w1", "wg", "w2", "out", "ws"):
         assert refine(d, **{n: None}) == INVALID, n
+    assert refine(d, wq=None) == INVALID                 # W_Q and q_next come together
+    assert refine(d, q=None) == INVALID
     assert refine(d, g1=40 * A + 4) == INVALID           # 16-byte alignment
     assert refine(d, ws=41 * A + 16) == INVALID          # 256-byte workspace alignment
     assert refine(d, ws_bytes=255) == L.SKA_ERR_WORKSPACE_TOO_SMALL
     assert refine(d, out=20 * A + 64) == INVALID         # the output overlaps x_tilde
-    assert refine(d, bar=29 * A + 1024) == INVALID       # x_bar overlaps x_next
+    assert refine(d, bar=30 * A + 1024) == INVALID       # x_bar overlaps x_next
+    assert refine(d, q=31 * A + 512) == INVALID          # q_next overlaps x_bar
     assert refine(d, ws=22 * A) == INVALID               # the workspace overlaps W_1
     # B = 0: nothing to do, no pointer is looked at
     assert refine(refine_desc(num_users=0), xt=None, xh=None, out=None, ws=None) == L.SKA_OK
+
+
+def project(B=2, H=2, k=300, d=128, **kw):
+    names = ["x", "wq", "q", "ws"]
+    ptrs = {n: (i + 50) * A for i, n in enumerate(names)}
+    ws_bytes = kw.pop("ws_bytes", 256)
+    ptrs.update(kw)
+    return L.lib().sa_project_queries(B, H, k, d, *[ptrs[n] for n in names], ws_bytes, None)
+
+
+def test_project_queries_host_checks():
+    assert project(H=0) == INVALID
+    assert project(k=0) == INVALID
+    assert project(B=-1) == INVALID
+    assert project(d=96) == UNSUP
+    assert project(B=1 << 12, H=64, k=64) == INVALID
+    assert project(B=0, x=None, wq=None, q=None, ws=None) == L.SKA_OK
+    for n in ("x", "wq", "q", "ws"):
+        assert project(**{n: None}) == INVALID, n
+    assert project(q=50 * A + 16) == INVALID             # q overlaps x
+    assert project(x=50 * A + 8) == INVALID              # alignment
+    assert project(ws_bytes=100) == L.SKA_ERR_WORKSPACE_TOO_SMALL
 
 
 def test_refine_without_a_device_reports_cuda_error():
@@ -231,6 +258,8 @@ def test_refine_without_a_device_reports_cuda_error():
     if torch.cuda.is_available():
         pytest.skip("a device is present")
     d = refine_desc()
-    # optional outputs and LayerNorm vectors may be NULL
-    assert refine(d, g1=None, b1=None, g2=None, b2=None, bar=None, bf=None) == L.SKA_ERR_CUDA
+    # optional outputs, W_Q and LayerNorm vectors may be NULL
+    assert refine(d, g1=None, b1=None, g2=None, b2=None, bar=None, bf=None, wq=None, q=None) == L.SKA_ERR_CUDA
     assert refine(refine_desc(head_dim=64, ffn_dim=128)) == L.SKA_ERR_CUDA
+    assert refine(refine_desc(x_tilde_shared=1)) == L.SKA_ERR_CUDA
+    assert project() == L.SKA_ERR_CUDA

@@ -34,9 +34,9 @@ def run_gpu(inp: W.RefineInputs, status=False):
     api = _api()
     dev = "cuda"
     g = lambda t: None if t is None else t.to(dev)
-    desc = api.refine_desc(inp.x_tilde, inp.w1)
+    desc = api.refine_desc(inp.x_tilde, inp.x_hat, inp.w1)
     ws = torch.empty(api.sa_refine_workspace_size(desc), dtype=torch.uint8, device=dev)
-    x_next, x_bar, x_bf = api.sa_refine(g(inp.x_tilde), g(inp.x_hat), g(inp.w1), g(inp.wg), g(inp.w2),
+    x_next, x_bar, x_bf, _ = api.sa_refine(g(inp.x_tilde), g(inp.x_hat), g(inp.w1), g(inp.wg), g(inp.w2),
                                         g(inp.gamma1), g(inp.beta1), g(inp.gamma2), g(inp.beta2),
                                         want_x_bar=True, want_bf16=True, workspace=ws)
     torch.cuda.synchronize()
@@ -132,3 +132,102 @@ def test_refine_timeout_reports_and_poisons():
     assert st == 5
     assert torch.isnan(x_next).all() and torch.isnan(x_bar).all() and torch.isnan(x_bf.float()).all()
     check(inp)
+
+
+# ------------------------------------------------------------------ queries of the next layer
+
+def assert_bf16_rounding_of(got, want, what, atol):
+    """got (bf16) is want (fp64) rounded to bf16: within one half-ulp of bf16, 2^-8 |want|, plus
+    atol for the error of the fp32 rows and products before the rounding."""
+    g = got.float().numpy().astype(np.float64)
+    err = np.abs(g - want)
+    bound = 2.0 ** -8 * np.abs(want) + atol
+    worst = float((err / bound).max())
+    print(f"[parity] {what}: worst error / half-ulp bound {worst:.3f}")
+    assert worst <= 1.0, what
+
+
+@pytest.mark.parametrize("B,H,k,d", [(1, 2, 256, 128), (3, 4, 200, 64), (2, 8, 512, 128)])
+def test_project_queries_parity(B, H, k, d):
+    api = _api()
+    r = W.make_refine(B, H, k, d, seed=900 + k)          # x_tilde as the rows, w1[:, :, :d] as W_Q
+    w_q = r.w1[:, :, :d].contiguous()
+    q = api.project_queries(r.x_tilde.cuda(), w_q.cuda())
+    torch.cuda.synchronize()
+    # the same fp32 rows on both sides: products off by 2^-17 relative, summed over d terms
+    assert_bf16_rounding_of(q.cpu(), oracle.project_queries(f64(r.x_tilde), f64(w_q)), "x W_Q", 1e-5)
+    # shared prototypes [H, k, d]
+    q0 = api.project_queries(r.x_tilde[0].cuda(), w_q.cuda())
+    torch.cuda.synchronize()
+    assert tuple(q0.shape) == (H, k, d)
+    assert torch.equal(q0.cpu(), q.cpu()[0])
+
+
+@pytest.mark.parametrize("B,H,k,d", [(2, 2, 200, 128), (3, 2, 130, 64)])
+def test_refine_with_next_queries_and_shared_residual(B, H, k, d):
+    api = _api()
+    r = W.make_refine(B, H, k, d, seed=950 + k)
+    w_q = r.wg[:, :, :d].contiguous()
+    g = lambda t: t.cuda()
+    # per-user residual, with the next layer's queries
+    x_next, _, _, q_next = api.sa_refine(g(r.x_tilde), g(r.x_hat), g(r.w1), g(r.wg), g(r.w2), g(r.gamma1),
+                                         g(r.beta1), g(r.gamma2), g(r.beta2), w_q_next=g(w_q))
+    torch.cuda.synchronize()
+    _, o_next = run_oracle(r)
+    assert_close(x_next.cpu(), o_next, "x_next (with W_Q)")
+    # the rows are the kernel's x_next (within 2e-5 of the oracle's), projected: atol 1e-4
+    assert_bf16_rounding_of(q_next.cpu(), oracle.project_queries(o_next, f64(w_q)), "x_next W_Q", 1e-4)
+    # one residual [H, k, d] for every user (layer 0: the prototypes)
+    shared = r.x_tilde[0]
+    x_s, _, _, _ = api.sa_refine(g(shared), g(r.x_hat), g(r.w1), g(r.wg), g(r.w2), g(r.gamma1), g(r.beta1),
+                                 g(r.gamma2), g(r.beta2))
+    torch.cuda.synchronize()
+    _, o_s = oracle.refine(np.broadcast_to(f64(shared), (B, H, k, d)), f64(r.x_hat), f64(r.w1), f64(r.wg),
+                           f64(r.w2), f64(r.gamma1), f64(r.beta1), f64(r.gamma2), f64(r.beta2))
+    assert_close(x_s.cpu(), o_s, "x_next (shared residual)")
+
+
+# ------------------------------------------------------- two stacked layers, end to end (N_sa = 2)
+
+STACK_MAX_ABS = 1e-2
+STACK_REL_L2 = 5e-3
+
+
+def _stack_close(got, want, what):
+    got = got.cpu().numpy().astype(np.float64)
+    err = np.abs(got - want)
+    rel = float(np.linalg.norm(got - want) / np.linalg.norm(want))
+    print(f"[parity] {what}: max abs {err.max():.3e}, rel L2 {rel:.3e}")
+    assert err.max() <= STACK_MAX_ABS and rel <= STACK_REL_L2, what
+
+
+@pytest.mark.parametrize("lengths,H,d,k", [([700, 129, 1], 2, 128, 256), ([1000, 300], 2, 64, 128),
+                                           ([513, 64], 1, 128, 512)])
+def test_two_layer_stack_end_to_end(lengths, H, d, k):
+    """Layer 0: q = P^(0) W_Q^(0) (sa_project_queries), SA over K^(0), refinement with the shared
+    residual P^(0) that also emits layer 1's per-user queries; layer 1: SA with those queries over
+    K^(1), refinement. Every step runs in the library's kernels; the oracle runs the same stack in
+    fp64 (queries unrounded). Tolerance: that of the SA forward, since the SA steps dominate the
+    error (the bf16 queries add about 2^-9 relative to the scores)."""
+    api = _api()
+    st = W.make_stack(lengths, H, d, k, 2, seed=77 + k)
+    g = lambda t: None if t is None else t.cuda()
+    cu = g(st.cu_seqlens)
+    v = g(st.v)
+    q0 = api.project_queries(g(st.p0), g(st.w_q[0]))
+    sk0, _, _ = api.sa_forward(q0, g(st.keys[0]), v, cu, scale=st.scale, norm="proto")
+    f0 = st.ffn[0]
+    x1, _, _, q1 = api.sa_refine(g(st.p0), sk0, g(f0.w1), g(f0.wg), g(f0.w2), g(f0.gamma1), g(f0.beta1),
+                                 g(f0.gamma2), g(f0.beta2), w_q_next=g(st.w_q[1]))
+    sk1, _, _ = api.sa_forward(q1, g(st.keys[1]), v, cu, scale=st.scale, norm="proto")
+    f1 = st.ffn[1]
+    x2, _, _, _ = api.sa_refine(x1, sk1, g(f1.w1), g(f1.wg), g(f1.w2), g(f1.gamma1), g(f1.beta1), g(f1.gamma2),
+                                g(f1.beta2))
+    torch.cuda.synchronize()
+    ffn = [(f64(f.w1), f64(f.wg), f64(f.w2), f64(f.gamma1), f64(f.beta1), f64(f.gamma2), f64(f.beta2))
+           for f in st.ffn]
+    o_out, o_sk = oracle.stacked_sa(f64(st.p0), [f64(w) for w in st.w_q], [f64(kk) for kk in st.keys], f64(st.v),
+                                    st.cu_seqlens.numpy(), None, st.scale, ffn)
+    _stack_close(sk0, o_sk[0], "layer 0 sketch")
+    _stack_close(sk1, o_sk[1], "layer 1 sketch")
+    _stack_close(x2, o_out, "X~(2)")
