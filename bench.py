@@ -46,6 +46,9 @@ METRICS = {
     "sa_fwd": ("SA fwd history-tokens/s and TFLOP/s (fraction of B200 bf16 peak) at L=100K", "history-tokens/s"),
     "sa_bwd": ("SA bwd history-tokens/s (dQ, dK, dV with A recomputed) and TFLOP/s", "history-tokens/s"),
     "stca": ("STCA targets/s over [10K suffix ; 256 sketch] keys and TFLOP/s", "targets/s"),
+    "refine": ("sketch refinement rows/s (LN, SwiGLU FFN, LN, next-layer query projection) and GB/s",
+               "sketch-rows/s"),
+    "sa_stack": ("stacked SA (N_sa = 2 layers) history-tokens/s at L=100K", "history-tokens/s"),
 }
 
 # name -> kind and shapes. lens: list, "ragged64" (64 users, log-uniform in [1K, 100K], seed 1) or
@@ -66,6 +69,10 @@ WORKLOADS = {
     "sa_bwd_b64_ragged_h4_d64_k256": dict(kind="sa_bwd", lens="ragged64", H=4, d=64, k=256, seqused=None),
     # profiling size for the backward: 2 x 100K, one head, same per-tile work
     "sa_bwd_b2_l100k_h1_d64_k256": dict(kind="sa_bwd", lens=[100_000] * 2, H=1, d=64, k=256, seqused=None),
+    # the refinement layer on the sketch of the 8 x 100K workload (8 users x 8 heads x 512 rows, d = 128)
+    "refine_b8_h8_k512_d128": dict(kind="refine", B=8, H=8, k=512, d=128),
+    # two stacked SA layers (§3.3) over the 8 x 100K workload, own keys per layer, V = the history
+    "sa_stack2_b8_l100k_h8_d128_k512": dict(kind="sa_stack", lens=[100_000] * 8, H=8, d=128, k=512, layers=2),
     "stca_b16_t512_h4_d64_l10k_s256": dict(kind="stca", users=16, targets=512, hist=10_000, ks=256, H=4, d=64,
                                            scale=0.125),
 }
@@ -342,7 +349,137 @@ class StcaJob:
         return done, time.perf_counter() - t0, f"{per_user} targets of each of {users} users (all heads), fp64 numpy"
 
 
-JOBS = {"sa_fwd": SaFwdJob, "sa_bwd": SaBwdJob, "stca": StcaJob}
+class RefineJob:
+    """One refinement layer (residual + LN, SwiGLU FFN, residual + LN, the next layer's queries) on
+    every sketch row. Its inputs (59 MB a set) fit in L2, so the steps rotate over four sets of
+    inputs and outputs (236 MB together): a step's data were last touched three steps earlier."""
+    SETS = 4
+
+    def __init__(self, spec, norm, rank, world, dev):
+        import torch
+        from sketch_attention_flashsa_b200 import api, flops
+        self.api = api
+        B, H, k, d = spec["B"], spec["H"], spec["k"], spec["d"]
+        F = 2 * d
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(4000 + rank)
+        rn = lambda *shape: torch.randn(shape, generator=gen, device=dev)  # noqa: E731
+        self.weights = {"w1": (rn(H, d, F) / math.sqrt(d)).bfloat16(), "wg": (rn(H, d, F) / math.sqrt(d)).bfloat16(),
+                        "w2": (rn(H, F, d) / math.sqrt(F)).bfloat16(), "wq": (rn(H, d, d) / math.sqrt(d)).bfloat16(),
+                        "g1": 1 + rn(H, d) / 10, "b1": rn(H, d) / 10, "g2": 1 + rn(H, d) / 10, "b2": rn(H, d) / 10}
+        self.sets = [{"x_tilde": rn(B, H, k, d), "x_hat": rn(B, H, k, d)} for _ in range(self.SETS)]
+        self.outs = [torch.empty((B, H, k, d), device=dev) for _ in range(self.SETS)]
+        self.inputs = self.sets[0]
+        self.turn = 0
+        self.ws = torch.empty(256, dtype=torch.uint8, device=dev)
+        rows = B * H * k
+        self.units = rows
+        self.flops = flops.refine_flops(rows, d)
+        self.bytes = flops.refine_bytes(rows, H, d)
+        self.kernel = "sa_refine_kernel"
+        self.launches = 2
+        self.config = {"users_per_gpu": B, "heads": H, "rows_per_user_head": k, "head_dim": d, "ffn_dim": F,
+                       "outputs": "x_next fp32, q_next bf16",
+                       "l2": f"rotating over {self.SETS} input/output sets of {rows * d * 14 / 1e6:.0f} MB each"}
+
+    def run(self, x):
+        if x is self.inputs:  # the timed steps rotate over the sets
+            i = self.turn % self.SETS
+            self.turn += 1
+            x, out = self.sets[i], self.outs[i]
+        else:
+            out = self.outs[0]
+        w = self.weights
+        x_next, _, _, q_next = self.api.sa_refine(x["x_tilde"], x["x_hat"], w["w1"], w["wg"], w["w2"], w["g1"],
+                                                  w["b1"], w["g2"], w["b2"], w_q_next=w["wq"], workspace=self.ws,
+                                                  out=out)
+        return x_next
+
+    def oracle_sample(self, budget_s):
+        import oracle
+        x, w = self.inputs, {n: f64(t) for n, t in self.weights.items()}
+        B = x["x_tilde"].shape[0]
+        done, users, t0 = 0.0, 0, time.perf_counter()
+        while time.perf_counter() - t0 < budget_s and users < 64:
+            b = users % B
+            xt, xh = f64(x["x_tilde"][b:b + 1]), f64(x["x_hat"][b:b + 1])
+            _, xn = oracle.refine(xt, xh, w["w1"], w["wg"], w["w2"], w["g1"], w["b1"], w["g2"], w["b2"])
+            oracle.project_queries(xn, w["wq"])
+            done += xt.shape[1] * xt.shape[2]
+            users += 1
+        return done, time.perf_counter() - t0, f"{users} whole users (all heads and rows), fp64 numpy"
+
+
+class StackJob:
+    """N_sa stacked SA layers (§3.3) through the public API: the layer-0 queries P^(0) W_Q, then per
+    layer the prototype-wise SA forward over that layer's keys with V = the history, and the
+    refinement that also emits the next layer's queries. The roofline is taken over the whole step
+    (several kernels), against the bf16 tensor peak."""
+
+    def __init__(self, spec, norm, rank, world, dev):
+        import torch
+        from sketch_attention_flashsa_b200 import api, flops
+        self.api = api
+        lens, _ = rank_users(spec, rank, world)
+        H, d, kp, nl = spec["H"], spec["d"], spec["k"], spec["layers"]
+        T, B = sum(lens), len(lens)
+        F = 2 * d
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(5000 + rank)
+        rn = lambda *shape: torch.randn(shape, generator=gen, device=dev)  # noqa: E731
+        x = {"p0": rn(H, kp, d), "v": rn(T, H, d).bfloat16(),
+             "cu": torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=dev)}
+        for l in range(nl):
+            x[f"k{l}"] = rn(T, H, d).bfloat16()
+            x[f"wq{l}"] = (rn(H, d, d) / math.sqrt(d)).bfloat16()
+            x[f"w1_{l}"] = (rn(H, d, F) / math.sqrt(d)).bfloat16()
+            x[f"wg_{l}"] = (rn(H, d, F) / math.sqrt(d)).bfloat16()
+            x[f"w2_{l}"] = (rn(H, F, d) / math.sqrt(F)).bfloat16()
+        self.inputs, self.nl, self.scale = x, nl, 1.0 / math.sqrt(d)
+        need = 0
+        for qshape in ((H, kp, d), (B, H, kp, d)):  # layer 0 shares its queries, later layers do not
+            q = torch.empty(qshape, dtype=torch.bfloat16, device=dev)
+            need = max(need, api.sa_forward_workspace_size(api.sa_desc(q, x["v"], x["cu"], scale=self.scale,
+                                                                         norm="proto")))
+        self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        rows = B * H * kp
+        self.units = T
+        self.flops = nl * (flops.sa_forward_flops(T, H, kp, d) + flops.refine_flops(rows, d)) + flops.gemm(H * kp, d, d)
+        self.bytes = nl * (flops.sa_forward_bytes(T, H, kp, d, B, norm=0) + flops.refine_bytes(rows, H, d))
+        self.kernel = "step: sa_proto_fwd_kernel x2, sa_refine_kernel x3 (one projection-only) and small kernels"
+        self.launches = 1 + nl * 6
+        self.hook = False
+        self.config = {"users_per_gpu": B, "heads": H, "head_dim": d, "protos": kp, "layers": nl, "norm": "proto",
+                       "valid_tokens_per_gpu": T, "keys": "one key tensor per layer; values = the history",
+                       "l2": "inputs larger than L2 (each K and V is %.2f GB per GPU)" % (T * H * d * 2 / 1e9)}
+
+    def run(self, x):
+        api = self.api
+        q = api.project_queries(x["p0"], x["wq0"])
+        x_t = x["p0"]
+        for l in range(self.nl):
+            sk, _, _ = api.sa_forward(q, x[f"k{l}"], x["v"], x["cu"], None, scale=self.scale, norm="proto",
+                                      want_lse=False, workspace=self.ws)
+            wq = x.get(f"wq{l + 1}")
+            x_t, _, _, q = api.sa_refine(x_t, sk, x[f"w1_{l}"], x[f"wg_{l}"], x[f"w2_{l}"], w_q_next=wq)
+        return x_t
+
+    def oracle_sample(self, budget_s):
+        import oracle
+        x = self.inputs
+        cu = x["cu"].cpu().numpy()
+        t0 = time.perf_counter()
+        n = min(2000, int(cu[1]))  # the first 2000 tokens of user 0, all heads, both layers
+        sub = lambda t: f64(t[:n])  # noqa: E731
+        ffn = [(f64(x[f"w1_{l}"]), f64(x[f"wg_{l}"]), f64(x[f"w2_{l}"]), None, None, None, None)
+               for l in range(self.nl)]
+        oracle.stacked_sa(f64(x["p0"]), [f64(x[f"wq{l}"]) for l in range(self.nl)],
+                          [sub(x[f"k{l}"]) for l in range(self.nl)], sub(x["v"]), np.array([0, n]), None,
+                          self.scale, ffn)
+        return n, time.perf_counter() - t0, f"the first {n} tokens of one user through {self.nl} layers, fp64 numpy"
+
+
+JOBS = {"sa_fwd": SaFwdJob, "sa_bwd": SaBwdJob, "stca": StcaJob, "refine": RefineJob, "sa_stack": StackJob}
 
 
 def traffic_for(workload, norm):
@@ -394,6 +531,29 @@ def _host_job(spec, norm):
     import torch
     g = torch.Generator().manual_seed(7)
     job = types.SimpleNamespace()
+    rn = lambda *shape: torch.randn(shape, generator=g)  # noqa: E731
+    if spec["kind"] == "refine":
+        H, k, d = spec["H"], spec["k"], spec["d"]
+        F = 2 * d
+        job.inputs = {"x_tilde": rn(2, H, k, d), "x_hat": rn(2, H, k, d)}
+        job.weights = {"w1": (rn(H, d, F) / math.sqrt(d)).bfloat16(), "wg": (rn(H, d, F) / math.sqrt(d)).bfloat16(),
+                       "w2": (rn(H, F, d) / math.sqrt(F)).bfloat16(), "wq": (rn(H, d, d) / math.sqrt(d)).bfloat16(),
+                       "g1": 1 + rn(H, d) / 10, "b1": rn(H, d) / 10, "g2": 1 + rn(H, d) / 10, "b2": rn(H, d) / 10}
+        job.oracle_sample = types.MethodType(RefineJob.oracle_sample, job)
+        return job
+    if spec["kind"] == "sa_stack":
+        H, kp, d, nl = spec["H"], spec["k"], spec["d"], spec["layers"]
+        F, T = 2 * d, 2000
+        x = {"p0": rn(H, kp, d), "v": rn(T, H, d).bfloat16(), "cu": torch.tensor([0, T], dtype=torch.int32)}
+        for l in range(nl):
+            x[f"k{l}"] = rn(T, H, d).bfloat16()
+            x[f"wq{l}"] = (rn(H, d, d) / math.sqrt(d)).bfloat16()
+            x[f"w1_{l}"] = (rn(H, d, F) / math.sqrt(d)).bfloat16()
+            x[f"wg_{l}"] = (rn(H, d, F) / math.sqrt(d)).bfloat16()
+            x[f"w2_{l}"] = (rn(H, F, d) / math.sqrt(F)).bfloat16()
+        job.inputs, job.nl, job.scale = x, nl, 1.0 / math.sqrt(d)
+        job.oracle_sample = types.MethodType(StackJob.oracle_sample, job)
+        return job
     if spec["kind"] == "stca":
         B, Tq, L, ks, H, d = 2, 64, spec["hist"], spec["ks"], spec["H"], spec["d"]
         job.inputs = {"q": torch.randn((B * Tq, H, d), generator=g).bfloat16(),
@@ -569,10 +729,12 @@ def time_job(job, args, world, dev, peaks):
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)
+    hook = getattr(job, "hook", True)  # False: several kernels a step, the step is the unit timed
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for i in range(args.steps):
-        api.set_timing_events(*kev[i])
+        if hook:
+            api.set_timing_events(*kev[i])
         job.run(job.inputs)
     e1.record()
     api.set_timing_events(None, None)
@@ -580,7 +742,7 @@ def time_job(job, args, world, dev, peaks):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    kern_mean = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    kern_mean = statistics.mean(a.elapsed_time(b) for a, b in kev) if hook else e0.elapsed_time(e1) / args.steps
     ms_total, kern_max = dp.max_over_ranks([e0.elapsed_time(e1), kern_mean], device=dev)
     units_all, flops_all = dp.sum_over_ranks([job.units, job.flops], device=dev)
     ms_per_step = ms_total / args.steps

@@ -104,8 +104,8 @@ __device__ __forceinline__ void store_pair8(uint8_t* hi, uint8_t* lo, int r, int
       make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]), pack_bf16x2(l[4], l[5]), pack_bf16x2(l[6], l[7]));
 }
 
-// LayerNorm of one row held by one thread: mean, biased variance (two passes), then the affine
-// map (gamma, beta may be null: 1 and 0).
+// LayerNorm of one row held by one thread: mean, biased variance (two passes), normalisation,
+// then the affine map (gamma, beta may be null: 1 and 0) in float4 steps.
 template <int D>
 __device__ __forceinline__ void layer_norm_row(float* x, const float* gamma, const float* beta, float eps) {
   float mean = 0.f;
@@ -120,11 +120,28 @@ __device__ __forceinline__ void layer_norm_row(float* x, const float* gamma, con
   }
   const float rs = rsqrtf(var * (1.f / D) + eps);
 #pragma unroll
-  for (int c = 0; c < D; ++c) {
-    float y = (x[c] - mean) * rs;
-    if (gamma) y *= __ldg(gamma + c);
-    if (beta) y += __ldg(beta + c);
-    x[c] = y;
+  for (int c = 0; c < D; ++c) x[c] = (x[c] - mean) * rs;
+  if (gamma) {
+    const float4* g4 = reinterpret_cast<const float4*>(gamma);
+#pragma unroll
+    for (int u = 0; u < D / 4; ++u) {
+      const float4 g = __ldg(g4 + u);
+      x[4 * u] *= g.x;
+      x[4 * u + 1] *= g.y;
+      x[4 * u + 2] *= g.z;
+      x[4 * u + 3] *= g.w;
+    }
+  }
+  if (beta) {
+    const float4* b4 = reinterpret_cast<const float4*>(beta);
+#pragma unroll
+    for (int u = 0; u < D / 4; ++u) {
+      const float4 b = __ldg(b4 + u);
+      x[4 * u] += b.x;
+      x[4 * u + 1] += b.y;
+      x[4 * u + 2] += b.z;
+      x[4 * u + 3] += b.w;
+    }
   }
 }
 
@@ -306,18 +323,22 @@ __global__ void __launch_bounds__(kRefThreads, 1)
     }
     // 3. G = swish(H1) * Hg into region B (W_1 / W_g are no longer read)
 #pragma unroll 1
-    for (int c = 0; c < F; c += 8) {
-      uint32_t v1[8], vg[8];
-      tmem_ld8(tb + lane_off + c, v1);
-      tmem_ld8(tb + lane_off + F + c, vg);
+    for (int c = 0; c < F; c += 32) {
+      uint32_t v1[32], vg[32];
+      tmem_ld32(tb + lane_off + c, v1);
+      tmem_ld32(tb + lane_off + F + c, vg);
       tmem_ld_wait();
-      float gv[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float a = __uint_as_float(v1[u]);
-        gv[u] = valid ? a / (1.f + __expf(-a)) * __uint_as_float(vg[u]) : 0.f;
+      for (int u = 0; u < 32; u += 8) {
+        float gv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float a = __uint_as_float(v1[u + e]);
+          // swish(a) = a / (1 + e^-a); the fast divide returns -0 for a < -88 (e^-a = inf)
+          gv[e] = valid ? __fdividef(a, 1.f + __expf(-a)) * __uint_as_float(vg[u + e]) : 0.f;
+        }
+        store_pair8(sGh, sGl, r, c + u, gv);
       }
-      store_pair8(sGh, sGl, r, c, gv);
     }
     fence_async_shared();
     tc_fence_before();
@@ -359,12 +380,12 @@ __global__ void __launch_bounds__(kRefThreads, 1)
       for (int u = 0; u < D; ++u) xb[u] = 0.f;
     }
 #pragma unroll
-    for (int c = 0; c < D; c += 16) {
-      uint32_t yv[16];
-      tmem_ld16(tb + lane_off + c, yv);
+    for (int c = 0; c < D; c += 32) {
+      uint32_t yv[32];
+      tmem_ld32(tb + lane_off + c, yv);
       tmem_ld_wait();
 #pragma unroll
-      for (int u = 0; u < 16; ++u) xb[c + u] += __uint_as_float(yv[u]);
+      for (int u = 0; u < 32; ++u) xb[c + u] += __uint_as_float(yv[u]);
     }
     tc_fence_before();
     if (valid) {
@@ -467,7 +488,10 @@ cudaError_t launch_sa_refine(int D, int F, int num_ctas, const CUtensorMap& m1, 
   cudaError_t e = cudaErrorInvalidValue;
   if (D == 64 && F == 128) e = refine_launch_t<64, 128>(num_ctas, m1, mg, m2, mq, p, stream);
   if (D == 128 && F == 256) e = refine_launch_t<128, 256>(num_ctas, m1, mg, m2, mq, p, stream);
-  if (e != cudaSuccess) return e;
+  return e;
+}
+
+cudaError_t launch_refine_poison(int D, const RefineParams& p, cudaStream_t stream) {
   const int64_t n = int64_t(p.B) * p.H * p.k * D;
   refine_poison_kernel<<<2 * 148, 256, 0, stream>>>(p.status, p.x_next, p.x_bar,
                                                     reinterpret_cast<uint16_t*>(p.x_next_bf16),

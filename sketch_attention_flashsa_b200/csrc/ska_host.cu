@@ -795,6 +795,7 @@ ska_status sa_refine(const ska_refine_desc* d, const float* x_tilde, const float
     TimedRegion tr(s);
     e = launch_sa_refine(D, F, ctas, m1, mg, m2, mq, p, s);
   }
+  if (e == cudaSuccess) e = launch_refine_poison(D, p, s);
   if (e != cudaSuccess) {
     record_error("refinement kernel launch", e);
     return SKA_ERR_CUDA;
@@ -841,6 +842,7 @@ ska_status sa_project_queries(int32_t num_users, int32_t num_heads, int32_t num_
   const int64_t tiles = int64_t(B) * H * ((k + 127) / 128);
   const int ctas = static_cast<int>(std::min<int64_t>(tiles, device_sm_count()));
   cudaError_t e = launch_sa_refine(D, 2 * D, ctas, mq, mq, mq, mq, p, s);
+  if (e == cudaSuccess) e = launch_refine_poison(D, p, s);
   if (e != cudaSuccess) {
     record_error("projection kernel launch", e);
     return SKA_ERR_CUDA;

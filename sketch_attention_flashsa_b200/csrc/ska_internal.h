@@ -149,11 +149,12 @@ struct RefineParams {
 };
 
 bool sa_refine_supported(int head_dim, int ffn_dim);
-// The fused refinement kernel on num_ctas persistent CTAs, then a kernel that turns the outputs
-// to NaN when the status word holds an error. mapWq is read only when p.q_next is set.
+// The fused refinement kernel on num_ctas persistent CTAs. mapWq is read only when p.q_next is set.
 cudaError_t launch_sa_refine(int head_dim, int ffn_dim, int num_ctas, const CUtensorMap& mapW1,
                              const CUtensorMap& mapWg, const CUtensorMap& mapW2, const CUtensorMap& mapWq,
                              const RefineParams& p, cudaStream_t stream);
+// Turns every output of the call to NaN when the status word holds an error (launched after it).
+cudaError_t launch_refine_poison(int head_dim, const RefineParams& p, cudaStream_t stream);
 
 // Small kernels (ska_small.cu).
 cudaError_t launch_schedule(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,

@@ -125,3 +125,18 @@ def sa_forward_bytes(valid_tokens: int, heads: int, protos: int, head_dim: int, 
 def stca_forward_flops(total_targets: int, keys_per_target: float, heads: int,
                        head_dim: int) -> float:
     return 4.0 * total_targets * keys_per_target * heads * head_dim
+
+
+def refine_flops(rows: float, d: float, project: bool = True) -> float:
+    """One refinement of `rows` sketch rows (all users and heads) of width d (§3.3, Eq. (13)-(14)):
+    the SwiGLU FFN at width 2d (App. G.3's 12 L_s d^2) and, with `project`, the next layer's query
+    projection X~ W_Q (App. G.3's 2 L_s d^2)."""
+    return swiglu(rows, d, 2 * d) + (gemm(rows, d, d) if project else 0.0)
+
+
+def refine_bytes(rows: float, heads: float, d: float, project: bool = True) -> float:
+    """Bytes a refinement moves at least once: x_tilde and x_hat read and x_next written in fp32,
+    q_next written in bf16, and the weights (bf16) and LayerNorm vectors (fp32) of every head."""
+    weights = heads * (3 * d * 2 * d + (d * d if project else 0)) * 2 + heads * 4 * d * 4
+    return rows * d * (4 + 4 + 4 + (2 if project else 0)) + weights
+
