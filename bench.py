@@ -628,7 +628,8 @@ def main():
     job = JOBS[spec["kind"]](spec, args.norm, rank, world, dev)
     peaks = load_peaks()
     res = time_job(job, args, world, dev, peaks)
-    res["roofline"]["traffic"] = traffic_for(args.workload, args.norm if spec["kind"] != "stca" else "stca")
+    res["roofline"]["traffic"] = traffic_for(args.workload, {"stca": "stca", "refine": "refine"}.get(spec["kind"],
+                                                                                                 args.norm))
 
     # End to end through the public API: pinned host inputs -> device, the call, result -> host.
     host = {n: t.cpu().pin_memory() for n, t in job.inputs.items()}
