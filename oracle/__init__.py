@@ -18,10 +18,10 @@ differences; none of them re-types the formulas below.
 """
 from .sa import (sa_forward_proto, sa_forward_token, sa_backward_proto,
                  sa_backward_token, sa_forward, sa_backward, sa_problem)
-from .stca import stca_forward
+from .stca import stca_forward, stca_backward
 from .refine import layer_norm, swish, swiglu_ffn, refine, project_queries, stacked_sa
 
 __all__ = ["sa_forward_proto", "sa_forward_token", "sa_backward_proto",
            "sa_backward_token", "sa_forward", "sa_backward", "sa_problem",
-           "stca_forward", "layer_norm", "swish", "swiglu_ffn", "refine", "project_queries",
+           "stca_forward", "stca_backward", "layer_norm", "swish", "swiglu_ffn", "refine", "project_queries",
            "stacked_sa"]

@@ -529,3 +529,40 @@ def test_stacked_sa_token_order_and_users():
     v2[6:] += rng.normal(size=(3, H, d))  # (a shift equal on every feature would be absorbed by LN)
     out2, _ = oracle.stacked_sa(p0, w_q, keys, v2, cu, None, 0.5, ffn)
     assert np.array_equal(out2[0], out[0]) and not np.allclose(out2[1], out[1])
+
+
+# ------------------------------------------------------------------- STCA backward (finite differences)
+
+@pytest.mark.parametrize("with_kv_len", [False, True])
+def test_stca_backward_matches_finite_differences(with_kv_len):
+    """Every gradient of <dO, out> against central differences of the forward oracle alone
+    (h = 1e-6): the query of each target, the suffix keys and values shared by a user's targets
+    (summed over them) and the sketch keys and values."""
+    q, cut, kh, vh, cuh, ksk, vsk = _stca_problem([2, 3], [4, 5], 3, H=2, d=4, seed=44)
+    kvl = np.array([2, 1, 0, 4, 3]) if with_kv_len else None
+    rng = np.random.default_rng(45)
+    do = rng.standard_normal(q.shape)
+    scale = 0.7
+    grads = oracle.stca_backward(q, cut, kh, vh, cuh, ksk, vsk, scale, do, kvl)
+
+    def f(args):
+        out, _ = oracle.stca_forward(args[0], cut, args[1], args[2], cuh, args[3], args[4], scale, kvl)
+        return float((out * do).sum())
+
+    base = [q, kh, vh, ksk, vsk]
+    h = 1e-6
+    for which, g in enumerate(grads):
+        flat = base[which].reshape(-1)
+        for idx in range(flat.size):
+            plus = [x.copy() for x in base]
+            minus = [x.copy() for x in base]
+            plus[which].reshape(-1)[idx] += h
+            minus[which].reshape(-1)[idx] -= h
+            fd = (f(plus) - f(minus)) / (2 * h)
+            assert abs(fd - g.reshape(-1)[idx]) < 1e-7, (which, idx, fd, g.reshape(-1)[idx])
+    if with_kv_len:
+        # suffix rows that no target of their user reaches get no gradient: rows 2, 3 of user 0
+        # (lengths 2, 1) and the last row of user 1 (lengths 0, 4, 3)
+        for rows in (slice(2, 4), slice(8, 9)):
+            assert not grads[1][rows].any() and not grads[2][rows].any()
+        assert grads[1][0:2].any() and grads[2][4:8].any()
