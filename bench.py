@@ -49,6 +49,7 @@ METRICS = {
     "refine": ("sketch refinement rows/s (LN, SwiGLU FFN, LN, next-layer query projection) and GB/s",
                "sketch-rows/s"),
     "sa_stack": ("stacked SA (N_sa = 2 layers) history-tokens/s at L=100K", "history-tokens/s"),
+    "stca_bwd": ("STCA bwd targets/s (dq, dK, dV over [10K suffix ; 256 sketch] keys) and TFLOP/s", "targets/s"),
 }
 
 # name -> kind and shapes. lens: list, "ragged64" (64 users, log-uniform in [1K, 100K], seed 1) or
@@ -73,6 +74,8 @@ WORKLOADS = {
     "refine_b8_h8_k512_d128": dict(kind="refine", B=8, H=8, k=512, d=128),
     # two stacked SA layers (§3.3) over the 8 x 100K workload, own keys per layer, V = the history
     "sa_stack2_b8_l100k_h8_d128_k512": dict(kind="sa_stack", lens=[100_000] * 8, H=8, d=128, k=512, layers=2),
+    "stca_bwd_b16_t512_h4_d64_l10k_s256": dict(kind="stca_bwd", users=16, targets=512, hist=10_000, ks=256, H=4,
+                                               d=64, scale=0.125),
     "stca_b16_t512_h4_d64_l10k_s256": dict(kind="stca", users=16, targets=512, hist=10_000, ks=256, H=4, d=64,
                                            scale=0.125),
 }
@@ -479,7 +482,61 @@ class StackJob:
         return n, time.perf_counter() - t0, f"the first {n} tokens of one user through {self.nl} layers, fp64 numpy"
 
 
-JOBS = {"sa_fwd": SaFwdJob, "sa_bwd": SaBwdJob, "stca": StcaJob, "refine": RefineJob, "sa_stack": StackJob}
+class StcaBwdJob(StcaJob):
+    """The STCA backward at the forward's shapes: the forward's out and lse are computed once
+    (inputs of the step), the upstream gradient is drawn; a step is one stca_backward call (its
+    key-major and query-major kernels are timed together)."""
+
+    def __init__(self, spec, norm, rank, world, dev):
+        import torch
+        from sketch_attention_flashsa_b200 import flops
+        super().__init__(spec, norm, rank, world, dev)
+        x = self.inputs
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(3500 + rank)
+        x["dout"] = torch.randn(x["q"].shape, generator=gen, device=dev, dtype=torch.bfloat16)
+        out, lse = self.api.stca_forward(x["q"], x["cu_t"], x["k_hist"], x["v_hist"], x["cu_h"], x["k_sk"], x["v_sk"],
+                                         scale=self.scale, max_targets=self.Tq)
+        x["out"], x["lse"] = out, lse
+        B, Tq, L, ks, H, d = spec["users"], spec["targets"], spec["hist"], spec["ks"], spec["H"], spec["d"]
+        desc = self.api.stca_desc(x["q"], x["k_hist"], x["k_sk"], x["cu_t"], x["cu_h"], scale=self.scale,
+                                  max_targets=Tq)
+        self.ws = torch.empty(max(int(self.api._lib.lib().stca_backward_workspace_size(
+            __import__("ctypes").byref(desc))), 256), dtype=torch.uint8, device=dev)
+        # five GEMM-shaped products per (target, key): S, dP, dV, dK, dq (App. G.1 counting)
+        self.flops = 2.5 * flops.stca_forward_flops(B * Tq, L + ks, H, d)
+        # read q, dO (bf16), out (fp32), K and V (bf16), lse; write dq, dK, dV (fp32)
+        self.bytes = (B * Tq * H * d * (2 + 2 + 4 + 4) + B * Tq * H * 4 + 2 * B * L * H * d * (2 + 4)
+                      + 2 * B * H * ks * d * (2 + 4))
+        self.kernel = "stca_bwd_dkv_kernel + stca_bwd_dq_kernel"
+        self.launches = 5
+        self.config["outputs"] = "dq, dK, dV fp32"
+
+    def run(self, x):
+        g = self.api.stca_backward(x["q"], x["cu_t"], x["k_hist"], x["v_hist"], x["cu_h"], x["k_sk"], x["v_sk"],
+                                   x["out"], x["lse"], x["dout"], scale=self.scale, workspace=self.ws)
+        return g[0]
+
+    def oracle_sample(self, budget_s):
+        import oracle
+        x = self.inputs
+        cut, cuh = x["cu_t"].cpu().numpy(), x["cu_h"].cpu().numpy()
+        done, users, t0 = 0.0, 0, time.perf_counter()
+        per_user = 16
+        while time.perf_counter() - t0 < budget_s and users < self.B:
+            b = users
+            rows = slice(int(cut[b]), int(cut[b]) + per_user)
+            oracle.stca_backward(f64(x["q"][rows]), np.array([0, per_user]), f64(x["k_hist"][cuh[b]:cuh[b + 1]]),
+                                 f64(x["v_hist"][cuh[b]:cuh[b + 1]]), np.array([0, cuh[b + 1] - cuh[b]]),
+                                 f64(x["k_sk"][b:b + 1]), f64(x["v_sk"][b:b + 1]), self.scale,
+                                 f64(x["dout"][rows]), None)
+            done += per_user
+            users += 1
+        return done, time.perf_counter() - t0, f"{per_user} targets of each of {users} users (all heads), fp64 numpy"
+
+
+JOBS = {"sa_fwd": SaFwdJob, "sa_bwd": SaBwdJob, "stca": StcaJob, "refine": RefineJob, "sa_stack": StackJob,
+        "stca_bwd": StcaBwdJob}
 
 
 def traffic_for(workload, norm):
@@ -554,7 +611,7 @@ def _host_job(spec, norm):
         job.inputs, job.nl, job.scale = x, nl, 1.0 / math.sqrt(d)
         job.oracle_sample = types.MethodType(StackJob.oracle_sample, job)
         return job
-    if spec["kind"] == "stca":
+    if spec["kind"] in ("stca", "stca_bwd"):
         B, Tq, L, ks, H, d = 2, 64, spec["hist"], spec["ks"], spec["H"], spec["d"]
         job.inputs = {"q": torch.randn((B * Tq, H, d), generator=g).bfloat16(),
                       "cu_t": torch.arange(0, B * Tq + 1, Tq, dtype=torch.int32),
@@ -564,7 +621,10 @@ def _host_job(spec, norm):
                       "k_sk": torch.randn((B, H, ks, d), generator=g).bfloat16(),
                       "v_sk": torch.randn((B, H, ks, d), generator=g).bfloat16()}
         job.scale, job.B = spec["scale"], B
-        job.oracle_sample = types.MethodType(StcaJob.oracle_sample, job)
+        if spec["kind"] == "stca_bwd":
+            job.inputs["dout"] = torch.randn((B * Tq, H, d), generator=g).bfloat16()
+        job.oracle_sample = types.MethodType((StcaBwdJob if spec["kind"] == "stca_bwd" else StcaJob).oracle_sample,
+                                             job)
         return job
     lens = lengths_for(spec["lens"])
     H, d, kp = spec["H"], spec["d"], spec["k"]
@@ -628,8 +688,8 @@ def main():
     job = JOBS[spec["kind"]](spec, args.norm, rank, world, dev)
     peaks = load_peaks()
     res = time_job(job, args, world, dev, peaks)
-    res["roofline"]["traffic"] = traffic_for(args.workload, {"stca": "stca", "refine": "refine"}.get(spec["kind"],
-                                                                                                 args.norm))
+    res["roofline"]["traffic"] = traffic_for(args.workload, {"stca": "stca", "refine": "refine",
+                                                             "stca_bwd": "stca_bwd"}.get(spec["kind"], args.norm))
 
     # End to end through the public API: pinned host inputs -> device, the call, result -> host.
     host = {n: t.cpu().pin_memory() for n, t in job.inputs.items()}

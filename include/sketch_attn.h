@@ -191,6 +191,28 @@ SKA_API ska_status stca_forward(const ska_stca_desc* desc, const void* q, const 
                         const int32_t* target_kv_len, const void* k_sk, const void* v_sk, float* out,
                         float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of workspace stca_backward needs (0 if the descriptor is invalid). */
+SKA_API size_t stca_backward_workspace_size(const ska_stca_desc* desc);
+
+/* STCA backward: gradients of <dout, out> through stca_forward (STCA is trained end to end with
+ * the ranker, §2.3; through its sketch branch the gradients reach the SA sketch, §3.4). Inputs as
+ * in stca_forward, plus:
+ *   out      fp32 [total_targets, H, d], the forward output (delta_t = <dout_t, out_t>)
+ *   lse      fp32 [total_targets, H], the forward's lse
+ *   dout     bf16 [total_targets, H, d]
+ *   dq       out, fp32 [total_targets, H, d]
+ *   dk_hist, dv_hist   out, fp32 [total_hist, H, d]: summed over the targets of the row's user
+ *                      that see it (target_kv_len); zero for rows no target sees
+ *   dk_sk, dv_sk       out, fp32 [B, H, num_sketch, d] (NULL when num_sketch == 0)
+ * head_dim 64 or 128. max_targets and max_hist are not used. dq takes dS as a two-term bf16 split
+ * (16 significant bits); dK and dV take P and dS in bf16, with fp32 accumulation.             */
+SKA_API ska_status stca_backward(const ska_stca_desc* desc, const void* q, const int32_t* cu_targets,
+                                 const void* k_hist, const void* v_hist, const int32_t* cu_hist,
+                                 const int32_t* target_kv_len, const void* k_sk, const void* v_sk,
+                                 const float* out, const float* lse, const void* dout, float* dq,
+                                 float* dk_hist, float* dv_hist, float* dk_sk, float* dv_sk, void* ws,
+                                 size_t ws_bytes, void* stream);
+
 /* Stacked refinement of the sketch (§3.3, Eq. (13)-(14)): one layer's update of the per-user
  * sketch after its SA aggregation,
  *   x_bar  = LN1(x_tilde + x_hat)                               Eq. (13)

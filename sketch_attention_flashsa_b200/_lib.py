@@ -24,7 +24,8 @@ EXPORTED = ("sa_forward_workspace_size", "sa_forward", "sa_backward_workspace_si
             "stca_forward_workspace_size", "stca_forward", "ska_status_string",
             "ska_read_device_status", "ska_set_debug", "ska_set_timing_events",
             "sa_forward_noalloc", "sa_forward_noalloc_scratch_bytes", "sa_forward_noalloc_read_status",
-            "ska_last_error_string", "sa_refine_workspace_size", "sa_refine", "sa_project_queries")
+            "ska_last_error_string", "sa_refine_workspace_size", "sa_refine", "sa_project_queries",
+            "stca_backward_workspace_size", "stca_backward")
 
 
 class SaDesc(ctypes.Structure):
@@ -98,6 +99,10 @@ def lib() -> ctypes.CDLL:
     L.sa_forward_noalloc_scratch_bytes.restype = sz
     L.sa_forward_noalloc_read_status.argtypes = [vp]
     L.sa_forward_noalloc_read_status.restype = ctypes.c_int
+    L.stca_backward_workspace_size.argtypes = [ctypes.POINTER(StcaDesc)]
+    L.stca_backward_workspace_size.restype = sz
+    L.stca_backward.argtypes = [ctypes.POINTER(StcaDesc)] + [vp] * 17 + [sz, vp]
+    L.stca_backward.restype = ctypes.c_int
     L.sa_refine_workspace_size.argtypes = [ctypes.POINTER(RefineDesc)]
     L.sa_refine_workspace_size.restype = sz
     L.sa_refine.argtypes = [ctypes.POINTER(RefineDesc)] + [vp] * 15 + [sz, vp]

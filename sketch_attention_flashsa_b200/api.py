@@ -269,6 +269,70 @@ def stca_forward(q: torch.Tensor, cu_targets: torch.Tensor, k_hist: torch.Tensor
     return out, lse
 
 
+def stca_backward(q: torch.Tensor, cu_targets: torch.Tensor, k_hist: torch.Tensor, v_hist: torch.Tensor,
+                  cu_hist: torch.Tensor, k_sk: Optional[torch.Tensor], v_sk: Optional[torch.Tensor],
+                  out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor, *, scale: float,
+                  target_kv_len: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None):
+    """STCA backward (SequenceO1 §2.3, §3.4): gradients of <dout, out> through stca_forward.
+
+    Inputs as in stca_forward, plus its outputs out fp32 [Tq,H,d] and lse fp32 [Tq,H], and dout
+    bf16 [Tq,H,d]. Returns (dq [Tq,H,d], dk_hist, dv_hist [Th,H,d], dk_sk, dv_sk [B,H,ks,d] or
+    None), all fp32.
+    """
+    for name, t in (("q", q), ("k_hist", k_hist), ("v_hist", v_hist), ("k_sk", k_sk), ("v_sk", v_sk),
+                    ("dout", dout)):
+        if t is not None and t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} has dtype {t.dtype}, expected torch.bfloat16")
+    if q.dim() != 3:
+        raise ValueError(f"q must be [Tq, H, d], got shape {tuple(q.shape)}")
+    Tq, H, D = q.shape
+    for name, t in (("cu_targets", cu_targets), ("cu_hist", cu_hist)):
+        if t.dtype != torch.int32 or t.dim() != 1 or t.numel() < 1:
+            raise ValueError(f"{name} must be a 1-D int32 tensor of B + 1 offsets")
+    B = cu_targets.numel() - 1
+    if cu_hist.numel() != B + 1:
+        raise ValueError(f"cu_hist has {cu_hist.numel()} entries, cu_targets {B + 1}")
+    if k_hist.dim() != 3 or k_hist.shape[1:] != (H, D):
+        raise ValueError(f"k_hist {tuple(k_hist.shape)} does not match q's heads and head_dim")
+    _shape("v_hist", v_hist, k_hist.shape)
+    if (k_sk is None) != (v_sk is None):
+        raise ValueError("k_sk and v_sk come together")
+    if k_sk is not None:
+        if k_sk.dim() != 4 or k_sk.shape[0] != B or k_sk.shape[1] != H or k_sk.shape[3] != D:
+            raise ValueError(f"k_sk must be [{B}, {H}, ks, {D}], got {tuple(k_sk.shape)}")
+        _shape("v_sk", v_sk, k_sk.shape)
+    _shape("out", out, (Tq, H, D))
+    _shape("lse", lse, (Tq, H))
+    _shape("dout", dout, (Tq, H, D))
+    if target_kv_len is not None and (target_kv_len.dtype != torch.int32 or tuple(target_kv_len.shape) != (Tq,)):
+        raise ValueError(f"target_kv_len must be int32 of shape ({Tq},)")
+    for name, t in (("q", q), ("k_hist", k_hist), ("v_hist", v_hist), ("k_sk", k_sk), ("v_sk", v_sk),
+                    ("dout", dout)):
+        _dev_tensor(name, t, (torch.bfloat16,))
+    for name, t in (("out", out), ("lse", lse)):
+        _dev_tensor(name, t, (torch.float32,))
+    for name, t in (("cu_targets", cu_targets), ("cu_hist", cu_hist), ("target_kv_len", target_kv_len)):
+        _dev_tensor(name, t, (torch.int32,))
+    desc = stca_desc(q, k_hist, k_sk, cu_targets, cu_hist, scale=scale, max_targets=max(Tq, 1))
+    L = _lib.lib()
+    need = int(L.stca_backward_workspace_size(ctypes.byref(desc)))
+    dev = q.device
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    dq = torch.empty((Tq, H, D), dtype=torch.float32, device=dev)
+    dkh = torch.empty(k_hist.shape, dtype=torch.float32, device=dev)
+    dvh = torch.empty(k_hist.shape, dtype=torch.float32, device=dev)
+    dks = torch.empty(k_sk.shape, dtype=torch.float32, device=dev) if k_sk is not None else None
+    dvs = torch.empty(k_sk.shape, dtype=torch.float32, device=dev) if k_sk is not None else None
+    rc = L.stca_backward(ctypes.byref(desc), _ptr(q), _ptr(cu_targets), _ptr(k_hist), _ptr(v_hist), _ptr(cu_hist),
+                         _ptr(target_kv_len), _ptr(k_sk), _ptr(v_sk), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                         _ptr(dkh), _ptr(dvh), _ptr(dks), _ptr(dvs), _ptr(workspace),
+                         ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check(rc, "stca_backward")
+    return dq, dkh, dvh, dks, dvs
+
+
 def sa_backward_workspace_size(desc: SaDesc) -> int:
     return int(_lib.lib().sa_backward_workspace_size(ctypes.byref(desc)))
 

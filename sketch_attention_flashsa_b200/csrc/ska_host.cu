@@ -717,6 +717,103 @@ ska_status stca_forward(const ska_stca_desc* d, const void* q, const int32_t* cu
   return SKA_OK;
 }
 
+size_t stca_backward_workspace_size(const ska_stca_desc* d) {
+  if (check_stca_desc(d) != SKA_OK) return 0;
+  size_t off = sizeof(WsHeader);
+  off = align256(off + size_t(d->num_users + 1) * 4);
+  off = align256(off + size_t(d->num_users + 1) * 4);
+  off = align256(off + size_t(d->total_targets) * d->num_heads * 4);
+  return off;
+}
+
+ska_status stca_backward(const ska_stca_desc* d, const void* q, const int32_t* cu_targets, const void* k_hist,
+                         const void* v_hist, const int32_t* cu_hist, const int32_t* target_kv_len, const void* k_sk,
+                         const void* v_sk, const float* out, const float* lse, const void* dout, float* dq,
+                         float* dk_hist, float* dv_hist, float* dk_sk, float* dv_sk, void* ws, size_t ws_bytes,
+                         void* stream) {
+  ska_status st = check_stca_desc(d);
+  if (st != SKA_OK) return st;
+  const int B = d->num_users, H = d->num_heads, D = d->head_dim, ks = d->num_sketch;
+  const int64_t Tq = d->total_targets, Th = d->total_hist;
+  if (!stca_bwd_supported(D)) return SKA_ERR_UNSUPPORTED;
+  if (B == 0) return SKA_OK;
+  if (!cu_targets || !cu_hist || !ws) return SKA_ERR_INVALID_VALUE;
+  if (Tq > 0 && (!q || !out || !lse || !dout || !dq)) return SKA_ERR_INVALID_VALUE;
+  if (Th > 0 && (!k_hist || !v_hist || !dk_hist || !dv_hist)) return SKA_ERR_INVALID_VALUE;
+  if (ks > 0 && (!k_sk || !v_sk || !dk_sk || !dv_sk)) return SKA_ERR_INVALID_VALUE;
+  const void* al[13] = {q, k_hist, v_hist, k_sk, v_sk, out, lse, dout, dq, dk_hist, dv_hist, dk_sk, dv_sk};
+  for (int i = 0; i < 13; ++i)
+    if (!aligned16(al[i])) return SKA_ERR_INVALID_VALUE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) || (reinterpret_cast<uintptr_t>(cu_targets) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_hist) & 3u) || (reinterpret_cast<uintptr_t>(target_kv_len) & 3u))
+    return SKA_ERR_INVALID_VALUE;
+  const size_t need = stca_backward_workspace_size(d);
+  if (ws_bytes < need) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  const size_t qb = size_t(Tq) * H * D * 2, hb = size_t(Th) * H * D * 2, sb = size_t(B) * H * ks * D * 2;
+  const void* ins[8] = {q, k_hist, v_hist, k_sk, v_sk, out, lse, dout};
+  const size_t insz[8] = {qb, hb, hb, sb, sb, qb * 2, size_t(Tq) * H * 4, qb};
+  const void* outs[6] = {dq, dk_hist, dv_hist, dk_sk, dv_sk, ws};
+  const size_t outsz[6] = {qb * 2, hb * 2, hb * 2, sb * 2, sb * 2, need};
+  for (int o = 0; o < 6; ++o) {
+    for (int i = 0; i < 8; ++i)
+      if (overlaps(outs[o], outsz[o], ins[i], insz[i])) return SKA_ERR_INVALID_VALUE;
+    for (int o2 = o + 1; o2 < 6; ++o2)
+      if (overlaps(outs[o], outsz[o], outs[o2], outsz[o2])) return SKA_ERR_INVALID_VALUE;
+  }
+  if (no_device()) return SKA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  StcaBwdParams p{};
+  size_t off = sizeof(WsHeader);
+  p.hdr = reinterpret_cast<WsHeader*>(wsb);
+  p.kprefix = reinterpret_cast<int32_t*>(wsb + off);
+  off = align256(off + size_t(B + 1) * 4);
+  p.qprefix = reinterpret_cast<int32_t*>(wsb + off);
+  off = align256(off + size_t(B + 1) * 4);
+  p.delta = reinterpret_cast<float*>(wsb + off);
+  p.cu_q = cu_targets;
+  p.cu_k = cu_hist;
+  p.kv_len = target_kv_len;
+  p.lse = lse;
+  p.dq = dq;
+  p.dk_hist = dk_hist;
+  p.dv_hist = dv_hist;
+  p.dk_sk = dk_sk;
+  p.dv_sk = dv_sk;
+  p.B = B;
+  p.H = H;
+  p.ks = ks;
+  p.scale = d->scale;
+  p.budget_ns = wait_budget();
+  if (cudaError_t e = launch_stca_bwd_prep(p, dout, out, Tq * H, D, s); e != cudaSuccess) {
+    record_error("launch_stca_bwd_prep", e);
+    return SKA_ERR_CUDA;
+  }
+  // maps over absent tensors point at the workspace's first row and are never loaded
+  const void* dummy = Tq > 0 ? q : ws;
+  CUtensorMap maps[6];
+  const uint64_t qrows = std::max<int64_t>(Tq, 1), hrows = std::max<int64_t>(Th, 1);
+  if (!encode_2d(&maps[0], Tq > 0 ? q : dummy, uint64_t(H) * D, qrows, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+  if (!encode_2d(&maps[1], Tq > 0 ? dout : dummy, uint64_t(H) * D, qrows, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+  if (!encode_2d(&maps[2], Th > 0 ? k_hist : dummy, uint64_t(H) * D, hrows, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+  if (!encode_2d(&maps[3], Th > 0 ? v_hist : dummy, uint64_t(H) * D, hrows, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+  const uint64_t srows = std::max<int64_t>(int64_t(B) * H * ks, 1);
+  if (!encode_2d(&maps[4], ks > 0 ? k_sk : dummy, D, srows, D, 64, 128)) return SKA_ERR_CUDA;
+  if (!encode_2d(&maps[5], ks > 0 ? v_sk : dummy, D, srows, D, 64, 128)) return SKA_ERR_CUDA;
+  const int sms = device_sm_count();
+  cudaError_t e;
+  {
+    TimedRegion tr(s);
+    e = launch_stca_bwd(D, sms, sms, maps, p, s);
+  }
+  if (e == cudaSuccess) e = launch_stca_bwd_poison(p, Tq * H * D, Th * H * D, int64_t(B) * H * ks * D, s);
+  if (e != cudaSuccess) {
+    record_error("STCA backward launch", e);
+    return SKA_ERR_CUDA;
+  }
+  return SKA_OK;
+}
+
 size_t sa_refine_workspace_size(const ska_refine_desc* d) {
   if (check_refine_desc(d) != SKA_OK) return 0;
   return sizeof(WsHeader);

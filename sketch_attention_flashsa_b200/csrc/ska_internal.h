@@ -156,6 +156,38 @@ cudaError_t launch_sa_refine(int head_dim, int ffn_dim, int num_ctas, const CUte
 // Turns every output of the call to NaN when the status word holds an error (launched after it).
 cudaError_t launch_refine_poison(int head_dim, const RefineParams& p, cudaStream_t stream);
 
+// Parameters of the STCA backward (stca_bwd.cu).
+struct StcaBwdParams {
+  const int32_t* cu_q;     // cu_targets [B+1]
+  const int32_t* cu_k;     // cu_hist [B+1]
+  const int32_t* kv_len;   // [total_targets] or null
+  const float* lse;        // [total_targets, H], natural log, from the forward
+  float* delta;            // [total_targets, H] workspace: <dO, out>
+  int32_t* kprefix;        // [B+1] workspace: H x key tiles of the users before b
+  int32_t* qprefix;        // [B+1] workspace: H x target tiles of the users before b
+  WsHeader* hdr;           // status; total_tiles = key items, tiles_per_cluster = target items
+  float* dq;               // [total_targets, H, D]
+  float* dk_hist;          // [total_hist, H, D]
+  float* dv_hist;
+  float* dk_sk;            // [B, H, ks, D]
+  float* dv_sk;
+  int B, H, ks;
+  float scale;
+  uint64_t budget_ns;
+};
+
+bool stca_bwd_supported(int head_dim);
+// The schedule (item prefixes, status cleared) and delta = <dO, out> per (target, head).
+cudaError_t launch_stca_bwd_prep(const StcaBwdParams& p, const void* dout, const float* out, int64_t rows,
+                                 int head_dim, cudaStream_t stream);
+// The key-major (dK, dV) then the query-major (dq) kernel. maps: Q, dO, K suffix, V suffix, K sketch,
+// V sketch.
+cudaError_t launch_stca_bwd(int head_dim, int ctas_kv, int ctas_q, const CUtensorMap* maps, const StcaBwdParams& p,
+                            cudaStream_t stream);
+// NaN into every gradient when the status word holds an error.
+cudaError_t launch_stca_bwd_poison(const StcaBwdParams& p, int64_t n_dq, int64_t n_hist, int64_t n_sketch,
+                                   cudaStream_t stream);
+
 // Small kernels (ska_small.cu).
 cudaError_t launch_schedule(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,
                             int num_clusters, int32_t* tile_prefix, WsHeader* hdr, cudaStream_t stream);

@@ -174,11 +174,12 @@ class STCAInputs:
     v_sk: torch.Tensor
     scale: float
     target_kv_len: Optional[torch.Tensor] = None
+    dout: Optional[torch.Tensor] = None  # bf16 [total_targets, H, d], the upstream gradient (backward)
 
 
 def make_stca(targets, hist, num_heads: int, head_dim: int, num_sketch: int, seed: int,
               *, scale: Optional[float] = None, sigma: float = 1.0,
-              with_kv_len: bool = False) -> STCAInputs:
+              with_kv_len: bool = False, with_dout: bool = False) -> STCAInputs:
     """Draw one STCA workload: per-user target counts ``targets`` and suffix lengths ``hist``."""
     rng = np.random.default_rng(seed)
     targets = [int(x) for x in targets]
@@ -195,8 +196,9 @@ def make_stca(targets, hist, num_heads: int, head_dim: int, num_sketch: int, see
         kvl = torch.from_numpy(np.concatenate(parts).astype(np.int32)) if parts else None
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    dout = to_bf16(normal(rng, (sum(targets), H, d))) if with_dout else None
     return STCAInputs(to_bf16(q), cu_from_lengths(targets), to_bf16(kh), to_bf16(vh),
-                      cu_from_lengths(hist), to_bf16(ks), to_bf16(vs), float(scale), kvl)
+                      cu_from_lengths(hist), to_bf16(ks), to_bf16(vs), float(scale), kvl, dout)
 
 
 # The five benchmark workloads plus the paper's production SA shape (App. G.5).

@@ -263,3 +263,40 @@ def test_refine_without_a_device_reports_cuda_error():
     assert refine(refine_desc(head_dim=64, ffn_dim=128)) == L.SKA_ERR_CUDA
     assert refine(refine_desc(x_tilde_shared=1)) == L.SKA_ERR_CUDA
     assert project() == L.SKA_ERR_CUDA
+
+
+STCA_BWD_ARGS = ["q", "cut", "kh", "vh", "cuh", "kvl", "ks", "vs", "out", "lse", "do", "dq", "dkh", "dvh", "dks",
+                 "dvs", "ws"]
+
+
+def stca_bwd(desc, **kw):
+    ptrs = {n: (i + 70) * A for i, n in enumerate(STCA_BWD_ARGS)}
+    ptrs["kvl"] = None
+    ws_bytes = kw.pop("ws_bytes", 1 << 30)
+    ptrs.update(kw)
+    return L.lib().stca_backward(ctypes.byref(desc) if desc is not None else None,
+                                 *[ptrs[n] for n in STCA_BWD_ARGS], ws_bytes, None)
+
+
+def test_stca_backward_host_checks():
+    d = stca_desc()
+    need = L.lib().stca_backward_workspace_size(ctypes.byref(d))
+    assert need >= 256 + 100 * 2 * 4  # header, prefixes, one delta per (target, head)
+    assert stca_bwd(None) == INVALID
+    assert stca_bwd(stca_desc(head_dim=32)) == UNSUP
+    assert stca_bwd(stca_desc(num_heads=0)) == INVALID
+    for n in ("q", "out", "lse", "do", "dq", "kh", "dkh", "dvs", "ws"):
+        assert stca_bwd(d, **{n: None}) == INVALID, n
+    assert stca_bwd(stca_desc(num_sketch=0), ks=None, vs=None, dks=None, dvs=None) != INVALID
+    assert stca_bwd(d, ws_bytes=need - 1) == L.SKA_ERR_WORKSPACE_TOO_SMALL
+    assert stca_bwd(d, dq=70 * A + 64) == INVALID      # dq overlaps q
+    assert stca_bwd(d, dvh=82 * A + 256) == INVALID    # dv_hist overlaps dk_hist
+    assert stca_bwd(d, kvl=2 * A + 2) == INVALID       # int32 alignment
+    assert stca_bwd(stca_desc(num_users=0, total_targets=0, total_hist=0), q=None, cut=None, ws=None) == L.SKA_OK
+
+
+def test_stca_backward_without_a_device_reports_cuda_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert stca_bwd(stca_desc()) == L.SKA_ERR_CUDA
