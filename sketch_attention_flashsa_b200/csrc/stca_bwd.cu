@@ -16,9 +16,11 @@
 //     dP = dO V^T; thread = target row: P, dS = P (dP - delta) split into bf16 hi + lo (hi over S,
 //     lo over dP); dq += dS_hi K + dS_lo K in TMEM, restarted every kDqChain key tiles and added
 //     into the output row in fp32 (the tensor core's fp32 accumulation is not round-to-nearest).
-// Warps 0-3 do the row work; warp 4 lane 0 issues the TMA loads, warp 5 lane 0 the MMAs. Operands
-// that stay for a whole item (K/V, or Q/dO) and the streamed ones are double-buffered where shared
-// memory allows (d = 64; d = 128 keeps one item stage).
+// Warps 0-7 do the row work, two warps per TMEM lane quarter, each on half of the 128 columns (its
+// bf16 pairs go over the first half of its own columns, so the halves never overwrite each other's
+// unread values; the MMAs read the A operand from both halves). Warp 8 lane 0 issues the TMA loads,
+// warp 9 lane 0 the MMAs. Operands that stay for a whole item (K/V, or Q/dO) and the streamed ones
+// are double-buffered where shared memory allows (d = 64; d = 128 keeps one item stage).
 #include <algorithm>
 #include <climits>
 #include <cmath>
@@ -30,7 +32,9 @@ namespace ska {
 
 namespace {
 
-constexpr int kSbThreads = 192;
+constexpr int kSbThreads = 320;
+constexpr int kRowWarps = 8;
+constexpr int kProdWarp = 8, kMmaWarp = 9;
 constexpr uint32_t kSbBlk = 16384;  // [128 rows x 64 bf16] swizzled block
 constexpr int kDqChain = 16;        // key tiles per dq accumulation chain in TMEM
 constexpr float kLog2e = 1.4426950408889634f;
@@ -134,12 +138,12 @@ __device__ __forceinline__ void sb_init(SbBars& bars, int is) {
     mbar_init(&bars.sempty2[i], 1);
   }
   mbar_init(&bars.sfull, 1);
-  mbar_init(&bars.pfull, 4);
+  mbar_init(&bars.pfull, kRowWarps);
   mbar_init(&bars.ofull, 1);
-  mbar_init(&bars.ofree, 4);
+  mbar_init(&bars.ofree, kRowWarps);
   mbar_init(&bars.drain, 1);
-  mbar_init(&bars.mready[0], 4);
-  mbar_init(&bars.mready[1], 4);
+  mbar_init(&bars.mready[0], kRowWarps);
+  mbar_init(&bars.mready[1], kRowWarps);
   bars.abort_flag = 0;
   fence_mbar_init();
 }
@@ -150,6 +154,10 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t base, int s) {
 }
 // MN-major B operand (rows = the K index, D contiguous) of K step s (16 rows)
 __device__ __forceinline__ uint64_t mndesc(uint32_t base, int s) { return sw128_desc(base + s * 2048, kSbBlk, 1024); }
+
+// A operand (bf16 pairs in TMEM) of K step s over 128 columns packed by two halves: half h holds the
+// pairs of columns [64 h, 64 h + 64) in its own TMEM columns [64 h, 64 h + 32)
+__device__ __forceinline__ uint32_t sb_pairs(uint32_t t, int s) { return t + (s >> 2) * 64 + (s & 3) * 8; }
 
 // ===================================================================== key-major: dK, dV
 template <int D>
@@ -173,7 +181,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
   float* sMeta = reinterpret_cast<float*>(smem + L::meta_off);  // stage m: lse2, delta, kv length
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) sb_init(bars, IS);
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     tmem_alloc(&bars.tmem_base, 512);
     tmem_relinquish();
   }
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
   SbWaiter wait{&bars, &p.hdr->status, p.budget_ns};
   const int nitems = (p.hdr->status == 0) ? p.hdr->total_tiles : 0;
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       int iuse = 0, suse = 0;
@@ -223,7 +231,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       sb_drain(wait, bars.ifull, IS, iuse);
       sb_drain(wait, bars.sfull2, 2, suse);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
@@ -256,9 +264,9 @@ __global__ void __launch_bounds__(kSbThreads, 1)
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int s = 0; s < 8; ++s) umma_bf16_ts(tdV, tS + s * 8, mndesc(dobase, s), idG, (qt | s) > 0);
+          for (int s = 0; s < 8; ++s) umma_bf16_ts(tdV, sb_pairs(tS, s), mndesc(dobase, s), idG, (qt | s) > 0);
 #pragma unroll
-          for (int s = 0; s < 8; ++s) umma_bf16_ts(tdK, tP + s * 8, mndesc(qbase, s), idG, (qt | s) > 0);
+          for (int s = 0; s < 8; ++s) umma_bf16_ts(tdK, sb_pairs(tP, s), mndesc(qbase, s), idG, (qt | s) > 0);
           umma_commit(&bars.sempty2[ss]);
           ++suse;
         }
@@ -272,9 +280,10 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       wait(&bars.drain, 0, true);
     }
   } else {
-    // ---------------------------------------------------------------- key rows (warps 0-3)
-    const int r = threadIdx.x;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // ---------------------------------------------------------------- key rows (warps 0-7)
+    const int r = threadIdx.x & 127;     // key row (TMEM lane)
+    const int half = warp >> 2;          // columns [64 half, 64 half + 64)
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c2 = p.scale * kLog2e;
     int npair = 0, nout = 0;
     bool ok = true;
@@ -292,7 +301,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       float* dk_row = sk ? p.dk_sk + ((static_cast<int64_t>(b) * p.H + h) * p.ks + (j - nh) * 128 + r) * D
                          : p.dk_hist + ((static_cast<int64_t>(p.cu_k[b]) + kk) * p.H + h) * D;
       if (nqt == 0) {  // no target reads these keys
-        if (keyok)
+        if (keyok && half == 0)
           for (int c = 0; c < D; c += 4) {
             *reinterpret_cast<float4*>(dv_row + c) = make_float4(0.f, 0.f, 0.f, 0.f);
             *reinterpret_cast<float4*>(dk_row + c) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -308,7 +317,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
         float* sLse = sMeta + m * 384;
         float* sDel = sLse + 128;
         int* sKvl = reinterpret_cast<int*>(sLse + 256);
-        {
+        if (half == 0) {
           const int tq = qt * 128 + r;
           const int64_t t = static_cast<int64_t>(p.cu_q[b]) + tq;
           const bool tv = tq < nt;
@@ -325,7 +334,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
         ++npair;
         tc_fence_after();
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
           uint32_t sv[32], dp[32];
           tmem_ld32(tS + lane_off + c0, sv);
           tmem_ld32(tP + lane_off + c0, dp);
@@ -350,9 +359,10 @@ __global__ void __launch_bounds__(kSbThreads, 1)
             dw[u / 2] = pack_bf16x2(ds[0], ds[1]);
             dw[u / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
           }
-          // bf16 pairs over columns [c0 / 2, c0 / 2 + 16): all already read
-          tmem_st16(tS + lane_off + c0 / 2, pw);
-          tmem_st16(tP + lane_off + c0 / 2, dw);
+          // bf16 pairs over this half's columns [64 half + (c0 - 64 half) / 2, + 16): already read
+          const int pc = 64 * half + (c0 - 64 * half) / 2;
+          tmem_st16(tS + lane_off + pc, pw);
+          tmem_st16(tP + lane_off + pc, dw);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -364,21 +374,22 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       if (!ok) break;
       ++nout;
       tc_fence_after();
+      {
+        // half 0 writes the dV row, half 1 the dK row (scaled)
+        const uint32_t src = half ? tdK : tdV;
+        float* dst = half ? dk_row : dv_row;
+        const float mul = half ? p.scale : 1.f;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t vv[32], kv[32];
-        tmem_ld32(tdV + lane_off + c, vv);
-        tmem_ld32(tdK + lane_off + c, kv);
-        tmem_ld_wait();
-        if (keyok) {
+        for (int c = 0; c < D; c += 32) {
+          uint32_t vv[32];
+          tmem_ld32(src + lane_off + c, vv);
+          tmem_ld_wait();
+          if (keyok) {
 #pragma unroll
-          for (int u = 0; u < 32; u += 4) {
-            *reinterpret_cast<float4*>(dv_row + c + u) =
-                make_float4(__uint_as_float(vv[u]), __uint_as_float(vv[u + 1]), __uint_as_float(vv[u + 2]),
-                            __uint_as_float(vv[u + 3]));
-            *reinterpret_cast<float4*>(dk_row + c + u) =
-                make_float4(p.scale * __uint_as_float(kv[u]), p.scale * __uint_as_float(kv[u + 1]),
-                            p.scale * __uint_as_float(kv[u + 2]), p.scale * __uint_as_float(kv[u + 3]));
+            for (int u = 0; u < 32; u += 4)
+              *reinterpret_cast<float4*>(dst + c + u) =
+                  make_float4(mul * __uint_as_float(vv[u]), mul * __uint_as_float(vv[u + 1]),
+                              mul * __uint_as_float(vv[u + 2]), mul * __uint_as_float(vv[u + 3]));
           }
         }
       }
@@ -389,7 +400,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     tc_fence_after();
     tmem_dealloc(tb, 512);
   }
@@ -416,7 +427,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
   uint8_t* sV = smem + L::d_off;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) sb_init(bars, IS);
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     tmem_alloc(&bars.tmem_base, 512);
     tmem_relinquish();
   }
@@ -428,7 +439,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
   SbWaiter wait{&bars, &p.hdr->status, p.budget_ns};
   const int nitems = (p.hdr->status == 0) ? p.hdr->tiles_per_cluster : 0;
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       int iuse = 0, suse = 0;
@@ -466,7 +477,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       sb_drain(wait, bars.ifull, IS, iuse);
       sb_drain(wait, bars.sfull2, 2, suse);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
@@ -500,9 +511,9 @@ __global__ void __launch_bounds__(kSbThreads, 1)
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int s = 0; s < 8; ++s) umma_bf16_ts(tdQ, tS + s * 8, mndesc(kbase, s), idG, (cj | s) > 0);
+          for (int s = 0; s < 8; ++s) umma_bf16_ts(tdQ, sb_pairs(tS, s), mndesc(kbase, s), idG, (cj | s) > 0);
 #pragma unroll
-          for (int s = 0; s < 8; ++s) umma_bf16_ts(tdQ, tP + s * 8, mndesc(kbase, s), idG, 1u);
+          for (int s = 0; s < 8; ++s) umma_bf16_ts(tdQ, sb_pairs(tP, s), mndesc(kbase, s), idG, 1u);
           umma_commit(&bars.sempty2[ss]);
           ++suse;
           if (cj == kDqChain - 1 || j == nkt - 1) {
@@ -518,9 +529,10 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       wait(&bars.drain, 0, true);
     }
   } else {
-    // ---------------------------------------------------------------- target rows (warps 0-3)
-    const int r = threadIdx.x;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // ---------------------------------------------------------------- target rows (warps 0-7)
+    const int r = threadIdx.x & 127;     // target row (TMEM lane)
+    const int half = warp >> 2;          // key columns [64 half, 64 half + 64), dq columns [D/2 half, ...)
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c2 = p.scale * kLog2e;
     int npair = 0, nchain = 0;
     bool ok = true;
@@ -534,7 +546,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       const int64_t t = static_cast<int64_t>(p.cu_q[b]) + tq;
       float* dq_row = p.dq + (t * p.H + h) * D;
       if (nkt == 0) {  // no keys: the output is zero
-        if (tv)
+        if (tv && half == 0)
           for (int c = 0; c < D; c += 4) *reinterpret_cast<float4*>(dq_row + c) = make_float4(0.f, 0.f, 0.f, 0.f);
         continue;
       }
@@ -549,7 +561,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
         ++npair;
         tc_fence_after();
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
           uint32_t sv[32], dp[32];
           tmem_ld32(tS + lane_off + c0, sv);
           tmem_ld32(tP + lane_off + c0, dp);
@@ -568,9 +580,10 @@ __global__ void __launch_bounds__(kSbThreads, 1)
             hw[u / 2] = pack_bf16x2(hi[0], hi[1]);
             lw[u / 2] = pack_bf16x2(lo[0], lo[1]);
           }
-          // hi over S, lo over dP: columns [c0 / 2, c0 / 2 + 16) of each, all already read
-          tmem_st16(tS + lane_off + c0 / 2, hw);
-          tmem_st16(tP + lane_off + c0 / 2, lw);
+          // hi over S, lo over dP: this half's columns [64 half + (c0 - 64 half) / 2, + 16), already read
+          const int pc = 64 * half + (c0 - 64 * half) / 2;
+          tmem_st16(tS + lane_off + pc, hw);
+          tmem_st16(tP + lane_off + pc, lw);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -584,7 +597,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
           tc_fence_after();
           const bool first = j < kDqChain;
 #pragma unroll 1
-          for (int c = 0; c < D; c += 32) {
+          for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 32) {
             uint32_t qv[32];
             tmem_ld32(tdQ + lane_off + c, qv);
             tmem_ld_wait();
@@ -613,7 +626,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     tc_fence_after();
     tmem_dealloc(tb, 512);
   }
