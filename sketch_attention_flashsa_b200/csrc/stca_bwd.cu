@@ -16,10 +16,10 @@
 //     dP = dO V^T; thread = target row: P, dS = P (dP - delta) split into bf16 hi + lo (hi over S,
 //     lo over dP); dq += dS_hi K + dS_lo K in TMEM, restarted every kDqChain key tiles and added
 //     into the output row in fp32 (the tensor core's fp32 accumulation is not round-to-nearest).
-// Warps 0-7 do the row work, two warps per TMEM lane quarter, each on half of the 128 columns (its
-// bf16 pairs go over the first half of its own columns, so the halves never overwrite each other's
-// unread values; the MMAs read the A operand from both halves). Warp 8 lane 0 issues the TMA loads,
-// warp 9 lane 0 the MMAs. Operands that stay for a whole item (K/V, or Q/dO) and the streamed ones
+// Warps 0-15 do the row work, four warps per TMEM lane quarter, each on a group of 32 of the 128
+// columns (its bf16 pairs go over the first half of its own columns, so the groups never overwrite
+// each other's unread values; the MMAs read the A operand from all groups). Warp 16 lane 0 issues the
+// TMA loads, warp 17 lane 0 the MMAs. Operands that stay for a whole item (K/V, or Q/dO) and the streamed ones
 // are double-buffered where shared memory allows (d = 64; d = 128 keeps one item stage).
 #include <algorithm>
 #include <climits>
@@ -32,9 +32,11 @@ namespace ska {
 
 namespace {
 
-constexpr int kSbThreads = 320;
-constexpr int kRowWarps = 8;
-constexpr int kProdWarp = 8, kMmaWarp = 9;
+constexpr int kGroups = 4;               // column groups of the row work
+constexpr int kCw = 128 / kGroups;        // columns per group
+constexpr int kRowWarps = 4 * kGroups;
+constexpr int kSbThreads = 32 * (kRowWarps + 2);
+constexpr int kProdWarp = kRowWarps, kMmaWarp = kRowWarps + 1;
 constexpr uint32_t kSbBlk = 16384;  // [128 rows x 64 bf16] swizzled block
 constexpr int kDqChain = 16;        // key tiles per dq accumulation chain in TMEM
 constexpr float kLog2e = 1.4426950408889634f;
@@ -155,9 +157,12 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t base, int s) {
 // MN-major B operand (rows = the K index, D contiguous) of K step s (16 rows)
 __device__ __forceinline__ uint64_t mndesc(uint32_t base, int s) { return sw128_desc(base + s * 2048, kSbBlk, 1024); }
 
-// A operand (bf16 pairs in TMEM) of K step s over 128 columns packed by two halves: half h holds the
-// pairs of columns [64 h, 64 h + 64) in its own TMEM columns [64 h, 64 h + 32)
-__device__ __forceinline__ uint32_t sb_pairs(uint32_t t, int s) { return t + (s >> 2) * 64 + (s & 3) * 8; }
+// A operand (bf16 pairs in TMEM) of K step s over 128 columns packed by column groups: group g holds
+// the pairs of columns [kCw g, kCw (g + 1)) in its own TMEM columns [kCw g, kCw g + kCw / 2)
+__device__ __forceinline__ uint32_t sb_pairs(uint32_t t, int s) {
+  constexpr int kSteps = kCw / 16;  // K steps per group
+  return t + (s / kSteps) * kCw + (s % kSteps) * 8;
+}
 
 // ===================================================================== key-major: dK, dV
 template <int D>
@@ -282,7 +287,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
   } else {
     // ---------------------------------------------------------------- key rows (warps 0-7)
     const int r = threadIdx.x & 127;     // key row (TMEM lane)
-    const int half = warp >> 2;          // columns [64 half, 64 half + 64)
+    const int grp = warp >> 2;           // columns [kCw grp, kCw (grp + 1))
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c2 = p.scale * kLog2e;
     int npair = 0, nout = 0;
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       float* dk_row = sk ? p.dk_sk + ((static_cast<int64_t>(b) * p.H + h) * p.ks + (j - nh) * 128 + r) * D
                          : p.dk_hist + ((static_cast<int64_t>(p.cu_k[b]) + kk) * p.H + h) * D;
       if (nqt == 0) {  // no target reads these keys
-        if (keyok && half == 0)
+        if (keyok && grp == 0)
           for (int c = 0; c < D; c += 4) {
             *reinterpret_cast<float4*>(dv_row + c) = make_float4(0.f, 0.f, 0.f, 0.f);
             *reinterpret_cast<float4*>(dk_row + c) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -317,7 +322,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
         float* sLse = sMeta + m * 384;
         float* sDel = sLse + 128;
         int* sKvl = reinterpret_cast<int*>(sLse + 256);
-        if (half == 0) {
+        if (grp == 0) {
           const int tq = qt * 128 + r;
           const int64_t t = static_cast<int64_t>(p.cu_q[b]) + tq;
           const bool tv = tq < nt;
@@ -333,8 +338,8 @@ __global__ void __launch_bounds__(kSbThreads, 1)
         if (!ok) break;
         ++npair;
         tc_fence_after();
-#pragma unroll 1
-        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+        {
+          const int c0 = kCw * grp;
           uint32_t sv[32], dp[32];
           tmem_ld32(tS + lane_off + c0, sv);
           tmem_ld32(tP + lane_off + c0, dp);
@@ -359,10 +364,9 @@ __global__ void __launch_bounds__(kSbThreads, 1)
             dw[u / 2] = pack_bf16x2(ds[0], ds[1]);
             dw[u / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
           }
-          // bf16 pairs over this half's columns [64 half + (c0 - 64 half) / 2, + 16): already read
-          const int pc = 64 * half + (c0 - 64 * half) / 2;
-          tmem_st16(tS + lane_off + pc, pw);
-          tmem_st16(tP + lane_off + pc, dw);
+          // bf16 pairs over this group's first 16 columns (already read)
+          tmem_st16(tS + lane_off + c0, pw);
+          tmem_st16(tP + lane_off + c0, dw);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -375,12 +379,16 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       ++nout;
       tc_fence_after();
       {
-        // half 0 writes the dV row, half 1 the dK row (scaled)
-        const uint32_t src = half ? tdK : tdV;
-        float* dst = half ? dk_row : dv_row;
-        const float mul = half ? p.scale : 1.f;
+        // groups 0 .. kGroups/2 - 1 write the dV row, the others the dK row (scaled), D / (kGroups/2)
+        // columns each
+        constexpr int kCols = D / (kGroups / 2);
+        const bool isk = grp >= kGroups / 2;
+        const uint32_t src = isk ? tdK : tdV;
+        float* dst = isk ? dk_row : dv_row;
+        const float mul = isk ? p.scale : 1.f;
+        const int cbeg = (grp % (kGroups / 2)) * kCols;
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
+        for (int c = cbeg; c < cbeg + kCols; c += 32) {
           uint32_t vv[32];
           tmem_ld32(src + lane_off + c, vv);
           tmem_ld_wait();
@@ -531,7 +539,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
   } else {
     // ---------------------------------------------------------------- target rows (warps 0-7)
     const int r = threadIdx.x & 127;     // target row (TMEM lane)
-    const int half = warp >> 2;          // key columns [64 half, 64 half + 64), dq columns [D/2 half, ...)
+    const int grp = warp >> 2;           // key columns [kCw grp, kCw (grp + 1)), dq columns [D/kGroups grp, ...)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c2 = p.scale * kLog2e;
     int npair = 0, nchain = 0;
@@ -546,7 +554,7 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       const int64_t t = static_cast<int64_t>(p.cu_q[b]) + tq;
       float* dq_row = p.dq + (t * p.H + h) * D;
       if (nkt == 0) {  // no keys: the output is zero
-        if (tv && half == 0)
+        if (tv && grp == 0)
           for (int c = 0; c < D; c += 4) *reinterpret_cast<float4*>(dq_row + c) = make_float4(0.f, 0.f, 0.f, 0.f);
         continue;
       }
@@ -560,8 +568,8 @@ __global__ void __launch_bounds__(kSbThreads, 1)
         if (!ok) break;
         ++npair;
         tc_fence_after();
-#pragma unroll 1
-        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+        {
+          const int c0 = kCw * grp;
           uint32_t sv[32], dp[32];
           tmem_ld32(tS + lane_off + c0, sv);
           tmem_ld32(tP + lane_off + c0, dp);
@@ -580,10 +588,9 @@ __global__ void __launch_bounds__(kSbThreads, 1)
             hw[u / 2] = pack_bf16x2(hi[0], hi[1]);
             lw[u / 2] = pack_bf16x2(lo[0], lo[1]);
           }
-          // hi over S, lo over dP: this half's columns [64 half + (c0 - 64 half) / 2, + 16), already read
-          const int pc = 64 * half + (c0 - 64 * half) / 2;
-          tmem_st16(tS + lane_off + pc, hw);
-          tmem_st16(tP + lane_off + pc, lw);
+          // hi over S, lo over dP: this group's first 16 columns of each (already read)
+          tmem_st16(tS + lane_off + c0, hw);
+          tmem_st16(tP + lane_off + c0, lw);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -597,13 +604,13 @@ __global__ void __launch_bounds__(kSbThreads, 1)
           tc_fence_after();
           const bool first = j < kDqChain;
 #pragma unroll 1
-          for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 32) {
-            uint32_t qv[32];
-            tmem_ld32(tdQ + lane_off + c, qv);
+          for (int c = grp * (D / kGroups); c < (grp + 1) * (D / kGroups); c += 16) {
+            uint32_t qv[16];
+            tmem_ld16(tdQ + lane_off + c, qv);
             tmem_ld_wait();
             if (tv) {
 #pragma unroll
-              for (int u = 0; u < 32; u += 4) {
+              for (int u = 0; u < 16; u += 4) {
                 float4 a = make_float4(p.scale * __uint_as_float(qv[u]), p.scale * __uint_as_float(qv[u + 1]),
                                        p.scale * __uint_as_float(qv[u + 2]), p.scale * __uint_as_float(qv[u + 3]));
                 if (!first) {
