@@ -19,9 +19,11 @@ differences; none of them re-types the formulas below.
 from .sa import (sa_forward_proto, sa_forward_token, sa_backward_proto,
                  sa_backward_token, sa_forward, sa_backward, sa_problem)
 from .stca import stca_forward, stca_backward
+from .diag import token_max_weight, weight_histogram, renormalized_sketch
 from .refine import layer_norm, swish, swiglu_ffn, refine, project_queries, stacked_sa
 
 __all__ = ["sa_forward_proto", "sa_forward_token", "sa_backward_proto",
            "sa_backward_token", "sa_forward", "sa_backward", "sa_problem",
-           "stca_forward", "stca_backward", "layer_norm", "swish", "swiglu_ffn", "refine", "project_queries",
+           "stca_forward", "stca_backward", "token_max_weight", "weight_histogram", "renormalized_sketch",
+           "layer_norm", "swish", "swiglu_ffn", "refine", "project_queries",
            "stacked_sa"]

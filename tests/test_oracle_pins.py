@@ -566,3 +566,42 @@ def test_stca_backward_matches_finite_differences(with_kv_len):
         for rows in (slice(2, 4), slice(8, 9)):
             assert not grads[1][rows].any() and not grads[2][rows].any()
         assert grads[1][0:2].any() and grads[2][4:8].any()
+
+
+# ------------------------------------------------------------- allocation diagnostics (Fig. 3, §2.4)
+
+def test_token_max_weight_hand_example():
+    """The hand example's PROTO columns are [1/4, 3/4], [2/3, 1/3], [1/4, 3/4]: maxima 3/4, 2/3, 3/4."""
+    mw = oracle.token_max_weight(HAND_Q, HAND_K, HAND_V, HAND_CU)
+    np.testing.assert_allclose(mw[:, 0], [0.75, 2.0 / 3.0, 0.75], atol=1e-15)
+
+
+def test_token_max_weight_bounds_and_even_split():
+    """Each token's weights sum to 1 over k prototypes, so its maximum lies in [1/k, 1]; with zero
+    queries it is exactly 1/k. Padding rows carry -1."""
+    q, k, v, cu = _rand_problem([7, 5], H=2, kp=5, seed=90)
+    mw = oracle.token_max_weight(q, k, v, cu, [7, 3], 1.0)
+    valid = np.r_[np.ones(7, bool), np.ones(3, bool), np.zeros(2, bool)]
+    assert (mw[valid] >= 1 / 5 - 1e-15).all() and (mw[valid] <= 1).all()
+    assert (mw[~valid] == -1).all()
+    np.testing.assert_allclose(oracle.token_max_weight(np.zeros_like(q), k, v, cu)[:, :], 0.2, atol=1e-15)
+
+
+def test_weight_histogram_counts():
+    vals = np.array([0.0, 0.1, 0.5, 0.999, 1.0, 0.25, -1.0, -1.0])
+    assert list(oracle.weight_histogram(vals, 4)) == [2, 1, 1, 2]   # [0,.25): 0, .1; [.25,.5): .25; ...
+    assert oracle.weight_histogram(vals, 4).sum() == 6                 # padding (-1) is skipped
+
+
+def test_renormalized_sketch_is_a_weighted_mean():
+    """Hand example: sketch row j = sum_i A_ji v_i and mass_j = sum_i A_ji, so the renormalised
+    row is the A-weighted mean of the values; with all values equal it is that value."""
+    sk, _, mass = oracle.sa_forward_proto(HAND_Q, HAND_K, HAND_V, HAND_CU)
+    r = oracle.renormalized_sketch(sk, mass)
+    A = np.array([[0.25, 2 / 3, 0.25], [0.75, 1 / 3, 0.75]])
+    want = (A @ HAND_V[:, 0]) / A.sum(axis=1)[:, None]
+    np.testing.assert_allclose(r[0, 0], want, atol=1e-14)
+    same = np.broadcast_to(np.array([[[2.0, -1.0]]]), HAND_V.shape)
+    sk2, _, m2 = oracle.sa_forward_proto(HAND_Q, HAND_K, same, HAND_CU)
+    np.testing.assert_allclose(oracle.renormalized_sketch(sk2, m2)[0, 0], [[2.0, -1.0]] * 2, atol=1e-14)
+    assert not oracle.renormalized_sketch(np.ones((1, 1, 2, 3)), np.array([[[0.0, 2.0]]]))[0, 0, 0].any()
