@@ -137,6 +137,25 @@ SKA_API ska_status sa_forward(const ska_sa_desc* desc, const void* q, const void
                       const int32_t* cu_seqlens, const int32_t* seqused, float* sketch, float* lse,
                       float* mass, void* ws, size_t ws_bytes, void* stream);
 
+/* SA forward with the allocation diagnostics (prototype-wise normalisation only; SKA_NORM_TOKEN
+ * returns SKA_ERR_UNSUPPORTED). Arguments as in sa_forward (same workspace size), plus:
+ *   token_max_weight  out, fp32 [total_tokens, H] or NULL: max_j A[j, i] for every token i, the
+ *                     "maximum normalized weight" whose distribution §5.1 / Fig. 3 reports; it lies
+ *                     in [1/k, 1]; -1 on padding rows
+ *   renormalize       nonzero: the sketch rows become sum_i A[j,i] v_i / sum_i A[j,i], the
+ *                     mass-weighted mean of the values (the Slot-Attention reading of the
+ *                     normalisation that §2.4 compares SA with); zero rows for zero mass. mass must
+ *                     then be given (it holds the divisors).                                      */
+SKA_API ska_status sa_forward_diag(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
+                                   const int32_t* cu_seqlens, const int32_t* seqused, float* sketch, float* lse,
+                                   float* mass, float* token_max_weight, int32_t renormalize, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* Histogram of n fp32 values in [0, 1] (e.g. token_max_weight): counts[b], int32, zeroed by the call,
+ * is the number of values in [b / bins, (b + 1) / bins), 1.0 counted in the last bin; negative
+ * (padding) and NaN values are skipped. 1 <= bins <= 4096. Counts are exact (integer sums).     */
+SKA_API ska_status sa_weight_histogram(const float* values, int64_t n, int32_t bins, int32_t* counts, void* stream);
+
 /* Bytes of workspace sa_backward needs (0 if the descriptor is invalid). */
 SKA_API size_t sa_backward_workspace_size(const ska_sa_desc* desc);
 

@@ -25,7 +25,7 @@ EXPORTED = ("sa_forward_workspace_size", "sa_forward", "sa_backward_workspace_si
             "ska_read_device_status", "ska_set_debug", "ska_set_timing_events",
             "sa_forward_noalloc", "sa_forward_noalloc_scratch_bytes", "sa_forward_noalloc_read_status",
             "ska_last_error_string", "sa_refine_workspace_size", "sa_refine", "sa_project_queries",
-            "stca_backward_workspace_size", "stca_backward")
+            "stca_backward_workspace_size", "stca_backward", "sa_forward_diag", "sa_weight_histogram")
 
 
 class SaDesc(ctypes.Structure):
@@ -99,6 +99,11 @@ def lib() -> ctypes.CDLL:
     L.sa_forward_noalloc_scratch_bytes.restype = sz
     L.sa_forward_noalloc_read_status.argtypes = [vp]
     L.sa_forward_noalloc_read_status.restype = ctypes.c_int
+    L.sa_forward_diag.argtypes = [ctypes.POINTER(SaDesc), vp, vp, vp, i32p, i32p, vp, vp, vp, vp, ctypes.c_int32,
+                                  vp, sz, vp]
+    L.sa_forward_diag.restype = ctypes.c_int
+    L.sa_weight_histogram.argtypes = [vp, ctypes.c_int64, ctypes.c_int32, vp, vp]
+    L.sa_weight_histogram.restype = ctypes.c_int
     L.stca_backward_workspace_size.argtypes = [ctypes.POINTER(StcaDesc)]
     L.stca_backward_workspace_size.restype = sz
     L.stca_backward.argtypes = [ctypes.POINTER(StcaDesc)] + [vp] * 17 + [sz, vp]

@@ -139,6 +139,49 @@ def sa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: to
     return sketch, lse, mass
 
 
+def sa_forward_diag(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                    seqused: Optional[torch.Tensor] = None, *, scale: float = 1.0, want_max_weight: bool = True,
+                    renormalize: bool = False, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Prototype-wise SA forward with the allocation diagnostics: each token's largest weight
+    max_j A[j,i] (SequenceO1 §5.1 Fig. 3; -1 on padding rows) and, with `renormalize`, the sketch
+    rows divided by their mass (the Slot-Attention weighted mean, §2.4).
+    Returns (sketch [B,H,k,d], lse [T,H], mass [B,H,k], max_weight [T,H] or None)."""
+    B, H, kp, D = _check_sa_inputs(q, k, v, cu_seqlens, seqused, (torch.bfloat16, torch.float32))
+    T = k.shape[0]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _dev_tensor(name, t, (torch.bfloat16, torch.float32))
+    _dev_tensor("cu_seqlens", cu_seqlens, (torch.int32,))
+    _dev_tensor("seqused", seqused, (torch.int32,))
+    desc = sa_desc(q, k, cu_seqlens, scale=scale, norm="proto")
+    dev = k.device
+    need = sa_forward_workspace_size(desc)
+    if need == 0 and B > 0:
+        raise SkaError(_lib.SKA_ERR_UNSUPPORTED, "sa_forward_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    sketch = torch.empty((B, H, kp, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((T, H), dtype=torch.float32, device=dev)
+    mass = torch.empty((B, H, kp), dtype=torch.float32, device=dev)
+    mw = torch.empty((T, H), dtype=torch.float32, device=dev) if want_max_weight else None
+    rc = _lib.lib().sa_forward_diag(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(seqused),
+                                    _ptr(sketch), _ptr(lse), _ptr(mass), _ptr(mw), 1 if renormalize else 0,
+                                    _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check(rc, "sa_forward_diag")
+    return sketch, lse, mass, mw
+
+
+def weight_histogram(values: torch.Tensor, bins: int, *, out: Optional[torch.Tensor] = None, stream=None):
+    """Counts of the values in `bins` equal bins over [0, 1] (1.0 in the last; negative values and
+    NaN skipped), as int32 on the device."""
+    _dev_tensor("values", values, (torch.float32,))
+    counts = torch.empty(bins, dtype=torch.int32, device=values.device) if out is None else out
+    _shape("out", counts, (bins,))
+    _dev_tensor("out", counts, (torch.int32,))
+    rc = _lib.lib().sa_weight_histogram(_ptr(values), int(values.numel()), int(bins), _ptr(counts), _stream(stream))
+    _check(rc, "sa_weight_histogram")
+    return counts
+
+
 def sa_forward_noalloc(q, k, v, cu_seqlens, seqused=None, *, scale: float = 1.0, norm="proto", out=None,
                        lse_out=None, mass_out=None, stream=None):
     """sa_forward for callers that cannot allocate device memory: scratch comes from a fixed array

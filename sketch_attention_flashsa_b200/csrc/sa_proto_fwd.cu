@@ -440,6 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (threadIdx.x == 128) mbar_expect_tx(&bars.xbar[xs], kXBytesPerTile * CS);  // arms tile i + 4
       if (p.lse && valid && rank == 0 && tok < p.total_tokens)
         p.lse[static_cast<int64_t>(tok) * p.H + t.h] = (M + __log2f(Lsum)) * 0.69314718055994531f;
+      // the token's largest weight over all k prototypes is 2^(M - M) / L
+      if (p.maxw && valid && rank == 0 && tok < p.total_tokens)
+        p.maxw[static_cast<int64_t>(tok) * p.H + t.h] = 1.f / Lsum;
 
       ok = __all_sync(0xffffffffu, wait(&bars.vfull[vent], (vuse / p.nv_entries) & 1));
       if (!ok) break;

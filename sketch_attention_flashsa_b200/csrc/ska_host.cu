@@ -410,20 +410,23 @@ size_t sa_forward_workspace_size(const ska_sa_desc* d) {
   return total;
 }
 
-ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
-                      const int32_t* seqused, float* sketch, float* lse, float* mass, void* ws, size_t ws_bytes,
-                      void* stream) {
+// sa_forward, plus (prototype-wise only) each token's largest weight and the mass-renormalised sketch.
+static ska_status sa_forward_impl(const ska_sa_desc* d, const void* q, const void* k, const void* v,
+                                  const int32_t* cu_seqlens, const int32_t* seqused, float* sketch, float* lse,
+                                  float* mass, float* maxw, bool renormalize, void* ws, size_t ws_bytes, void* stream) {
   ska_status st = check_sa_desc(d);
   if (st != SKA_OK) return st;
   const int B = d->num_users, H = d->num_heads, D = d->head_dim, kp = d->num_protos;
   const int64_t T = d->total_tokens;
+  if ((maxw || renormalize) && d->norm != SKA_NORM_PROTO) return SKA_ERR_UNSUPPORTED;
   if (B == 0) return SKA_OK;
   // pointers and alignment
   if (!q || !cu_seqlens || !sketch || !ws) return SKA_ERR_INVALID_VALUE;
   if (T > 0 && (!k || !v)) return SKA_ERR_INVALID_VALUE;
+  if (renormalize && !mass) return SKA_ERR_INVALID_VALUE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(sketch) || !aligned16(lse) ||
-      !aligned16(mass) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
-      (reinterpret_cast<uintptr_t>(seqused) & 3u))
+      !aligned16(mass) || !aligned16(maxw) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(seqused) & 3u))
     return SKA_ERR_INVALID_VALUE;
   // outputs against inputs and each other (host-only checks, before any device query)
   const size_t esz = d->in_dtype == SKA_F32 ? 4 : 2;
@@ -439,13 +442,19 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
       overlaps(mass, mass_bytes, k, kvn * esz) || overlaps(mass, mass_bytes, v, kvn * esz) ||
       overlaps(mass, mass_bytes, sketch, sk_bytes) || overlaps(mass, mass_bytes, lse, lse_bytes))
     return SKA_ERR_INVALID_VALUE;
+  const size_t mw_bytes = size_t(T) * H * 4;
+  if (overlaps(maxw, mw_bytes, q, qn * esz) || overlaps(maxw, mw_bytes, k, kvn * esz) ||
+      overlaps(maxw, mw_bytes, v, kvn * esz) || overlaps(maxw, mw_bytes, sketch, sk_bytes) ||
+      overlaps(maxw, mw_bytes, lse, lse_bytes) || overlaps(maxw, mw_bytes, mass, mass_bytes))
+    return SKA_ERR_INVALID_VALUE;
   if (no_device()) return SKA_ERR_CUDA;
   const size_t ws_need = sa_forward_workspace_size(d);
   if (ws_need == 0) return SKA_ERR_UNSUPPORTED;
   if (ws_bytes < ws_need) return SKA_ERR_WORKSPACE_TOO_SMALL;
   if (overlaps(ws, ws_need, sketch, sk_bytes) || overlaps(ws, ws_need, lse, lse_bytes) ||
       overlaps(ws, ws_need, q, qn * esz) || overlaps(ws, ws_need, k, kvn * esz) ||
-      overlaps(ws, ws_need, v, kvn * esz) || overlaps(mass, mass_bytes, ws, ws_need))
+      overlaps(ws, ws_need, v, kvn * esz) || overlaps(mass, mass_bytes, ws, ws_need) ||
+      overlaps(maxw, mw_bytes, ws, ws_need))
     return SKA_ERR_INVALID_VALUE;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -493,6 +502,7 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
     p.partial = partial;
     p.lse = lse;
     p.mass_partial = mass ? mass_partial : nullptr;
+    p.maxw = maxw;
     p.B = B;
     p.H = H;
     p.k = kp;
@@ -514,13 +524,41 @@ ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const 
     }
   }
   if (cudaError_t e_ = launch_proto_combine(prefix, hdr, partial, mass ? mass_partial : nullptr, B, H, kp, D, sketch,
-                                            mass, s);
+                                            mass, renormalize, s);
       e_ != cudaSuccess) {
     record_error("launch_proto_combine", e_);
     return SKA_ERR_CUDA;
   }
-  if (lse && T > 0) {
-    if (cudaError_t e_ = launch_fill_padding_lse(cu_seqlens, seqused, B, H, T, lse, s); e_ != cudaSuccess) { record_error("launch_fill_padding_lse", e_); return SKA_ERR_CUDA; }
+  if ((lse || maxw) && T > 0) {
+    if (cudaError_t e_ = launch_fill_padding_lse(cu_seqlens, seqused, B, H, T, lse, maxw, s); e_ != cudaSuccess) { record_error("launch_fill_padding_lse", e_); return SKA_ERR_CUDA; }
+  }
+  return SKA_OK;
+}
+
+ska_status sa_forward(const ska_sa_desc* d, const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                      const int32_t* seqused, float* sketch, float* lse, float* mass, void* ws, size_t ws_bytes,
+                      void* stream) {
+  return sa_forward_impl(d, q, k, v, cu_seqlens, seqused, sketch, lse, mass, nullptr, false, ws, ws_bytes, stream);
+}
+
+ska_status sa_forward_diag(const ska_sa_desc* d, const void* q, const void* k, const void* v,
+                           const int32_t* cu_seqlens, const int32_t* seqused, float* sketch, float* lse, float* mass,
+                           float* token_max_weight, int32_t renormalize, void* ws, size_t ws_bytes, void* stream) {
+  return sa_forward_impl(d, q, k, v, cu_seqlens, seqused, sketch, lse, mass, token_max_weight, renormalize != 0, ws,
+                         ws_bytes, stream);
+}
+
+ska_status sa_weight_histogram(const float* values, int64_t n, int32_t bins, int32_t* counts, void* stream) {
+  if (n < 0 || bins < 1 || bins > 4096) return SKA_ERR_INVALID_VALUE;
+  if (!counts || (n > 0 && !values)) return SKA_ERR_INVALID_VALUE;
+  if ((reinterpret_cast<uintptr_t>(values) & 3u) || (reinterpret_cast<uintptr_t>(counts) & 3u))
+    return SKA_ERR_INVALID_VALUE;
+  if (overlaps(values, size_t(n) * 4, counts, size_t(bins) * 4)) return SKA_ERR_INVALID_VALUE;
+  if (no_device()) return SKA_ERR_CUDA;
+  if (cudaError_t e = launch_weight_histogram(values, n, bins, counts, static_cast<cudaStream_t>(stream));
+      e != cudaSuccess) {
+    record_error("weight histogram launch", e);
+    return SKA_ERR_CUDA;
   }
   return SKA_OK;
 }

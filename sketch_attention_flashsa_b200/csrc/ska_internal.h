@@ -31,6 +31,7 @@ struct ProtoFwdParams {
   float* partial;              // [(num_segments + num_clusters) * k * D] fp32
   float* lse;                  // [T, H] or null
   float* mass_partial;         // [(num_segments + num_clusters) * k] or null
+  float* maxw;                 // [T, H] or null: each token's largest weight, 1 / L (Fig. 3 diagnostic)
   int B, H, k;
   int total_tokens;
   int q_per_user;
@@ -193,11 +194,16 @@ cudaError_t launch_schedule(const int32_t* cu_seqlens, const int32_t* seqused, i
                             int num_clusters, int32_t* tile_prefix, WsHeader* hdr, cudaStream_t stream);
 // Also marks the call SKA_ERR_RANGE in hdr->status when a summed sketch value is not finite (an
 // fp16 overflow of a scaled value row), and writes NaN when hdr->status reports an error.
+// With `renormalize` every sketch row is divided by its prototype's mass (zero rows for zero mass).
 cudaError_t launch_proto_combine(const int32_t* tile_prefix, WsHeader* hdr, const float* partial,
                                  const float* mass_partial, int B, int H, int k, int D, float* sketch,
-                                 float* mass, cudaStream_t stream);
+                                 float* mass, bool renormalize, cudaStream_t stream);
+// -inf lse and -1 maximum weight (either may be null) on the padding rows of every user.
 cudaError_t launch_fill_padding_lse(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,
-                                    int64_t T, float* lse, cudaStream_t stream);
+                                    int64_t T, float* lse, float* maxw, cudaStream_t stream);
+// counts[b] (zeroed first) = number of values in [b / bins, (b + 1) / bins), 1.0 in the last bin;
+// negative and NaN values are skipped.
+cudaError_t launch_weight_histogram(const float* values, int64_t n, int bins, int32_t* counts, cudaStream_t stream);
 cudaError_t launch_cast_f32_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream);
 
 }  // namespace ska

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restric
 __global__ void proto_combine_kernel(const int32_t* __restrict__ prefix, WsHeader* __restrict__ hdr,
                                      const float* __restrict__ partial, const float* __restrict__ mass_partial,
                                      int B, int H, int k, int D, float* __restrict__ sketch,
-                                     float* __restrict__ mass) {
+                                     float* __restrict__ mass, bool renormalize) {
   const int s = blockIdx.x;
   const bool failed = *reinterpret_cast<volatile int32_t*>(&hdr->status) != 0;
   bool finite = true;
@@ -83,6 +83,14 @@ __global__ void proto_combine_kernel(const int32_t* __restrict__ prefix, WsHeade
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
     finite = finite && isfinite(acc.x) && isfinite(acc.y) && isfinite(acc.z) && isfinite(acc.w);
+    if (renormalize) {
+      // the prototype's mass, summed in the same order as its mass output
+      const int j = static_cast<int>(e / D);
+      float mj = 0.f;
+      for (int pc = p0; pc <= p1; ++pc) mj += mass_partial[static_cast<int64_t>(s + pc) * k + j];
+      const float inv = mj > 0.f ? 1.f / mj : 0.f;
+      acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+    }
     if (failed) acc = make_float4(NAN, NAN, NAN, NAN);
     *reinterpret_cast<float4*>(sketch + static_cast<int64_t>(s) * per + e) = acc;
   }
@@ -97,16 +105,38 @@ __global__ void proto_combine_kernel(const int32_t* __restrict__ prefix, WsHeade
   if (!finite && !failed) atomicCAS(&hdr->status, 0, static_cast<int>(SKA_ERR_RANGE));
 }
 
-// lse rows of padding tokens (positions >= seqused[b] inside user b) are -inf.
+// lse rows of padding tokens (positions >= seqused[b] inside user b) are -inf, their maximum
+// weights -1.
 __global__ void fill_padding_lse_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ seqused,
-                                        int B, int H, int64_t T, float* __restrict__ lse) {
+                                        int B, int H, int64_t T, float* __restrict__ lse, float* __restrict__ maxw) {
   const int b = blockIdx.x;
   if (b >= B) return;
   const int64_t lo = cu[b] + used_len(cu, seqused, b);
   const int64_t hi = (static_cast<int64_t>(cu[b + 1]) < T) ? static_cast<int64_t>(cu[b + 1]) : T;
   if (hi <= lo) return;
   const int64_t n = static_cast<int64_t>(hi - lo) * H;
-  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) lse[lo * H + i] = -INFINITY;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+    if (lse) lse[lo * H + i] = -INFINITY;
+    if (maxw) maxw[lo * H + i] = -1.f;
+  }
+}
+
+// Histogram of values in [0, 1]: per-block counts in shared memory, then added into the global
+// counts (integer additions: the result does not depend on their order).
+__global__ void weight_histogram_kernel(const float* __restrict__ v, int64_t n, int bins, int32_t* __restrict__ counts) {
+  extern __shared__ int32_t local[];
+  for (int b = threadIdx.x; b < bins; b += blockDim.x) local[b] = 0;
+  __syncthreads();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float x = v[i];
+    if (!(x >= 0.f)) continue;  // padding (-1) and NaN
+    const int b = min(static_cast<int>(x * bins), bins - 1);
+    atomicAdd(&local[b], 1);
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < bins; b += blockDim.x)
+    if (local[b]) atomicAdd(&counts[b], local[b]);
 }
 
 __global__ void cast_f32_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t n) {
@@ -125,18 +155,28 @@ cudaError_t launch_schedule(const int32_t* cu, const int32_t* seqused, int B, in
 
 cudaError_t launch_proto_combine(const int32_t* prefix, WsHeader* hdr, const float* partial,
                                  const float* mass_partial, int B, int H, int k, int D, float* sketch,
-                                 float* mass, cudaStream_t stream) {
+                                 float* mass, bool renormalize, cudaStream_t stream) {
   const int per4 = (k * D) / 4;
   const int threads = 256;
   const int bx = std::min(32, (per4 + threads - 1) / threads);
   dim3 grid(B * H, bx, 1);
-  proto_combine_kernel<<<grid, threads, 0, stream>>>(prefix, hdr, partial, mass_partial, B, H, k, D, sketch, mass);
+  proto_combine_kernel<<<grid, threads, 0, stream>>>(prefix, hdr, partial, mass_partial, B, H, k, D, sketch, mass,
+                                                     renormalize);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fill_padding_lse(const int32_t* cu, const int32_t* seqused, int B, int H, int64_t T,
-                                    float* lse, cudaStream_t stream) {
-  fill_padding_lse_kernel<<<B, 256, 0, stream>>>(cu, seqused, B, H, T, lse);
+                                    float* lse, float* maxw, cudaStream_t stream) {
+  fill_padding_lse_kernel<<<B, 256, 0, stream>>>(cu, seqused, B, H, T, lse, maxw);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weight_histogram(const float* values, int64_t n, int bins, int32_t* counts, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(counts, 0, size_t(bins) * sizeof(int32_t), stream);
+  if (e != cudaSuccess || n == 0) return e;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 4);
+  weight_histogram_kernel<<<static_cast<unsigned>(blocks), 256, size_t(bins) * sizeof(int32_t), stream>>>(
+      values, n, bins, counts);
   return cudaGetLastError();
 }
 

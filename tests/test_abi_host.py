@@ -300,3 +300,28 @@ def test_stca_backward_without_a_device_reports_cuda_error():
     if torch.cuda.is_available():
         pytest.skip("a device is present")
     assert stca_bwd(stca_desc()) == L.SKA_ERR_CUDA
+
+
+def diag(desc, mw=12 * A, renorm=0, mass=11 * A, **kw):
+    args = dict(q=A, k=2 * A, v=3 * A, cu=4 * A, su=None, sk=5 * A, lse=6 * A, ws=256 * A)
+    args.update(kw)
+    return L.lib().sa_forward_diag(ctypes.byref(desc), args["q"], args["k"], args["v"], args["cu"], args["su"],
+                                   args["sk"], args["lse"], mass, mw, renorm, args["ws"], 1 << 30, None)
+
+
+def test_forward_diag_and_histogram_host_checks():
+    assert diag(sa_desc(norm=L.SKA_NORM_TOKEN)) == UNSUP          # prototype-wise only
+    assert diag(sa_desc(norm=L.SKA_NORM_TOKEN), mw=None, renorm=1) == UNSUP
+    assert diag(sa_desc(), renorm=1, mass=None) == INVALID        # the divisors are the mass output
+    assert diag(sa_desc(), mw=12 * A + 8) == INVALID              # alignment
+    assert diag(sa_desc(), mw=5 * A + 64) == INVALID              # overlaps the sketch
+    h = L.lib().sa_weight_histogram
+    assert h(None, 10, 4, 20 * A, None) == INVALID
+    assert h(21 * A, 10, 0, 20 * A, None) == INVALID
+    assert h(21 * A, 10, 5000, 20 * A, None) == INVALID
+    assert h(21 * A, -1, 4, 20 * A, None) == INVALID
+    assert h(21 * A, 10, 4, 21 * A + 8, None) == INVALID          # counts overlap the values
+    import torch
+    if not torch.cuda.is_available():
+        assert diag(sa_desc()) == L.SKA_ERR_CUDA
+        assert h(21 * A, 10, 4, 20 * A, None) == L.SKA_ERR_CUDA
