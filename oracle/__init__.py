@@ -20,10 +20,11 @@ from .sa import (sa_forward_proto, sa_forward_token, sa_backward_proto,
                  sa_backward_token, sa_forward, sa_backward, sa_problem)
 from .stca import stca_forward, stca_backward
 from .diag import token_max_weight, weight_histogram, renormalized_sketch
+from .cache import SketchCache, splitmix64, key_hash
 from .refine import layer_norm, swish, swiglu_ffn, refine, project_queries, stacked_sa
 
 __all__ = ["sa_forward_proto", "sa_forward_token", "sa_backward_proto",
            "sa_backward_token", "sa_forward", "sa_backward", "sa_problem",
            "stca_forward", "stca_backward", "token_max_weight", "weight_histogram", "renormalized_sketch",
-           "layer_norm", "swish", "swiglu_ffn", "refine", "project_queries",
+           "SketchCache", "splitmix64", "key_hash", "layer_norm", "swish", "swiglu_ffn", "refine", "project_queries",
            "stacked_sa"]

@@ -605,3 +605,49 @@ def test_renormalized_sketch_is_a_weighted_mean():
     sk2, _, m2 = oracle.sa_forward_proto(HAND_Q, HAND_K, same, HAND_CU)
     np.testing.assert_allclose(oracle.renormalized_sketch(sk2, m2)[0, 0], [[2.0, -1.0]] * 2, atol=1e-14)
     assert not oracle.renormalized_sketch(np.ones((1, 1, 2, 3)), np.array([[[0.0, 2.0]]]))[0, 0, 0].any()
+
+
+# ------------------------------------------------------------------------ sketch cache (§4.1)
+
+def test_splitmix64_published_vectors():
+    """The first three outputs of SplitMix64 from seed 0 (the generator's reference test vectors)."""
+    g = 0x9E3779B97F4A7C15
+    assert oracle.splitmix64(0) == 0xE220A8397B1DCDAF
+    assert oracle.splitmix64(g) == 0x6E789E6AA1B965F4
+    assert oracle.splitmix64((2 * g) & ((1 << 64) - 1)) == 0x06C45D188009454F
+
+
+def test_cache_hand_worked_sequence():
+    """One set of two ways, ttl 10: A at t=0 and B at t=1 both hit; C at t=2 evicts the oldest (A);
+    at t=12 B (stored at 1) has expired, so D at t=12 takes B's way, not C's; re-putting C keeps
+    its way and refreshes its time."""
+    c = oracle.SketchCache(1, 2, 3, 10)
+    A, B, C, D = (1, 7, 0, 100), (2, 7, 0, 100), (3, 7, 0, 100), (4, 7, 0, 100)
+    row = lambda x: np.full(3, float(x))  # noqa: E731
+    assert c.put([A, B], [row(1), row(2)], 0) == [0, 1]
+    hits, rows = c.get([A, B, C], 1)
+    assert list(hits) == [True, True, False] and rows[1][0] == 2.0
+    assert c.put([C], [row(3)], 2) == [0]                 # A (time 0) is the oldest
+    assert list(c.get([A, C], 2)[0]) == [False, True]
+    assert list(c.get([B], 12)[0]) == [False]             # 12 - 1 > 10
+    assert list(c.get([C], 12)[0]) == [True]              # 12 - 2 <= 10
+    assert c.put([D], [row(4)], 12) == [1]                # B's way: expired before the oldest rule
+    assert c.put([C], [row(5)], 13) == [0]                # same key, same way, new data and time
+    hits, rows = c.get([C, D], 22)                          # 22 - 12 = 10: D still live
+    assert list(hits) == [True, True] and rows[0][0] == 5.0 and rows[1][0] == 4.0
+    assert list(c.get([C, D], 23)[0]) == [True, False]     # 23 - 12 > 10
+    # at 24 both ways have expired: the first (way 0) takes A; a duplicate in the same batch is the
+    # same key, so it lands on the same way and the later data wins
+    assert c.put([A, A], [row(6), row(7)], 24) == [0, 0]
+    assert c.get([A], 24)[1][0][0] == 7.0
+
+
+def test_cache_keys_differ_by_every_field():
+    """Version, configuration and history timestamp are all part of the key (a new model version or
+    a newer history must not hit an old sketch)."""
+    c = oracle.SketchCache(4, 4, 2, 100)
+    base = (5, 1, 2, 3)
+    c.put([base], [np.ones(2)], 0)
+    for other in [(6, 1, 2, 3), (5, 2, 2, 3), (5, 1, 3, 3), (5, 1, 2, 4)]:
+        assert not c.get([other], 0)[0][0]
+    assert c.get([base], 0)[0][0]
