@@ -293,6 +293,47 @@ SKA_API ska_status sa_project_queries(int32_t num_users, int32_t num_heads, int3
                                       const float* x, const void* w_q, void* q_out, void* ws,
                                       size_t ws_bytes, void* stream);
 
+/* Sketch cache (§4.1): the user-only sketch X~_u (any fixed number of floats per user, e.g.
+ * H x k x d) cached in device memory, keyed by user id, model version, history timestamp and sketch
+ * configuration, with TTL invalidation and capacity eviction, one get/put interface for training
+ * and serving.
+ * Layout: num_sets sets (a power of two, <= 2^24) of `ways` ways (1..32); a key's set is SplitMix64
+ * folded over the four key fields (user id, version, configuration, timestamp, in that order, each
+ * mixed in by xor), masked to num_sets - 1. Times are the caller's integer clock (e.g. seconds);
+ * an entry stored at time t is live while now - t <= ttl.
+ *   get: a key hits when a way of its set holds it live; its row is copied out (a miss: zeros).
+ *   put: keys are applied in batch order: a way holding the same key is overwritten, else the
+ *        first empty or expired way is used, else the oldest (ties: the lowest way).
+ * The cache memory is the caller's (sa_cache_bytes, 256-byte aligned); calls on one cache must be
+ * ordered on one stream. row_floats is a multiple of 4; rows are 16-byte aligned.                 */
+typedef struct {
+  uint64_t user_id;
+  uint32_t model_version;
+  uint32_t sketch_config;
+  int64_t history_timestamp;
+} ska_cache_key;
+
+typedef struct {
+  int32_t num_sets;
+  int32_t ways;
+  int32_t row_floats;
+  int32_t reserved;
+  int64_t ttl;
+} ska_cache_desc;
+
+/* Bytes of device memory a cache needs (0 if the descriptor is invalid). */
+SKA_API size_t sa_cache_bytes(const ska_cache_desc* desc);
+/* Marks every way empty. */
+SKA_API ska_status sa_cache_init(const ska_cache_desc* desc, void* cache, size_t cache_bytes, void* stream);
+/* keys: device array of n keys; rows: fp32 [n, row_floats]; slots: out, int32 [n], the slot
+ * (set * ways + way) each key was written to. */
+SKA_API ska_status sa_cache_put(const ska_cache_desc* desc, void* cache, size_t cache_bytes, const ska_cache_key* keys,
+                                const float* rows, int32_t n, int64_t now, int32_t* slots, void* stream);
+/* out: fp32 [n, row_floats]; hits: out, int32 [n], 1 for a hit and 0 for a miss. */
+SKA_API ska_status sa_cache_get(const ska_cache_desc* desc, const void* cache, size_t cache_bytes,
+                                const ska_cache_key* keys, int32_t n, int64_t now, float* out, int32_t* hits,
+                                void* stream);
+
 /* Human-readable name of a status code (static string). */
 SKA_API const char* ska_status_string(ska_status status);
 

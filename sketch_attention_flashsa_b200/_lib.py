@@ -25,7 +25,8 @@ EXPORTED = ("sa_forward_workspace_size", "sa_forward", "sa_backward_workspace_si
             "ska_read_device_status", "ska_set_debug", "ska_set_timing_events",
             "sa_forward_noalloc", "sa_forward_noalloc_scratch_bytes", "sa_forward_noalloc_read_status",
             "ska_last_error_string", "sa_refine_workspace_size", "sa_refine", "sa_project_queries",
-            "stca_backward_workspace_size", "stca_backward", "sa_forward_diag", "sa_weight_histogram")
+            "stca_backward_workspace_size", "stca_backward", "sa_forward_diag", "sa_weight_histogram",
+            "sa_cache_bytes", "sa_cache_init", "sa_cache_put", "sa_cache_get")
 
 
 class SaDesc(ctypes.Structure):
@@ -49,6 +50,16 @@ class RefineDesc(ctypes.Structure):
                 ("num_protos", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("ffn_dim", ctypes.c_int32), ("eps", ctypes.c_float), ("x_tilde_shared", ctypes.c_int32),
                 ("reserved", ctypes.c_int32)]
+
+
+class CacheKey(ctypes.Structure):
+    _fields_ = [("user_id", ctypes.c_uint64), ("model_version", ctypes.c_uint32), ("sketch_config", ctypes.c_uint32),
+                ("history_timestamp", ctypes.c_int64)]
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("num_sets", ctypes.c_int32), ("ways", ctypes.c_int32), ("row_floats", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("ttl", ctypes.c_int64)]
 
 
 class SkaError(RuntimeError):
@@ -99,6 +110,14 @@ def lib() -> ctypes.CDLL:
     L.sa_forward_noalloc_scratch_bytes.restype = sz
     L.sa_forward_noalloc_read_status.argtypes = [vp]
     L.sa_forward_noalloc_read_status.restype = ctypes.c_int
+    L.sa_cache_bytes.argtypes = [ctypes.POINTER(CacheDesc)]
+    L.sa_cache_bytes.restype = sz
+    L.sa_cache_init.argtypes = [ctypes.POINTER(CacheDesc), vp, sz, vp]
+    L.sa_cache_init.restype = ctypes.c_int
+    L.sa_cache_put.argtypes = [ctypes.POINTER(CacheDesc), vp, sz, vp, vp, ctypes.c_int32, ctypes.c_int64, vp, vp]
+    L.sa_cache_put.restype = ctypes.c_int
+    L.sa_cache_get.argtypes = [ctypes.POINTER(CacheDesc), vp, sz, vp, ctypes.c_int32, ctypes.c_int64, vp, vp, vp]
+    L.sa_cache_get.restype = ctypes.c_int
     L.sa_forward_diag.argtypes = [ctypes.POINTER(SaDesc), vp, vp, vp, i32p, i32p, vp, vp, vp, vp, ctypes.c_int32,
                                   vp, sz, vp]
     L.sa_forward_diag.restype = ctypes.c_int

@@ -522,3 +522,58 @@ def project_queries(x: torch.Tensor, w_q: torch.Tensor, *, workspace: Optional[t
                                        ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check(rc, "sa_project_queries")
     return out
+
+
+def cache_keys(user_id, model_version, sketch_config, history_timestamp, device="cuda") -> torch.Tensor:
+    """Keys of the sketch cache as the C ABI lays them out (ska_cache_key, 24 bytes): an int64
+    tensor [n, 3] holding the user id, the version in the low and the configuration in the high
+    32 bits, and the history timestamp."""
+    u = torch.as_tensor(user_id, dtype=torch.int64).reshape(-1)
+    v = torch.as_tensor(model_version, dtype=torch.int64).reshape(-1) & 0xFFFFFFFF
+    c = torch.as_tensor(sketch_config, dtype=torch.int64).reshape(-1) & 0xFFFFFFFF
+    t = torch.as_tensor(history_timestamp, dtype=torch.int64).reshape(-1)
+    n = max(u.numel(), v.numel(), c.numel(), t.numel())
+    word1 = v.expand(n) | (c.expand(n) << 32)
+    return torch.stack([u.expand(n), word1, t.expand(n)], dim=1).contiguous().to(device)
+
+
+class SketchCache:
+    """Device-side sketch cache of SequenceO1 §4.1 (see sa_cache_* in include/sketch_attn.h):
+    num_sets sets x ways ways of rows of row_floats floats, entries live for ttl time units."""
+
+    def __init__(self, num_sets: int, ways: int, row_floats: int, ttl: int, device="cuda", stream=None):
+        from ._lib import CacheDesc
+        self.desc = CacheDesc(num_sets, ways, row_floats, 0, ttl)
+        L = _lib.lib()
+        nbytes = int(L.sa_cache_bytes(ctypes.byref(self.desc)))
+        if nbytes == 0:
+            raise SkaError(_lib.SKA_ERR_INVALID_VALUE, "sa_cache_bytes")
+        self.mem = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.row_floats = row_floats
+        _check(L.sa_cache_init(ctypes.byref(self.desc), _ptr(self.mem), ctypes.c_size_t(nbytes), _stream(stream)),
+               "sa_cache_init")
+
+    def put(self, keys: torch.Tensor, rows: torch.Tensor, now: int, stream=None) -> torch.Tensor:
+        if keys.dim() != 2 or keys.shape[1] != 3 or keys.dtype != torch.int64:
+            raise ValueError("keys must be an int64 [n, 3] tensor (see cache_keys)")
+        n = keys.shape[0]
+        _shape("rows", rows, (n, self.row_floats))
+        _dev_tensor("keys", keys, (torch.int64,))
+        _dev_tensor("rows", rows, (torch.float32,))
+        slots = torch.empty(n, dtype=torch.int32, device=keys.device)
+        _check(_lib.lib().sa_cache_put(ctypes.byref(self.desc), _ptr(self.mem), ctypes.c_size_t(self.mem.numel()),
+                                       _ptr(keys), _ptr(rows), n, int(now), _ptr(slots), _stream(stream)),
+               "sa_cache_put")
+        return slots
+
+    def get(self, keys: torch.Tensor, now: int, stream=None):
+        if keys.dim() != 2 or keys.shape[1] != 3 or keys.dtype != torch.int64:
+            raise ValueError("keys must be an int64 [n, 3] tensor (see cache_keys)")
+        _dev_tensor("keys", keys, (torch.int64,))
+        n = keys.shape[0]
+        out = torch.empty((n, self.row_floats), dtype=torch.float32, device=keys.device)
+        hits = torch.empty(n, dtype=torch.int32, device=keys.device)
+        _check(_lib.lib().sa_cache_get(ctypes.byref(self.desc), _ptr(self.mem), ctypes.c_size_t(self.mem.numel()),
+                                       _ptr(keys), n, int(now), _ptr(out), _ptr(hits), _stream(stream)),
+               "sa_cache_get")
+        return out, hits

@@ -985,4 +985,64 @@ ska_status sa_project_queries(int32_t num_users, int32_t num_heads, int32_t num_
   return SKA_OK;
 }
 
+size_t sa_cache_bytes(const ska_cache_desc* d) { return cache_desc_ok(d) ? cache_bytes(*d) : 0; }
+
+ska_status sa_cache_init(const ska_cache_desc* d, void* cache, size_t nbytes, void* stream) {
+  if (!cache_desc_ok(d)) return SKA_ERR_INVALID_VALUE;
+  if (!cache || (reinterpret_cast<uintptr_t>(cache) & 255u)) return SKA_ERR_INVALID_VALUE;
+  if (nbytes < cache_bytes(*d)) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  if (no_device()) return SKA_ERR_CUDA;
+  if (cudaError_t e = launch_cache_init(*d, cache, static_cast<cudaStream_t>(stream)); e != cudaSuccess) {
+    record_error("cache init launch", e);
+    return SKA_ERR_CUDA;
+  }
+  return SKA_OK;
+}
+
+ska_status sa_cache_put(const ska_cache_desc* d, void* cache, size_t nbytes, const ska_cache_key* keys,
+                        const float* rows, int32_t n, int64_t now, int32_t* slots, void* stream) {
+  if (!cache_desc_ok(d) || n < 0) return SKA_ERR_INVALID_VALUE;
+  if (!cache || (reinterpret_cast<uintptr_t>(cache) & 255u)) return SKA_ERR_INVALID_VALUE;
+  if (nbytes < cache_bytes(*d)) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  if (n == 0) return SKA_OK;
+  if (!keys || !rows || !slots || !aligned16(rows) || (reinterpret_cast<uintptr_t>(keys) & 7u) ||
+      (reinterpret_cast<uintptr_t>(slots) & 3u))
+    return SKA_ERR_INVALID_VALUE;
+  const size_t cb = cache_bytes(*d), rb = size_t(n) * d->row_floats * 4;
+  if (overlaps(cache, cb, keys, size_t(n) * sizeof(ska_cache_key)) || overlaps(cache, cb, rows, rb) ||
+      overlaps(cache, cb, slots, size_t(n) * 4) || overlaps(slots, size_t(n) * 4, rows, rb) ||
+      overlaps(slots, size_t(n) * 4, keys, size_t(n) * sizeof(ska_cache_key)))
+    return SKA_ERR_INVALID_VALUE;
+  if (no_device()) return SKA_ERR_CUDA;
+  if (cudaError_t e = launch_cache_put(*d, cache, keys, rows, n, now, slots, static_cast<cudaStream_t>(stream));
+      e != cudaSuccess) {
+    record_error("cache put launch", e);
+    return SKA_ERR_CUDA;
+  }
+  return SKA_OK;
+}
+
+ska_status sa_cache_get(const ska_cache_desc* d, const void* cache, size_t nbytes, const ska_cache_key* keys,
+                        int32_t n, int64_t now, float* out, int32_t* hits, void* stream) {
+  if (!cache_desc_ok(d) || n < 0) return SKA_ERR_INVALID_VALUE;
+  if (!cache || (reinterpret_cast<uintptr_t>(cache) & 255u)) return SKA_ERR_INVALID_VALUE;
+  if (nbytes < cache_bytes(*d)) return SKA_ERR_WORKSPACE_TOO_SMALL;
+  if (n == 0) return SKA_OK;
+  if (!keys || !out || !hits || !aligned16(out) || (reinterpret_cast<uintptr_t>(keys) & 7u) ||
+      (reinterpret_cast<uintptr_t>(hits) & 3u))
+    return SKA_ERR_INVALID_VALUE;
+  const size_t cb = cache_bytes(*d), ob = size_t(n) * d->row_floats * 4;
+  if (overlaps(out, ob, cache, cb) || overlaps(out, ob, keys, size_t(n) * sizeof(ska_cache_key)) ||
+      overlaps(hits, size_t(n) * 4, cache, cb) || overlaps(hits, size_t(n) * 4, out, ob) ||
+      overlaps(hits, size_t(n) * 4, keys, size_t(n) * sizeof(ska_cache_key)))
+    return SKA_ERR_INVALID_VALUE;
+  if (no_device()) return SKA_ERR_CUDA;
+  if (cudaError_t e = launch_cache_get(*d, cache, keys, n, now, out, hits, static_cast<cudaStream_t>(stream));
+      e != cudaSuccess) {
+    record_error("cache get launch", e);
+    return SKA_ERR_CUDA;
+  }
+  return SKA_OK;
+}
+
 }  // extern "C"

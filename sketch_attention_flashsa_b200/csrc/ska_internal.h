@@ -189,6 +189,15 @@ cudaError_t launch_stca_bwd(int head_dim, int ctas_kv, int ctas_q, const CUtenso
 cudaError_t launch_stca_bwd_poison(const StcaBwdParams& p, int64_t n_dq, int64_t n_hist, int64_t n_sketch,
                                    cudaStream_t stream);
 
+// Sketch cache (sketch_cache.cu).
+bool cache_desc_ok(const ska_cache_desc* d);
+size_t cache_bytes(const ska_cache_desc& d);
+cudaError_t launch_cache_init(const ska_cache_desc& d, void* cache, cudaStream_t stream);
+cudaError_t launch_cache_put(const ska_cache_desc& d, void* cache, const ska_cache_key* keys, const float* rows, int n,
+                             int64_t now, int32_t* slots, cudaStream_t stream);
+cudaError_t launch_cache_get(const ska_cache_desc& d, const void* cache, const ska_cache_key* keys, int n, int64_t now,
+                             float* out, int32_t* hits, cudaStream_t stream);
+
 // Small kernels (ska_small.cu).
 cudaError_t launch_schedule(const int32_t* cu_seqlens, const int32_t* seqused, int B, int H,
                             int num_clusters, int32_t* tile_prefix, WsHeader* hdr, cudaStream_t stream);

@@ -325,3 +325,30 @@ def test_forward_diag_and_histogram_host_checks():
     if not torch.cuda.is_available():
         assert diag(sa_desc()) == L.SKA_ERR_CUDA
         assert h(21 * A, 10, 4, 20 * A, None) == L.SKA_ERR_CUDA
+
+
+def test_cache_host_checks():
+    lib = L.lib()
+    good = L.CacheDesc(64, 8, 16, 0, 100)
+    nb = lib.sa_cache_bytes(ctypes.byref(good))
+    assert nb >= 256 + 64 * 8 * (32 + 16 * 4)
+    for bad in (L.CacheDesc(48, 8, 16, 0, 100), L.CacheDesc(64, 33, 16, 0, 100), L.CacheDesc(64, 8, 6, 0, 100),
+                L.CacheDesc(64, 8, 16, 0, -1), L.CacheDesc(0, 8, 16, 0, 1)):
+        assert lib.sa_cache_bytes(ctypes.byref(bad)) == 0
+        assert lib.sa_cache_init(ctypes.byref(bad), 90 * A, nb, None) == INVALID
+    assert lib.sa_cache_init(ctypes.byref(good), 90 * A, nb - 1, None) == L.SKA_ERR_WORKSPACE_TOO_SMALL
+    assert lib.sa_cache_init(ctypes.byref(good), 90 * A + 128, nb, None) == INVALID
+    put = lambda **kw: lib.sa_cache_put(ctypes.byref(good), kw.get("c", 90 * A), nb, kw.get("k", 91 * A),  # noqa: E731
+                                        kw.get("r", 92 * A), kw.get("n", 10), 5, kw.get("s", 93 * A), None)
+    assert put(n=-1) == INVALID
+    assert put(n=0, k=None, r=None, s=None) == L.SKA_OK
+    assert put(k=91 * A + 4) == INVALID                 # keys are 8-byte aligned
+    assert put(r=92 * A + 8) == INVALID                 # rows 16-byte aligned
+    assert put(s=92 * A + 64) == INVALID                # slots overlap the rows
+    get = lambda **kw: lib.sa_cache_get(ctypes.byref(good), 90 * A, nb, kw.get("k", 91 * A), 10, 5,  # noqa: E731
+                                        kw.get("o", 92 * A), kw.get("h", 93 * A), None)
+    assert get(o=90 * A + 1024) == INVALID              # output overlaps the cache
+    assert get(h=None) == INVALID
+    import torch
+    if not torch.cuda.is_available():
+        assert put() == L.SKA_ERR_CUDA and get() == L.SKA_ERR_CUDA
