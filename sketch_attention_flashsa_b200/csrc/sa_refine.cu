@@ -33,7 +33,8 @@ namespace ska {
 
 namespace {
 
-constexpr int kRefThreads = 128;
+constexpr int kGroups = 4;                    // threads per row, each on a column slice
+constexpr int kRefThreads = 128 * kGroups;
 constexpr uint32_t kRefBlk = 16384;  // [128 rows x 64 bf16] swizzled block
 
 template <int D, int F>
@@ -53,7 +54,8 @@ struct RefLayout {
   static constexpr uint32_t wg = a_bytes + w_bytes;
   static constexpr uint32_t g_hi = a_bytes;
   static constexpr uint32_t g_lo = a_bytes + g_bytes;
-  static constexpr uint32_t bars = a_bytes + b_bytes;
+  static constexpr uint32_t red = a_bytes + b_bytes;         // kGroups x 128 partial row sums
+  static constexpr uint32_t bars = red + kGroups * 128 * 4;
   static constexpr uint32_t total = bars + 128;
   static_assert(a_bytes % 1024 == 0 && w_bytes % 1024 == 0 && g_bytes % 1024 == 0, "1024-byte aligned blocks");
   static_assert(total <= 227 * 1024, "fits in shared memory");
@@ -161,6 +163,74 @@ __device__ __forceinline__ void store_row_bf16(uint8_t* dst, const float* x) {
                        pack_bf16x2(x[8 * u + 4], x[8 * u + 5]), pack_bf16x2(x[8 * u + 6], x[8 * u + 7]));
 }
 
+// Row statistics of a LayerNorm whose row is split over the kGroups threads of one TMEM lane: each
+// passes its partial sum and receives the row's total through shared memory (CTA barriers: every
+// thread of the CTA calls this at the same point).
+__device__ __forceinline__ float row_total(float part, float* red, int grp, int r) {
+  red[grp * 128 + r] = part;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int g = 0; g < kGroups; ++g) t += red[g * 128 + r];
+  __syncthreads();  // the slots are free for the next use
+  return t;
+}
+
+// LayerNorm of a row held as kGroups slices of C values (this thread: columns [c0, c0 + C)); the
+// statistics are over the whole row of D values, in two passes (mean, then squared deviations).
+template <int C, int D>
+__device__ __forceinline__ void layer_norm_slice(float* x, int c0, const float* gamma, const float* beta, float eps,
+                                                 float* red, int grp, int r) {
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < C; ++c) s += x[c];
+  const float mean = row_total(s, red, grp, r) * (1.f / D);
+  float v = 0.f;
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    const float t = x[c] - mean;
+    v = fmaf(t, t, v);
+  }
+  const float rs = rsqrtf(row_total(v, red, grp, r) * (1.f / D) + eps);
+#pragma unroll
+  for (int c = 0; c < C; ++c) x[c] = (x[c] - mean) * rs;
+  if (gamma) {
+    const float4* g4 = reinterpret_cast<const float4*>(gamma + c0);
+#pragma unroll
+    for (int u = 0; u < C / 4; ++u) {
+      const float4 g = __ldg(g4 + u);
+      x[4 * u] *= g.x;
+      x[4 * u + 1] *= g.y;
+      x[4 * u + 2] *= g.z;
+      x[4 * u + 3] *= g.w;
+    }
+  }
+  if (beta) {
+    const float4* b4 = reinterpret_cast<const float4*>(beta + c0);
+#pragma unroll
+    for (int u = 0; u < C / 4; ++u) {
+      const float4 b = __ldg(b4 + u);
+      x[4 * u] += b.x;
+      x[4 * u + 1] += b.y;
+      x[4 * u + 2] += b.z;
+      x[4 * u + 3] += b.w;
+    }
+  }
+}
+
+template <int C>
+__device__ __forceinline__ void load_slice(const float* src, float* x) {
+  const float4* a = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int u = 0; u < C / 4; ++u) {
+    const float4 v = a[u];
+    x[4 * u] = v.x;
+    x[4 * u + 1] = v.y;
+    x[4 * u + 2] = v.z;
+    x[4 * u + 3] = v.w;
+  }
+}
+
 template <int D, int F>
 __global__ void __launch_bounds__(kRefThreads, 1)
     sa_refine_kernel(const __grid_constant__ CUtensorMap mapW1, const __grid_constant__ CUtensorMap mapWg,
@@ -168,24 +238,31 @@ __global__ void __launch_bounds__(kRefThreads, 1)
                      const RefineParams p) {
   using L = RefLayout<D, F>;
   constexpr uint32_t kCols = 2 * F;  // H1 | Hg
+  constexpr int XC = D / kGroups;    // columns of X, Y and q per thread
+  constexpr int GC = F / kGroups;    // columns of G per thread
   static_assert(kCols <= 512 && (kCols & (kCols - 1)) == 0, "TMEM allocation is a power of two <= 512");
+  static_assert(XC % 16 == 0 && GC % 32 == 0, "column slices");
   extern __shared__ __align__(1024) uint8_t smem[];
   RefBars& bars = *reinterpret_cast<RefBars*>(smem + L::bars);
+  float* red = reinterpret_cast<float*>(smem + L::red);
   if ((smem_u32(smem) & 1023u) != 0) {
     if (threadIdx.x == 0) atomicCAS(p.status, 0, (int)SKA_ERR_UNSUPPORTED);
     return;
   }
-  const int r = threadIdx.x, warp = r >> 5;
+  const int warp = threadIdx.x >> 5;
+  const int r = threadIdx.x & 127;  // the row (TMEM lane) of this thread
+  const int grp = warp >> 2;        // its column slice
   const bool ctl = (threadIdx.x == 0);
+  constexpr uint32_t kArrivals = kRefThreads / 32;
   if (ctl) {
     mbar_init(&bars.w1g, 1);
     mbar_init(&bars.w2, 1);
-    mbar_init(&bars.x, 4);
+    mbar_init(&bars.x, kArrivals);
     mbar_init(&bars.m1, 1);
-    mbar_init(&bars.g, 4);
+    mbar_init(&bars.g, kArrivals);
     mbar_init(&bars.m2, 1);
     mbar_init(&bars.wq, 1);
-    mbar_init(&bars.xq, 4);
+    mbar_init(&bars.xq, kArrivals);
     mbar_init(&bars.m3, 1);
     mbar_init(&bars.drain, 1);
     bars.abort_flag = 0;
@@ -199,7 +276,7 @@ __global__ void __launch_bounds__(kRefThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = bars.tmem_base;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
   RefWaiter wait{&bars, p.status, p.budget_ns};
   uint8_t* sXh = smem + L::x_hi;
   uint8_t* sXl = smem + L::x_lo;
@@ -213,22 +290,24 @@ __global__ void __launch_bounds__(kRefThreads, 1)
   constexpr uint32_t i2 = idesc_bf16_f32(128, D, false, true);
   const int tiles_per_bh = (p.k + 127) / 128;
   const int ntiles = p.B * p.H * tiles_per_bh;
+  const int xc0 = grp * XC, gc0 = grp * GC;
   int it = 0;
   bool w1g_pending = false, w2_pending = false, wq_pending = false;  // thread 0: loads not yet waited for
   const bool project_only = p.mode == 1;
-  // the rows to project, as a bf16 hi + lo pair in region A, then the arrival on xq
-  auto stage_x = [&](const float* x) {
-#pragma unroll
-    for (int c = 0; c < D; c += 8) store_pair8(sXh, sXl, r, c, x + c);
-    fence_async_shared();
-    __syncwarp();
-    if ((r & 31) == 0) mbar_arrive(&bars.xq);
-  };
   // thread 0: W_Q of head h into region B
   auto load_wq = [&](int h) {
     mbar_expect_tx(&bars.wq, L::wq_bytes);
     for (int nb = 0; nb < D / 64; ++nb) tma_load_2d(sWq + nb * D * 128, &mapWq, &bars.wq, nb * 64, h * D);
     wq_pending = true;
+  };
+  // this thread's slice of the rows to project, as a bf16 hi + lo pair in region A, then the
+  // warp's arrival on xq
+  auto stage_x = [&](const float* x) {
+#pragma unroll
+    for (int c = 0; c < XC; c += 8) store_pair8(sXh, sXl, r, xc0 + c, x + c);
+    fence_async_shared();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&bars.xq);
   };
   // tiles in (h, b, row tile) order
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
@@ -241,162 +320,147 @@ __global__ void __launch_bounds__(kRefThreads, 1)
     const int64_t xrow = p.x_tilde_shared ? static_cast<int64_t>(h) * p.k + j : row;
     const uint32_t par = it & 1;
     bool ok = true;
-    float xb[D];
+    float xb[XC];
     if (project_only) {
       if (ctl) load_wq(h);
       if (valid) {
-        const float4* a = reinterpret_cast<const float4*>(p.x_tilde + xrow * D);
-#pragma unroll
-        for (int u = 0; u < D / 4; ++u) {
-          const float4 va = a[u];
-          xb[4 * u] = va.x;
-          xb[4 * u + 1] = va.y;
-          xb[4 * u + 2] = va.z;
-          xb[4 * u + 3] = va.w;
-        }
+        load_slice<XC>(p.x_tilde + xrow * D + xc0, xb);
       } else {
 #pragma unroll
-        for (int u = 0; u < D; ++u) xb[u] = 0.f;
+        for (int u = 0; u < XC; ++u) xb[u] = 0.f;
       }
       stage_x(xb);
     } else {
-    if (ctl) {  // W_1, W_g of head h into region B (the previous tile's MMAs have all completed)
-      mbar_expect_tx(&bars.w1g, 2 * L::w_bytes);
-      for (int nb = 0; nb < F / 64; ++nb) {
-        tma_load_2d(sW1 + nb * D * 128, &mapW1, &bars.w1g, nb * 64, h * D);
-        tma_load_2d(sWg + nb * D * 128, &mapWg, &bars.w1g, nb * 64, h * D);
+      if (ctl) {  // W_1, W_g of head h into region B (the previous tile's MMAs have all completed)
+        mbar_expect_tx(&bars.w1g, 2 * L::w_bytes);
+        for (int nb = 0; nb < F / 64; ++nb) {
+          tma_load_2d(sW1 + nb * D * 128, &mapW1, &bars.w1g, nb * 64, h * D);
+          tma_load_2d(sWg + nb * D * 128, &mapWg, &bars.w1g, nb * 64, h * D);
+        }
+        w1g_pending = true;
       }
-      w1g_pending = true;
-    }
-    // 1. X- = LN1(x_tilde + x_hat)
-    if (valid) {
-      const float4* a = reinterpret_cast<const float4*>(p.x_tilde + xrow * D);
-      const float4* c = reinterpret_cast<const float4*>(p.x_hat + row * D);
+      // 1. X- = LN1(x_tilde + x_hat)
+      if (valid) {
+        float xh[XC];
+        load_slice<XC>(p.x_tilde + xrow * D + xc0, xb);
+        load_slice<XC>(p.x_hat + row * D + xc0, xh);
 #pragma unroll
-      for (int u = 0; u < D / 4; ++u) {
-        const float4 va = a[u], vc = c[u];
-        xb[4 * u] = va.x + vc.x;
-        xb[4 * u + 1] = va.y + vc.y;
-        xb[4 * u + 2] = va.z + vc.z;
-        xb[4 * u + 3] = va.w + vc.w;
+        for (int u = 0; u < XC; ++u) xb[u] += xh[u];
+      } else {
+#pragma unroll
+        for (int u = 0; u < XC; ++u) xb[u] = 0.f;
       }
-      layer_norm_row<D>(xb, p.gamma1 ? p.gamma1 + h * D : nullptr, p.beta1 ? p.beta1 + h * D : nullptr, p.eps);
-      if (p.x_bar) store_row_f32<D>(p.x_bar + row * D, xb);
-      // X- in fp32 waits in this thread's own output row for the residual of step 5, so that it
-      // does not occupy registers across the products
-      store_row_f32<D>(p.x_next + row * D, xb);
-    } else {
+      layer_norm_slice<XC, D>(xb, xc0, p.gamma1 ? p.gamma1 + h * D : nullptr, p.beta1 ? p.beta1 + h * D : nullptr,
+                              p.eps, red, grp, r);
+      if (valid) {
+        if (p.x_bar) store_row_f32<XC>(p.x_bar + row * D + xc0, xb);
+        // X- in fp32 waits in this thread's slice of its output row for the residual of step 5
+        store_row_f32<XC>(p.x_next + row * D + xc0, xb);
+      } else {
 #pragma unroll
-      for (int u = 0; u < D; ++u) xb[u] = 0.f;
-    }
+        for (int u = 0; u < XC; ++u) xb[u] = 0.f;
+      }
 #pragma unroll
-    for (int c = 0; c < D; c += 8) store_pair8(sXh, sXl, r, c, xb + c);
-    fence_async_shared();
-    __syncwarp();
-    if ((r & 31) == 0) mbar_arrive(&bars.x);
-    // 2. H1 = X- W_1, Hg = X- W_g
-    if (ctl) {
-      ok = wait(&bars.x, par) && wait(&bars.w1g, par);
-      if (ok) {
-        w1g_pending = false;
-        tc_fence_after();
+      for (int c = 0; c < XC; c += 8) store_pair8(sXh, sXl, r, xc0 + c, xb + c);
+      fence_async_shared();
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&bars.x);
+      // 2. H1 = X- W_1, Hg = X- W_g
+      if (ctl) {
+        ok = wait(&bars.x, par) && wait(&bars.w1g, par);
+        if (ok) {
+          w1g_pending = false;
+          tc_fence_after();
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t xa = smem_u32(half ? sXl : sXh);
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t xa = smem_u32(half ? sXl : sXh);
 #pragma unroll
-          for (int s = 0; s < D / 16; ++s) {
-            const uint64_t ad = sw128_desc(xa + (s / 4) * kRefBlk + (s % 4) * 32, 16, 1024);
-            const uint32_t acc = (half | s) > 0;
-            umma_bf16(tb, ad, sw128_desc(smem_u32(sW1) + s * 2048, D * 128, 1024), i1, acc);
-            umma_bf16(tb + F, ad, sw128_desc(smem_u32(sWg) + s * 2048, D * 128, 1024), i1, acc);
+            for (int s = 0; s < D / 16; ++s) {
+              const uint64_t ad = sw128_desc(xa + (s / 4) * kRefBlk + (s % 4) * 32, 16, 1024);
+              const uint32_t acc = (half | s) > 0;
+              umma_bf16(tb, ad, sw128_desc(smem_u32(sW1) + s * 2048, D * 128, 1024), i1, acc);
+              umma_bf16(tb + F, ad, sw128_desc(smem_u32(sWg) + s * 2048, D * 128, 1024), i1, acc);
+            }
           }
+          if (!(p.debug_flags & 2u)) umma_commit(&bars.m1);  // the test hook withholds it
         }
-        if (!(p.debug_flags & 2u)) umma_commit(&bars.m1);  // the test hook withholds it
       }
-    }
-    if (!__syncthreads_and(ok && wait(&bars.m1, par))) break;
-    tc_fence_after();
-    if (ctl) {  // W_2 into region A, whose X hi / lo MMA1 has finished reading
-      mbar_expect_tx(&bars.w2, L::w_bytes);
-      for (int nb = 0; nb < D / 64; ++nb) tma_load_2d(sW2 + nb * F * 128, &mapW2, &bars.w2, nb * 64, h * F);
-      w2_pending = true;
-    }
-    // 3. G = swish(H1) * Hg into region B (W_1 / W_g are no longer read)
+      if (!__syncthreads_and(ok && wait(&bars.m1, par))) break;
+      tc_fence_after();
+      if (ctl) {  // W_2 into region A, whose X hi / lo MMA1 has finished reading
+        mbar_expect_tx(&bars.w2, L::w_bytes);
+        for (int nb = 0; nb < D / 64; ++nb) tma_load_2d(sW2 + nb * F * 128, &mapW2, &bars.w2, nb * 64, h * F);
+        w2_pending = true;
+      }
+      // 3. G = swish(H1) * Hg into region B (W_1 / W_g are no longer read), this thread's slice
 #pragma unroll 1
-    for (int c = 0; c < F; c += 32) {
-      uint32_t v1[32], vg[32];
-      tmem_ld32(tb + lane_off + c, v1);
-      tmem_ld32(tb + lane_off + F + c, vg);
-      tmem_ld_wait();
+      for (int c = gc0; c < gc0 + GC; c += 32) {
+        uint32_t v1[32], vg[32];
+        tmem_ld32(tb + lane_off + c, v1);
+        tmem_ld32(tb + lane_off + F + c, vg);
+        tmem_ld_wait();
 #pragma unroll
-      for (int u = 0; u < 32; u += 8) {
-        float gv[8];
+        for (int u = 0; u < 32; u += 8) {
+          float gv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float a = __uint_as_float(v1[u + e]);
-          // swish(a) = a / (1 + e^-a); the fast divide returns -0 for a < -88 (e^-a = inf)
-          gv[e] = valid ? __fdividef(a, 1.f + __expf(-a)) * __uint_as_float(vg[u + e]) : 0.f;
+          for (int e = 0; e < 8; ++e) {
+            const float a = __uint_as_float(v1[u + e]);
+            // swish(a) = a / (1 + e^-a); the fast divide returns -0 for a < -88 (e^-a = inf)
+            gv[e] = valid ? __fdividef(a, 1.f + __expf(-a)) * __uint_as_float(vg[u + e]) : 0.f;
+          }
+          store_pair8(sGh, sGl, r, c + u, gv);
         }
-        store_pair8(sGh, sGl, r, c + u, gv);
       }
-    }
-    fence_async_shared();
-    tc_fence_before();
-    __syncwarp();
-    if ((r & 31) == 0) mbar_arrive(&bars.g);
-    // 4. Y = G W_2 into TMEM columns [0, D)
-    if (ctl) {
-      ok = wait(&bars.g, par) && wait(&bars.w2, par);
-      if (ok) {
-        w2_pending = false;
-        tc_fence_after();
+      fence_async_shared();
+      tc_fence_before();
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&bars.g);
+      // 4. Y = G W_2 into TMEM columns [0, D)
+      if (ctl) {
+        ok = wait(&bars.g, par) && wait(&bars.w2, par);
+        if (ok) {
+          w2_pending = false;
+          tc_fence_after();
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t ga = smem_u32(half ? sGl : sGh);
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t ga = smem_u32(half ? sGl : sGh);
 #pragma unroll
-          for (int s = 0; s < F / 16; ++s)
-            umma_bf16(tb, sw128_desc(ga + (s / 4) * kRefBlk + (s % 4) * 32, 16, 1024),
-                      sw128_desc(smem_u32(sW2) + s * 2048, F * 128, 1024), i2, (half | s) > 0);
+            for (int s = 0; s < F / 16; ++s)
+              umma_bf16(tb, sw128_desc(ga + (s / 4) * kRefBlk + (s % 4) * 32, 16, 1024),
+                        sw128_desc(smem_u32(sW2) + s * 2048, F * 128, 1024), i2, (half | s) > 0);
+          }
+          umma_commit(&bars.m2);
         }
-        umma_commit(&bars.m2);
       }
-    }
-    if (!__syncthreads_and(ok && wait(&bars.m2, par))) break;
-    tc_fence_after();
-    if (ctl && p.q_next) load_wq(h);  // region B is free: MMA2 has read G
-    // 5. X~' = LN2(X- + Y)
-    if (valid) {
-      const float4* a = reinterpret_cast<const float4*>(p.x_next + row * D);
+      if (!__syncthreads_and(ok && wait(&bars.m2, par))) break;
+      tc_fence_after();
+      if (ctl && p.q_next) load_wq(h);  // region B is free: MMA2 has read G
+      // 5. X~' = LN2(X- + Y)
+      if (valid) {
+        load_slice<XC>(p.x_next + row * D + xc0, xb);
+      } else {
 #pragma unroll
-      for (int u = 0; u < D / 4; ++u) {
-        const float4 va = a[u];
-        xb[4 * u] = va.x;
-        xb[4 * u + 1] = va.y;
-        xb[4 * u + 2] = va.z;
-        xb[4 * u + 3] = va.w;
+        for (int u = 0; u < XC; ++u) xb[u] = 0.f;
       }
-    } else {
 #pragma unroll
-      for (int u = 0; u < D; ++u) xb[u] = 0.f;
-    }
+      for (int c = 0; c < XC; c += 16) {
+        uint32_t yv[16];
+        tmem_ld16(tb + lane_off + xc0 + c, yv);
+        tmem_ld_wait();
 #pragma unroll
-    for (int c = 0; c < D; c += 32) {
-      uint32_t yv[32];
-      tmem_ld32(tb + lane_off + c, yv);
-      tmem_ld_wait();
+        for (int u = 0; u < 16; ++u) xb[c + u] += __uint_as_float(yv[u]);
+      }
+      tc_fence_before();
+      layer_norm_slice<XC, D>(xb, xc0, p.gamma2 ? p.gamma2 + h * D : nullptr, p.beta2 ? p.beta2 + h * D : nullptr,
+                              p.eps, red, grp, r);
+      if (valid) {
+        store_row_f32<XC>(p.x_next + row * D + xc0, xb);
+        if (p.x_next_bf16) store_row_bf16<XC>(p.x_next_bf16 + (row * D + xc0) * 2, xb);
+      } else {
 #pragma unroll
-      for (int u = 0; u < 32; ++u) xb[c + u] += __uint_as_float(yv[u]);
-    }
-    tc_fence_before();
-    if (valid) {
-      layer_norm_row<D>(xb, p.gamma2 ? p.gamma2 + h * D : nullptr, p.beta2 ? p.beta2 + h * D : nullptr, p.eps);
-      store_row_f32<D>(p.x_next + row * D, xb);
-      if (p.x_next_bf16) store_row_bf16<D>(p.x_next_bf16 + row * D * 2, xb);
-    } else {
-#pragma unroll
-      for (int u = 0; u < D; ++u) xb[u] = 0.f;
-    }
-    if (p.q_next) stage_x(xb);  // region A: W_2 there has been read by MMA2
+        for (int u = 0; u < XC; ++u) xb[u] = 0.f;
+      }
+      if (p.q_next) stage_x(xb);  // region A: W_2 there has been read by MMA2
     }  // full refinement
     if (p.q_next) {
       // 6. the next layer's queries: X~' W_Q from the hi + lo pair staged in region A
@@ -418,15 +482,15 @@ __global__ void __launch_bounds__(kRefThreads, 1)
       }
       if (!__syncthreads_and(ok && wait(&bars.m3, par))) break;
       tc_fence_after();
-      uint4* qo = reinterpret_cast<uint4*>(p.q_next + row * D * 2);
-#pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t qv[32];
-        tmem_ld32(tb + lane_off + c, qv);
+      uint4* qo = reinterpret_cast<uint4*>(p.q_next + (row * D + xc0) * 2);
+#pragma unroll
+      for (int c = 0; c < XC; c += 16) {
+        uint32_t qv[16];
+        tmem_ld16(tb + lane_off + xc0 + c, qv);
         tmem_ld_wait();
         if (valid) {
 #pragma unroll
-          for (int u = 0; u < 32; u += 8)
+          for (int u = 0; u < 16; u += 8)
             qo[(c + u) / 8] = make_uint4(pack_bf16x2(__uint_as_float(qv[u]), __uint_as_float(qv[u + 1])),
                                          pack_bf16x2(__uint_as_float(qv[u + 2]), __uint_as_float(qv[u + 3])),
                                          pack_bf16x2(__uint_as_float(qv[u + 4]), __uint_as_float(qv[u + 5])),
