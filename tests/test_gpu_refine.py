@@ -231,3 +231,32 @@ def test_two_layer_stack_end_to_end(lengths, H, d, k):
     _stack_close(sk0, o_sk[0], "layer 0 sketch")
     _stack_close(sk1, o_sk[1], "layer 1 sketch")
     _stack_close(x2, o_out, "X~(2)")
+
+
+@pytest.mark.slow
+def test_two_layer_stack_full_size_sampled_user():
+    """The two-layer stack at the headline shapes (8 users x 100,000 tokens, H = 8, d = 128,
+    k = 512) through the library; user 3's final sketch (all heads) against the fp64 oracle stack
+    run on that user alone (every step is per user)."""
+    api = _api()
+    st = W.make_stack([100_000] * 8, 8, 128, 512, 2, seed=79)
+    g = lambda t: None if t is None else t.cuda()  # noqa: E731
+    cu = g(st.cu_seqlens)
+    v = g(st.v)
+    q0 = api.project_queries(g(st.p0), g(st.w_q[0]))
+    sk0, _, _ = api.sa_forward(q0, g(st.keys[0]), v, cu, scale=st.scale, norm="proto")
+    f0 = st.ffn[0]
+    x1, _, _, q1 = api.sa_refine(g(st.p0), sk0, g(f0.w1), g(f0.wg), g(f0.w2), g(f0.gamma1), g(f0.beta1),
+                                 g(f0.gamma2), g(f0.beta2), w_q_next=g(st.w_q[1]))
+    sk1, _, _ = api.sa_forward(q1, g(st.keys[1]), v, cu, scale=st.scale, norm="proto")
+    f1 = st.ffn[1]
+    x2, _, _, _ = api.sa_refine(x1, sk1, g(f1.w1), g(f1.wg), g(f1.w2), g(f1.gamma1), g(f1.beta1), g(f1.gamma2),
+                                g(f1.beta2))
+    torch.cuda.synchronize()
+    b = 3
+    lo, hi = b * 100_000, (b + 1) * 100_000
+    ffn = [(f64(f.w1), f64(f.wg), f64(f.w2), f64(f.gamma1), f64(f.beta1), f64(f.gamma2), f64(f.beta2))
+           for f in st.ffn]
+    o_out, _ = oracle.stacked_sa(f64(st.p0), [f64(w) for w in st.w_q], [f64(kk[lo:hi]) for kk in st.keys],
+                                 f64(st.v[lo:hi]), np.array([0, 100_000]), None, st.scale, ffn)
+    _stack_close(x2[b:b + 1], o_out, "X~(2), user 3 of 8 x 100K")
