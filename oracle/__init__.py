@@ -21,10 +21,10 @@ from .sa import (sa_forward_proto, sa_forward_token, sa_backward_proto,
 from .stca import stca_forward, stca_backward
 from .diag import token_max_weight, weight_histogram, renormalized_sketch
 from .cache import SketchCache, splitmix64, key_hash
-from .refine import layer_norm, swish, swiglu_ffn, refine, project_queries, stacked_sa
+from .refine import layer_norm, swish, swiglu_ffn, refine, project_queries, stacked_sa, round_bf16
 
 __all__ = ["sa_forward_proto", "sa_forward_token", "sa_backward_proto",
            "sa_backward_token", "sa_forward", "sa_backward", "sa_problem",
            "stca_forward", "stca_backward", "token_max_weight", "weight_histogram", "renormalized_sketch",
            "SketchCache", "splitmix64", "key_hash", "layer_norm", "swish", "swiglu_ffn", "refine", "project_queries",
-           "stacked_sa"]
+           "stacked_sa", "round_bf16"]

@@ -21,6 +21,8 @@ Readings taken here (the pages name LN and the FFN but not their details):
   that S^(0) of Eq. (10) is Eq. (7)'s (P^(0) W_Q)(X W_K)^T and its residual in Eq. (13) adds P^(0).
 * The keys K^(l) = X W_K^(l) of each layer are inputs (the key projection of the history is not
   part of this oracle); the values are X itself (Eq. (9), Eq. (12)).
+* Optionally (``query_bf16``) each layer's queries X~^(l) W_Q^(l) are rounded to bf16 before the
+  SA step, the input precision of SA (bf16 inputs, fp32 softmax); everything else stays fp64.
 """
 from __future__ import annotations
 
@@ -93,7 +95,15 @@ def project_queries(x, w_q):
     return out
 
 
-def stacked_sa(p0, w_q, keys, v, cu_seqlens, seqused, scale, ffn):
+def round_bf16(x):
+    """x rounded to the nearest bfloat16 value (8 significant bits, ties to even), returned as
+    float64; finite normal range only (|x| well inside [2^-126, 2^127]), zeros kept."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                      # x = m 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.round(m * 256.0) / 256.0, e)  # np.round: half to even
+
+
+def stacked_sa(p0, w_q, keys, v, cu_seqlens, seqused, scale, ffn, query_bf16=False):
     """N_sa stacked SA layers (§3.3, Eq. (10)-(14)), N_sa = len(w_q).
 
     p0: [H, k, d] prototypes P^(0) (= X~^(0), shared by all users); w_q: N_sa arrays [H, d, d];
@@ -101,6 +111,7 @@ def stacked_sa(p0, w_q, keys, v, cu_seqlens, seqused, scale, ffn):
     ffn: N_sa tuples (w1, wg, w2, gamma1, beta1, gamma2, beta2) as in `refine`.
     Layer l: Q = X~^(l) W_Q^(l); X^^(l+1) = A^(l) X with A^(l) the prototype-wise softmax of
     scale Q K^(l)T (Eq. (10)-(12)); X~^(l+1) from Eq. (13)-(14).
+    query_bf16: round each layer's queries to bf16 before its SA step (the SA input precision).
     Returns X~^(N_sa) as [B, H, k, d] and the per-layer sketches X^^(l+1).
     """
     p0 = np.asarray(p0, dtype=np.float64)
@@ -109,6 +120,8 @@ def stacked_sa(p0, w_q, keys, v, cu_seqlens, seqused, scale, ffn):
     sketches = []
     for l in range(len(w_q)):
         q = project_queries(x_t, w_q[l])
+        if query_bf16:
+            q = round_bf16(q)
         x_hat, _, _ = sa_forward(q, keys[l], v, cu_seqlens, seqused, scale, NORM_PROTO)
         sketches.append(x_hat)
         _, x_t = refine(x_t, x_hat, *ffn[l])

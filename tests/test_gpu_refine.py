@@ -207,8 +207,9 @@ def test_two_layer_stack_end_to_end(lengths, H, d, k):
     """Layer 0: q = P^(0) W_Q^(0) (sa_project_queries), SA over K^(0), refinement with the shared
     residual P^(0) that also emits layer 1's per-user queries; layer 1: SA with those queries over
     K^(1), refinement. Every step runs in the library's kernels; the oracle runs the same stack in
-    fp64 (queries unrounded). Tolerance: that of the SA forward, since the SA steps dominate the
-    error (the bf16 queries add about 2^-9 relative to the scores)."""
+    fp64 with each layer's queries rounded to bf16, the precision in which SA takes them (else the
+    rounding alone moves X~(2) by about 1e-2 at 100K tokens a user). Tolerance: that of the SA
+    forward, since the SA steps dominate the error."""
     api = _api()
     st = W.make_stack(lengths, H, d, k, 2, seed=77 + k)
     g = lambda t: None if t is None else t.cuda()
@@ -227,7 +228,7 @@ def test_two_layer_stack_end_to_end(lengths, H, d, k):
     ffn = [(f64(f.w1), f64(f.wg), f64(f.w2), f64(f.gamma1), f64(f.beta1), f64(f.gamma2), f64(f.beta2))
            for f in st.ffn]
     o_out, o_sk = oracle.stacked_sa(f64(st.p0), [f64(w) for w in st.w_q], [f64(kk) for kk in st.keys], f64(st.v),
-                                    st.cu_seqlens.numpy(), None, st.scale, ffn)
+                                    st.cu_seqlens.numpy(), None, st.scale, ffn, query_bf16=True)
     _stack_close(sk0, o_sk[0], "layer 0 sketch")
     _stack_close(sk1, o_sk[1], "layer 1 sketch")
     _stack_close(x2, o_out, "X~(2)")
@@ -237,7 +238,7 @@ def test_two_layer_stack_end_to_end(lengths, H, d, k):
 def test_two_layer_stack_full_size_sampled_user():
     """The two-layer stack at the headline shapes (8 users x 100,000 tokens, H = 8, d = 128,
     k = 512) through the library; user 3's final sketch (all heads) against the fp64 oracle stack
-    run on that user alone (every step is per user)."""
+    (bf16 queries, as above) run on that user alone (every step is per user)."""
     api = _api()
     st = W.make_stack([100_000] * 8, 8, 128, 512, 2, seed=79)
     g = lambda t: None if t is None else t.cuda()  # noqa: E731
@@ -258,5 +259,5 @@ def test_two_layer_stack_full_size_sampled_user():
     ffn = [(f64(f.w1), f64(f.wg), f64(f.w2), f64(f.gamma1), f64(f.beta1), f64(f.gamma2), f64(f.beta2))
            for f in st.ffn]
     o_out, _ = oracle.stacked_sa(f64(st.p0), [f64(w) for w in st.w_q], [f64(kk[lo:hi]) for kk in st.keys],
-                                 f64(st.v[lo:hi]), np.array([0, 100_000]), None, st.scale, ffn)
+                                 f64(st.v[lo:hi]), np.array([0, 100_000]), None, st.scale, ffn, query_bf16=True)
     _stack_close(x2[b:b + 1], o_out, "X~(2), user 3 of 8 x 100K")

@@ -12,6 +12,7 @@ import math
 from fractions import Fraction
 
 import numpy as np
+import torch
 import pytest
 
 import oracle
@@ -529,6 +530,45 @@ def test_stacked_sa_token_order_and_users():
     v2[6:] += rng.normal(size=(3, H, d))  # (a shift equal on every feature would be absorbed by LN)
     out2, _ = oracle.stacked_sa(p0, w_q, keys, v2, cu, None, 0.5, ffn)
     assert np.array_equal(out2[0], out[0]) and not np.allclose(out2[1], out[1])
+
+
+def test_round_bf16_hand_cases_ties_to_even():
+    """bf16 keeps 8 significant bits: near 1 the spacing is 2^-7. 1 + 2^-8 is halfway between 1
+    (even mantissa) and 1 + 2^-7, so it goes to 1; 1 + 3 2^-8 is halfway between 1 + 2^-7 (odd) and
+    1 + 2^-6 (even), so it goes up; a hair above a tie rounds up; signs are symmetric."""
+    x = np.array([1 + 2.0**-8, 1 + 3 * 2.0**-8, 1 + 2.0**-8 + 2.0**-40, -(1 + 2.0**-8), 0.0, 3.0, 2.0**-20 * 255])
+    want = np.array([1.0, 1 + 2.0**-6, 1 + 2.0**-7, -1.0, 0.0, 3.0, 2.0**-20 * 255])
+    assert np.array_equal(oracle.round_bf16(x), want)
+
+
+def test_round_bf16_matches_a_library_conversion_on_fp32_values():
+    """On values that fp32 holds exactly, a single rounding to bf16 is what torch's fp32 -> bf16
+    conversion (round to nearest even) computes."""
+    rng = np.random.default_rng(83)
+    x = (rng.standard_normal(200_000) * np.exp(rng.uniform(-30, 30, 200_000))).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(oracle.round_bf16(x.astype(np.float64)), want)
+
+
+def test_stacked_sa_bf16_queries_no_op_when_queries_are_bf16():
+    """One layer with W_Q = I and bf16-valued prototypes: the queries are already bf16, so the
+    rounding option changes nothing; with W_Q scaled by 1 + 2^-12 it does change the result."""
+    rng = np.random.default_rng(84)
+    H, k, d, f = 2, 3, 8, 16
+    cu = np.array([0, 5, 9])
+    v = rng.normal(size=(9, H, d))
+    keys = [rng.normal(size=(9, H, d))]
+    p0 = oracle.round_bf16(rng.normal(size=(H, k, d)))
+    ffn = [(rng.normal(size=(H, d, f)) / 3, rng.normal(size=(H, d, f)) / 3, rng.normal(size=(H, f, d)) / 3,
+            None, None, None, None)]
+    eye = [np.broadcast_to(np.eye(d), (H, d, d)).copy()]
+    a, _ = oracle.stacked_sa(p0, eye, keys, v, cu, None, 1.0, ffn)
+    b, _ = oracle.stacked_sa(p0, eye, keys, v, cu, None, 1.0, ffn, query_bf16=True)
+    assert np.array_equal(a, b)
+    off = [eye[0] * (1 + 2.0**-12)]
+    c, _ = oracle.stacked_sa(p0, off, keys, v, cu, None, 1.0, ffn)
+    e, _ = oracle.stacked_sa(p0, off, keys, v, cu, None, 1.0, ffn, query_bf16=True)
+    assert np.array_equal(e, a) and not np.array_equal(c, a)
 
 
 # ------------------------------------------------------------------- STCA backward (finite differences)
