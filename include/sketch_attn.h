@@ -168,9 +168,15 @@ SKA_API size_t sa_backward_workspace_size(const ska_sa_desc* desc);
  *   dq       out, fp32, q's shape: [H,k,d] summed over all users when the prototypes are shared,
  *            else [B,H,k,d]
  *   dk, dv   out, fp32 [total_tokens, H, d]; zero rows on padding tokens
- * Supported: num_protos in {16, 32, 64, 128, 256} for head_dim 64, up to 128 for head_dim 128
- * (SKA_ERR_UNSUPPORTED otherwise). dQ is formed from a two-term bf16 split of dS (16
- * significant bits) and reduced over users in a fixed order.                                  */
+ * Supported (SKA_ERR_UNSUPPORTED otherwise): num_protos in {16, 32, 64, 128, 256} for head_dim
+ * 64 and {16, 32, 64, 128} for head_dim 128 in one fused launch; larger sets up to 4096 that are
+ * multiples of 256 (head_dim 64) or 128 (head_dim 128) in one launch per chunk of that many
+ * prototypes, dK and dV summed over the chunks in chunk order. In PROTO mode those first run
+ * one pass per chunk for delta_i = sum_j A_ij dA_ij, kept in the workspace: 1.4x the FLOPs of
+ * one fused pass, and the keys and values are read 2 k / chunk times (TOKEN: k / chunk). dQ is
+ * formed from a two-term bf16 split of dS (16 significant bits), and over chunks so are dK (from
+ * dS) and dV (from A); dQ is reduced over users in a fixed order. Results are bitwise
+ * reproducible run to run.                                                                     */
 SKA_API ska_status sa_backward(const ska_sa_desc* desc, const void* q, const void* k, const void* v,
                        const int32_t* cu_seqlens, const int32_t* seqused, const float* sketch,
                        const float* lse, const void* dsketch, float* dq, float* dk, float* dv, void* ws,

@@ -5,19 +5,27 @@
 // TMEM lanes (S^T orientation):
 //   MMA  S^T  = K . Q^T                        -> A = exp(scale s - lse) (PROTO: per-token lse;
 //                                                 TOKEN: per-prototype lse), to smem in bf16
-//   MMA  dV   = A^T . dO        (M=tok, N=d)   -> TMEM
+//   MMA  dV   = A^T . dO        (M=tok, N=d)   -> TMEM (A as hi + lo over prototype chunks)
 //   MMA  dA^T = V . dO^T        (M=tok, N=k)   -> TMEM (over S^T)
 //   softmax-gradient: PROTO dS = A (dA - delta_i) with delta_i = sum_j A_ji dA_ji in fp32 (each
 //        warpgroup sums its half of the prototypes, the halves are added in a fixed order);
 //        TOKEN dS = A (dA - D_j) with D_j = dO_j . O_j from the forward sketch. dS goes to smem
 //        as a bf16 pair hi + lo.
-//   MMA  dK   = dS^T . Q        (M=tok, N=d)   -> TMEM from the hi half, scaled on the way out
+//   MMA  dK   = dS^T . Q        (M=tok, N=d)   -> TMEM from the hi half (both halves over prototype
+//        chunks), scaled on the way out
 //   MMA  dQ  += dS . K          (M=proto, N=d) -> TMEM, both halves; restarted every 16 tiles and
 //        added into the CTA's partial slot (the tensor core's fp32 accumulation is not
 //        round-to-nearest, so one chain over a whole segment would drift); a second kernel sums
 //        the partial slots of every prototype set in a fixed order.
 // Warps 0-7 (two warpgroups, each owning half of the prototype columns) do the elementwise
 // work; thread 0 also issues the TMA loads and MMAs. The phases of a tile run one after another.
+//
+// Prototype sets larger than one CTA holds (TMEM: S^T, dV, dK and the dQ blocks) run as one
+// launch per chunk of KP prototypes (rows j0 .. j0 + KP - 1 of Q, dO, the sketch and TOKEN's lse):
+// every chunk but the first adds its dK and dV to the previous chunk's, and the chunk's dQ slots
+// are reduced into dq's rows j0 ... PROTO's delta_i sums over all k prototypes of the token, so
+// a first pass per chunk (pass 1: S, A and dA^T only) adds its part into a [T, H] buffer in chunk
+// order, and the gradient pass (pass 2) reads delta_i from there.
 #include <algorithm>
 #include <cmath>
 
@@ -32,6 +40,8 @@ constexpr int kBwdThreads = 256;
 constexpr int kBwdWarps = 8;
 constexpr int kBlk = 16384;  // [128 rows x 64 bf16] swizzled block
 constexpr int kDqFlush = 16;  // tiles per dQ accumulation chain in TMEM
+// Larger prototype sets run as launches over chunks of prototypes (see sa_bwd_chunk).
+constexpr int kMaxChunkedProtos = 4096;
 
 struct BwdLayout {
   uint32_t q_off, do_off, k_off, v_off, a_off, lo_off, lse_off, d_off, bar_off, total;
@@ -132,13 +142,14 @@ struct BwdWaiter {
 };
 
 
-template <int D, int KP>
+// CHUNK: this launch is one chunk of a larger prototype set (passes 1 and 2, dK/dV accumulation);
+// without it those paths are compiled out.
+template <int D, int KP, bool CHUNK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     sa_bwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapDO,
                   const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
-                  const SaBwdParams p) {
+                  const SaBwdParams p, const __grid_constant__ SaBwdChunk ck) {
   constexpr int KB = D / 64;
-  constexpr int PB = (KP + 63) / 64;
   constexpr int NCOL = KP / 2;                  // prototype columns per worker thread
   constexpr int QBLK = (KP * 128 + 1023) & ~1023;
   constexpr int CV = (KP + 31) / 32 * 32;      // TMEM columns: S^T/dA^T at 0, dV, dK, dQ blocks
@@ -202,6 +213,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr uint32_t iV = idesc_bf16_f32(128, D, false, true);
   constexpr uint32_t iQ = idesc_bf16_f32(128, D, true, true);
   const bool ctl = (threadIdx.x == 0);
+  const int pass = CHUNK ? ck.pass : 0;
+  const bool accumulate = CHUNK && ck.accumulate;
   const int wg = warp >> 2, q4 = warp & 3;
   const int r = q4 * 32 + lane;
   const int col0 = wg * NCOL;
@@ -212,8 +225,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   int nk_seen = 0, nv_seen = 0;                        // fills waited for
   auto load_qdo = [&](const BwdPos& u) {
     ++nq_issued;
-    const int qrow = (p.q_per_user ? u.b * p.H * p.k : 0) + u.h * p.k;
-    const int orow = (u.b * p.H + u.h) * p.k;
+    const int qrow = (p.q_per_user ? u.b * p.H * ck.kt : 0) + u.h * ck.kt + ck.j0;
+    const int orow = (u.b * p.H + u.h) * ck.kt + ck.j0;
     mbar_expect_tx(&bars.qd, 2 * KB * KP * 128);
     for (int kb = 0; kb < KB; ++kb) {
       tma_load_2d(sQ + kb * QBLK, &mapQ, &bars.qd, kb * 64, qrow);
@@ -270,7 +283,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // per-prototype lse (log2 units) and D_j = dO_j . O_j of this (user, head)
       const int jj = threadIdx.x;
       if (jj < p.k) {
-        const int64_t row = (static_cast<int64_t>(t.b) * p.H + t.h) * p.k + jj;
+        const int64_t row = (static_cast<int64_t>(t.b) * p.H + t.h) * ck.kt + ck.j0 + jj;
         sLse[jj] = p.lse[row] * L2E;
         float acc = 0.f;
         for (int dd = 0; dd < D; ++dd) acc += __bfloat162float(p.dsketch[row * D + dd]) * p.sketch[row * D + dd];
@@ -311,12 +324,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     // A in bf16 for dV = A^T dO (fp32 A stays in registers for dS): dV_i is a weighted mean of
     // dO rows, so rounding the weights to 8 significant bits leaves ~1e-3 relative error in dV
+    // (over chunks of a larger prototype set, dV sums more prototypes and grows with them: A then
+    // enters as a bf16 pair hi + lo)
+    if (pass != 1) {
 #pragma unroll
-    for (int c = 0; c < NCOL; c += 8) {
-      const int jj = col0 + c;
-      const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
-      *reinterpret_cast<uint4*>(sA + off) = make_uint4(pack_bf16x2(a[c], a[c + 1]), pack_bf16x2(a[c + 2], a[c + 3]),
-                                                       pack_bf16x2(a[c + 4], a[c + 5]), pack_bf16x2(a[c + 6], a[c + 7]));
+      for (int c = 0; c < NCOL; c += 8) {
+        const int jj = col0 + c;
+        const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
+        if constexpr (CHUNK) {
+          float hi[8], lo[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            hi[u] = __bfloat162float(__float2bfloat16_rn(a[c + u]));
+            lo[u] = a[c + u] - hi[u];
+          }
+          *reinterpret_cast<uint4*>(sA + off) = make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]),
+                                                           pack_bf16x2(hi[4], hi[5]), pack_bf16x2(hi[6], hi[7]));
+          *reinterpret_cast<uint4*>(sLo + off) = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]),
+                                                            pack_bf16x2(lo[4], lo[5]), pack_bf16x2(lo[6], lo[7]));
+        } else {
+          *reinterpret_cast<uint4*>(sA + off) = make_uint4(pack_bf16x2(a[c], a[c + 1]), pack_bf16x2(a[c + 2], a[c + 3]),
+                                                           pack_bf16x2(a[c + 4], a[c + 5]), pack_bf16x2(a[c + 6], a[c + 7]));
+        }
+      }
     }
     fence_async_shared();
     tc_fence_before();
@@ -326,10 +356,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = wait(&bars.a, i & 1);
       if (ok) {
         tc_fence_after();
+        if (pass != 1) {
 #pragma unroll
-        for (int s = 0; s < KP / 16; ++s)
-          umma_bf16(tb + CV, sw128_desc(smem_u32(sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
-                    sw128_desc(smem_u32(sDO) + s * 2048, QBLK, 1024), iV, s > 0);
+          for (int s = 0; s < KP / 16; ++s)
+            umma_bf16(tb + CV, sw128_desc(smem_u32(sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                      sw128_desc(smem_u32(sDO) + s * 2048, QBLK, 1024), iV, s > 0);
+          if constexpr (CHUNK) {
+#pragma unroll
+            for (int s = 0; s < KP / 16; ++s)
+              umma_bf16(tb + CV, sw128_desc(smem_u32(sLo) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                        sw128_desc(smem_u32(sDO) + s * 2048, QBLK, 1024), iV, 1u);
+          }
+        }
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
           umma_bf16(tb, sw128_desc(smem_u32(sV) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
@@ -346,7 +384,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // PROTO: delta_i = sum_j A_ij dA_ij in fp32; each warpgroup sums its half of the
     // prototypes and the two halves are added in a fixed order
     float delta = 0.f;
-    if (p.norm == SKA_NORM_PROTO) {
+    if (p.norm == SKA_NORM_PROTO && pass == 2) {
+      delta = (valid && tok < p.total_tokens) ? ck.delta[static_cast<int64_t>(tok) * p.H + t.h] : 0.f;
+    } else if (p.norm == SKA_NORM_PROTO) {
       float part = 0.f;
 #pragma unroll
       for (int c = 0; c < NCOL; c += 16) {
@@ -366,6 +406,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, wait(&bars.dl, i & 1));
       if (!ok) break;
       delta = sDl[r] + sDl[128 + r];
+    }
+    if (pass == 1) {
+      // this chunk's part of delta_i, added in chunk order (launches run one after another)
+      if (wg == 0 && valid && tok < p.total_tokens) {
+        float* dp = ck.delta + static_cast<int64_t>(tok) * p.H + t.h;
+        *dp = (ck.j0 == 0 ? 0.f : *dp) + delta;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (ctl && i + 1 < ntiles) {  // the MMAs of this tile are complete: K, Q and dO are free
+        if (tn.j == 0) load_qdo(tn);
+        load_k(tn);
+      }
+      if (first) ++nseg;
+      t = tn;
+      continue;
     }
     // dS = A (dA - delta) as a bf16 pair hi + lo
     constexpr int DC = (NCOL >= 16) ? 16 : 8;  // columns per TMEM round trip
@@ -408,12 +464,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = wait(&bars.ds, i & 1);
       if (ok) {
         tc_fence_after();
-        // dK from the hi half of dS alone (~1e-3 relative); dQ, a sum over every token of every
-        // user, takes both halves
+        // dK from the hi half of dS alone (~1e-3 relative) when one launch holds every prototype;
+        // over chunks of a larger set (dK sums more prototypes and grows with them) from both
+        // halves. dQ, a sum over every token of every user, always takes both.
 #pragma unroll
         for (int s = 0; s < KP / 16; ++s)
           umma_bf16(tb + CK, sw128_desc(smem_u32(sA) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
                     sw128_desc(smem_u32(sQ) + s * 2048, QBLK, 1024), iV, s > 0);
+        if constexpr (CHUNK) {
+#pragma unroll
+          for (int s = 0; s < KP / 16; ++s)
+            umma_bf16(tb + CK, sw128_desc(smem_u32(sLo) + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+                      sw128_desc(smem_u32(sQ) + s * 2048, QBLK, 1024), iV, 1u);
+        }
 #pragma unroll
         for (int g = 0; g < QBLOCKS; ++g)
 #pragma unroll
@@ -470,8 +533,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int64_t tk = static_cast<int64_t>(tok0) + row;
           if (row < urows && tk < p.total_tokens) {
             const int64_t off = (tk * p.H + t.h) * D + cc + (lane & 7) * 4;
-            *reinterpret_cast<float4*>(p.dk + off) = staged(stk, u);
-            *reinterpret_cast<float4*>(p.dv + off) = staged(stv, u);
+            float4 gk = staged(stk, u), gv = staged(stv, u);
+            if (accumulate) {
+              const float4 pk = *reinterpret_cast<const float4*>(p.dk + off);
+              const float4 pv = *reinterpret_cast<const float4*>(p.dv + off);
+              gk.x += pk.x; gk.y += pk.y; gk.z += pk.z; gk.w += pk.w;
+              gv.x += pv.x; gv.y += pv.y; gv.z += pv.z; gv.w += pv.w;
+            }
+            *reinterpret_cast<float4*>(p.dk + off) = gk;
+            *reinterpret_cast<float4*>(p.dv + off) = gv;
           }
         }
         __syncwarp();
@@ -481,11 +551,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           float* dv = p.dv + (static_cast<int64_t>(tok) * p.H + t.h) * D + cc;
 #pragma unroll
           for (int u = 0; u < 32; u += 4) {
-            *reinterpret_cast<float4*>(dk + u) =
-                make_float4(p.scale * __uint_as_float(kr[u]), p.scale * __uint_as_float(kr[u + 1]),
-                            p.scale * __uint_as_float(kr[u + 2]), p.scale * __uint_as_float(kr[u + 3]));
-            *reinterpret_cast<float4*>(dv + u) = make_float4(__uint_as_float(vr[u]), __uint_as_float(vr[u + 1]),
-                                                             __uint_as_float(vr[u + 2]), __uint_as_float(vr[u + 3]));
+            float4 gk = make_float4(p.scale * __uint_as_float(kr[u]), p.scale * __uint_as_float(kr[u + 1]),
+                                    p.scale * __uint_as_float(kr[u + 2]), p.scale * __uint_as_float(kr[u + 3]));
+            float4 gv = make_float4(__uint_as_float(vr[u]), __uint_as_float(vr[u + 1]), __uint_as_float(vr[u + 2]),
+                                    __uint_as_float(vr[u + 3]));
+            if (accumulate) {
+              const float4 pk = *reinterpret_cast<const float4*>(dk + u);
+              const float4 pv = *reinterpret_cast<const float4*>(dv + u);
+              gk.x += pk.x; gk.y += pk.y; gk.z += pk.z; gk.w += pk.w;
+              gv.x += pv.x; gv.y += pv.y; gv.z += pv.z; gv.w += pv.w;
+            }
+            *reinterpret_cast<float4*>(dk + u) = gk;
+            *reinterpret_cast<float4*>(dv + u) = gv;
           }
         }
       }
@@ -568,7 +645,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // dq[(b?) h] = sum over the segments it collects of their partial slots, fixed order.
-__global__ void sa_bwd_dq_reduce(const SaBwdParams p, int D, float* __restrict__ dq) {
+__global__ void sa_bwd_dq_reduce(const SaBwdParams p, const SaBwdChunk ck, int D, float* __restrict__ dq) {
   const int64_t per = static_cast<int64_t>(p.k) * D;
   const int qsets = p.q_per_user ? p.B * p.H : p.H;
   const int64_t n = static_cast<int64_t>(qsets) * per;
@@ -587,7 +664,7 @@ __global__ void sa_bwd_dq_reduce(const SaBwdParams p, int D, float* __restrict__
       const int s = b * p.H + h;
       for (int c = t0 / W; c <= (t0 + nb - 1) / W; ++c) acc += p.dq_partial[static_cast<int64_t>(s + c) * per + within];
     }
-    dq[e] = acc;
+    dq[(static_cast<int64_t>(qs) * ck.kt + ck.j0) * D + within] = acc;
   }
 }
 
@@ -605,33 +682,49 @@ __global__ void sa_bwd_zero_padding(const SaBwdParams p, int D) {
   }
 }
 
-template <int D, int KP>
+template <int D, int KP, bool CHUNK = false>
 cudaError_t bwd_launch_t(int num_ctas, const CUtensorMap& mQ, const CUtensorMap& mDO, const CUtensorMap& mK,
-                         const CUtensorMap& mV, const SaBwdParams& p, cudaStream_t stream) {
-  auto kern = sa_bwd_kernel<D, KP>;
+                         const CUtensorMap& mV, const SaBwdParams& p, const SaBwdChunk& ck, cudaStream_t stream) {
+  auto kern = sa_bwd_kernel<D, KP, CHUNK>;
   const size_t smem = bwd_layout(D, KP).total;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<num_ctas, kBwdThreads, smem, stream>>>(mQ, mDO, mK, mV, p);
+  kern<<<num_ctas, kBwdThreads, smem, stream>>>(mQ, mDO, mK, mV, p, ck);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-bool sa_bwd_supported(int D, int k) {
+namespace {
+// One CTA holds all k prototypes of a tile (TMEM: S^T / dA^T, dV, dK and the dQ blocks).
+bool bwd_one_launch(int D, int k) {
   if (D != 64 && D != 128) return false;
   if (!(k == 16 || k == 32 || k == 64 || k == 128 || k == 256)) return false;
   if (bwd_tmem_cols(D, k) + ((k + 31) / 32 * 32 - k) > 512) return false;
   return bwd_layout(D, k).total <= 227 * 1024;
 }
+}  // namespace
+
+int sa_bwd_chunk(int D, int k) {
+  if (bwd_one_launch(D, k)) return k;
+  if (D != 64 && D != 128) return 0;
+  const int c = (D == 128) ? 128 : 256;
+  return (k > c && k % c == 0 && k <= kMaxChunkedProtos) ? c : 0;
+}
+
+bool sa_bwd_supported(int D, int k) { return sa_bwd_chunk(D, k) > 0; }
 
 size_t sa_bwd_smem_bytes(int D, int k) { return bwd_layout(D, k).total; }
 
 cudaError_t launch_sa_bwd(int D, int num_ctas, const CUtensorMap& mQ, const CUtensorMap& mDO,
                           const CUtensorMap& mK, const CUtensorMap& mV, const SaBwdParams& p,
-                          cudaStream_t stream) {
+                          const SaBwdChunk& ck, cudaStream_t stream) {
+  const bool chunk = ck.kt != p.k;
+  if (chunk && D == 64 && p.k == 256) return bwd_launch_t<64, 256, true>(num_ctas, mQ, mDO, mK, mV, p, ck, stream);
+  if (chunk && D == 128 && p.k == 128) return bwd_launch_t<128, 128, true>(num_ctas, mQ, mDO, mK, mV, p, ck, stream);
+  if (chunk) return cudaErrorInvalidValue;
 #define SKA_BWD_CASE(DD, KK) \
-  if (D == DD && p.k == KK) return bwd_launch_t<DD, KK>(num_ctas, mQ, mDO, mK, mV, p, stream);
+  if (D == DD && p.k == KK) return bwd_launch_t<DD, KK>(num_ctas, mQ, mDO, mK, mV, p, ck, stream);
   SKA_BWD_CASE(64, 16)
   SKA_BWD_CASE(64, 32)
   SKA_BWD_CASE(64, 64)
@@ -645,8 +738,8 @@ cudaError_t launch_sa_bwd(int D, int num_ctas, const CUtensorMap& mQ, const CUte
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_sa_bwd_finish(const SaBwdParams& p, int D, float* dq, cudaStream_t stream) {
-  sa_bwd_dq_reduce<<<592, 256, 0, stream>>>(p, D, dq);
+cudaError_t launch_sa_bwd_finish(const SaBwdParams& p, const SaBwdChunk& ck, int D, float* dq, cudaStream_t stream) {
+  sa_bwd_dq_reduce<<<592, 256, 0, stream>>>(p, ck, D, dq);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (p.B > 0) sa_bwd_zero_padding<<<p.B, 256, 0, stream>>>(p, D);

@@ -563,15 +563,29 @@ ska_status sa_weight_histogram(const float* values, int64_t n, int32_t bins, int
   return SKA_OK;
 }
 
+// Workspace of sa_backward: header, tile prefix, the dQ partial slots of one launch (one chunk of
+// prototypes), then, for PROTO over several chunks, delta_i [T, H].
+struct BwdWs {
+  size_t dqp, delta, total;
+};
+
+bool bwd_ws_layout(const ska_sa_desc* d, int sms, BwdWs* w) {
+  const int kc = sa_bwd_chunk(d->head_dim, d->num_protos);
+  if (kc <= 0 || sms <= 0) return false;
+  size_t off = sizeof(WsHeader);
+  w->dqp = off = align256(off + size_t(d->num_users + 1) * 4);
+  off = align256(off + (size_t(d->num_users) * d->num_heads + sms) * kc * d->head_dim * 4);
+  w->delta = off;
+  if (d->norm == SKA_NORM_PROTO && kc < d->num_protos) off = align256(off + size_t(d->total_tokens) * d->num_heads * 4);
+  w->total = off;
+  return true;
+}
+
 size_t sa_backward_workspace_size(const ska_sa_desc* d) {
   if (check_sa_desc(d) != SKA_OK) return 0;
   if (d->in_dtype != SKA_BF16 || !sa_bwd_supported(d->head_dim, d->num_protos)) return 0;
-  const int sms = device_sm_count();
-  if (sms <= 0) return 0;
-  size_t off = sizeof(WsHeader);
-  off = align256(off + size_t(d->num_users + 1) * 4);
-  off = align256(off + (size_t(d->num_users) * d->num_heads + sms) * d->num_protos * d->head_dim * 4);
-  return off;
+  BwdWs w;
+  return bwd_ws_layout(d, device_sm_count(), &w) ? w.total : 0;
 }
 
 ska_status sa_backward(const ska_sa_desc* d, const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
@@ -613,10 +627,14 @@ ska_status sa_backward(const ska_sa_desc* d, const void* q, const void* k, const
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (B == 0) return SKA_OK;
   const int sms = device_sm_count();
+  BwdWs w;
+  if (!bwd_ws_layout(d, sms, &w)) return SKA_ERR_UNSUPPORTED;
+  const int kc = sa_bwd_chunk(D, kp);  // prototypes per launch
+  const int nchunks = kp / kc;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
   int32_t* prefix = reinterpret_cast<int32_t*>(wsb + sizeof(WsHeader));
-  float* dqp = reinterpret_cast<float*>(wsb + align256(sizeof(WsHeader) + size_t(B + 1) * 4));
+  float* dqp = reinterpret_cast<float*>(wsb + w.dqp);
   if (cudaError_t e_ = launch_schedule(cu_seqlens, seqused, B, H, sms, prefix, hdr, s); e_ != cudaSuccess) { record_error("launch_schedule", e_); return SKA_ERR_CUDA; }
   SaBwdParams p{};
   p.norm = d->norm;
@@ -632,29 +650,68 @@ ska_status sa_backward(const ska_sa_desc* d, const void* q, const void* k, const
   p.dq_partial = dqp;
   p.B = B;
   p.H = H;
-  p.k = kp;
+  p.k = kc;
+  SaBwdChunk ck{};
+  ck.delta = (d->norm == SKA_NORM_PROTO && nchunks > 1) ? reinterpret_cast<float*>(wsb + w.delta) : nullptr;
+  ck.kt = kp;
+  ck.j0 = 0;
+  ck.pass = 0;
+  ck.accumulate = 0;
   p.total_tokens = static_cast<int>(T);
   p.q_per_user = d->q_per_user;
   p.scale = d->scale;
   p.budget_ns = wait_budget();
-  if (T > 0) {
-    CUtensorMap mQ, mDO, mK, mV;
-    const uint64_t qrows = uint64_t(d->q_per_user ? B : 1) * H * kp;
-    if (!encode_2d(&mQ, q, D, qrows, D, 64, kp)) return SKA_ERR_CUDA;
-    if (!encode_2d(&mDO, dsketch, D, uint64_t(B) * H * kp, D, 64, kp)) return SKA_ERR_CUDA;
-    if (!encode_2d(&mK, k, uint64_t(H) * D, T, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
-    if (!encode_2d(&mV, v, uint64_t(H) * D, T, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+  if (T == 0) {  // no tiles: the reduction writes zeros
+    for (int c = 0; c < nchunks; ++c) {
+      ck.j0 = c * kc;
+      if (cudaError_t e_ = launch_sa_bwd_finish(p, ck, D, dq, s); e_ != cudaSuccess) { record_error("launch_sa_bwd_finish", e_); return SKA_ERR_CUDA; }
+    }
+    return SKA_OK;
+  }
+  CUtensorMap mQ, mDO, mK, mV;
+  const uint64_t qrows = uint64_t(d->q_per_user ? B : 1) * H * kp;
+  if (!encode_2d(&mQ, q, D, qrows, D, 64, kc)) return SKA_ERR_CUDA;
+  if (!encode_2d(&mDO, dsketch, D, uint64_t(B) * H * kp, D, 64, kc)) return SKA_ERR_CUDA;
+  if (!encode_2d(&mK, k, uint64_t(H) * D, T, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+  if (!encode_2d(&mV, v, uint64_t(H) * D, T, uint64_t(H) * D, 64, 128)) return SKA_ERR_CUDA;
+  if (nchunks == 1) {
     cudaError_t e;
     {
       TimedRegion tr(s);
-      e = launch_sa_bwd(D, sms, mQ, mDO, mK, mV, p, s);
+      e = launch_sa_bwd(D, sms, mQ, mDO, mK, mV, p, ck, s);
     }
     if (e != cudaSuccess) {
       record_error("fused kernel launch", e);
       return SKA_ERR_CUDA;
     }
+    if (cudaError_t e_ = launch_sa_bwd_finish(p, ck, D, dq, s); e_ != cudaSuccess) { record_error("launch_sa_bwd_finish", e_); return SKA_ERR_CUDA; }
+    return SKA_OK;
   }
-  if (cudaError_t e_ = launch_sa_bwd_finish(p, D, dq, s); e_ != cudaSuccess) { record_error("launch_sa_bwd_finish", e_); return SKA_ERR_CUDA; }
+  // More prototypes than one CTA holds (the timed region spans every launch): PROTO first sums
+  // delta_i = sum_j A_ij dA_ij over the chunks, one pass each; then every chunk forms its
+  // gradients (with that delta_i in PROTO). dK and dV are summed over the chunks in chunk order,
+  // and each chunk's dQ is reduced before the next chunk reuses the partial slots.
+  TimedRegion tr(s);
+  if (ck.delta) {
+    ck.pass = 1;
+    for (int c = 0; c < nchunks; ++c) {
+      ck.j0 = c * kc;
+      if (cudaError_t e = launch_sa_bwd(D, sms, mQ, mDO, mK, mV, p, ck, s); e != cudaSuccess) {
+        record_error("fused kernel launch (delta)", e);
+        return SKA_ERR_CUDA;
+      }
+    }
+    ck.pass = 2;
+  }
+  for (int c = 0; c < nchunks; ++c) {
+    ck.j0 = c * kc;
+    ck.accumulate = c > 0;
+    if (cudaError_t e = launch_sa_bwd(D, sms, mQ, mDO, mK, mV, p, ck, s); e != cudaSuccess) {
+      record_error("fused kernel launch", e);
+      return SKA_ERR_CUDA;
+    }
+    if (cudaError_t e_ = launch_sa_bwd_finish(p, ck, D, dq, s); e_ != cudaSuccess) { record_error("launch_sa_bwd_finish", e_); return SKA_ERR_CUDA; }
+  }
   return SKA_OK;
 }
 

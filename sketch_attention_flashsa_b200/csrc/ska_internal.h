@@ -112,20 +112,34 @@ struct SaBwdParams {
   const __nv_bfloat16* dsketch;// [B,H,k,d] (TOKEN: D_j)
   float* dk;                   // [T,H,d]
   float* dv;                   // [T,H,d]
-  float* dq_partial;           // [(B*H + ctas) * k * d]
+  float* dq_partial;           // [(B*H + ctas) * k * d], k = this launch's prototypes
   int B, H, k, total_tokens, q_per_user;
   float scale;
   uint64_t budget_ns;
 };
 
+// One launch over a chunk of a larger prototype set (its own kernel parameter: kept apart from
+// SaBwdParams, whose size the register allocation of the fused kernel turned out sensitive to).
+struct SaBwdChunk {
+  float* delta;    // PROTO: [T,H], delta_i summed over the chunks
+  int kt, j0;      // all prototypes, and the first one of this launch (one launch: k, 0)
+  int pass;        // 0: every gradient; 1: PROTO delta_i only, this chunk's part added into
+                   // delta; 2: every gradient with delta_i read from delta
+  int accumulate;  // dK, dV added to the previous chunk's
+};
+
 bool sa_bwd_supported(int head_dim, int num_protos);
+// Prototypes per launch: num_protos itself when one CTA holds them all, else the chunk size
+// (128 for head_dim 128, 256 for 64) dividing num_protos; 0 if unsupported.
+int sa_bwd_chunk(int head_dim, int num_protos);
 size_t sa_bwd_smem_bytes(int head_dim, int num_protos);
 cudaError_t launch_sa_bwd(int head_dim, int num_ctas, const CUtensorMap& mapQ, const CUtensorMap& mapDO,
                           const CUtensorMap& mapK, const CUtensorMap& mapV, const SaBwdParams& p,
-                          cudaStream_t stream);
+                          const SaBwdChunk& ck, cudaStream_t stream);
 // dq = scale * sum of the partial slots of every segment with head h (shared prototypes) or of
 // segment (b, h) (per-user queries), in a fixed order; also zeroes dK/dV rows of padding tokens.
-cudaError_t launch_sa_bwd_finish(const SaBwdParams& p, int head_dim, float* dq, cudaStream_t stream);
+cudaError_t launch_sa_bwd_finish(const SaBwdParams& p, const SaBwdChunk& ck, int head_dim, float* dq,
+                                 cudaStream_t stream);
 
 // Parameters of the stacked refinement of the sketch (sa_refine.cu): rows (b, h, j) of
 // [B, H, k, D] fp32 tensors; per-head LayerNorm vectors [H, D] (nullable: gamma 1, beta 0).

@@ -124,11 +124,20 @@ def test_empty_batch_is_a_no_op_on_the_host():
 
 
 @pytest.mark.parametrize("kw,code", [
-    ({"in_dtype": L.SKA_F32}, UNSUP), ({"num_protos": 512}, UNSUP), ({"num_protos": 48}, UNSUP),
-    ({"head_dim": 128, "num_protos": 256}, UNSUP), ({"scale": 0.0}, INVALID), ({"norm": 3}, INVALID),
+    ({"in_dtype": L.SKA_F32}, UNSUP), ({"num_protos": 48}, UNSUP),
+    # beyond one CTA: multiples of the chunk (256 at d = 64, 128 at d = 128) up to 4096 only
+    ({"num_protos": 640}, UNSUP), ({"num_protos": 8192}, UNSUP), ({"head_dim": 128, "num_protos": 200}, UNSUP),
+    ({"head_dim": 128, "num_protos": 4224}, UNSUP), ({"scale": 0.0}, INVALID), ({"norm": 3}, INVALID),
 ])
 def test_sa_backward_rejects(kw, code):
     assert bwd(sa_desc(**kw)) == code
+
+
+@pytest.mark.parametrize("kw", [{"num_protos": 512}, {"num_protos": 4096}, {"head_dim": 128, "num_protos": 256},
+                                {"head_dim": 128, "num_protos": 384}, {"head_dim": 128, "num_protos": 1024}])
+def test_sa_backward_accepts_prototype_chunks(kw):
+    # supported shapes pass the host checks and stop only at the missing device
+    assert bwd(sa_desc(**kw)) == L.SKA_ERR_CUDA
 
 
 def test_sa_backward_pointer_checks():

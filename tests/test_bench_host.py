@@ -24,7 +24,7 @@ def test_committed_traffic_entries_name_real_workloads_and_sources():
             continue
         assert workload in bench.WORKLOADS, workload
         for norm, entry in per_norm.items():
-            assert norm in ("proto", "token", "stca", "refine"), (workload, norm)
+            assert norm in ("proto", "token", "stca", "refine", "stca_bwd"), (workload, norm)
             assert os.path.exists(os.path.join(bench.ROOT, entry["source"])), entry["source"]
             assert entry["bytes"] > 0 and len(entry["source_sha256"]) == 16
 

@@ -60,6 +60,45 @@ def test_backward_parity_small(name, norm):
     check_bwd(inp, norm)
 
 
+# More prototypes than one CTA holds: one launch per chunk of 128 (d = 128) or 256 (d = 64)
+# prototypes, PROTO's delta_i summed over the chunks by a first pass.
+CHUNK_CASES = {
+    "d128_k256": ([1, 127, 129, 600], 2, 128, 256),
+    "d128_k384": ([250, 3], 1, 128, 384),
+    "d128_k512": ([300, 0, 517], 2, 128, 512),
+    "d64_k512": ([700, 129], 2, 64, 512),
+    "d64_k1024": ([400], 1, 64, 1024),
+}
+
+
+@pytest.mark.parametrize("norm", ["proto", "token"])
+@pytest.mark.parametrize("name", sorted(CHUNK_CASES))
+def test_backward_parity_prototype_chunks(name, norm):
+    lengths, H, d, k = CHUNK_CASES[name]
+    inp = W.make_sa(lengths, H, d, k, seed=540 + len(name) + k, with_dsketch=True, dsketch_seed=17)
+    check_bwd(inp, norm)
+
+
+@pytest.mark.parametrize("norm", ["proto", "token"])
+def test_backward_prototype_chunks_padding_per_user(norm):
+    inp = W.make_sa([200, 0, 300, 130], 2, 128, 512, seed=57, seqused=[150, 0, 1, 130], per_user_q=True,
+                    with_dsketch=True, dsketch_seed=18)
+    dq, dk, dv = check_bwd(inp, norm)
+    assert (dk[150:200] == 0).all() and (dv[150:200] == 0).all()
+    assert (dk[201:500] == 0).all() and (dv[201:500] == 0).all()
+
+
+@pytest.mark.parametrize("norm", ["proto", "token"])
+def test_backward_prototype_chunks_deterministic(norm):
+    inp = W.make_sa([3000, 1700], 2, 128, 512, seed=58, with_dsketch=True, dsketch_seed=19)
+    nid = W.NORM_PROTO if norm == "proto" else W.NORM_TOKEN
+    osk, olse, _ = oracle.sa_forward(f64(inp.q), f64(inp.k), f64(inp.v), inp.cu_seqlens.numpy(), None, 1.0, nid)
+    a = run_bwd(inp, norm, osk, olse)
+    b = run_bwd(inp, norm, osk, olse)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
 @pytest.mark.parametrize("norm", ["proto", "token"])
 def test_backward_padding_empty_per_user(norm):
     inp = W.make_sa([200, 0, 300, 130], 2, 64, 256, seed=51, seqused=[150, 0, 1, 130], per_user_q=True,
@@ -123,3 +162,13 @@ def test_backward_config4_full(norm):
         worst = max(worst, mk, mv)
     assert_close(dq, odq, f"{norm} dq (all users)")
     print(f"[parity] dK, dV of all {B} users, worst max abs {worst:.3e}")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("norm", ["proto", "token"])
+def test_backward_production_shape_k1024(norm):
+    """App. G.5's shapes (d = 128, k up to 1024): 6 ragged users up to 24K tokens, H = 2,
+    k = 1024 (eight chunks of 128 prototypes); dQ, dK and dV of every user against the oracle."""
+    inp = W.make_sa([24_000, 9_001, 1, 16_384, 130, 20_000], 2, 128, 1024, seed=59, with_dsketch=True,
+                    dsketch_seed=20)
+    check_bwd(inp, norm)
