@@ -9,6 +9,8 @@ combine, lse fill). The other rows of the path run with --workload (same JSON co
   sa_fwd_*                          one step = one sa_forward call (--norm proto|token)
   sa_bwd_b64_ragged_h4_d64_k256     one step = one sa_backward call: 64 ragged users (1.45M
                                     tokens), H=4, d=64, k=256 -> dQ, dK, dV (--norm proto|token)
+  sa_bwd_b8_l100k_h8_d128_k512      the same at the headline shapes (launches over chunks of 128
+                                    prototypes; the kernel time spans all of them)
   stca_b16_t512_h4_d64_l10k_s256    one step = one stca_forward call: 16 users x 512 targets over
                                     [10,000 suffix ; 256 sketch] keys, H=4, d=64
 
@@ -70,6 +72,9 @@ WORKLOADS = {
     "sa_bwd_b64_ragged_h4_d64_k256": dict(kind="sa_bwd", lens="ragged64", H=4, d=64, k=256, seqused=None),
     # profiling size for the backward: 2 x 100K, one head, same per-tile work
     "sa_bwd_b2_l100k_h1_d64_k256": dict(kind="sa_bwd", lens=[100_000] * 2, H=1, d=64, k=256, seqused=None),
+    # the backward at the headline forward's shapes (k = 512, d = 128: four launches over chunks of 128
+    # prototypes, PROTO with a delta pass per chunk first)
+    "sa_bwd_b8_l100k_h8_d128_k512": dict(kind="sa_bwd", lens=[100_000] * 8, H=8, d=128, k=512, seqused=None),
     # the refinement layer on the sketch of the 8 x 100K workload (8 users x 8 heads x 512 rows, d = 128)
     "refine_b8_h8_k512_d128": dict(kind="refine", B=8, H=8, k=512, d=128),
     # two stacked SA layers (§3.3) over the 8 x 100K workload, own keys per layer, V = the history
@@ -268,9 +273,14 @@ class SaBwdJob:
         self.bytes = (T * H * d * (2 + 2 + 4 + 4) + (T * H * 4 if norm == "proto" else B * H * kp * 4)
                       + B * H * kp * d * (2 + (4 if norm == "token" else 0)) + H * kp * d * (2 + 4))
         self.kernel = "sa_bwd_kernel"
-        self.launches = 4
+        # schedule, then per chunk of prototypes the fused kernel, the dQ reduction and the padding
+        # zeroing (PROTO over several chunks: one delta pass per chunk first)
+        one = kp <= (256 if d == 64 else 128)
+        nch = 1 if one else kp // (256 if d == 64 else 128)
+        self.launches = 1 + 3 * nch + (nch if (norm == "proto" and nch > 1) else 0)
+        self.chunks = nch
         self.config = {"users_per_gpu": B, "heads": H, "head_dim": d, "protos": kp, "norm": norm,
-                       "tokens_per_gpu": T, "outputs": "dQ, dK, dV fp32",
+                       "tokens_per_gpu": T, "outputs": "dQ, dK, dV fp32", "prototype_chunks": nch,
                        "l2": "inputs larger than L2 (K and V are %.2f GB each per GPU)" % (T * H * d * 2 / 1e9)}
 
     def run(self, x):
