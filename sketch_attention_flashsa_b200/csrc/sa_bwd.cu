@@ -10,7 +10,7 @@
 //   softmax-gradient: PROTO dS = A (dA - delta_i) with delta_i = sum_j A_ji dA_ji in fp32 (each
 //        warpgroup sums its half of the prototypes, the halves are added in a fixed order);
 //        TOKEN dS = A (dA - D_j) with D_j = dO_j . O_j from the forward sketch. dS goes to smem
-//        as a bf16 pair hi + lo.
+//        as a bf16 pair hi + lo (16 significant bits).
 //   MMA  dK   = dS^T . Q        (M=tok, N=d)   -> TMEM from the hi half (both halves over prototype
 //        chunks), scaled on the way out
 //   MMA  dQ  += dS . K          (M=proto, N=d) -> TMEM, both halves; restarted every 16 tiles and
@@ -332,16 +332,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int jj = col0 + c;
         const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
         if constexpr (CHUNK) {
-          float hi[8], lo[8];
+          uint32_t wh[4], wl[4];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            hi[u] = __bfloat162float(__float2bfloat16_rn(a[c + u]));
-            lo[u] = a[c + u] - hi[u];
-          }
-          *reinterpret_cast<uint4*>(sA + off) = make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]),
-                                                           pack_bf16x2(hi[4], hi[5]), pack_bf16x2(hi[6], hi[7]));
-          *reinterpret_cast<uint4*>(sLo + off) = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]),
-                                                            pack_bf16x2(lo[4], lo[5]), pack_bf16x2(lo[6], lo[7]));
+          for (int u = 0; u < 8; u += 2) split_bf16x2(f2_pack(a[c + u], a[c + u + 1]), wh[u / 2], wl[u / 2]);
+          *reinterpret_cast<uint4*>(sA + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          *reinterpret_cast<uint4*>(sLo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
         } else {
           *reinterpret_cast<uint4*>(sA + off) = make_uint4(pack_bf16x2(a[c], a[c + 1]), pack_bf16x2(a[c + 2], a[c + 3]),
                                                            pack_bf16x2(a[c + 4], a[c + 5]), pack_bf16x2(a[c + 6], a[c + 7]));
@@ -437,23 +432,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int h8 = 0; h8 < DC; h8 += 8) {
         const int c = c0 + h8;
-        float hi[8], lo[8];
+        uint32_t wh[4], wl[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float sub = (p.norm == SKA_NORM_PROTO) ? delta : sDj[col0 + c + u];
-          const float ds = a[c + u] * (__uint_as_float(da[h8 + u]) - sub);
-          hi[u] = __bfloat162float(__float2bfloat16_rn(ds));
-          lo[u] = ds - hi[u];
+        for (int u = 0; u < 8; u += 2) {  // in fp32 pairs
+          const uint64_t sub = (p.norm == SKA_NORM_PROTO) ? f2_pack(delta, delta)
+                                                          : f2_pack(sDj[col0 + c + u], sDj[col0 + c + u + 1]);
+          const uint64_t ds = f2_mul(f2_pack(a[c + u], a[c + u + 1]),
+                                     f2_sub(f2_pack(__uint_as_float(da[h8 + u]), __uint_as_float(da[h8 + u + 1])), sub));
+          split_bf16x2(ds, wh[u / 2], wl[u / 2]);
         }
         const int jj = col0 + c;
-        uint4 wh, wl;
-        wh.x = pack_bf16x2(hi[0], hi[1]); wh.y = pack_bf16x2(hi[2], hi[3]);
-        wh.z = pack_bf16x2(hi[4], hi[5]); wh.w = pack_bf16x2(hi[6], hi[7]);
-        wl.x = pack_bf16x2(lo[0], lo[1]); wl.y = pack_bf16x2(lo[2], lo[3]);
-        wl.z = pack_bf16x2(lo[4], lo[5]); wl.w = pack_bf16x2(lo[6], lo[7]);
         const uint32_t off = (jj >> 6) * kBlk + sw128_offset(r, (jj & 63) * 2);
-        *reinterpret_cast<uint4*>(sA + off) = wh;
-        *reinterpret_cast<uint4*>(sLo + off) = wl;
+        *reinterpret_cast<uint4*>(sA + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        *reinterpret_cast<uint4*>(sLo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
       }
     }
     fence_async_shared();

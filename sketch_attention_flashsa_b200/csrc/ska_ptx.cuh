@@ -400,6 +400,22 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   return r;
 }
 
+// Two-term bf16 split of a packed fp32 pair x = (x0, x1) for the hi + lo MMA passes: hi = each value
+// rounded to 8 significant bits on its integer bits (add half a bf16 unit, keep the top 16 bits:
+// ties away from zero), lo = bf16(x - hi) rounded to nearest. x - hi is exact in fp32 and at most
+// 2^-8 |x|, so hi + lo is x to within 2^-17 |x|, and hi alone is a rounded (unbiased) bf16 value.
+// x0 goes to the low halves of both words (the MMA's element order). Finite x only.
+__device__ __forceinline__ void split_bf16x2(uint64_t x, uint32_t& hi, uint32_t& lo) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint32_t b0 = __float_as_uint(x0) + 0x8000u, b1 = __float_as_uint(x1) + 0x8000u;
+  hi = __byte_perm(b0, b1, 0x7632);
+  const uint64_t h = f2_pack(__uint_as_float(b0 & 0xffff0000u), __uint_as_float(b1 & 0xffff0000u));
+  float l0, l1;
+  f2_unpack(f2_sub(x, h), l0, l1);
+  lo = pack_bf16x2(l0, l1);
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

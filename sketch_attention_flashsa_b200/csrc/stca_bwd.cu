@@ -575,18 +575,16 @@ __global__ void __launch_bounds__(kSbThreads, 1)
           tmem_ld32(tP + lane_off + c0, dp);
           tmem_ld_wait();
           uint32_t hw[16], lw[16];
+          const uint64_t del2 = f2_pack(del, del);
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
-            float hi[2], lo[2];
+            float pe[2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const float pe = (c0 + u + e < nvalid) ? ex2_approx(fmaf(__uint_as_float(sv[u + e]), c2, -lse2)) : 0.f;
-              const float ds = pe * (__uint_as_float(dp[u + e]) - del);
-              hi[e] = __bfloat162float(__float2bfloat16_rn(ds));
-              lo[e] = ds - hi[e];
-            }
-            hw[u / 2] = pack_bf16x2(hi[0], hi[1]);
-            lw[u / 2] = pack_bf16x2(lo[0], lo[1]);
+            for (int e = 0; e < 2; ++e)
+              pe[e] = (c0 + u + e < nvalid) ? ex2_approx(fmaf(__uint_as_float(sv[u + e]), c2, -lse2)) : 0.f;
+            const uint64_t ds = f2_mul(f2_pack(pe[0], pe[1]),
+                                       f2_sub(f2_pack(__uint_as_float(dp[u]), __uint_as_float(dp[u + 1])), del2));
+            split_bf16x2(ds, hw[u / 2], lw[u / 2]);
           }
           // hi over S, lo over dP: this group's first 16 columns of each (already read)
           tmem_st16(tS + lane_off + c0, hw);
