@@ -3,10 +3,12 @@
 // The FFN is the SwiGLU of App. G.1 with intermediate width F = 2d (App. G.3). It is applied to
 // every sketch row (b, h, j), using the weights and LayerNorm parameters of head h.
 //
-// One CTA of 128 threads takes 128 rows of one (user, head) at a time, one thread per row:
-//   1. X- = LN1(x_tilde + x_hat) in fp32. The thread parks it in its own row of the output for the
+// One CTA of 512 threads takes 128 rows of one (user, head) at a time, four threads per row, each
+// on a quarter of the columns (LayerNorm statistics combined through shared memory):
+//   1. X- = LN1(x_tilde + x_hat) in fp32. The thread keeps its slice in registers for the
 //      residual of step 5. It is also written to shared memory as a bf16 pair hi + lo
-//      (16 significant bits) in the K-major A-operand layout.
+//      (16 significant bits) in the K-major A-operand layout. Thread 0 then prefetches the CTA's
+//      next tile of x_tilde and x_hat into L2.
 //   2. MMA: H1 = X- W_1 and Hg = X- W_g (M = 128, N = F, K = d; one pass for hi, one for lo),
 //      accumulated in TMEM.
 //   3. G = swish(H1) * Hg, again as a bf16 hi + lo pair in shared memory.
@@ -354,8 +356,6 @@ __global__ void __launch_bounds__(kRefThreads, 1)
                               p.eps, red, grp, r);
       if (valid) {
         if (p.x_bar) store_row_f32<XC>(p.x_bar + row * D + xc0, xb);
-        // X- in fp32 waits in this thread's slice of its output row for the residual of step 5
-        store_row_f32<XC>(p.x_next + row * D + xc0, xb);
       } else {
 #pragma unroll
         for (int u = 0; u < XC; ++u) xb[u] = 0.f;
@@ -365,6 +365,17 @@ __global__ void __launch_bounds__(kRefThreads, 1)
       fence_async_shared();
       __syncwarp();
       if ((threadIdx.x & 31) == 0) mbar_arrive(&bars.x);
+      if (ctl && tile + static_cast<int>(gridDim.x) < ntiles) {
+        // the next tile's rows of x_tilde and x_hat into L2 while this tile computes
+        const int nt = tile + gridDim.x;
+        const int nh = nt / (p.B * tiles_per_bh), nrem = nt - nh * p.B * tiles_per_bh;
+        const int nb = nrem / tiles_per_bh, nj0 = (nrem - nb * tiles_per_bh) * 128;
+        const uint32_t bytes = static_cast<uint32_t>(min(128, p.k - nj0)) * D * 4;
+        const int64_t nrow = (static_cast<int64_t>(nb) * p.H + nh) * p.k + nj0;
+        const int64_t nxrow = p.x_tilde_shared ? static_cast<int64_t>(nh) * p.k + nj0 : nrow;
+        bulk_prefetch_l2(p.x_tilde + nxrow * D, bytes);
+        bulk_prefetch_l2(p.x_hat + nrow * D, bytes);
+      }
       // 2. H1 = X- W_1, Hg = X- W_g
       if (ctl) {
         ok = wait(&bars.x, par) && wait(&bars.w1g, par);
@@ -394,13 +405,13 @@ __global__ void __launch_bounds__(kRefThreads, 1)
       }
       // 3. G = swish(H1) * Hg into region B (W_1 / W_g are no longer read), this thread's slice
 #pragma unroll 1
-      for (int c = gc0; c < gc0 + GC; c += 32) {
-        uint32_t v1[32], vg[32];
-        tmem_ld32(tb + lane_off + c, v1);
-        tmem_ld32(tb + lane_off + F + c, vg);
+      for (int c = gc0; c < gc0 + GC; c += 16) {  // (16 columns at a time: X- stays in registers)
+        uint32_t v1[16], vg[16];
+        tmem_ld16(tb + lane_off + c, v1);
+        tmem_ld16(tb + lane_off + F + c, vg);
         tmem_ld_wait();
 #pragma unroll
-        for (int u = 0; u < 32; u += 8) {
+        for (int u = 0; u < 16; u += 8) {
           float gv[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -435,13 +446,7 @@ __global__ void __launch_bounds__(kRefThreads, 1)
       if (!__syncthreads_and(ok && wait(&bars.m2, par))) break;
       tc_fence_after();
       if (ctl && p.q_next) load_wq(h);  // region B is free: MMA2 has read G
-      // 5. X~' = LN2(X- + Y)
-      if (valid) {
-        load_slice<XC>(p.x_next + row * D + xc0, xb);
-      } else {
-#pragma unroll
-        for (int u = 0; u < XC; ++u) xb[u] = 0.f;
-      }
+      // 5. X~' = LN2(X- + Y), X- still in xb (zero on rows past k)
 #pragma unroll
       for (int c = 0; c < XC; c += 16) {
         uint32_t yv[16];
