@@ -1,7 +1,7 @@
 // SA backward on sm_100a: gradients of <dSketch, sketch> through SequenceO1 §3.1 Eq. (7)-(9)
 // (SA is trained end to end, App. A.4), for both normalisations.
 //
-// Per 128-token tile of one (user, head), one CTA holding all k <= 256 prototypes, tokens on
+// Per 128-token tile of one (user, head), one CTA holding the launch's KP <= 256 prototypes, tokens on
 // TMEM lanes (S^T orientation):
 //   MMA  S^T  = K . Q^T                        -> A = exp(scale s - lse) (PROTO: per-token lse;
 //                                                 TOKEN: per-prototype lse), to smem in bf16
