@@ -75,6 +75,8 @@ WORKLOADS = {
     # the backward at the headline forward's shapes (k = 512, d = 128: four launches over chunks of 128
     # prototypes, PROTO with a delta pass per chunk first)
     "sa_bwd_b8_l100k_h8_d128_k512": dict(kind="sa_bwd", lens=[100_000] * 8, H=8, d=128, k=512, seqused=None),
+    # profiling size for it: 2 x 100K, one head, the same per-tile work
+    "sa_bwd_b2_l100k_h1_d128_k512": dict(kind="sa_bwd", lens=[100_000] * 2, H=1, d=128, k=512, seqused=None),
     # the refinement layer on the sketch of the 8 x 100K workload (8 users x 8 heads x 512 rows, d = 128)
     "refine_b8_h8_k512_d128": dict(kind="refine", B=8, H=8, k=512, d=128),
     # two stacked SA layers (§3.3) over the 8 x 100K workload, own keys per layer, V = the history

@@ -518,21 +518,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         stage_row(stk, kr, p.scale);
         stage_row(stv, vr, 1.f);
         __syncwarp();
+        if (accumulate) {
+          // the previous chunks' values, all in flight together before any store (a load placed
+          // after a store of the same arrays cannot be moved ahead of it)
+          float4 pk[8], pv[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int row = q4 * 32 + 4 * u + (lane >> 3);  // token row in the tile
-          const int64_t tk = static_cast<int64_t>(tok0) + row;
-          if (row < urows && tk < p.total_tokens) {
+          for (int u = 0; u < 8; ++u) {
+            const int row = q4 * 32 + 4 * u + (lane >> 3);
+            const int64_t tk = static_cast<int64_t>(tok0) + row;
             const int64_t off = (tk * p.H + t.h) * D + cc + (lane & 7) * 4;
-            float4 gk = staged(stk, u), gv = staged(stv, u);
-            if (accumulate) {
-              const float4 pk = *reinterpret_cast<const float4*>(p.dk + off);
-              const float4 pv = *reinterpret_cast<const float4*>(p.dv + off);
-              gk.x += pk.x; gk.y += pk.y; gk.z += pk.z; gk.w += pk.w;
-              gv.x += pv.x; gv.y += pv.y; gv.z += pv.z; gv.w += pv.w;
+            const bool in = row < urows && tk < p.total_tokens;
+            pk[u] = in ? *reinterpret_cast<const float4*>(p.dk + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+            pv[u] = in ? *reinterpret_cast<const float4*>(p.dv + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int row = q4 * 32 + 4 * u + (lane >> 3);
+            const int64_t tk = static_cast<int64_t>(tok0) + row;
+            if (row < urows && tk < p.total_tokens) {
+              const int64_t off = (tk * p.H + t.h) * D + cc + (lane & 7) * 4;
+              float4 gk = staged(stk, u), gv = staged(stv, u);
+              gk.x += pk[u].x; gk.y += pk[u].y; gk.z += pk[u].z; gk.w += pk[u].w;
+              gv.x += pv[u].x; gv.y += pv[u].y; gv.z += pv[u].z; gv.w += pv[u].w;
+              *reinterpret_cast<float4*>(p.dk + off) = gk;
+              *reinterpret_cast<float4*>(p.dv + off) = gv;
             }
-            *reinterpret_cast<float4*>(p.dk + off) = gk;
-            *reinterpret_cast<float4*>(p.dv + off) = gv;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int row = q4 * 32 + 4 * u + (lane >> 3);  // token row in the tile
+            const int64_t tk = static_cast<int64_t>(tok0) + row;
+            if (row < urows && tk < p.total_tokens) {
+              const int64_t off = (tk * p.H + t.h) * D + cc + (lane & 7) * 4;
+              *reinterpret_cast<float4*>(p.dk + off) = staged(stk, u);
+              *reinterpret_cast<float4*>(p.dv + off) = staged(stv, u);
+            }
           }
         }
         __syncwarp();
