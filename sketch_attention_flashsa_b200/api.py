@@ -35,6 +35,14 @@ def _dev_tensor(name, t, dtypes):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _dtypes(pairs, dtypes):
+    """Dtype checks of several tensors, ahead of any device check (a wrong dtype is reported as such
+    wherever the tensor lives)."""
+    for name, t in pairs:
+        if t is not None and t.dtype not in dtypes:
+            raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+
+
 def _shape(name, t, want):
     if t is not None and tuple(t.shape) != tuple(want):
         raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(want)}")
@@ -475,10 +483,14 @@ def sa_refine(x_tilde: torch.Tensor, x_hat: torch.Tensor, w1: torch.Tensor, wg: 
     for name, t in (("gamma1", gamma1), ("beta1", beta1), ("gamma2", gamma2), ("beta2", beta2)):
         _shape(name, t, (H, D))
     _shape("out", out, x_hat.shape)
-    for name, t in (("x_tilde", x_tilde), ("x_hat", x_hat), ("gamma1", gamma1), ("beta1", beta1),
-                    ("gamma2", gamma2), ("beta2", beta2), ("out", out)):
+    acts = (("x_tilde", x_tilde), ("x_hat", x_hat), ("gamma1", gamma1), ("beta1", beta1), ("gamma2", gamma2),
+            ("beta2", beta2), ("out", out))
+    weights = (("w1", w1), ("wg", wg), ("w2", w2), ("w_q_next", w_q_next))
+    _dtypes(acts, (torch.float32,))
+    _dtypes(weights, (torch.bfloat16,))
+    for name, t in acts:
         _dev_tensor(name, t, (torch.float32,))
-    for name, t in (("w1", w1), ("wg", wg), ("w2", w2), ("w_q_next", w_q_next)):
+    for name, t in weights:
         _dev_tensor(name, t, (torch.bfloat16,))
     desc = refine_desc(x_tilde, x_hat, w1, eps=eps)
     L = _lib.lib()
@@ -512,6 +524,8 @@ def project_queries(x: torch.Tensor, w_q: torch.Tensor, *, workspace: Optional[t
     B, H, k, D = shape4
     _shape("w_q", w_q, (H, D, D))
     _shape("out", out, x.shape)
+    _dtypes((("x", x),), (torch.float32,))
+    _dtypes((("w_q", w_q), ("out", out)), (torch.bfloat16,))
     _dev_tensor("x", x, (torch.float32,))
     _dev_tensor("w_q", w_q, (torch.bfloat16,))
     _dev_tensor("out", out, (torch.bfloat16,))

@@ -114,3 +114,78 @@ def stca(**over):
 def test_stca_rejects_mismatched_tensors(over, msg):
     with pytest.raises(ValueError, match=msg):
         stca(**over)
+
+
+def stca_bwd(**over):
+    a = dict(q=torch.zeros(Tq, H, D, dtype=bf), cu_targets=torch.tensor([0, 15, 40], dtype=i32),
+             k_hist=torch.zeros(Th, H, D, dtype=bf), v_hist=torch.zeros(Th, H, D, dtype=bf),
+             cu_hist=torch.tensor([0, 30, 70], dtype=i32), k_sk=torch.zeros(2, H, KS, D, dtype=bf),
+             v_sk=torch.zeros(2, H, KS, D, dtype=bf), out=torch.zeros(Tq, H, D, dtype=f32),
+             lse=torch.zeros(Tq, H, dtype=f32), dout=torch.zeros(Tq, H, D, dtype=bf))
+    kw = {k: v for k, v in over.items() if k not in a}
+    a.update({k: v for k, v in over.items() if k in a})
+    return api.stca_backward(a["q"], a["cu_targets"], a["k_hist"], a["v_hist"], a["cu_hist"], a["k_sk"], a["v_sk"],
+                             a["out"], a["lse"], a["dout"], scale=0.125, **kw)
+
+
+@pytest.mark.parametrize("over,msg", [
+    (dict(q=torch.zeros(Tq, H, D, dtype=f32)), "dtype"),
+    (dict(dout=torch.zeros(Tq, H, D, dtype=f32)), "dtype"),
+    (dict(q=torch.zeros(Tq, H * D, dtype=bf)), "q must be"),
+    (dict(cu_targets=torch.tensor([0, 15, 40], dtype=torch.int64)), "cu_targets"),
+    (dict(cu_hist=torch.tensor([0, 70], dtype=i32)), "cu_hist"),
+    (dict(k_hist=torch.zeros(Th, H + 1, D, dtype=bf)), "k_hist"),
+    (dict(v_hist=torch.zeros(Th + 1, H, D, dtype=bf)), "v_hist"),
+    (dict(v_sk=None), "together"),
+    (dict(k_sk=torch.zeros(3, H, KS, D, dtype=bf)), "k_sk"),
+    (dict(out=torch.zeros(Tq, H, D + 1, dtype=f32)), "out"),
+    (dict(lse=torch.zeros(Tq + 1, H, dtype=f32)), "lse"),
+    (dict(dout=torch.zeros(Tq, H, D + 1, dtype=bf)), "dout"),
+    (dict(target_kv_len=torch.zeros(Tq, dtype=torch.int64)), "target_kv_len"),
+])
+def test_stca_backward_rejects_mismatched_tensors(over, msg):
+    with pytest.raises(ValueError, match=msg):
+        stca_bwd(**over)
+
+
+KR, F = 128, 2 * D
+
+
+def refine(**over):
+    a = dict(x_tilde=torch.zeros(B, H, KR, D, dtype=f32), x_hat=torch.zeros(B, H, KR, D, dtype=f32),
+             w1=torch.zeros(H, D, F, dtype=bf), wg=torch.zeros(H, D, F, dtype=bf), w2=torch.zeros(H, F, D, dtype=bf))
+    kw = {k: v for k, v in over.items() if k not in a}
+    a.update({k: v for k, v in over.items() if k in a})
+    return api.sa_refine(a["x_tilde"], a["x_hat"], a["w1"], a["wg"], a["w2"], **kw)
+
+
+@pytest.mark.parametrize("over,msg", [
+    (dict(x_hat=torch.zeros(H, KR, D, dtype=f32)), "x_hat must be"),
+    (dict(x_tilde=torch.zeros(B, H, KR + 1, D, dtype=f32)), "x_tilde"),
+    (dict(x_tilde=torch.zeros(H + 1, KR, D, dtype=f32)), "x_tilde"),       # shared rows: [H, k, d]
+    (dict(w1=torch.zeros(H, D + 1, F, dtype=bf)), "w1 must be"),
+    (dict(wg=torch.zeros(H, D, F + 8, dtype=bf)), "wg"),
+    (dict(w2=torch.zeros(H, D, F, dtype=bf)), "w2"),                         # [H, F, d], not [H, d, F]
+    (dict(w_q_next=torch.zeros(H, D, D + 1, dtype=bf)), "w_q_next"),
+    (dict(gamma1=torch.zeros(H, D + 1, dtype=f32)), "gamma1"),
+    (dict(beta2=torch.zeros(H + 1, D, dtype=f32)), "beta2"),
+    (dict(out=torch.zeros(B, H, KR, D + 1, dtype=f32)), "out"),
+    (dict(x_hat=torch.zeros(B, H, KR, D, dtype=bf), x_tilde=torch.zeros(B, H, KR, D, dtype=bf)), "dtype"),
+    (dict(w1=torch.zeros(H, D, F, dtype=f32)), "dtype"),
+])
+def test_refine_rejects_mismatched_tensors(over, msg):
+    with pytest.raises(ValueError, match=msg):
+        refine(**over)
+
+
+@pytest.mark.parametrize("x,w_q,out,msg", [
+    (torch.zeros(KR, D, dtype=f32), torch.zeros(H, D, D, dtype=bf), None, "x must be"),
+    (torch.zeros(H, KR, D, dtype=f32), torch.zeros(H + 1, D, D, dtype=bf), None, "w_q"),
+    (torch.zeros(B, H, KR, D, dtype=f32), torch.zeros(H, D, D, dtype=bf), torch.zeros(B, H, KR, D + 1, dtype=bf),
+     "out"),
+    (torch.zeros(H, KR, D, dtype=bf), torch.zeros(H, D, D, dtype=bf), None, "dtype"),
+    (torch.zeros(H, KR, D, dtype=f32), torch.zeros(H, D, D, dtype=f32), None, "dtype"),
+])
+def test_project_queries_rejects_mismatched_tensors(x, w_q, out, msg):
+    with pytest.raises(ValueError, match=msg):
+        api.project_queries(x, w_q, out=out)
