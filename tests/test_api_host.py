@@ -189,3 +189,29 @@ def test_refine_rejects_mismatched_tensors(over, msg):
 def test_project_queries_rejects_mismatched_tensors(x, w_q, out, msg):
     with pytest.raises(ValueError, match=msg):
         api.project_queries(x, w_q, out=out)
+
+
+def test_cache_keys_have_the_c_layout():
+    """cache_keys packs the fields into the 24 bytes of ska_cache_key (user id, version and
+    configuration as two 32-bit words, timestamp), with scalars broadcast over the batch."""
+    import ctypes
+    from sketch_attention_flashsa_b200 import _lib
+    keys = api.cache_keys([5, 2**40 + 3], 0xFFFFFFFE, [0x12345678, 0x9ABCDEF0], -7, device="cpu")
+    assert keys.dtype == torch.int64 and tuple(keys.shape) == (2, 3)
+    want = b"".join(bytes(_lib.CacheKey(u, 0xFFFFFFFE, c, -7))
+                    for u, c in ((5, 0x12345678), (2**40 + 3, 0x9ABCDEF0)))
+    assert ctypes.sizeof(_lib.CacheKey) == 24
+    assert keys.numpy().tobytes() == want
+
+
+@pytest.mark.parametrize("call,msg", [
+    (lambda: api.weight_histogram(torch.zeros(10, dtype=torch.float64), 8), "dtype"),
+    (lambda: api.sa_forward_diag(torch.zeros(H, K, D, dtype=f32), torch.zeros(T, H, D, dtype=bf),
+                                 torch.zeros(T, H, D, dtype=bf), torch.tensor([0, 10, 30, 50], dtype=i32)),
+     "share one dtype"),
+    (lambda: api.sa_forward_diag(torch.zeros(H + 1, K, D, dtype=bf), torch.zeros(T, H, D, dtype=bf),
+                                 torch.zeros(T, H, D, dtype=bf), torch.tensor([0, 10, 30, 50], dtype=i32)), "heads"),
+])
+def test_diagnostics_reject_mismatched_tensors(call, msg):
+    with pytest.raises(ValueError, match=msg):
+        call()
